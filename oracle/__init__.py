@@ -1,0 +1,146 @@
+"""fp64 CPU oracle for the sum-of-Kronecker-products linear layer.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The CUDA library never calls it and shares no code with it.
+
+The arithmetic lives in ``kron_oracle.c`` (plain C, double precision): it builds
+W = sum_i kron(S (.) A_i, B_i) entry by entry and multiplies naively, as the
+page "kronecker-layer-benchmark", section "1. Build W, then multiply" defines
+the layer; the backward is the chain rule through that explicit W.  This module
+only marshals numpy arrays into that library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kron_oracle.c")
+_LIB = os.path.join(_HERE, "_kron_oracle.so")
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile a C source of the oracle into a shared library (gcc, OpenMP)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-o", tmp, src]
+        )
+        os.replace(tmp, out)
+    return out
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shapes(S, A, B):
+    r, p, q = A.shape
+    r2, m1, m2 = B.shape
+    if S.shape != (p, q) or r2 != r:
+        raise ValueError(f"inconsistent factor shapes S{S.shape} A{A.shape} B{B.shape}")
+    return p, q, m1, m2, r
+
+
+class Oracle:
+    """numpy front end of one compiled copy of kron_oracle.c."""
+
+    def __init__(self, so_path: str):
+        lib = ctypes.CDLL(so_path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        L, I = ctypes.c_long, ctypes.c_int
+        lib.oracle_build_weight.argtypes = [dp, dp, dp, I, I, I, I, I, dp]
+        lib.oracle_matmul_bias.argtypes = [dp, dp, dp, L, L, L, dp]
+        lib.oracle_forward.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, dp]
+        lib.oracle_backward.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I,
+                                        dp, dp, dp, dp, dp]
+        lib.oracle_set_threads.argtypes = [I]
+        lib.oracle_get_threads.restype = I
+        self._lib = lib
+
+    def set_threads(self, n: int) -> None:
+        self._lib.oracle_set_threads(int(n))
+
+    def get_threads(self) -> int:
+        return int(self._lib.oracle_get_threads())
+
+    def weight(self, S, A, B) -> np.ndarray:
+        """Dense W = sum_i kron(S (.) A_i, B_i), shape (p*m1, q*m2)."""
+        S, A, B = _f64(S), _f64(A), _f64(B)
+        p, q, m1, m2, r = _shapes(S, A, B)
+        W = np.empty((p * m1, q * m2), dtype=np.float64)
+        self._lib.oracle_build_weight(_ptr(S), _ptr(A), _ptr(B), p, q, m1, m2, r, _ptr(W))
+        return W
+
+    def forward(self, x, S, A, B, bias=None) -> np.ndarray:
+        """y = x W + bias for x of shape (N, p*m1); returns (N, q*m2) float64."""
+        x, S, A, B = _f64(x), _f64(S), _f64(A), _f64(B)
+        p, q, m1, m2, r = _shapes(S, A, B)
+        N = x.shape[0]
+        if x.shape != (N, p * m1):
+            raise ValueError(f"x has shape {x.shape}, expected (N, {p * m1})")
+        bias = None if bias is None else _f64(bias)
+        y = np.empty((N, q * m2), dtype=np.float64)
+        self._lib.oracle_forward(_ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(bias),
+                                 N, p, q, m1, m2, r, _ptr(y))
+        return y
+
+    def backward(self, x, S, A, B, G, need_dx: bool = True, need_params: bool = True) -> dict:
+        """Gradients of <G, y> with respect to x, S, A, B and bias (float64).
+
+        Returns a dict with keys dX, dS, dA, dB, dbias (None where not requested).
+        """
+        x, S, A, B, G = _f64(x), _f64(S), _f64(A), _f64(B), _f64(G)
+        p, q, m1, m2, r = _shapes(S, A, B)
+        N = x.shape[0]
+        if x.shape != (N, p * m1) or G.shape != (N, q * m2):
+            raise ValueError("x / G shapes do not match the factors")
+        dX = np.empty_like(x) if need_dx else None
+        dS = np.empty((p, q)) if need_params else None
+        dA = np.empty((r, p, q)) if need_params else None
+        dB = np.empty((r, m1, m2)) if need_params else None
+        dbias = np.empty((q * m2,)) if need_params else None
+        self._lib.oracle_backward(_ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(G),
+                                  N, p, q, m1, m2, r,
+                                  _ptr(dX), _ptr(dS), _ptr(dA), _ptr(dB), _ptr(dbias))
+        return {"dX": dX, "dS": dS, "dA": dA, "dB": dB, "dbias": dbias}
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def set_threads(n: int) -> None:
+    default().set_threads(n)
+
+
+def get_threads() -> int:
+    return default().get_threads()
+
+
+def weight(S, A, B) -> np.ndarray:
+    return default().weight(S, A, B)
+
+
+def forward(x, S, A, B, bias=None) -> np.ndarray:
+    return default().forward(x, S, A, B, bias)
+
+
+def backward(x, S, A, B, G, need_dx: bool = True, need_params: bool = True) -> dict:
+    return default().backward(x, S, A, B, G, need_dx, need_params)

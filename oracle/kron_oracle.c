@@ -1,0 +1,194 @@
+/*
+ * kron_oracle.c -- plain, slow, fp64 CPU oracle for the sum-of-Kronecker-products
+ * linear layer.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg call it; the product path never does.  It shares
+ * no code, header or constant with the CUDA library.
+ *
+ * What it computes (page "kronecker-layer-benchmark", section "1. Build W, then
+ * multiply", the `weight()` and `forward()` methods of KronLinear):
+ *
+ *     C_i = S (.) A_i                         (elementwise, p x q)
+ *     W   = sum_i kron(C_i, B_i)              ((p*m1) x (q*m2), torch.kron order)
+ *     y   = x W + bias                        (row vectors, x is N x (p*m1))
+ *
+ * i.e. W[a*m1 + j][c*m2 + k] = sum_i C_i[a][c] * B_i[j][k].  B_i is m1 x m2
+ * (the section "2. The vec trick" allows a rectangular B: `m, n = B.shape[1:]`).
+ *
+ * The backward pass is the gradient of L = <G, y> for an upstream gradient
+ * G = dL/dy, by the chain rule through the explicit W (the page leaves the
+ * backward to autograd, section "Setup", "Training step"):
+ *
+ *     dX        = G W^T
+ *     dW        = x^T G
+ *     dC_i[a,c] = sum_{j,k} dW[a*m1+j][c*m2+k] * B_i[j][k]
+ *     dB_i[j,k] = sum_{a,c} dW[a*m1+j][c*m2+k] * C_i[a][c]
+ *     dA_i      = dC_i (.) S
+ *     dS        = sum_i dC_i (.) A_i
+ *     dbias     = sum_n G[n]
+ *
+ * Everything is double precision, row-major and contiguous:
+ *   x [N][p*m1], y and G [N][q*m2], S [p][q], A [r][p][q], B [r][m1][m2],
+ *   bias [q*m2], W [p*m1][q*m2].
+ * Loops are the definitions written out; OpenMP only splits independent output
+ * rows across threads, the summation order inside one output stays sequential.
+ */
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* W = sum_i kron(S (.) A_i, B_i), built entry by entry. */
+void oracle_build_weight(const double *S, const double *A, const double *B,
+                         int p, int q, int m1, int m2, int r, double *W)
+{
+    const long in = (long)p * m1, out = (long)q * m2;
+    memset(W, 0, sizeof(double) * (size_t)(in * out));
+    for (int i = 0; i < r; ++i)
+        for (int a = 0; a < p; ++a)
+            for (int c = 0; c < q; ++c) {
+                const double Cac = S[(long)a * q + c] * A[((long)i * p + a) * q + c];
+                for (int j = 0; j < m1; ++j)
+                    for (int k = 0; k < m2; ++k)
+                        W[((long)a * m1 + j) * out + (long)c * m2 + k] +=
+                            Cac * B[((long)i * m1 + j) * m2 + k];
+            }
+}
+
+/* y = x W + bias (bias may be NULL).  Naive triple loop, one output row per task. */
+void oracle_matmul_bias(const double *x, const double *W, const double *bias,
+                        long N, long in, long out, double *y)
+{
+    #pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n) {
+        double *yn = y + n * out;
+        for (long o = 0; o < out; ++o) yn[o] = bias ? bias[o] : 0.0;
+        const double *xn = x + n * in;
+        for (long u = 0; u < in; ++u) {
+            const double xv = xn[u];
+            const double *Wu = W + u * out;
+            for (long o = 0; o < out; ++o) yn[o] += xv * Wu[o];
+        }
+    }
+}
+
+/* Forward: builds W, then y = x W + bias. */
+void oracle_forward(const double *x, const double *S, const double *A, const double *B,
+                    const double *bias, long N, int p, int q, int m1, int m2, int r,
+                    double *y)
+{
+    const long in = (long)p * m1, out = (long)q * m2;
+    double *W = (double *)malloc(sizeof(double) * (size_t)(in * out));
+    oracle_build_weight(S, A, B, p, q, m1, m2, r, W);
+    oracle_matmul_bias(x, W, bias, N, in, out, y);
+    free(W);
+}
+
+/*
+ * Backward through the explicit W.  Any output pointer may be NULL to skip it
+ * (dX is the costly one; dW is needed by dS, dA and dB).
+ */
+void oracle_backward(const double *x, const double *S, const double *A, const double *B,
+                     const double *G, long N, int p, int q, int m1, int m2, int r,
+                     double *dX, double *dS, double *dA, double *dB, double *dbias)
+{
+    const long in = (long)p * m1, out = (long)q * m2;
+    double *W = (double *)malloc(sizeof(double) * (size_t)(in * out));
+    oracle_build_weight(S, A, B, p, q, m1, m2, r, W);
+
+    if (dX) {
+        /* dX[n][u] = sum_o G[n][o] * W[u][o] */
+        #pragma omp parallel for schedule(static)
+        for (long n = 0; n < N; ++n) {
+            const double *Gn = G + n * out;
+            for (long u = 0; u < in; ++u) {
+                const double *Wu = W + u * out;
+                double s = 0.0;
+                for (long o = 0; o < out; ++o) s += Gn[o] * Wu[o];
+                dX[n * in + u] = s;
+            }
+        }
+    }
+
+    if (dS || dA || dB) {
+        /* dW[u][o] = sum_n x[n][u] * G[n][o] */
+        double *dW = (double *)calloc((size_t)(in * out), sizeof(double));
+        #pragma omp parallel for schedule(static)
+        for (long u = 0; u < in; ++u) {
+            double *dWu = dW + u * out;
+            for (long n = 0; n < N; ++n) {
+                const double xv = x[n * in + u];
+                const double *Gn = G + n * out;
+                for (long o = 0; o < out; ++o) dWu[o] += xv * Gn[o];
+            }
+        }
+        /* dC_i[a][c] = sum_{j,k} dW[a*m1+j][c*m2+k] * B_i[j][k] */
+        double *dC = (double *)calloc((size_t)r * p * q, sizeof(double));
+        for (int i = 0; i < r; ++i)
+            for (int a = 0; a < p; ++a)
+                for (int c = 0; c < q; ++c) {
+                    double s = 0.0;
+                    for (int j = 0; j < m1; ++j)
+                        for (int k = 0; k < m2; ++k)
+                            s += dW[((long)a * m1 + j) * out + (long)c * m2 + k] *
+                                 B[((long)i * m1 + j) * m2 + k];
+                    dC[((long)i * p + a) * q + c] = s;
+                }
+        if (dB) {
+            /* dB_i[j][k] = sum_{a,c} dW[a*m1+j][c*m2+k] * C_i[a][c] */
+            for (int i = 0; i < r; ++i)
+                for (int j = 0; j < m1; ++j)
+                    for (int k = 0; k < m2; ++k) {
+                        double s = 0.0;
+                        for (int a = 0; a < p; ++a)
+                            for (int c = 0; c < q; ++c)
+                                s += dW[((long)a * m1 + j) * out + (long)c * m2 + k] *
+                                     S[(long)a * q + c] * A[((long)i * p + a) * q + c];
+                        dB[((long)i * m1 + j) * m2 + k] = s;
+                    }
+        }
+        if (dA) {
+            for (int i = 0; i < r; ++i)
+                for (long ac = 0; ac < (long)p * q; ++ac)
+                    dA[(long)i * p * q + ac] = dC[(long)i * p * q + ac] * S[ac];
+        }
+        if (dS) {
+            for (long ac = 0; ac < (long)p * q; ++ac) {
+                double s = 0.0;
+                for (int i = 0; i < r; ++i)
+                    s += dC[(long)i * p * q + ac] * A[(long)i * p * q + ac];
+                dS[ac] = s;
+            }
+        }
+        free(dC);
+        free(dW);
+    }
+
+    if (dbias) {
+        for (long o = 0; o < out; ++o) {
+            double s = 0.0;
+            for (long n = 0; n < N; ++n) s += G[n * out + o];
+            dbias[o] = s;
+        }
+    }
+    free(W);
+}

@@ -1,0 +1,260 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the oracle.
+
+Each ``pin_*`` function takes an oracle object (``oracle.Oracle``) and raises
+AssertionError when the oracle disagrees with something the pages or plain
+mathematics fix.  ``test_oracle_pins.py`` runs them on the real oracle and
+``test_oracle_mutations.py`` runs them on deliberately broken copies of it, to
+show that a dropped term, a swapped index or a transposed operand is caught.
+
+Sources of truth used here (none of them is the oracle's own loop):
+  * numpy's ``np.kron`` and ``@`` (library routines),
+  * pure-Python scalar sums on tiny inputs (brute force),
+  * Kronecker algebra: mixed product, transpose, block structure, rank one,
+  * the Van Loan rearrangement of a sum of r Kronecker products has rank <= r
+    (page "LLM Compression via Kronecker Product Decomposition", section
+    "Van Loan Rearrangement (1993)"),
+  * special shapes that reduce to a plain GEMM,
+  * central finite differences of L = <G, y> (exact here: L is affine in each
+    single parameter coordinate), and Euler's identity for functions that are
+    linear in one argument.
+"""
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+
+
+def _rand_layer(rng, p, q, m1, m2, r, s_zero=0.25, N=3):
+    S = np.ones((p, q))
+    S[rng.random((p, q)) < s_zero] = 0.0
+    A = rng.standard_normal((r, p, q))
+    B = rng.standard_normal((r, m1, m2))
+    bias = rng.standard_normal(q * m2)
+    x = rng.standard_normal((N, p * m1))
+    G = rng.standard_normal((N, q * m2))
+    return S, A, B, bias, x, G
+
+
+def pin_weight_is_sum_of_numpy_krons(orc):
+    """W equals sum_i np.kron(S*A_i, B_i) (page "kronecker-layer-benchmark", KronLinear.weight)."""
+    rng = np.random.default_rng(101)
+    for (p, q, m1, m2, r) in [(2, 3, 4, 5, 2), (3, 2, 1, 3, 3), (4, 4, 2, 2, 1), (1, 2, 3, 1, 2)]:
+        S, A, B, *_ = _rand_layer(rng, p, q, m1, m2, r)
+        ref = sum(np.kron(S * A[i], B[i]) for i in range(r))
+        W = orc.weight(S, A, B)
+        assert W.shape == (p * m1, q * m2)
+        assert np.allclose(W, ref, rtol=0, atol=1e-13), (p, q, m1, m2, r)
+
+
+def pin_forward_brute_force(orc):
+    """Tiny case: y[n, c*m2+k] = bias + sum_{i,a,j} x[n, a*m1+j] S[a,c] A_i[a,c] B_i[j,k]."""
+    rng = np.random.default_rng(102)
+    p, q, m1, m2, r, N = 2, 3, 2, 3, 2, 2
+    S, A, B, bias, x, _ = _rand_layer(rng, p, q, m1, m2, r, N=N)
+    y = orc.forward(x, S, A, B, bias)
+    for n, c, k in itertools.product(range(N), range(q), range(m2)):
+        s = bias[c * m2 + k]
+        for i, a, j in itertools.product(range(r), range(p), range(m1)):
+            s += x[n, a * m1 + j] * S[a, c] * A[i, a, c] * B[i, j, k]
+        assert abs(y[n, c * m2 + k] - s) < 1e-12, (n, c, k)
+
+
+def pin_forward_vec_trick(orc):
+    """The row-wise vec trick Y_n = sum_i C_i^T X_n B_i gives the same y
+    (page "kronecker-layer-benchmark", section "2. The vec trick": all variants agree)."""
+    rng = np.random.default_rng(103)
+    for (p, q, m1, m2, r, N) in [(8, 8, 8, 8, 2, 16), (3, 5, 4, 2, 3, 7), (6, 4, 2, 5, 1, 5)]:
+        S, A, B, bias, x, _ = _rand_layer(rng, p, q, m1, m2, r, N=N)
+        X = x.reshape(N, p, m1)
+        Y = np.zeros((N, q, m2))
+        for i in range(r):
+            Y += np.swapaxes(S * A[i], 0, 1)[None] @ (X @ B[i])
+        ref = Y.reshape(N, q * m2) + bias
+        assert np.allclose(orc.forward(x, S, A, B, bias), ref, rtol=0, atol=1e-12)
+
+
+def pin_forward_is_gemm_with_numpy_weight(orc):
+    """y = x @ W + bias with numpy's matmul on the numpy-built W (larger, ragged shapes)."""
+    rng = np.random.default_rng(104)
+    p, q, m1, m2, r, N = 5, 3, 3, 4, 3, 37
+    S, A, B, bias, x, _ = _rand_layer(rng, p, q, m1, m2, r, N=N)
+    W = sum(np.kron(S * A[i], B[i]) for i in range(r))
+    assert np.allclose(orc.forward(x, S, A, B, bias), x @ W + bias, rtol=0, atol=1e-11)
+    assert np.allclose(orc.forward(x, S, A, B, None), x @ W, rtol=0, atol=1e-11)
+
+
+def pin_mixed_product(orc):
+    """(C kron B)(C' kron B') = (C C') kron (B B') (r = 1, S = 1)."""
+    rng = np.random.default_rng(105)
+    p, q, s, m1, m2, m3 = 3, 4, 2, 2, 3, 5
+    C1, C2 = rng.standard_normal((p, q)), rng.standard_normal((q, s))
+    B1, B2 = rng.standard_normal((m1, m2)), rng.standard_normal((m2, m3))
+    W1 = orc.weight(np.ones((p, q)), C1[None], B1[None])
+    W2 = orc.weight(np.ones((q, s)), C2[None], B2[None])
+    W12 = orc.weight(np.ones((p, s)), (C1 @ C2)[None], (B1 @ B2)[None])
+    assert np.allclose(W1 @ W2, W12, rtol=0, atol=1e-12)
+
+
+def pin_transpose(orc):
+    """(sum_i C_i kron B_i)^T = sum_i C_i^T kron B_i^T; also maps the out x in convention."""
+    rng = np.random.default_rng(106)
+    p, q, m1, m2, r = 3, 5, 2, 4, 2
+    S, A, B, *_ = _rand_layer(rng, p, q, m1, m2, r)
+    W = orc.weight(S, A, B)
+    Wt = orc.weight(S.T, np.swapaxes(A, 1, 2), np.swapaxes(B, 1, 2))
+    assert np.allclose(W.T, Wt, rtol=0, atol=1e-13)
+
+
+def pin_block_structure(orc):
+    """S[a,c] = 0 makes the m1 x m2 block (a, c) of W exactly zero, other blocks are not
+    (page "kronecker-layer-benchmark", introduction: sparse S gives a block-sparse W)."""
+    rng = np.random.default_rng(107)
+    p, q, m1, m2, r = 6, 5, 3, 2, 3
+    S, A, B, *_ = _rand_layer(rng, p, q, m1, m2, r, s_zero=0.4)
+    W = orc.weight(S, A, B)
+    for a, c in itertools.product(range(p), range(q)):
+        blk = W[a * m1:(a + 1) * m1, c * m2:(c + 1) * m2]
+        if S[a, c] == 0:
+            assert np.all(blk == 0.0), (a, c)
+        else:
+            assert np.abs(blk).max() > 1e-6, (a, c)
+
+
+def pin_rank_one(orc):
+    """r = 1, S = ones: W = A kron B exactly."""
+    rng = np.random.default_rng(108)
+    A = rng.standard_normal((1, 4, 3))
+    B = rng.standard_normal((1, 2, 5))
+    W = orc.weight(np.ones((4, 3)), A, B)
+    assert np.array_equal(W, np.kron(A[0], B[0]))
+
+
+def pin_van_loan_rank(orc):
+    """The rearranged W~ (rows (a,c), columns (j,k)) equals sum_i vec(C_i) vec(B_i)^T and
+    has exactly r non-zero singular values (page "LLM Compression via Kronecker Product
+    Decomposition", section "Core Algorithm -- Van Loan Kronecker Decomposition")."""
+    rng = np.random.default_rng(109)
+    p, q, m1, m2, r = 4, 3, 3, 4, 3
+    S, A, B, *_ = _rand_layer(rng, p, q, m1, m2, r, s_zero=0.0)
+    W = orc.weight(S, A, B)
+    Wt = W.reshape(p, m1, q, m2).transpose(0, 2, 1, 3).reshape(p * q, m1 * m2)
+    outer = sum(np.outer((S * A[i]).ravel(), B[i].ravel()) for i in range(r))
+    assert np.allclose(Wt, outer, rtol=0, atol=1e-12)
+    sv = np.linalg.svd(Wt, compute_uv=False)
+    assert sv[r - 1] > 1e-6 * sv[0]
+    assert np.all(sv[r:] < 1e-10 * sv[0])
+
+
+def pin_special_shapes(orc):
+    """Shapes that reduce to a plain GEMM: m1 = m2 = 1 (W = S (.) sum_i b_i A_i, b_i the
+    1 x 1 block B_i),
+    p = q = 1 (W = S * sum_i A_i B_i) and C = I, r = 1 (W = blockdiag(B, ..., B))."""
+    rng = np.random.default_rng(110)
+    N = 6
+    # m1 = m2 = 1
+    p, q, r = 5, 4, 3
+    S, A, B, bias, x, _ = _rand_layer(rng, p, q, 1, 1, r, N=N)
+    assert np.allclose(orc.forward(x, S, A, B, bias),
+                       x @ (S * (B[:, 0, 0, None, None] * A).sum(0)) + bias, atol=1e-12)
+    # p = q = 1
+    m1, m2, r = 3, 4, 2
+    S, A, B, bias, x, _ = _rand_layer(rng, 1, 1, m1, m2, r, s_zero=0.0, N=N)
+    W = S[0, 0] * sum(A[i, 0, 0] * B[i] for i in range(r))
+    assert np.allclose(orc.forward(x, S, A, B, bias), x @ W + bias, atol=1e-12)
+    # C = I, r = 1: block-diagonal copy of B
+    p, m1, m2 = 4, 3, 2
+    B = rng.standard_normal((1, m1, m2))
+    x = rng.standard_normal((N, p * m1))
+    y = orc.forward(x, np.ones((p, p)), np.eye(p)[None], B, None)
+    for c in range(p):
+        assert np.allclose(y[:, c * m2:(c + 1) * m2], x[:, c * m1:(c + 1) * m1] @ B[0], atol=1e-12)
+
+
+def _loss(orc, x, S, A, B, bias, G):
+    return float(np.sum(G * orc.forward(x, S, A, B, bias)))
+
+
+def pin_finite_differences(orc):
+    """Central differences of L = <G, y>.  L is affine in every single coordinate of
+    x, S, A, B and bias, so the difference quotient is exact up to rounding."""
+    rng = np.random.default_rng(111)
+    p, q, m1, m2, r, N = 3, 2, 2, 3, 2, 4
+    S, A, B, bias, x, G = _rand_layer(rng, p, q, m1, m2, r, N=N)
+    g = orc.backward(x, S, A, B, G)
+    h = 0.5
+    for name, arr in (("dX", x), ("dS", S), ("dA", A), ("dB", B), ("dbias", bias)):
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            lp = _loss(orc, x, S, A, B, bias, G)
+            arr[idx] = old - h
+            lm = _loss(orc, x, S, A, B, bias, G)
+            arr[idx] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - g[name][idx]) < 1e-9 * (1 + abs(fd)), (name, idx, fd, g[name][idx])
+
+
+def pin_linearity_identities(orc):
+    """y - bias is linear in each of x, S, A and B, so by Euler's identity
+    <dX, x> = <dS, S> = <dA, A> = <dB, B> = <G, y - bias>, and <dbias, 1> = sum G."""
+    rng = np.random.default_rng(112)
+    p, q, m1, m2, r, N = 6, 5, 4, 3, 3, 29
+    S, A, B, bias, x, G = _rand_layer(rng, p, q, m1, m2, r, N=N)
+    S = S * rng.standard_normal((p, q))          # a general (not 0/1) S
+    g = orc.backward(x, S, A, B, G)
+    ref = float(np.sum(G * orc.forward(x, S, A, B, None)))
+    tol = 1e-10 * (1 + abs(ref))
+    assert abs(np.sum(g["dX"] * x) - ref) < tol
+    assert abs(np.sum(g["dS"] * S) - ref) < tol
+    assert abs(np.sum(g["dA"] * A) - ref) < tol
+    assert abs(np.sum(g["dB"] * B) - ref) < tol
+    assert np.allclose(g["dbias"], G.sum(0), atol=1e-12)
+
+
+def pin_backward_numpy_chain_rule(orc):
+    """dX = G W^T and dW = x^T G with numpy on the numpy-built W; dC, dB by contracting dW
+    with the other factor; dA = dC (.) S and dS = sum_i dC_i (.) A_i."""
+    rng = np.random.default_rng(113)
+    p, q, m1, m2, r, N = 4, 3, 2, 5, 2, 11
+    S, A, B, bias, x, G = _rand_layer(rng, p, q, m1, m2, r, N=N)
+    W = sum(np.kron(S * A[i], B[i]) for i in range(r))
+    dW = (x.T @ G).reshape(p, m1, q, m2)
+    dC = np.einsum("ajck,ijk->iac", dW, B)
+    dB = np.einsum("ajck,iac->ijk", dW, S[None] * A)
+    g = orc.backward(x, S, A, B, G)
+    assert np.allclose(g["dX"], G @ W.T, atol=1e-11)
+    assert np.allclose(g["dA"], dC * S[None], atol=1e-11)
+    assert np.allclose(g["dS"], (dC * A).sum(0), atol=1e-11)
+    assert np.allclose(g["dB"], dB, atol=1e-11)
+    assert np.allclose(g["dbias"], G.sum(0), atol=1e-12)
+
+
+def pin_zero_s_gradient(orc):
+    """Where S[a,c] = 0, dA is zero but dS is in general not (sum_i dC_i (.) A_i)."""
+    rng = np.random.default_rng(114)
+    p, q, m1, m2, r, N = 4, 4, 2, 2, 2, 9
+    S, A, B, bias, x, G = _rand_layer(rng, p, q, m1, m2, r, s_zero=0.5, N=N)
+    assert (S == 0).any()
+    g = orc.backward(x, S, A, B, G)
+    z = S == 0
+    assert np.all(g["dA"][:, z] == 0.0)
+    assert np.abs(g["dS"][z]).min() > 1e-8
+
+
+ALL_PINS = [
+    pin_weight_is_sum_of_numpy_krons,
+    pin_forward_brute_force,
+    pin_forward_vec_trick,
+    pin_forward_is_gemm_with_numpy_weight,
+    pin_mixed_product,
+    pin_transpose,
+    pin_block_structure,
+    pin_rank_one,
+    pin_van_loan_rank,
+    pin_special_shapes,
+    pin_finite_differences,
+    pin_linearity_identities,
+    pin_backward_numpy_chain_rule,
+    pin_zero_s_gradient,
+]

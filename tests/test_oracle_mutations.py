@@ -1,0 +1,64 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check that the
+pins catch every one of them (a dropped term, a wrong sign or index, a missing
+factor).  The copies are compiled and run on the CPU only."""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "kron_oracle.c")
+
+# (name, exact text in kron_oracle.c, replacement, occurrence index)
+MUTATIONS = [
+    ("weight_drops_S",
+     "const double Cac = S[(long)a * q + c] * A[((long)i * p + a) * q + c];",
+     "const double Cac = A[((long)i * p + a) * q + c];", 0),
+    ("weight_row_interleave_swapped",
+     "W[((long)a * m1 + j) * out + (long)c * m2 + k] +=",
+     "W[((long)j * p + a) * out + (long)c * m2 + k] +=", 0),
+    ("weight_col_interleave_swapped",
+     "W[((long)a * m1 + j) * out + (long)c * m2 + k] +=",
+     "W[((long)a * m1 + j) * out + (long)k * q + c] +=", 0),
+    ("bias_dropped", "yn[o] = bias ? bias[o] : 0.0;", "yn[o] = 0.0;", 0),
+    ("dx_wrong_sign", "s += Gn[o] * Wu[o];", "s -= Gn[o] * Wu[o];", 0),
+    ("dw_reads_wrong_column", "const double xv = x[n * in + u];",
+     "const double xv = x[n * in + (in - 1 - u)];", 0),
+    ("dB_drops_S",
+     "S[(long)a * q + c] * A[((long)i * p + a) * q + c];\n                        dB",
+     "A[((long)i * p + a) * q + c];\n                        dB", 0),
+    ("dA_forgets_S", "dA[(long)i * p * q + ac] = dC[(long)i * p * q + ac] * S[ac];",
+     "dA[(long)i * p * q + ac] = dC[(long)i * p * q + ac];", 0),
+    ("dS_uses_S_not_A", "s += dC[(long)i * p * q + ac] * A[(long)i * p * q + ac];",
+     "s += dC[(long)i * p * q + ac] * S[ac];", 0),
+    ("dbias_skips_first_row", "for (long n = 0; n < N; ++n) s += G[n * out + o];",
+     "for (long n = 1; n < N; ++n) s += G[n * out + o];", 0),
+    ("dC_uses_only_first_rank_of_B",
+     "B[((long)i * m1 + j) * m2 + k];\n                    dC",
+     "B[((long)0 * m1 + j) * m2 + k];\n                    dC", 0),
+]
+
+
+def _mutate(text, old, new, occ):
+    pos = -1
+    for _ in range(occ + 1):
+        pos = text.index(old, pos + 1)
+    return text[:pos] + new + text[pos + len(old):]
+
+
+@pytest.mark.parametrize("name,old,new,occ", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(tmp_path, name, old, new, occ):
+    text = open(SRC).read()
+    assert old in text, f"mutation anchor for {name} not found in the oracle source"
+    src = tmp_path / f"mut_{name}.c"
+    src.write_text(_mutate(text, old, new, occ))
+    so = oracle.build(force=True, src=str(src), out=str(tmp_path / f"mut_{name}.so"))
+    orc = oracle.Oracle(so)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
