@@ -1,0 +1,347 @@
+"""Benchmark: Kronecker-layer rows/s, forward + backward, on the tutorial layer
+(N = 20000 rows, 1024 x 1024, m = 32 (p = q = 32), r = 4, fp32 I/O, half of S zeroed),
+with the achieved fraction of the dominant kernel's roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--path tf32|f32|bf16]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+One step = forward (y = x W + bias) and backward (dX, dS, dA, dB, dbias) of one batch
+through the C ABI.  With N > 1 GPUs (torchrun, NCCL) every rank runs the full batch
+on its own GPU (weak scaling) and the factor gradients are summed across ranks with
+one NCCL all-reduce per step, the data-parallel exchange.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Kron-layer rows/s fwd+bwd (1024², m=32, r=4) & achieved % of roofline"
+UNIT = "rows/s"
+WORKLOAD = "tutorial"
+ROTATE = 3  # independent input sets cycled through, so the working set exceeds L2
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def _workload_desc(w):
+    zero = f", {w.s_zero_entries} of {w.p * w.q} entries of S zeroed" if w.s_zero_entries else ""
+    return (f"{w.name}: N={w.N} rows, {w.d_in}x{w.d_out} layer, p={w.p} q={w.q} "
+            f"m1={w.m1} m2={w.m2}, r={w.r}, {w.dtype} I/O{zero}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(w, rows: int, threads: int | None = None):
+    """Time the fp64 oracle (forward + backward) on the first `rows` rows."""
+    import numpy as np
+
+    import kron_workloads as kw
+    import oracle
+    if threads:
+        oracle.set_threads(threads)
+    f = {k: v.float().numpy().astype(np.float64) for k, v in kw.factors(w).items()}
+    x = kw.rows(w, "x", 0, rows).float().numpy().astype(np.float64)
+    G = kw.rows(w, "G", 0, rows).float().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.forward(x, f["S"], f["A"], f["B"], f["bias"])
+    oracle.backward(x, f["S"], f["A"], f["B"], G)
+    dt = time.perf_counter() - t0
+    return rows / dt, dt, oracle.get_threads()
+
+
+def run_reference(args, w):
+    """--impl reference: the fp64 oracle on the host cores, a bounded row sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        cpu_baseline(w, rows)
+    t0 = time.perf_counter()
+    threads = 1
+    for _ in range(args.steps):
+        _, _, threads = cpu_baseline(w, rows)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": _workload_desc(w), "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"first {rows} of {w.N} rows per step, forward + backward"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--path", default=None, help="tf32 | f32 | bf16 (default: headline path)")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import kron_workloads as kw
+    w = kw.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    import kronecker_factored_structured_b200 as kfs
+    from kronecker_factored_structured_b200 import accounting as acc
+
+    path = args.path or ("tf32" if "tf32" in kfs.native.IMPLEMENTED_PATHS else "f32")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if path == "bf16" and w.dtype != "bf16":
+        w = dataclasses.replace(w, dtype="bf16")
+    kfs.native.load()
+
+    # ---- inputs resident in HBM: ROTATE independent (x, G) sets, factors shared ----
+    fac = {k: v.to(dev) for k, v in kw.factors(w).items()}
+    sets = []
+    for s in range(ROTATE):
+        ws = dataclasses.replace(w, seed=w.seed + 1000 * s) if s else w
+        sets.append((kw.rows(ws, "x").to(dev), kw.rows(ws, "G").to(dev)))
+    p, q, m1, m2, r, N = w.p, w.q, w.m1, w.m2, w.r, w.N
+    t_io = kfs.native.io_dtype(path)
+    elt = 2 if path == "bf16" else 4
+    y = torch.empty(N, q * m2, dtype=t_io, device=dev)
+    grads = {"dX": torch.empty(N, p * m1, dtype=t_io, device=dev)}
+    flat = torch.empty(p * q + r * p * q + r * m1 * m2 + q * m2, dtype=torch.float32, device=dev)
+    o = 0
+    for k, shp in (("dS", (p, q)), ("dA", (r, p, q)), ("dB", (r, m1, m2)), ("dbias", (q * m2,))):
+        n = 1
+        for d in shp:
+            n *= d
+        grads[k] = flat[o:o + n].view(*shp)
+        o += n
+    wsb = torch.empty(max(kfs.workspace_size(N, p, q, m1, m2, r, path), 1), dtype=torch.uint8,
+                      device=dev)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(i, timing=None):
+        x, G = sets[i % ROTATE]
+        if timing is not None:
+            timing[0].record(stream)
+        kfs.forward(x, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, out=y)
+        if timing is not None:
+            timing[1].record(stream)
+        kfs.backward(x, fac["S"], fac["A"], fac["B"], G, dtype=path, workspace=wsb, grads=grads)
+        if timing is not None:
+            timing[2].record(stream)
+        if world > 1:
+            dist.all_reduce(flat)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-call events on the launching stream ----
+    marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
+    start, end = ev(), ev()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, marks[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = start.elapsed_time(end)
+    t_fwd = statistics.mean(a.elapsed_time(b) for a, b, _ in marks)
+    t_bwd = statistics.mean(b.elapsed_time(c) for _, b, c in marks)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * N * args.steps / (ms / 1e3)
+
+    # ---- end to end through the public API with pinned host buffers ----
+    xh = [s[0].cpu().pin_memory() for s in sets]
+    gh = [s[1].cpu().pin_memory() for s in sets]
+    yh = torch.empty(N, q * m2, dtype=t_io).pin_memory()
+    dxh = torch.empty(N, p * m1, dtype=t_io).pin_memory()
+    fh = torch.empty_like(flat, device="cpu").pin_memory()
+    xd, gd = torch.empty_like(sets[0][0]), torch.empty_like(sets[0][1])
+
+    def e2e_step(i):
+        xd.copy_(xh[i % ROTATE], non_blocking=True)
+        gd.copy_(gh[i % ROTATE], non_blocking=True)
+        kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, out=y)
+        kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, workspace=wsb, grads=grads)
+        if world > 1:
+            dist.all_reduce(flat)
+        yh.copy_(y, non_blocking=True)
+        dxh.copy_(grads["dX"], non_blocking=True)
+        fh.copy_(flat, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s0, s1 = ev(), ev()
+    s0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s0.elapsed_time(s1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * N * e2e_steps / (e2e_ms / 1e3)
+    h2d = xh[0].numel() * xh[0].element_size() + gh[0].numel() * gh[0].element_size()
+    d2h = yh.numel() * yh.element_size() + dxh.numel() * dxh.element_size() + fh.numel() * 4
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---- roofline of the dominant kernel (the fused backward call) ----
+    peaks = _peaks()
+    bwd_bytes = N * elt * (2 * p * m1 + q * m2)
+    bwd_flops = N * (acc.flops_per_row(p, q, m1, m2, r) - acc.flops_per_row(p, q, m1, m2, r, False))
+    if path == "f32":
+        peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12   # FFMA TFLOP/s at max clock
+        achieved = bwd_flops / (t_bwd / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "kron_bwd_simt_kernel + reduction (one backward call)",
+                "peak_source": "derived: 148 SMs x 128 FFMA/clk x 2 x max SM clock"}
+    else:
+        achieved = bwd_bytes / (t_bwd / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "fused backward call", "peak_source": peaks["source"]}
+
+    step_bytes = N * acc.bytes_per_row(p * m1, q * m2, elt)
+    step_flops = N * acc.flops_per_row(p, q, m1, m2, r)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": path, "data": "synthetic",
+        "config": {"workload": _workload_desc(w), "N": N, "p": p, "q": q, "m1": m1, "m2": m2,
+                   "r": r, "path": path, "parallelism": f"dp{world}",
+                   "l2": f"inputs rotated over {ROTATE} independent (x, dY) sets "
+                         f"({ROTATE * N * elt * (p * m1 + q * m2) / 1e6:.0f} MB > 126 MB L2)"},
+        "fwd_ms": t_fwd, "bwd_ms": t_bwd,
+        "tflops": step_flops / (ms_step / 1e3) / 1e12,
+        "gbs": step_bytes / (ms_step / 1e3) / 1e9,
+        "step_roofline_frac_hbm": (step_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3),
+        "roofline": roof,
+        "gpu_launches": args.steps * 3,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rows_s, dt, cores = cpu_baseline(w, args.cpu_rows)
+        line["cpu_baseline"] = {"value": rows_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {args.cpu_rows} of {N} rows, forward + "
+                                          f"backward, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,135 @@
+/*
+ * kron_linear.h -- C ABI of libkronlinear.so, the B200 (sm_100a) implementation of
+ * the sum-of-Kronecker-products linear layer
+ *
+ *     y = x W + bias,   W = sum_{i<r} kron(C_i, B_i),   C_i = S (.) A_i,
+ *
+ * as defined on the page "kronecker-layer-benchmark" (section "1. Build W, then
+ * multiply", KronLinear.weight/forward; rectangular B_i as in section "2. The vec
+ * trick").  W is never formed: each row x_n is viewed as X_n (p x m1) and
+ * Y_n = sum_i C_i^T X_n B_i (section "2. The vec trick" and "3. The vec trick
+ * without the loop"), with both contractions fused on chip.
+ *
+ * Layouts (all row-major, contiguous, no padding):
+ *   x, dX   [N][p*m1]      X_n[a][j]  = x[n][a*m1 + j]
+ *   y, dY   [N][q*m2]      Y_n[c][k]  = y[n][c*m2 + k]
+ *   S, dS   [p][q]
+ *   A, dA   [r][p][q]
+ *   B, dB   [r][m1][m2]
+ *   bias, dbias [q*m2]
+ *
+ * Element types by path (kron_dtype_t):
+ *   KRON_F32   every tensor is float32; exact FP32 arithmetic on the CUDA cores.
+ *   KRON_TF32  every tensor is float32; both contractions run on the tcgen05 tensor
+ *              cores with TF32 operands and FP32 accumulation.
+ *   KRON_BF16  x, y, dY, dX, S, A, B and bias are bfloat16; dS, dA, dB and dbias are
+ *              float32.  tcgen05 tensor cores with BF16 operands, FP32 accumulation.
+ *
+ * Ownership and synchronisation: every pointer except `stream` is a DEVICE pointer
+ * owned by the caller.  The library allocates no memory, keeps no state between
+ * calls and never synchronises; all work is enqueued on `stream` (a cudaStream_t
+ * passed as void*, NULL = legacy default stream).
+ *
+ * Errors: arguments, shapes, alignment and workspace size are checked on the host
+ * before anything is launched; a failing check returns its status and launches
+ * nothing.  Shapes a path does not cover return KRON_ERR_UNSUPPORTED (there is no
+ * fallback to another path or to the CPU).  A failed launch returns KRON_ERR_CUDA;
+ * faults during execution surface at the caller's next synchronisation.
+ * kron_last_error() gives a one-line description of the last failure on the
+ * calling host thread.
+ */
+#ifndef KRON_LINEAR_H
+#define KRON_LINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KRON_LINEAR_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define KRON_API __attribute__((visibility("default")))
+#else
+#define KRON_API
+#endif
+
+typedef enum {
+    KRON_F32 = 0,   /* exact FP32 (FFMA)                          */
+    KRON_TF32 = 1,  /* FP32 I/O, TF32 tensor cores, FP32 accumulate */
+    KRON_BF16 = 2   /* BF16 I/O, BF16 tensor cores, FP32 accumulate */
+} kron_dtype_t;
+
+typedef enum {
+    KRON_OK = 0,
+    KRON_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad dtype or flag   */
+    KRON_ERR_UNSUPPORTED = 2,  /* valid shape that this path does not implement          */
+    KRON_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                       */
+    KRON_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than kron_linear_workspace_size */
+    KRON_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed            */
+    KRON_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait gave up           */
+} kron_status_t;
+
+/* Skip the work of (a, c) blocks where S is zero (the m1 x m2 block of W is zero,
+ * page "kronecker-layer-benchmark", introduction).  Only provably-zero products are
+ * skipped: dS stays exact at zero entries of S.  Results equal the unflagged call
+ * up to rounding. */
+#define KRON_FLAG_SKIP_ZERO_BLOCKS 1u
+
+/*
+ * Forward: y = x W + bias.
+ *   x     [N][p*m1]  input rows
+ *   S, A, B          factors as above
+ *   bias  [q*m2]     may be NULL (no bias)
+ *   y     [N][q*m2]  output, overwritten
+ *   N >= 0 rows (N == 0 is a no-op); p, q, m1, m2, r >= 1.
+ * Requirements: x, y, S, A, B, bias 16-byte aligned (KRON_ERR_ALIGNMENT);
+ * m1 and m2 multiples of 4 (F32/TF32) or 8 (BF16), else KRON_ERR_UNSUPPORTED.
+ */
+KRON_API kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, const void *B,
+                                  const void *bias, void *y,
+                                  int64_t N, int p, int q, int m1, int m2, int r,
+                                  kron_dtype_t dtype, unsigned flags, void *stream);
+
+/*
+ * Backward: gradients of L = <dY, y> (dY = dL/dy).
+ *   dX    [N][p*m1]   = dY W^T                                   (may be NULL: skipped)
+ *   dS    [p][q]      = sum_i dC_i (.) A_i
+ *   dA    [r][p][q]   = dC_i (.) S,   dC_i = sum_n (X_n B_i) dY_n^T
+ *   dB    [r][m1][m2] = sum_n X_n^T C_i dY_n
+ *   dbias [q*m2]      = sum_n dY_n                                (may be NULL: skipped)
+ * Gradients OVERWRITE their outputs.  T = X_n B_i is recomputed, nothing is kept
+ * from the forward call.  The sums over rows are split into a fixed number of
+ * contiguous row ranges whose partials are added in a fixed order, so results are
+ * bitwise identical across calls with the same inputs on the same GPU model.
+ * `workspace` is device scratch of at least kron_linear_workspace_size(...) bytes,
+ * 256-byte aligned, owned by the caller; its contents on entry are ignored.
+ */
+KRON_API kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, const void *B,
+                                   const void *dY, void *dX, void *dS, void *dA, void *dB,
+                                   void *dbias,
+                                   int64_t N, int p, int q, int m1, int m2, int r,
+                                   kron_dtype_t dtype, unsigned flags,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace kron_linear_backward needs for this problem (0 if the
+ * arguments are invalid).  Depends only on the arguments, not on the device. */
+KRON_API size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r,
+                                  kron_dtype_t dtype);
+
+/* Static description of a status code. */
+KRON_API const char *kron_status_string(kron_status_t status);
+
+/* One-line description of the last failure on this host thread ("" if none). */
+KRON_API const char *kron_last_error(void);
+
+/* KRON_LINEAR_ABI_VERSION of the loaded library. */
+KRON_API int kron_linear_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRON_LINEAR_H */

@@ -1,0 +1,167 @@
+// api.cu -- the extern "C" entry points of libkronlinear.so (include/kron_linear.h):
+// host-side validation, then dispatch to the kernels of the requested path.
+// Nothing here computes any part of the layer.
+#include "../../include/kron_linear.h"
+#include "internal.h"
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+kron_status_t fail(kron_status_t st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+kron_status_t fail(kron_status_t st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+kron_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(KRON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+kron_status_t check_shape(int64_t N, int p, int q, int m1, int m2, int r, kron_dtype_t dtype,
+                          unsigned flags) {
+    if (dtype != KRON_F32 && dtype != KRON_TF32 && dtype != KRON_BF16)
+        return fail(KRON_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (flags & ~KRON_FLAG_SKIP_ZERO_BLOCKS)
+        return fail(KRON_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if (N < 0 || p < 1 || q < 1 || m1 < 1 || m2 < 1 || r < 1)
+        return fail(KRON_ERR_INVALID_ARG,
+                    "sizes must be N >= 0 and p, q, m1, m2, r >= 1 (got N=%lld p=%d q=%d m1=%d "
+                    "m2=%d r=%d)", (long long)N, p, q, m1, m2, r);
+    if ((int64_t)p * m1 > (1 << 20) || (int64_t)q * m2 > (1 << 20) || r > 4096 ||
+        N > ((int64_t)1 << 40))
+        return fail(KRON_ERR_INVALID_ARG, "sizes out of range");
+    const int mult = dtype == KRON_BF16 ? 8 : 4;
+    if (m1 % mult || m2 % mult)
+        return fail(KRON_ERR_UNSUPPORTED, "m1 and m2 must be multiples of %d for this dtype", mult);
+    return KRON_OK;
+}
+
+int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
+    (void)dtype;
+    const int R = kron::simt_backward_rows(s);
+    if (R <= 0) return 0;
+    int64_t tiles = (s.N + R - 1) / R;
+    if (tiles < 1) tiles = 1;
+    return tiles < kron::kRowParts ? (int)tiles : kron::kRowParts;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kron_linear_abi_version(void) { return KRON_LINEAR_ABI_VERSION; }
+
+const char *kron_last_error(void) { return g_last_error; }
+
+const char *kron_status_string(kron_status_t status) {
+    switch (status) {
+        case KRON_OK: return "KRON_OK";
+        case KRON_ERR_INVALID_ARG: return "KRON_ERR_INVALID_ARG: invalid argument";
+        case KRON_ERR_UNSUPPORTED: return "KRON_ERR_UNSUPPORTED: shape or dtype not implemented";
+        case KRON_ERR_ALIGNMENT: return "KRON_ERR_ALIGNMENT: pointer not 16-byte aligned";
+        case KRON_ERR_WORKSPACE: return "KRON_ERR_WORKSPACE: workspace missing or too small";
+        case KRON_ERR_CUDA: return "KRON_ERR_CUDA: CUDA error";
+        case KRON_ERR_TIMEOUT: return "KRON_ERR_TIMEOUT: device-side wait timed out";
+    }
+    return "unknown kron_status_t";
+}
+
+size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r,
+                                  kron_dtype_t dtype) {
+    if (check_shape(N, p, q, m1, m2, r, dtype, 0) != KRON_OK) return 0;
+    const kron::Shape s{N, p, q, m1, m2, r};
+    const int parts = backward_parts(s, dtype);
+    return (size_t)parts * kron::partial_stride(s) * sizeof(float);
+}
+
+kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, const void *B,
+                                  const void *bias, void *y, int64_t N, int p, int q, int m1,
+                                  int m2, int r, kron_dtype_t dtype, unsigned flags,
+                                  void *stream) {
+    g_last_error[0] = 0;
+    kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
+    if (st != KRON_OK) return st;
+    if (!x || !S || !A || !B || !y)
+        return fail(KRON_ERR_INVALID_ARG, "x, S, A, B and y must be non-null");
+    if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(y) ||
+        (bias && !aligned16(bias)))
+        return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
+    if (N == 0) return KRON_OK;
+    const kron::Shape s{N, p, q, m1, m2, r};
+    cudaStream_t cs = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    switch (dtype) {
+        case KRON_F32:
+            if (kron::simt_forward_rows(s) <= 0)
+                return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
+            e = kron::simt_forward((const float *)x, (const float *)S, (const float *)A,
+                                   (const float *)B, (const float *)bias, (float *)y, s, cs);
+            break;
+        default:
+            return fail(KRON_ERR_UNSUPPORTED, "dtype %d forward not implemented", (int)dtype);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return KRON_OK;
+}
+
+kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, const void *B,
+                                   const void *dY, void *dX, void *dS, void *dA, void *dB,
+                                   void *dbias, int64_t N, int p, int q, int m1, int m2, int r,
+                                   kron_dtype_t dtype, unsigned flags, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    g_last_error[0] = 0;
+    kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
+    if (st != KRON_OK) return st;
+    if (!x || !S || !A || !B || !dY || !dS || !dA || !dB)
+        return fail(KRON_ERR_INVALID_ARG, "x, S, A, B, dY, dS, dA and dB must be non-null");
+    if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(dY) ||
+        !aligned16(dS) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
+        (dbias && !aligned16(dbias)))
+        return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
+    const kron::Shape s{N, p, q, m1, m2, r};
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (N == 0) {  // empty batch: every gradient is zero
+        cudaError_t e = cudaMemsetAsync(dS, 0, (size_t)p * q * sizeof(float), cs);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, (size_t)r * p * q * sizeof(float), cs);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, (size_t)r * m1 * m2 * sizeof(float), cs);
+        if (e == cudaSuccess && dbias)
+            e = cudaMemsetAsync(dbias, 0, (size_t)q * m2 * sizeof(float), cs);
+        return e == cudaSuccess ? KRON_OK : cuda_fail(e, "zero gradients");
+    }
+    const size_t need = kron_linear_workspace_size(N, p, q, m1, m2, r, dtype);
+    if (!workspace || workspace_bytes < need)
+        return fail(KRON_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if ((uintptr_t)workspace & 255u)
+        return fail(KRON_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    const int parts = backward_parts(s, dtype);
+    cudaError_t e = cudaSuccess;
+    switch (dtype) {
+        case KRON_F32:
+            if (kron::simt_backward_rows(s) <= 0)
+                return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
+            e = kron::simt_backward((const float *)x, (const float *)S, (const float *)A,
+                                    (const float *)B, (const float *)dY, (float *)dX,
+                                    (float *)workspace, parts, s, cs);
+            if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+            e = kron::reduce_partials((const float *)workspace, parts, S, A, false, (float *)dS,
+                                      (float *)dA, (float *)dB, (float *)dbias, s, cs);
+            break;
+        default:
+            return fail(KRON_ERR_UNSUPPORTED, "dtype %d backward not implemented", (int)dtype);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "reduction launch");
+    return KRON_OK;
+}
+
+}  // extern "C"

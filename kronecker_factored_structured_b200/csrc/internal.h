@@ -1,0 +1,47 @@
+// internal.h -- declarations shared by the translation units of libkronlinear.so.
+// Not part of the public ABI (include/kron_linear.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kron {
+
+struct Shape {
+    int64_t N;
+    int p, q, m1, m2, r;
+    int64_t d_in() const { return (int64_t)p * m1; }
+    int64_t d_out() const { return (int64_t)q * m2; }
+};
+
+// Number of contiguous row ranges the backward splits N into.  A fixed constant
+// (the SM count of a B200), so the partition, and with it the summation order of
+// dS/dA/dB/dbias, does not depend on scheduling or on the device.
+constexpr int kRowParts = 148;
+
+// Floats of one row range's partial sums in the workspace:
+// [dC: r*p*q][dB: r*m1*m2][dbias: q*m2], each range padded to 64 floats.
+inline size_t partial_stride(const Shape &s) {
+    size_t n = (size_t)s.r * s.p * s.q + (size_t)s.r * s.m1 * s.m2 + (size_t)s.q * s.m2;
+    return (n + 63) & ~(size_t)63;
+}
+
+// ---- exact FP32 path on the CUDA cores (simt_f32.cu) ----
+// Rows per tile for the SIMT kernels; 0 when the shape does not fit shared memory.
+int simt_forward_rows(const Shape &s);
+int simt_backward_rows(const Shape &s);
+cudaError_t simt_forward(const float *x, const float *S, const float *A, const float *B,
+                         const float *bias, float *y, const Shape &s, cudaStream_t st);
+// Writes dX (if non-null) and the per-range partials into ws (parts x partial_stride).
+cudaError_t simt_backward(const float *x, const float *S, const float *A, const float *B,
+                          const float *dY, float *dX, float *ws, int parts, const Shape &s,
+                          cudaStream_t st);
+
+// ---- deterministic reduction of the row-range partials (reduce.cu) ----
+// S and A are float (is_bf16 = false) or bfloat16 (is_bf16 = true).
+cudaError_t reduce_partials(const float *ws, int parts, const void *S, const void *A,
+                            bool is_bf16, float *dS, float *dA, float *dB, float *dbias,
+                            const Shape &s, cudaStream_t st);
+
+}  // namespace kron

@@ -1,0 +1,369 @@
+// simt_f32.cu -- exact-FP32 path of the Kronecker layer on the CUDA cores (FFMA).
+//
+// Both contractions of the vec trick (page "kronecker-layer-benchmark", sections
+// "2. The vec trick" and "3. The vec trick without the loop") are fused per tile of
+// R rows: the intermediate T_i = X_n B_i lives only in shared memory, so the
+// permute/reshape copies of the loop-free PyTorch version never touch HBM.
+//
+// Forward, per tile and rank i:
+//   T[(n,a),k]  = sum_j X[(n,a),j] * B_i[j,k]              (stage 1)
+//   Y[(n,c),k] += sum_a C_i[a,c]  * T[(n,a),k]              (stage 2)
+// Backward, per tile and rank i (G = dY):
+//   U[(n,a),k]  = sum_c C_i[a,c]  * G[(n,c),k]
+//   T[(n,a),k]  = sum_j X[(n,a),j] * B_i[j,k]              (recomputed)
+//   dX[(n,a),j]+= sum_k U[(n,a),k] * B_i[j,k]
+//   dB_i[j,k]  += sum_(n,a) X[(n,a),j] * U[(n,a),k]
+//   dC_i[a,c]  += sum_(n,k) T[(n,a),k] * G[(n,c),k]
+// dB, dC and dbias are accumulated per CTA over one fixed contiguous row range and
+// written as partials; reduce.cu adds the partials in a fixed order.
+#include "internal.h"
+
+#include <algorithm>
+
+namespace kron {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// Register-tiled product of shared-memory operands:
+//   Cm(m,n) (+)= sum_{k1<K1, k0<K0} Am(m,k1,k0) * Bm(k1,k0,n)   for every batch b
+// with Am(m,k1,k0) = A[b*sab + m*sam + k1*sak1 + k0*sak0],
+//      Bm(k1,k0,n) = B[b*sbb + k1*sbk1 + k0*sbk0 + n*sbn],
+//      Cm(m,n)     = C[b*scb + m*scm + n].
+// Thread-owned outputs are the 4x4 grid {tm + u*MT} x {tn + v*NT}: neighbouring
+// threads read neighbouring columns of B, and rows of A differ by one row stride
+// (odd strides keep those reads on distinct banks).
+struct MM {
+    const float *A; int sab, sam, sak1, sak0;
+    const float *B; int sbb, sbk1, sbk0, sbn;
+    float *C; int scb, scm;
+    int batch, M, N, K1, K0;
+};
+
+__device__ __forceinline__ void smem_mm(const MM &g, bool accumulate) {
+    const int MT = (g.M + 3) >> 2, NT = (g.N + 3) >> 2;
+    const int tiles = MT * NT;
+    for (int t = threadIdx.x; t < g.batch * tiles; t += blockDim.x) {
+        const int b = t / tiles;
+        const int tt = t - b * tiles;
+        const int tm = tt / NT, tn = tt - tm * NT;
+        int row[4], col[4];
+        bool rv[4], cv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            row[u] = tm + u * MT;
+            rv[u] = row[u] < g.M;
+            if (!rv[u]) row[u] = 0;
+            col[u] = tn + u * NT;
+            cv[u] = col[u] < g.N;
+            if (!cv[u]) col[u] = 0;
+        }
+        const float *Ab = g.A + (size_t)b * g.sab;
+        const float *Bb = g.B + (size_t)b * g.sbb;
+        float acc[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+        for (int k1 = 0; k1 < g.K1; ++k1) {
+            const float *Ak = Ab + k1 * g.sak1;
+            const float *Bk = Bb + k1 * g.sbk1;
+#pragma unroll 4
+            for (int k0 = 0; k0 < g.K0; ++k0) {
+                float a[4], bb[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) a[u] = Ak[row[u] * g.sam + k0 * g.sak0];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) bb[v] = Bk[k0 * g.sbk0 + col[v] * g.sbn];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], bb[v], acc[u][v]);
+            }
+        }
+        float *Cb = g.C + (size_t)b * g.scb;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                if (rv[u] && cv[v]) {
+                    float *c = Cb + row[u] * g.scm + col[v];
+                    *c = accumulate ? *c + acc[u][v] : acc[u][v];
+                }
+    }
+}
+
+// Row r of a [rows][width] global matrix -> shared rows with stride ld; rows at or
+// beyond N read as zero.  `width` floats per row, 16-byte aligned rows.
+__device__ __forceinline__ void load_rows(const float *__restrict__ g, int64_t n0, int64_t N,
+                                          int rows, int width, float *s, int blk, int ld) {
+    // width = nblk * blk; shared row (n, b) of length blk starts at ((n*nblk)+b)*ld
+    const int nblk = width / blk;
+    const int w4 = width >> 2;
+    for (int e = threadIdx.x; e < rows * w4; e += blockDim.x) {
+        const int n = e / w4, c4 = (e - n * w4) << 2;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + n < N) v = *reinterpret_cast<const float4 *>(g + (n0 + n) * width + c4);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int c = c4 + t, bi = c / blk, j = c - bi * blk;
+            s[(n * nblk + bi) * ld + j] = vv[t];
+        }
+    }
+}
+
+struct FwdLayout {
+    int R, ldx, ldb, ldc, ldt;
+    size_t offX, offB, offC, offT, offY, total;  // in floats
+};
+
+inline size_t up4(size_t v) { return (v + 3) & ~(size_t)3; }  // 16-byte aligned offsets
+
+FwdLayout fwd_layout(const Shape &s, int R) {
+    FwdLayout L;
+    L.R = R;
+    L.ldx = s.m1 + 1;
+    L.ldb = s.m2 + 1;
+    L.ldc = s.q + 1;
+    L.ldt = s.m2 + 1;
+    size_t o = 0;
+    L.offX = o; o = up4(o + (size_t)R * s.p * L.ldx);
+    L.offB = o; o = up4(o + (size_t)s.m1 * L.ldb);
+    L.offC = o; o = up4(o + (size_t)s.p * L.ldc);
+    L.offT = o; o = up4(o + (size_t)R * s.p * L.ldt);
+    L.offY = o; o = up4(o + (size_t)R * s.q * s.m2);
+    L.total = o;
+    return L;
+}
+
+// acc_smem: the dC/dB/dbias accumulators live in shared memory; otherwise (large
+// r*p*q) they are accumulated in place in the CTA's own workspace partial.
+struct BwdLayout {
+    int R, ldx, ldg, ldb, ldc, ldt, acc_smem;
+    size_t offX, offG, offDX, offU, offT, offB, offC, offDC, offDB, offDb, total;
+};
+
+BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem) {
+    BwdLayout L;
+    L.R = R;
+    L.acc_smem = acc_smem;
+    L.ldx = s.m1 + 1;
+    L.ldg = s.m2 + 1;
+    L.ldb = s.m2 + 1;
+    L.ldc = s.q + 1;
+    L.ldt = s.m2 + 1;
+    size_t o = 0;
+    L.offX = o; o = up4(o + (size_t)R * s.p * L.ldx);
+    L.offG = o; o = up4(o + (size_t)R * s.q * L.ldg);
+    L.offDX = o; o = up4(o + (size_t)R * s.p * L.ldx);
+    L.offU = o; o = up4(o + (size_t)R * s.p * L.ldt);
+    L.offT = o; o = up4(o + (size_t)R * s.p * L.ldt);
+    L.offB = o; o = up4(o + (size_t)s.m1 * L.ldb);
+    L.offC = o; o = up4(o + (size_t)s.p * L.ldc);
+    L.offDC = L.offDB = L.offDb = o;
+    if (acc_smem) {
+        L.offDC = o; o = up4(o + (size_t)s.r * s.p * s.q);
+        L.offDB = o; o = up4(o + (size_t)s.r * s.m1 * s.m2);
+        L.offDb = o; o = up4(o + (size_t)s.q * s.m2);
+    }
+    L.total = o;
+    return L;
+}
+
+// Factor i into shared memory: Bs[j*ldb + k] = B_i[j,k], Cs[a*ldc + c] = S[a,c]*A_i[a,c].
+__device__ __forceinline__ void load_factors(const float *__restrict__ S,
+                                             const float *__restrict__ A,
+                                             const float *__restrict__ B, int i, const Shape &s,
+                                             float *Bs, int ldb, float *Cs, int ldc) {
+    const float *Bi = B + (size_t)i * s.m1 * s.m2;
+    for (int e = threadIdx.x; e < s.m1 * s.m2; e += blockDim.x) {
+        const int j = e / s.m2, k = e - j * s.m2;
+        Bs[j * ldb + k] = Bi[e];
+    }
+    const float *Ai = A + (size_t)i * s.p * s.q;
+    for (int e = threadIdx.x; e < s.p * s.q; e += blockDim.x) {
+        const int a = e / s.q, c = e - a * s.q;
+        Cs[a * ldc + c] = S[e] * Ai[e];
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+kron_fwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
+                     const float *__restrict__ A, const float *__restrict__ B,
+                     const float *__restrict__ bias, float *__restrict__ y, Shape s,
+                     FwdLayout L) {
+    extern __shared__ __align__(16) float smem[];
+    float *Xs = smem + L.offX, *Bs = smem + L.offB, *Cs = smem + L.offC;
+    float *Ts = smem + L.offT, *Ys = smem + L.offY;
+    const int R = L.R;
+    const int64_t n0 = (int64_t)blockIdx.x * R;
+    const int P = s.p, Q = s.q, M1 = s.m1, M2 = s.m2;
+
+    load_rows(x, n0, s.N, R, P * M1, Xs, M1, L.ldx);
+
+    for (int i = 0; i < s.r; ++i) {
+        __syncthreads();  // previous stage 2 done with Bs/Cs/Ts
+        load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
+        __syncthreads();
+        // stage 1: T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
+        MM g1{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
+        smem_mm(g1, false);
+        __syncthreads();
+        // stage 2, batched over rows n: Y[(n,c),k] += sum_a C_i[a,c] T[(n,a),k]
+        MM g2{Cs, 0, 1, 0, L.ldc, Ts, P * L.ldt, 0, L.ldt, 1, Ys, Q * M2, M2, R, Q, M2, 1, P};
+        smem_mm(g2, i > 0);
+    }
+    __syncthreads();
+    // y = Y + bias, coalesced float4 stores
+    const int out = Q * M2, o4 = out >> 2;
+    for (int e = threadIdx.x; e < R * o4; e += blockDim.x) {
+        const int n = e / o4, c4 = (e - n * o4) << 2;
+        if (n0 + n >= s.N) continue;
+        float4 v = *reinterpret_cast<const float4 *>(Ys + n * out + c4);
+        if (bias) {
+            const float4 bv = *reinterpret_cast<const float4 *>(bias + c4);
+            v.x += bv.x; v.y += bv.y; v.z += bv.z; v.w += bv.w;
+        }
+        *reinterpret_cast<float4 *>(y + (n0 + n) * out + c4) = v;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+kron_bwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
+                     const float *__restrict__ A, const float *__restrict__ B,
+                     const float *__restrict__ G, float *__restrict__ dX,
+                     float *__restrict__ ws, int64_t rows_per_part, size_t ws_stride, Shape s,
+                     BwdLayout L) {
+    extern __shared__ __align__(16) float smem[];
+    float *Xs = smem + L.offX, *Gs = smem + L.offG, *dXs = smem + L.offDX;
+    float *Us = smem + L.offU, *Ts = smem + L.offT, *Bs = smem + L.offB, *Cs = smem + L.offC;
+    const int R = L.R;
+    const int P = s.p, Q = s.q, M1 = s.m1, M2 = s.m2;
+    const size_t n_dc = (size_t)s.r * P * Q, n_db = (size_t)s.r * M1 * M2;
+    float *part = ws + (size_t)blockIdx.x * ws_stride;
+    float *dCs = L.acc_smem ? smem + L.offDC : part;
+    float *dBs = L.acc_smem ? smem + L.offDB : part + n_dc;
+    float *dbs = L.acc_smem ? smem + L.offDb : part + n_dc + n_db;
+    const int64_t lo = (int64_t)blockIdx.x * rows_per_part;
+    const int64_t hi = lo + rows_per_part < s.N ? lo + rows_per_part : s.N;
+
+    for (size_t e = threadIdx.x; e < n_dc; e += blockDim.x) dCs[e] = 0.f;
+    for (size_t e = threadIdx.x; e < n_db; e += blockDim.x) dBs[e] = 0.f;
+    for (int e = threadIdx.x; e < Q * M2; e += blockDim.x) dbs[e] = 0.f;
+
+    for (int64_t n0 = lo; n0 < hi; n0 += R) {
+        __syncthreads();
+        load_rows(x, n0, hi, R, P * M1, Xs, M1, L.ldx);
+        load_rows(G, n0, hi, R, Q * M2, Gs, M2, L.ldg);
+        __syncthreads();
+        // dbias partial: rows beyond the range were loaded as zero
+        for (int o = threadIdx.x; o < Q * M2; o += blockDim.x) {
+            const int c = o / M2, k = o - c * M2;
+            float acc = 0.f;
+            for (int n = 0; n < R; ++n) acc += Gs[(n * Q + c) * L.ldg + k];
+            dbs[o] += acc;
+        }
+        for (int i = 0; i < s.r; ++i) {
+            __syncthreads();
+            load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
+            __syncthreads();
+            // U[(n,a),k] = sum_c C_i[a,c] G[(n,c),k]          (batched over n)
+            MM gu{Cs, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
+                  R, P, M2, 1, Q};
+            smem_mm(gu, false);
+            // T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
+            MM gt{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
+            smem_mm(gt, false);
+            __syncthreads();
+            // dX[(n,a),j] += sum_k U[(n,a),k] B_i[j,k]
+            MM gx{Us, 0, L.ldt, 0, 1, Bs, 0, 0, 1, L.ldb, dXs, 0, L.ldx, 1, R * P, M1, 1, M2};
+            smem_mm(gx, i > 0);
+            // dB_i[j,k] += sum_(n,a) X[(n,a),j] U[(n,a),k]
+            MM gb{Xs, 0, 1, 0, L.ldx, Us, 0, 0, L.ldt, 1, dBs + (size_t)i * M1 * M2, 0, M2,
+                  1, M1, M2, 1, R * P};
+            smem_mm(gb, true);
+            // dC_i[a,c] += sum_n sum_k T[(n,a),k] G[(n,c),k]
+            MM gc{Ts, 0, L.ldt, P * L.ldt, 1, Gs, 0, Q * L.ldg, 1, L.ldg,
+                  dCs + (size_t)i * P * Q, 0, Q, 1, P, Q, R, M2};
+            smem_mm(gc, true);
+        }
+        __syncthreads();
+        if (dX) {
+            const int w = P * M1, w4 = w >> 2;
+            for (int e = threadIdx.x; e < R * w4; e += blockDim.x) {
+                const int n = e / w4, c4 = (e - n * w4) << 2;
+                if (n0 + n >= hi) continue;
+                float v[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int c = c4 + t, a = c / M1, j = c - a * M1;
+                    v[t] = dXs[(n * P + a) * L.ldx + j];
+                }
+                *reinterpret_cast<float4 *>(dX + (n0 + n) * w + c4) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
+    }
+    if (!L.acc_smem) return;  // accumulated in place
+    __syncthreads();
+    for (size_t e = threadIdx.x; e < n_dc; e += blockDim.x) part[e] = dCs[e];
+    for (size_t e = threadIdx.x; e < n_db; e += blockDim.x) part[n_dc + e] = dBs[e];
+    for (size_t e = threadIdx.x; e < (size_t)Q * M2; e += blockDim.x)
+        part[n_dc + n_db + e] = dbs[e];
+}
+
+size_t fwd_bytes(const Shape &s, int R) { return fwd_layout(s, R).total * sizeof(float); }
+size_t bwd_bytes(const Shape &s, int R, bool acc_smem) {
+    return bwd_layout(s, R, acc_smem).total * sizeof(float);
+}
+
+// Backward tile choice: rows per tile R and where the accumulators live.
+BwdLayout bwd_choose(const Shape &s) {
+    for (int acc = 1; acc >= 0; --acc)
+        for (int R : {4, 2, 1})
+            if (bwd_bytes(s, R, acc) <= kMaxSmem) return bwd_layout(s, R, acc);
+    BwdLayout none = bwd_layout(s, 1, false);
+    none.R = 0;
+    return none;
+}
+
+}  // namespace
+
+int simt_forward_rows(const Shape &s) {
+    for (int R : {8, 4, 2, 1})
+        if (fwd_bytes(s, R) <= kMaxSmem) return R;
+    return 0;
+}
+
+int simt_backward_rows(const Shape &s) { return bwd_choose(s).R; }
+
+cudaError_t simt_forward(const float *x, const float *S, const float *A, const float *B,
+                         const float *bias, float *y, const Shape &s, cudaStream_t st) {
+    const int R = simt_forward_rows(s);
+    const FwdLayout L = fwd_layout(s, R);
+    const size_t smem = L.total * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(kron_fwd_simt_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (s.N + R - 1) / R;
+    kron_fwd_simt_kernel<<<(unsigned)tiles, kThreads, smem, st>>>(x, S, A, B, bias, y, s, L);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_backward(const float *x, const float *S, const float *A, const float *B,
+                          const float *dY, float *dX, float *ws, int parts, const Shape &s,
+                          cudaStream_t st) {
+    const BwdLayout L = bwd_choose(s);
+    const size_t smem = L.total * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(kron_bwd_simt_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t rows_per_part = (s.N + parts - 1) / parts;
+    kron_bwd_simt_kernel<<<parts, kThreads, smem, st>>>(x, S, A, B, dY, dX, ws, rows_per_part,
+                                                        partial_stride(s), s, L);
+    return cudaGetLastError();
+}
+
+}  // namespace kron

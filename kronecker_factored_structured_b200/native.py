@@ -1,0 +1,167 @@
+"""ctypes binding of libkronlinear.so (include/kron_linear.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current CUDA stream.  If the
+library has not been built, or a call fails, this module raises -- it never
+computes anything itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkronlinear.so")
+
+KRON_F32, KRON_TF32, KRON_BF16 = 0, 1, 2
+DTYPES = {"f32": KRON_F32, "tf32": KRON_TF32, "bf16": KRON_BF16}
+KRON_FLAG_SKIP_ZERO_BLOCKS = 1
+
+# Paths whose kernels are built into the library.
+IMPLEMENTED_PATHS = ("f32",)
+
+STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
+          3: "KRON_ERR_ALIGNMENT", 4: "KRON_ERR_WORKSPACE", 5: "KRON_ERR_CUDA",
+          6: "KRON_ERR_TIMEOUT"}
+
+# Every symbol include/kron_linear.h declares.
+EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_workspace_size",
+           "kron_status_string", "kron_last_error", "kron_linear_abi_version")
+
+
+class KronError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{self.name}: {detail}")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the shared library (raises if it is missing: no fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing; build it with `python -m kronecker_factored_structured_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i64, I, U, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+    lib.kron_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, I, I, I, I, I, I, U, vp]
+    lib.kron_linear_forward.restype = I
+    lib.kron_linear_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                         i64, I, I, I, I, I, I, U, vp, sz, vp]
+    lib.kron_linear_backward.restype = I
+    lib.kron_linear_workspace_size.argtypes = [i64, I, I, I, I, I, I]
+    lib.kron_linear_workspace_size.restype = sz
+    lib.kron_status_string.argtypes = [I]
+    lib.kron_status_string.restype = ctypes.c_char_p
+    lib.kron_last_error.argtypes = []
+    lib.kron_last_error.restype = ctypes.c_char_p
+    lib.kron_linear_abi_version.argtypes = []
+    lib.kron_linear_abi_version.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != 0:
+        detail = load().kron_last_error().decode()
+        raise KronError(status, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def io_dtype(dtype: str) -> torch.dtype:
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def _expect(t, name, dtype, shape):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def shapes(S, A, B):
+    r, p, q = A.shape
+    r2, m1, m2 = B.shape
+    if tuple(S.shape) != (p, q) or r2 != r:
+        raise ValueError(f"inconsistent factor shapes S{tuple(S.shape)} A{tuple(A.shape)} "
+                         f"B{tuple(B.shape)}")
+    return p, q, m1, m2, r
+
+
+def workspace_size(N, p, q, m1, m2, r, dtype="tf32") -> int:
+    return int(load().kron_linear_workspace_size(N, p, q, m1, m2, r, DTYPES[dtype]))
+
+
+def forward(x, S, A, B, bias=None, dtype="tf32", flags=0, out=None, stream=None):
+    """y = x W + bias with W = sum_i kron(S*A_i, B_i), on the library's kernels."""
+    p, q, m1, m2, r = shapes(S, A, B)
+    N = x.shape[0]
+    t = io_dtype(dtype)
+    _expect(x, "x", t, (N, p * m1))
+    for name, v, shp in (("S", S, (p, q)), ("A", A, (r, p, q)), ("B", B, (r, m1, m2))):
+        _expect(v, name, t, shp)
+    if bias is not None:
+        _expect(bias, "bias", t, (q * m2,))
+    if out is None:
+        out = torch.empty(N, q * m2, dtype=t, device=x.device)
+    _expect(out, "y", t, (N, q * m2))
+    _check(load().kron_linear_forward(_ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(bias), _ptr(out),
+                                      N, p, q, m1, m2, r, DTYPES[dtype], flags, _stream(stream)))
+    return out
+
+
+def backward(x, S, A, B, dY, dtype="tf32", flags=0, need_dx=True, need_dbias=True,
+             workspace=None, grads=None, stream=None):
+    """Gradients of <dY, y>: returns dict(dX, dS, dA, dB, dbias).
+
+    dX has the I/O dtype; dS, dA, dB and dbias are float32.  ``grads`` may hold
+    preallocated outputs (same keys); ``workspace`` a preallocated uint8 buffer.
+    """
+    p, q, m1, m2, r = shapes(S, A, B)
+    N = x.shape[0]
+    t = io_dtype(dtype)
+    _expect(x, "x", t, (N, p * m1))
+    _expect(dY, "dY", t, (N, q * m2))
+    for name, v, shp in (("S", S, (p, q)), ("A", A, (r, p, q)), ("B", B, (r, m1, m2))):
+        _expect(v, name, t, shp)
+    dev = x.device
+    g = dict(grads or {})
+    f32 = torch.float32
+    if need_dx and g.get("dX") is None:
+        g["dX"] = torch.empty(N, p * m1, dtype=t, device=dev)
+    if not need_dx:
+        g["dX"] = None
+    for k, shp in (("dS", (p, q)), ("dA", (r, p, q)), ("dB", (r, m1, m2))):
+        if g.get(k) is None:
+            g[k] = torch.empty(shp, dtype=f32, device=dev)
+        _expect(g[k], k, f32, shp)
+    if need_dbias and g.get("dbias") is None:
+        g["dbias"] = torch.empty(q * m2, dtype=f32, device=dev)
+    if not need_dbias:
+        g["dbias"] = None
+    ws_bytes = workspace_size(N, p, q, m1, m2, r, dtype)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    _check(load().kron_linear_backward(
+        _ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(dY), _ptr(g["dX"]), _ptr(g["dS"]),
+        _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dbias"]), N, p, q, m1, m2, r, DTYPES[dtype], flags,
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return g

@@ -1,0 +1,103 @@
+"""The C ABI: the library loads, exports every symbol the header declares, and its
+host-side checks reject bad arguments before launching anything (no GPU needed:
+every call below fails validation, so no kernel is ever launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kronecker_factored_structured_b200 as kfs
+from kronecker_factored_structured_b200 import native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kron_linear.h")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KRON_API\s+[\w\s\*]*?\b(kron_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = native.load()
+    syms = header_symbols()
+    assert set(syms) == set(native.EXPORTS), syms
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_abi_version_and_status_strings():
+    lib = native.load()
+    assert lib.kron_linear_abi_version() == 1
+    for code, name in native.STATUS.items():
+        assert lib.kron_status_string(code).decode().startswith(name)
+
+
+def test_workspace_size_depends_on_shape_only():
+    a = kfs.workspace_size(20000, 32, 32, 32, 32, 4, "f32")
+    assert a > 0 and a % 256 == 0
+    assert a == kfs.workspace_size(20000, 32, 32, 32, 32, 4, "f32")
+    assert kfs.workspace_size(0, 0, 32, 32, 32, 4, "f32") == 0      # invalid p
+    assert kfs.workspace_size(10, 8, 8, 6, 8, 1, "f32") == 0        # m1 not a multiple of 4
+
+
+V = ctypes.c_void_p
+ALIGNED = V(0x10000)          # never dereferenced: each call below fails a host check
+MISALIGNED = V(0x10004)
+
+
+def fwd(x=ALIGNED, S=ALIGNED, A=ALIGNED, B=ALIGNED, bias=None, y=ALIGNED, N=8, p=2, q=2, m1=4,
+        m2=4, r=1, dtype=0, flags=0):
+    lib = native.load()
+    return lib.kron_linear_forward(x, S, A, B, bias, y, N, p, q, m1, m2, r, dtype, flags, None)
+
+
+def bwd(ws=None, ws_bytes=0, dtype=0, flags=0, dS=ALIGNED, x=ALIGNED, N=8, m1=4):
+    lib = native.load()
+    return lib.kron_linear_backward(x, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, dS, ALIGNED,
+                                    ALIGNED, None, N, 2, 2, m1, 4, 1, dtype, flags, ws, ws_bytes,
+                                    None)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(dtype=7), 1),
+    (dict(flags=4), 1),
+    (dict(N=-1), 1),
+    (dict(p=0), 1),
+    (dict(r=0), 1),
+    (dict(x=None), 1),
+    (dict(y=None), 1),
+    (dict(m1=6), 2),               # not a multiple of 4 (F32)
+    (dict(m1=4, dtype=2), 2),      # not a multiple of 8 (BF16)
+    (dict(x=MISALIGNED), 3),
+    (dict(bias=MISALIGNED), 3),
+])
+def test_forward_rejects(kwargs, status):
+    assert fwd(**kwargs) == status
+    assert native.load().kron_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(dtype=5), 1),
+    (dict(dS=None), 1),
+    (dict(x=MISALIGNED), 3),
+    (dict(m1=3), 2),
+    (dict(ws=None, ws_bytes=0), 4),                 # no workspace
+    (dict(ws=ALIGNED, ws_bytes=16), 4),             # too small
+])
+def test_backward_rejects(kwargs, status):
+    assert bwd(**kwargs) == status
+
+
+def test_backward_rejects_misaligned_workspace():
+    need = kfs.workspace_size(8, 2, 2, 4, 4, 1, "f32")
+    assert bwd(ws=V(0x10010), ws_bytes=need) == 3
+
+
+def test_python_binding_raises_without_cuda_tensors():
+    import torch
+    x = torch.zeros(4, 8)
+    S, A, B = torch.ones(2, 2), torch.zeros(1, 2, 2), torch.zeros(1, 4, 4)
+    with pytest.raises(ValueError):
+        kfs.forward(x, S, A, B, dtype="f32")
