@@ -125,6 +125,13 @@ KRON_API const char *kron_status_string(kron_status_t status);
 /* One-line description of the last failure on this host thread ("" if none). */
 KRON_API const char *kron_last_error(void);
 
+/* Device-side error state of the tensor-core kernels.  Every wait inside those
+ * kernels is bounded: if one makes no progress for 2 s the kernel raises an error
+ * word in device memory and returns instead of hanging.  This call synchronises the
+ * current device, reads that word and returns KRON_ERR_TIMEOUT if it is set
+ * (KRON_OK otherwise); clear != 0 resets it. */
+KRON_API kron_status_t kron_linear_device_error(int clear);
+
 /* KRON_LINEAR_ABI_VERSION of the loaded library. */
 KRON_API int kron_linear_abi_version(void);
 

@@ -107,6 +107,16 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
             e = kron::simt_forward((const float *)x, (const float *)S, (const float *)A,
                                    (const float *)B, (const float *)bias, (float *)y, s, cs);
             break;
+        case KRON_TF32:
+        case KRON_BF16: {
+            const bool bf16 = dtype == KRON_BF16;
+            if (!kron::tc_forward_supported(s, bf16))
+                return fail(KRON_ERR_UNSUPPORTED,
+                            "no tensor-core forward for p=%d q=%d m1=%d m2=%d r=%d (%s)", p, q, m1,
+                            m2, r, bf16 ? "bf16" : "tf32");
+            e = kron::tc_forward(x, S, A, B, bias, y, s, bf16, cs);
+            break;
+        }
         default:
             return fail(KRON_ERR_UNSUPPORTED, "dtype %d forward not implemented", (int)dtype);
     }
@@ -161,6 +171,13 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
             return fail(KRON_ERR_UNSUPPORTED, "dtype %d backward not implemented", (int)dtype);
     }
     if (e != cudaSuccess) return cuda_fail(e, "reduction launch");
+    return KRON_OK;
+}
+
+kron_status_t kron_linear_device_error(int clear) {
+    const int v = kron::tc_read_device_error(clear != 0);
+    if (v < 0) return fail(KRON_ERR_CUDA, "could not read the device error word");
+    if (v) return fail(KRON_ERR_TIMEOUT, "a kernel's bounded wait gave up (device error 0x%x)", v);
     return KRON_OK;
 }
 

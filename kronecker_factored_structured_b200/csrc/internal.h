@@ -38,6 +38,13 @@ cudaError_t simt_backward(const float *x, const float *S, const float *A, const 
                           const float *dY, float *dX, float *ws, int parts, const Shape &s,
                           cudaStream_t st);
 
+// ---- tensor-core paths (tc_fwd.cu, tc_bwd.cu): TF32 (fp32 I/O) or BF16 ----
+bool tc_forward_supported(const Shape &s, bool bf16);
+cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
+                       const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st);
+// Device error word of the tensor-core kernels (bounded waits); -1 if unreadable.
+int tc_read_device_error(bool clear);
+
 // ---- deterministic reduction of the row-range partials (reduce.cu) ----
 // S and A are float (is_bf16 = false) or bfloat16 (is_bf16 = true).
 cudaError_t reduce_partials(const float *ws, int parts, const void *S, const void *A,

@@ -1,0 +1,456 @@
+// tc_fwd.cu -- forward of the Kronecker layer on the sm_100a tensor cores (tcgen05).
+//
+// Vec trick (page "kronecker-layer-benchmark", section "3. The vec trick without the
+// loop"): per tile of NT = 128/m2 rows of x,
+//   stage 1   T[(i,k),(n,a)] = sum_j B_i[j,k] X_n[a,j]        one MMA chain, M = r*m2,
+//                                                             N = NT*p, K = m1
+//   stage 2   Y[(n,k),c]     = sum_(i,a) T[n,a,i,k] C_i[a,c]   M = NT*m2 = 128, N = q,
+//                                                             K = r*p
+//   y[n, c*m2 + k] = Y[(n,k),c] + bias[c*m2 + k]
+// Stage 1 is computed transposed, so each accumulator lane (i,k) holds a whole row of
+// stage 2's A operand: the epilogue moves it TMEM -> registers -> shared memory with
+// 16-byte stores straight into the K-major swizzled layout stage 2 reads.  That is the
+// page's permute of Z, done on chip; T never reaches HBM.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over tiles):
+//   warp 0     TMA producer: x tiles into an S-stage ring (128B-swizzled)
+//   warp 1     TMEM allocator + single-thread MMA issuer
+//   warps 2-5  epilogue 1: stage-1 accumulator -> T in shared memory (operand of stage 2)
+//   warps 6-9  epilogue 2: stage-2 accumulator + bias -> y in HBM (coalesced rows)
+// Accumulators and T are double-buffered so stage 1 of tile t+1 overlaps the epilogues.
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+namespace kron {
+namespace tc {
+
+__device__ int g_device_error = 0;
+
+template <typename T> struct Elt;
+template <> struct Elt<float> {
+    static constexpr int bytes = 4;
+    static constexpr uint32_t fmt = 2;  // TF32
+    static constexpr bool tf32 = true;
+};
+template <> struct Elt<__nv_bfloat16> {
+    static constexpr int bytes = 2;
+    static constexpr uint32_t fmt = 1;  // BF16
+    static constexpr bool tf32 = false;
+};
+
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
+struct FwdCfg {
+    using T = T_;
+    static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_;
+    static constexpr int E = Elt<T>::bytes;
+    static constexpr int NT = 128 / M2;        // rows of x per tile
+    static constexpr int N1 = NT * P;          // stage-1 N: (n,a)
+    static constexpr int SW1 = cmin(128, M1 * E);
+    static constexpr int KC1 = M1 * E / SW1;   // 128B K-chunks along j
+    static constexpr int K2B = R * P * E;      // stage-2 K in bytes: (i,a)
+    static constexpr int SW2 = cmin(128, K2B);
+    static constexpr int KC2 = K2B / SW2;
+    static constexpr int STAGES = 3;
+    // shared-memory regions (bytes, each 1024-aligned)
+    static constexpr int A1_BYTES = 128 * M1 * E;      // B_all^T [(i,k)][j]
+    static constexpr int B2_BYTES = Q * K2B;           // C'      [c][(i,a)]
+    static constexpr int X_BYTES = N1 * M1 * E;        // x tile  [(n,a)][j]
+    static constexpr int T_BYTES = 128 * K2B;          // T       [(n,k)][(i,a)]
+    static constexpr int OFF_A1 = 0;
+    static constexpr int OFF_B2 = OFF_A1 + A1_BYTES;
+    static constexpr int OFF_X = OFF_B2 + B2_BYTES;
+    static constexpr int OFF_T = OFF_X + STAGES * X_BYTES;
+    static constexpr int OFF_BAR = OFF_T + 2 * T_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+    // TMEM columns: D1[2] (N1 each), D2[2] (Q each)
+    static constexpr int TM_D1 = 0, TM_D2 = 2 * N1;
+    static constexpr int TM_COLS_USED = 2 * N1 + 2 * Q;
+    static constexpr int TM_COLS = TM_COLS_USED <= 32 ? 32 : TM_COLS_USED <= 64 ? 64
+                                 : TM_COLS_USED <= 128 ? 128 : TM_COLS_USED <= 256 ? 256 : 512;
+    static constexpr uint32_t IDESC1 = idesc_f32acc(128, N1, Elt<T>::fmt);
+    static constexpr uint32_t IDESC2 = idesc_f32acc(128, Q, Elt<T>::fmt);
+
+    static_assert(R * M2 == 128, "stage-1 M = r*m2 must be 128");
+    static_assert(128 % M2 == 0, "m2 must divide 128");
+    static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 256, "stage-1 N = (128/m2)*p out of range");
+    static_assert(Q % 32 == 0 && Q <= 256, "q must be a multiple of 32, at most 256");
+    static_assert(M1 * E % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
+    static_assert(K2B % 32 == 0 && (K2B <= 128 || K2B % 128 == 0), "r*p bytes");
+    static_assert((P * E) % 16 == 0, "p*elt must be a multiple of 16 bytes");
+    static_assert(TM_COLS_USED <= 512, "TMEM budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct FwdArgs {
+    const void *S, *A, *B, *bias;
+    void *y;
+    int64_t N;
+    int num_tiles;
+    int *device_error;
+};
+
+// Byte offset of element (row, kbyte) of a K-major operand with `rows` rows, K split
+// into chunks of `sw` bytes (chunk-major), 8-row atoms of 8*sw bytes, swizzled.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int kbyte, int rows, int sw) {
+    const int chunk = kbyte / sw, inner = kbyte % sw;
+    const uint32_t off = (uint32_t)chunk * rows * sw + (uint32_t)(row >> 3) * 8 * sw +
+                         (uint32_t)(row & 7) * sw + inner;
+    return swz(off, sw);
+}
+
+template <typename T>
+__device__ __forceinline__ float ldf(const void *p, size_t i) {
+    if constexpr (Elt<T>::tf32) return static_cast<const float *>(p)[i];
+    else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+// Write 16 bytes worth of operand values (4 tf32 / 8 bf16) from floats.
+template <typename T>
+__device__ __forceinline__ void st16(uint32_t addr, const float *v) {
+    if constexpr (Elt<T>::tf32) {
+        st_shared_v4(addr, f32_to_tf32(v[0]), f32_to_tf32(v[1]), f32_to_tf32(v[2]),
+                     f32_to_tf32(v[3]));
+    } else {
+        st_shared_v4(addr, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(320, 1)
+kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
+    using T = typename Cfg::T;
+    constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
+    constexpr int NT = Cfg::NT, N1 = Cfg::N1, S = Cfg::STAGES;
+    constexpr int VPC = 16 / E;  // values per 16-byte chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sA1 = sbase + Cfg::OFF_A1, sB2 = sbase + Cfg::OFF_B2;
+    const uint32_t sX = sbase + Cfg::OFF_X, sT = sbase + Cfg::OFF_T;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    // barrier indices
+    constexpr int B_XFULL = 0, B_XEMPTY = S, B_D1FULL = 2 * S, B_D1EMPTY = 2 * S + 2,
+                  B_TFULL = 2 * S + 4, B_TEMPTY = 2 * S + 6, B_D2FULL = 2 * S + 8,
+                  B_D2EMPTY = 2 * S + 10, NBARS = 2 * S + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
+    const Abort abort_flag{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    // ---------------- set-up: barriers, TMEM, packed factors ----------------
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar(B_XFULL + s), 1);
+            mbar_init(bar(B_XEMPTY + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_D1FULL + b), 1);
+            mbar_init(bar(B_D1EMPTY + b), 128);
+            mbar_init(bar(B_TFULL + b), 128);
+            mbar_init(bar(B_TEMPTY + b), 1);
+            mbar_init(bar(B_D2FULL + b), 1);
+            mbar_init(bar(B_D2EMPTY + b), 128);
+        }
+        *abort_flag.flag = 0;
+        mbar_init_fence();
+        prefetch_tmap(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
+    }
+    // stage-1 A operand: B_all^T[(i,k)][j] = B_i[j][k]
+    for (int e = threadIdx.x; e < 128 * (M1 / VPC); e += blockDim.x) {
+        const int row = e / (M1 / VPC), j0 = (e % (M1 / VPC)) * VPC;
+        const int i = row / M2, k = row % M2;
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < VPC; ++t) v[t] = ldf<T>(args.B, ((size_t)i * M1 + j0 + t) * M2 + k);
+        st16<T>(sA1 + kmajor_off(row, j0 * E, 128, Cfg::SW1), v);
+    }
+    // stage-2 B operand: C'[c][(i,a)] = S[a][c] * A_i[a][c]
+    for (int e = threadIdx.x; e < Q * (R * P / VPC); e += blockDim.x) {
+        const int c = e / (R * P / VPC), ia0 = (e % (R * P / VPC)) * VPC;
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < VPC; ++t) {
+            const int ia = ia0 + t, i = ia / P, a = ia % P;
+            v[t] = ldf<T>(args.S, (size_t)a * Q + c) * ldf<T>(args.A, ((size_t)i * P + a) * Q + c);
+        }
+        st16<T>(sB2 + kmajor_off(c, ia0 * E, Q, Cfg::SW2), v);
+    }
+    fence_proxy_async();  // generic-proxy writes of the factors -> visible to the MMA
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int my_tiles = (args.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int t = 0; t < my_tiles; ++t) {
+                const int s = t % S;
+                const uint32_t ph = (t / S) & 1;
+                if (!mbar_wait(bar(B_XEMPTY + s), ph ^ 1, abort_flag)) break;
+                const int tile = blockIdx.x + t * gridDim.x;
+                mbar_arrive_expect_tx(bar(B_XFULL + s), Cfg::X_BYTES);
+#pragma unroll
+                for (int kc = 0; kc < Cfg::KC1; ++kc)
+                    tma_load_2d(sX + s * Cfg::X_BYTES + kc * N1 * Cfg::SW1, &tmap_x,
+                                kc * (Cfg::SW1 / E), tile * N1, bar(B_XFULL + s));
+                issued = t + 1;
+            }
+            // drain: loads still in flight complete before the CTA may exit
+            for (int t = (issued > S ? issued - S : 0); t < issued; ++t)
+                mbar_wait(bar(B_XFULL + t % S), (t / S) & 1, abort_flag);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            auto stage2 = [&](int u) -> bool {
+                const int b = u & 1;
+                const uint32_t pb = (u >> 1) & 1;
+                if (!mbar_wait(bar(B_TFULL + b), pb, abort_flag)) return false;
+                if (!mbar_wait(bar(B_D2EMPTY + b), pb ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t d = tmem + Cfg::TM_D2 + b * Q;
+#pragma unroll
+                for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
+                    const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
+                    const uint64_t ad = sdesc_kmajor(sT + b * Cfg::T_BYTES + ch * 128 * Cfg::SW2 + in, Cfg::SW2);
+                    const uint64_t bd = sdesc_kmajor(sB2 + ch * Q * Cfg::SW2 + in, Cfg::SW2);
+                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC2, kk > 0);
+                }
+                mma_commit(bar(B_TEMPTY + b));
+                mma_commit(bar(B_D2FULL + b));
+                return true;
+            };
+            bool ok = true;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                const int s = t % S, b = t & 1;
+                const uint32_t ph = (t / S) & 1, pb = (t >> 1) & 1;
+                if (!mbar_wait(bar(B_XFULL + s), ph, abort_flag)) break;
+                if (!mbar_wait(bar(B_D1EMPTY + b), pb ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + Cfg::TM_D1 + b * N1;
+#pragma unroll
+                for (int kk = 0; kk < M1 * E / 32; ++kk) {
+                    const int kb = kk * 32, ch = kb / Cfg::SW1, in = kb % Cfg::SW1;
+                    const uint64_t ad = sdesc_kmajor(sA1 + ch * 128 * Cfg::SW1 + in, Cfg::SW1);
+                    const uint64_t bd = sdesc_kmajor(sX + s * Cfg::X_BYTES + ch * N1 * Cfg::SW1 + in, Cfg::SW1);
+                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC1, kk > 0);
+                }
+                mma_commit(bar(B_XEMPTY + s));
+                mma_commit(bar(B_D1FULL + b));
+                if (t > 0) ok = stage2(t - 1);
+            }
+            if (ok && my_tiles > 0) stage2(my_tiles - 1);
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue 1: D1 (lanes (i,k), columns (n,a)) -> T smem ----------------
+        const int quad = warp & 3;
+        const int L = quad * 32 + lane;  // (i,k)
+        const int i = L / M2, k = L % M2;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        for (int t = 0; t < my_tiles; ++t) {
+            const int b = t & 1;
+            const uint32_t pb = (t >> 1) & 1;
+            if (!mbar_wait(bar(B_D1FULL + b), pb, abort_flag)) break;
+            if (!mbar_wait(bar(B_TEMPTY + b), pb ^ 1, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t tb = sT + b * Cfg::T_BYTES;
+#pragma unroll 1
+            for (int c0 = 0; c0 < N1; c0 += 32) {
+                uint32_t r[32];
+                tmem_load32(tmem + lane_addr + Cfg::TM_D1 + b * N1 + c0, r);
+                if (c0 + 32 >= N1) {  // all of D1[b] read by this thread
+                    tc_fence_before();
+                    mbar_arrive(bar(B_D1EMPTY + b));
+                }
+#pragma unroll
+                for (int g = 0; g < 32 / VPC; ++g) {
+                    const int col = c0 + g * VPC;   // (n,a) of the first value
+                    const int n = col / P, a = col % P;
+                    float v[8];
+#pragma unroll
+                    for (int u = 0; u < VPC; ++u) v[u] = __uint_as_float(r[g * VPC + u]);
+                    st16<T>(tb + kmajor_off(n * M2 + k, (i * P + a) * E, 128, Cfg::SW2), v);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(B_TFULL + b));
+        }
+    } else {
+        // ---------------- epilogue 2: D2 (lanes (n,k), columns c) + bias -> y ----------------
+        const int quad = warp & 3;
+        const int L = quad * 32 + lane;  // (n,k)
+        const int n = L / M2, k = L % M2;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        float bias[Q];
+#pragma unroll
+        for (int c = 0; c < Q; ++c) bias[c] = args.bias ? ldf<T>(args.bias, (size_t)c * M2 + k) : 0.f;
+        for (int t = 0; t < my_tiles; ++t) {
+            const int b = t & 1;
+            const uint32_t pb = (t >> 1) & 1;
+            if (!mbar_wait(bar(B_D2FULL + b), pb, abort_flag)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
+#pragma unroll
+            for (int c0 = 0; c0 < Q; c0 += 32) {
+                uint32_t r[32];
+                tmem_load32(tmem + lane_addr + Cfg::TM_D2 + b * Q + c0, r);
+                if (c0 + 32 >= Q) {
+                    tc_fence_before();
+                    mbar_arrive(bar(B_D2EMPTY + b));
+                }
+                if (row < args.N) {
+#pragma unroll
+                    for (int u = 0; u < 32 && c0 + u < Q; ++u) {
+                        const float v = __uint_as_float(r[u]) + bias[c0 + u];
+                        const size_t o = (size_t)row * (Q * M2) + (size_t)(c0 + u) * M2 + k;
+                        if constexpr (Elt<T>::tf32) static_cast<float *>(args.y)[o] = v;
+                        else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------- teardown ----------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D tensor map of a row-major [rows][cols] matrix, box = box_cols x box_rows, swizzled.
+cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
+                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw) {
+    auto enc = get_encode();
+    if (!enc) return cudaErrorNotSupported;
+    const int E = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * E};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUtensorMapSwizzle swm = sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : sw == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                           : sw == 32  ? CU_TENSOR_MAP_SWIZZLE_32B
+                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
+    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                     2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swm, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Address of the device error word on the current device (looked up once per device).
+int *device_error_ptr() {
+    static int *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = (int *)p;
+    }
+    return ptrs[dev];
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+template <class Cfg>
+cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *B,
+                       const void *bias, void *y, const Shape &s, cudaStream_t st) {
+    using T = typename Cfg::T;
+    const bool bf16 = !Elt<T>::tf32;
+    CUtensorMap tm;
+    cudaError_t e = make_tmap_2d(&tm, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1,
+                                 Cfg::SW1 / Cfg::E, Cfg::N1, Cfg::SW1);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kron_fwd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    FwdArgs a{S, A, B, bias, y, s.N, (int)((s.N + Cfg::NT - 1) / Cfg::NT), device_error_ptr()};
+    const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+    kron_fwd_tc_kernel<Cfg><<<grid, 320, Cfg::SMEM, st>>>(tm, a);
+    return cudaGetLastError();
+}
+
+using FwdFn = cudaError_t (*)(const void *, const void *, const void *, const void *,
+                              const void *, void *, const Shape &, cudaStream_t);
+
+struct FwdEntry {
+    int p, q, m1, m2, r;
+    bool bf16;
+    FwdFn fn;
+};
+
+// Shapes with a compiled tensor-core forward.
+const FwdEntry kFwdTable[] = {
+    {32, 32, 32, 32, 4, false, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, float>>},
+    {32, 32, 32, 32, 4, true, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, __nv_bfloat16>>},
+};
+
+FwdFn find_fwd(const Shape &s, bool bf16) {
+    for (const auto &f : kFwdTable)
+        if (f.p == s.p && f.q == s.q && f.m1 == s.m1 && f.m2 == s.m2 && f.r == s.r && f.bf16 == bf16)
+            return f.fn;
+    return nullptr;
+}
+
+}  // namespace tc
+
+bool tc_forward_supported(const Shape &s, bool bf16) { return tc::find_fwd(s, bf16) != nullptr; }
+
+cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
+                       const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st) {
+    tc::FwdFn fn = tc::find_fwd(s, bf16);
+    if (!fn) return cudaErrorNotSupported;
+    return fn(x, S, A, B, bias, y, s, st);
+}
+
+int tc_read_device_error(bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, tc::g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(tc::g_device_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace kron

@@ -28,7 +28,8 @@ STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
 
 # Every symbol include/kron_linear.h declares.
 EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_workspace_size",
-           "kron_status_string", "kron_last_error", "kron_linear_abi_version")
+           "kron_status_string", "kron_last_error", "kron_linear_device_error",
+           "kron_linear_abi_version")
 
 
 class KronError(RuntimeError):
@@ -62,6 +63,8 @@ def load(path: str = LIB_PATH):
     lib.kron_status_string.restype = ctypes.c_char_p
     lib.kron_last_error.argtypes = []
     lib.kron_last_error.restype = ctypes.c_char_p
+    lib.kron_linear_device_error.argtypes = [I]
+    lib.kron_linear_device_error.restype = I
     lib.kron_linear_abi_version.argtypes = []
     lib.kron_linear_abi_version.restype = I
     _lib = lib
@@ -104,6 +107,11 @@ def shapes(S, A, B):
         raise ValueError(f"inconsistent factor shapes S{tuple(S.shape)} A{tuple(A.shape)} "
                          f"B{tuple(B.shape)}")
     return p, q, m1, m2, r
+
+
+def device_error(clear: bool = False) -> None:
+    """Raise KronError(KRON_ERR_TIMEOUT) if a kernel's bounded wait gave up."""
+    _check(load().kron_linear_device_error(1 if clear else 0))
 
 
 def workspace_size(N, p, q, m1, m2, r, dtype="tf32") -> int:
