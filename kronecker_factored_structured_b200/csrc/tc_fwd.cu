@@ -12,12 +12,21 @@
 // 16-byte stores straight into the K-major swizzled layout stage 2 reads.  That is the
 // page's permute of Z, done on chip; T never reaches HBM.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over tiles):
-//   warp 0     TMA producer: x tiles into an S-stage ring (128B-swizzled)
-//   warp 1     TMEM allocator + single-thread MMA issuer
-//   warps 2-5  epilogue 1: stage-1 accumulator -> T in shared memory (operand of stage 2)
-//   warps 6-9  epilogue 2: stage-2 accumulator + bias -> y in HBM (coalesced rows)
-// Accumulators and T are double-buffered so stage 1 of tile t+1 overlaps the epilogues.
+// Warp roles (480 threads, one CTA per SM, persistent over tiles):
+//   warp 0       TMA producer: x tiles into an S-stage ring (128B-swizzled)
+//   warps 1, 2   MMA issuers for even / odd tiles (warp 1 also owns the TMEM allocation)
+//   warps 3-10   epilogue 1: stage-1 accumulator -> T in shared memory (stage 2's A
+//                operand); every tile is handled by all 8 warps, two per TMEM lane
+//                quadrant, each taking half of the columns
+//   warps 11-14  epilogue 2: stage-2 accumulator + bias -> y in HBM (coalesced rows)
+// Any shared-memory access by an MMA-issuing thread (an mbarrier wait included) first
+// drains that thread's queued MMAs, leaving the tensor pipe idle.  So each issuer
+// synchronises once per tile -- round k waits for everything it needs, then issues
+// stage 2 of tile k and stage 1 of tile k+2 in one burst -- and two issuers own
+// alternate tiles, so while one drains at its sync point the other keeps the tensor
+// core busy.  Stage-1 accumulators are triple-buffered; T and the stage-2 accumulator
+// are one per tile parity.  The epilogues take the tiles strictly in order, which keeps
+// every mbarrier's phases in order (a consumer can never test a phase two ahead).
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -68,9 +77,10 @@ struct FwdCfg {
     static constexpr int OFF_T = OFF_X + STAGES * X_BYTES;
     static constexpr int OFF_BAR = OFF_T + 2 * T_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + alignment slack
-    // TMEM columns: D1[2] (N1 each), D2[2] (Q each)
-    static constexpr int TM_D1 = 0, TM_D2 = 2 * N1;
-    static constexpr int TM_COLS_USED = 2 * N1 + 2 * Q;
+    // TMEM columns: D1[3] (N1 each; stage 1 runs two tiles ahead), D2[2] (Q each)
+    static constexpr int D1_SLOTS = 3;
+    static constexpr int TM_D1 = 0, TM_D2 = D1_SLOTS * N1;
+    static constexpr int TM_COLS_USED = D1_SLOTS * N1 + 2 * Q;
     static constexpr int TM_COLS = TM_COLS_USED <= 32 ? 32 : TM_COLS_USED <= 64 ? 64
                                  : TM_COLS_USED <= 128 ? 128 : TM_COLS_USED <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC1 = idesc_f32acc(128, N1, Elt<T>::fmt);
@@ -78,7 +88,7 @@ struct FwdCfg {
 
     static_assert(R * M2 == 128, "stage-1 M = r*m2 must be 128");
     static_assert(128 % M2 == 0, "m2 must divide 128");
-    static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 256, "stage-1 N = (128/m2)*p out of range");
+    static_assert(N1 % 64 == 0 && N1 <= 256, "stage-1 N = (128/m2)*p: multiple of 64, at most 256");
     static_assert(Q % 32 == 0 && Q <= 256, "q must be a multiple of 32, at most 256");
     static_assert(M1 * E % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
     static_assert(K2B % 32 == 0 && (K2B <= 128 || K2B % 128 == 0), "r*p bytes");
@@ -123,7 +133,7 @@ __device__ __forceinline__ void st16(uint32_t addr, const float *v) {
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(480, 1)
 kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     using T = typename Cfg::T;
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
@@ -138,9 +148,10 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     const uint32_t sX = sbase + Cfg::OFF_X, sT = sbase + Cfg::OFF_T;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     // barrier indices
-    constexpr int B_XFULL = 0, B_XEMPTY = S, B_D1FULL = 2 * S, B_D1EMPTY = 2 * S + 2,
-                  B_TFULL = 2 * S + 4, B_TEMPTY = 2 * S + 6, B_D2FULL = 2 * S + 8,
-                  B_D2EMPTY = 2 * S + 10, NBARS = 2 * S + 12;
+    constexpr int D1S = Cfg::D1_SLOTS;
+    constexpr int B_XFULL = 0, B_XEMPTY = S, B_D1FULL = 2 * S, B_D1EMPTY = 2 * S + D1S,
+                  B_TFULL = 2 * S + 2 * D1S, B_TEMPTY = B_TFULL + 2, B_D2FULL = B_TFULL + 4,
+                  B_D2EMPTY = B_TFULL + 6, B_DRAIN = B_TFULL + 8, NBARS = B_TFULL + 10;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
     const Abort abort_flag{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
     auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -153,13 +164,16 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             mbar_init(bar(B_XFULL + s), 1);
             mbar_init(bar(B_XEMPTY + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < D1S; ++b) {
             mbar_init(bar(B_D1FULL + b), 1);
-            mbar_init(bar(B_D1EMPTY + b), 128);
-            mbar_init(bar(B_TFULL + b), 128);
+            mbar_init(bar(B_D1EMPTY + b), 256);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_TFULL + b), 256);
             mbar_init(bar(B_TEMPTY + b), 1);
             mbar_init(bar(B_D2FULL + b), 1);
             mbar_init(bar(B_D2EMPTY + b), 128);
+            mbar_init(bar(B_DRAIN + b), 1);
         }
         *abort_flag.flag = 0;
         mbar_init_fence();
@@ -214,37 +228,16 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             }
             // drain: loads still in flight complete before the CTA may exit
             for (int t = (issued > S ? issued - S : 0); t < issued; ++t)
-                mbar_wait(bar(B_XFULL + t % S), (t / S) & 1, abort_flag);
+                mbar_wait_drain(bar(B_XFULL + t % S), (t / S) & 1);
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 || warp == 2) {
+        // ---------------- MMA issuers: warp 1 even tiles, warp 2 odd tiles ----------------
+        const int par = warp - 1;
         if (lane == 0) {
-            auto stage2 = [&](int u) -> bool {
-                const int b = u & 1;
-                const uint32_t pb = (u >> 1) & 1;
-                if (!mbar_wait(bar(B_TFULL + b), pb, abort_flag)) return false;
-                if (!mbar_wait(bar(B_D2EMPTY + b), pb ^ 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t d = tmem + Cfg::TM_D2 + b * Q;
-#pragma unroll
-                for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
-                    const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
-                    const uint64_t ad = sdesc_kmajor(sT + b * Cfg::T_BYTES + ch * 128 * Cfg::SW2 + in, Cfg::SW2);
-                    const uint64_t bd = sdesc_kmajor(sB2 + ch * Q * Cfg::SW2 + in, Cfg::SW2);
-                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC2, kk > 0);
-                }
-                mma_commit(bar(B_TEMPTY + b));
-                mma_commit(bar(B_D2FULL + b));
-                return true;
-            };
-            bool ok = true;
-            for (int t = 0; t < my_tiles && ok; ++t) {
-                const int s = t % S, b = t & 1;
-                const uint32_t ph = (t / S) & 1, pb = (t >> 1) & 1;
-                if (!mbar_wait(bar(B_XFULL + s), ph, abort_flag)) break;
-                if (!mbar_wait(bar(B_D1EMPTY + b), pb ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + Cfg::TM_D1 + b * N1;
+            // stage 1 of tile u into D1 slot u % 3 (its waits already done)
+            auto issue_stage1 = [&](int u) {
+                const int s = u % S, d1 = u % D1S;
+                const uint32_t d = tmem + Cfg::TM_D1 + d1 * N1;
 #pragma unroll
                 for (int kk = 0; kk < M1 * E / 32; ++kk) {
                     const int kb = kk * 32, ch = kb / Cfg::SW1, in = kb % Cfg::SW1;
@@ -253,31 +246,66 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
                     mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC1, kk > 0);
                 }
                 mma_commit(bar(B_XEMPTY + s));
-                mma_commit(bar(B_D1FULL + b));
-                if (t > 0) ok = stage2(t - 1);
+                mma_commit(bar(B_D1FULL + d1));
+            };
+            auto wait_stage1 = [&](int u) -> bool {
+                return mbar_wait(bar(B_XFULL + u % S), (u / S) & 1, abort_flag) &&
+                       mbar_wait(bar(B_D1EMPTY + u % D1S), ((u / D1S) & 1) ^ 1, abort_flag);
+            };
+            bool ok = true;
+            if (par < my_tiles) {  // prologue: stage 1 of this issuer's first tile
+                ok = wait_stage1(par);
+                if (ok) {
+                    tc_fence_after();
+                    issue_stage1(par);
+                }
             }
-            if (ok && my_tiles > 0) stage2(my_tiles - 1);
+            const uint32_t d = tmem + Cfg::TM_D2 + par * Q;
+            const uint32_t tb = sT + par * Cfg::T_BYTES;
+            for (int k = par; k < my_tiles && ok; k += 2) {
+                const uint32_t pb = (k >> 1) & 1;
+                // one synchronisation point per round
+                if (!mbar_wait(bar(B_TFULL + par), pb, abort_flag)) break;
+                if (!mbar_wait(bar(B_D2EMPTY + par), pb ^ 1, abort_flag)) break;
+                if (k + 2 < my_tiles && !wait_stage1(k + 2)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
+                    const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
+                    const uint64_t ad = sdesc_kmajor(tb + ch * 128 * Cfg::SW2 + in, Cfg::SW2);
+                    const uint64_t bd = sdesc_kmajor(sB2 + ch * Q * Cfg::SW2 + in, Cfg::SW2);
+                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC2, kk > 0);
+                }
+                mma_commit(bar(B_TEMPTY + par));
+                mma_commit(bar(B_D2FULL + par));
+                if (k + 2 < my_tiles) issue_stage1(k + 2);
+            }
+            // every MMA of this issuer has completed before TMEM can be released
+            mma_commit(bar(B_DRAIN + par));
+            mbar_wait_drain(bar(B_DRAIN + par), 0);
         }
-    } else if (warp < 6) {
+    } else if (warp < 11) {
         // ---------------- epilogue 1: D1 (lanes (i,k), columns (n,a)) -> T smem ----------------
+        const int half = (warp - 3) / 4;          // which half of the columns
         const int quad = warp & 3;
         const int L = quad * 32 + lane;  // (i,k)
         const int i = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        constexpr int HC = N1 / 2;                // columns per warp
         for (int t = 0; t < my_tiles; ++t) {
-            const int b = t & 1;
+            const int b = t & 1, d1 = t % D1S;
             const uint32_t pb = (t >> 1) & 1;
-            if (!mbar_wait(bar(B_D1FULL + b), pb, abort_flag)) break;
+            if (!mbar_wait(bar(B_D1FULL + d1), (t / D1S) & 1, abort_flag)) break;
             if (!mbar_wait(bar(B_TEMPTY + b), pb ^ 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t tb = sT + b * Cfg::T_BYTES;
 #pragma unroll 1
-            for (int c0 = 0; c0 < N1; c0 += 32) {
+            for (int c0 = half * HC; c0 < (half + 1) * HC; c0 += 32) {
                 uint32_t r[32];
-                tmem_load32(tmem + lane_addr + Cfg::TM_D1 + b * N1 + c0, r);
-                if (c0 + 32 >= N1) {  // all of D1[b] read by this thread
+                tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1 + c0, r);
+                if (c0 + 32 >= (half + 1) * HC) {  // this thread's columns of the slot are read
                     tc_fence_before();
-                    mbar_arrive(bar(B_D1EMPTY + b));
+                    mbar_arrive(bar(B_D1EMPTY + d1));
                 }
 #pragma unroll
                 for (int g = 0; g < 32 / VPC; ++g) {
@@ -309,8 +337,13 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
 #pragma unroll
             for (int c0 = 0; c0 < Q; c0 += 32) {
-                uint32_t r[32];
-                tmem_load32(tmem + lane_addr + Cfg::TM_D2 + b * Q + c0, r);
+                float acc[32];
+                {
+                    uint32_t r[32];
+                    tmem_load32(tmem + lane_addr + Cfg::TM_D2 + b * Q + c0, r);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) acc[u] = __uint_as_float(r[u]);
+                }
                 if (c0 + 32 >= Q) {
                     tc_fence_before();
                     mbar_arrive(bar(B_D2EMPTY + b));
@@ -318,7 +351,7 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
                 if (row < args.N) {
 #pragma unroll
                     for (int u = 0; u < 32 && c0 + u < Q; ++u) {
-                        const float v = __uint_as_float(r[u]) + bias[c0 + u];
+                        const float v = acc[u] + bias[c0 + u];
                         const size_t o = (size_t)row * (Q * M2) + (size_t)(c0 + u) * M2 + k;
                         if constexpr (Elt<T>::tf32) static_cast<float *>(args.y)[o] = v;
                         else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
@@ -406,7 +439,7 @@ cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *
     if (e != cudaSuccess) return e;
     FwdArgs a{S, A, B, bias, y, s.N, (int)((s.N + Cfg::NT - 1) / Cfg::NT), device_error_ptr()};
     const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-    kron_fwd_tc_kernel<Cfg><<<grid, 320, Cfg::SMEM, st>>>(tm, a);
+    kron_fwd_tc_kernel<Cfg><<<grid, 480, Cfg::SMEM, st>>>(tm, a);
     return cudaGetLastError();
 }
 
