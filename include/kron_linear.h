@@ -84,7 +84,7 @@ typedef enum {
  *   S, A, B          factors as above
  *   bias  [q*m2]     may be NULL (no bias)
  *   y     [N][q*m2]  output, overwritten
- *   N >= 0 rows (N == 0 is a no-op); p, q, m1, m2, r >= 1.
+ *   N >= 0 rows (N == 0 is a no-op and x, y may then be NULL); p, q, m1, m2, r >= 1.
  * Requirements: x, y, S, A, B, bias 16-byte aligned (KRON_ERR_ALIGNMENT);
  * m1 and m2 multiples of 4 (F32/TF32) or 8 (BF16), else KRON_ERR_UNSUPPORTED.
  */
@@ -100,6 +100,7 @@ KRON_API kron_status_t kron_linear_forward(const void *x, const void *S, const v
  *   dA    [r][p][q]   = dC_i (.) S,   dC_i = sum_n (X_n B_i) dY_n^T
  *   dB    [r][m1][m2] = sum_n X_n^T C_i dY_n
  *   dbias [q*m2]      = sum_n dY_n                                (may be NULL: skipped)
+ * With N == 0, x, dY and dX may be NULL and the factor gradients are set to zero.
  * Gradients OVERWRITE their outputs.  T = X_n B_i is recomputed, nothing is kept
  * from the forward call.  The sums over rows are split into a fixed number of
  * contiguous row ranges whose partials are added in a fixed order, so results are

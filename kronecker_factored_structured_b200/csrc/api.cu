@@ -46,13 +46,18 @@ kron_status_t check_shape(int64_t N, int p, int q, int m1, int m2, int r, kron_d
     return KRON_OK;
 }
 
+// Number of contiguous row ranges of the backward: at most kRowParts, none empty.  A
+// function of the shape and path only, so the summation order is fixed.
 int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
-    (void)dtype;
-    const int R = kron::simt_backward_rows(s);
-    if (R <= 0) return 0;
-    int64_t tiles = (s.N + R - 1) / R;
+    int rows_per_tile = 0;
+    if (dtype == KRON_F32) rows_per_tile = kron::simt_backward_rows(s);
+    else if (kron::tc_backward_supported(s, dtype == KRON_BF16)) rows_per_tile = kron::tc_backward_tile_rows(s);
+    if (rows_per_tile <= 0) return 0;
+    int64_t tiles = (s.N + rows_per_tile - 1) / rows_per_tile;
     if (tiles < 1) tiles = 1;
-    return tiles < kron::kRowParts ? (int)tiles : kron::kRowParts;
+    const int64_t parts0 = tiles < kron::kRowParts ? tiles : kron::kRowParts;
+    const int64_t per = (tiles + parts0 - 1) / parts0;
+    return (int)((tiles + per - 1) / per);
 }
 
 }  // namespace
@@ -91,8 +96,8 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
     g_last_error[0] = 0;
     kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
     if (st != KRON_OK) return st;
-    if (!x || !S || !A || !B || !y)
-        return fail(KRON_ERR_INVALID_ARG, "x, S, A, B and y must be non-null");
+    if (!S || !A || !B || (N > 0 && (!x || !y)))
+        return fail(KRON_ERR_INVALID_ARG, "S, A, B (and x, y when N > 0) must be non-null");
     if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(y) ||
         (bias && !aligned16(bias)))
         return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
@@ -132,8 +137,9 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
     g_last_error[0] = 0;
     kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
     if (st != KRON_OK) return st;
-    if (!x || !S || !A || !B || !dY || !dS || !dA || !dB)
-        return fail(KRON_ERR_INVALID_ARG, "x, S, A, B, dY, dS, dA and dB must be non-null");
+    if (!S || !A || !B || !dS || !dA || !dB || (N > 0 && (!x || !dY)))
+        return fail(KRON_ERR_INVALID_ARG,
+                    "S, A, B, dS, dA, dB (and x, dY when N > 0) must be non-null");
     if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(dY) ||
         !aligned16(dS) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
         (dbias && !aligned16(dbias)))
@@ -148,6 +154,11 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
             e = cudaMemsetAsync(dbias, 0, (size_t)q * m2 * sizeof(float), cs);
         return e == cudaSuccess ? KRON_OK : cuda_fail(e, "zero gradients");
     }
+    if (dtype != KRON_F32 && !kron::tc_backward_supported(s, dtype == KRON_BF16))
+        return fail(KRON_ERR_UNSUPPORTED, "no tensor-core backward for p=%d q=%d m1=%d m2=%d r=%d",
+                    p, q, m1, m2, r);
+    if (dtype == KRON_F32 && kron::simt_backward_rows(s) <= 0)
+        return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
     const size_t need = kron_linear_workspace_size(N, p, q, m1, m2, r, dtype);
     if (!workspace || workspace_bytes < need)
         return fail(KRON_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
@@ -167,6 +178,19 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
             e = kron::reduce_partials((const float *)workspace, parts, S, A, false, (float *)dS,
                                       (float *)dA, (float *)dB, (float *)dbias, s, cs);
             break;
+        case KRON_TF32:
+        case KRON_BF16: {
+            const bool bf16 = dtype == KRON_BF16;
+            if (!kron::tc_backward_supported(s, bf16))
+                return fail(KRON_ERR_UNSUPPORTED,
+                            "no tensor-core backward for p=%d q=%d m1=%d m2=%d r=%d (%s)", p, q,
+                            m1, m2, r, bf16 ? "bf16" : "tf32");
+            e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16, cs);
+            if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+            e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
+                                      (float *)dA, (float *)dB, (float *)dbias, s, cs);
+            break;
+        }
         default:
             return fail(KRON_ERR_UNSUPPORTED, "dtype %d backward not implemented", (int)dtype);
     }

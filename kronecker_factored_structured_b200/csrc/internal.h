@@ -42,6 +42,12 @@ cudaError_t simt_backward(const float *x, const float *S, const float *A, const 
 bool tc_forward_supported(const Shape &s, bool bf16);
 cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
                        const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st);
+bool tc_backward_supported(const Shape &s, bool bf16);
+int tc_backward_tile_rows(const Shape &s);
+// Writes dX (if non-null) and the per-range partials (parts x partial_stride floats).
+cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
+                        const void *dY, void *dX, float *ws, int parts, const Shape &s,
+                        bool bf16, cudaStream_t st);
 // Device error word of the tensor-core kernels (bounded waits); -1 if unreadable.
 int tc_read_device_error(bool clear);
 

@@ -20,7 +20,7 @@ DTYPES = {"f32": KRON_F32, "tf32": KRON_TF32, "bf16": KRON_BF16}
 KRON_FLAG_SKIP_ZERO_BLOCKS = 1
 
 # Paths whose kernels are built into the library.
-IMPLEMENTED_PATHS = ("f32",)
+IMPLEMENTED_PATHS = ("f32", "tf32", "bf16")
 
 STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
           3: "KRON_ERR_ALIGNMENT", 4: "KRON_ERR_WORKSPACE", 5: "KRON_ERR_CUDA",

@@ -68,6 +68,7 @@ def bwd(ws=None, ws_bytes=0, dtype=0, flags=0, dS=ALIGNED, x=ALIGNED, N=8, m1=4)
     (dict(r=0), 1),
     (dict(x=None), 1),
     (dict(y=None), 1),
+    (dict(S=None, N=0), 1),
     (dict(m1=6), 2),               # not a multiple of 4 (F32)
     (dict(m1=4, dtype=2), 2),      # not a multiple of 8 (BF16)
     (dict(x=MISALIGNED), 3),
