@@ -63,11 +63,20 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def wait_started(self, timeout=5.0):
+        """Block until nvidia-smi has printed its first sample (it takes ~0.5 s to start)."""
+        import select
+        if self.proc is None:
+            return
+        r, _, _ = select.select([self.proc.stdout], [], [], timeout)
+        if r:
+            self.first = self.proc.stdout.readline()
 
     def __exit__(self, *exc):
         self.lines = []
@@ -78,7 +87,7 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.lines = [ln for ln in (getattr(self, "first", "") + out).splitlines() if ln.strip()]
 
     def summary(self):
         if not getattr(self, "lines", None):
@@ -149,7 +158,7 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--path", default=None, help="tf32 | f32 | bf16 (default: headline path)")
@@ -230,6 +239,7 @@ def main():
     marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
     start, end = ev(), ev()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.wait_started()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()

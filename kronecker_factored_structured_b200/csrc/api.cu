@@ -8,6 +8,13 @@
 #include <stdio.h>
 #include <string.h>
 
+namespace kron {
+const char *&launch_step() {
+    thread_local const char *step = "launch";
+    return step;
+}
+}  // namespace kron
+
 namespace {
 
 thread_local char g_last_error[256] = "";
@@ -22,7 +29,7 @@ kron_status_t fail(kron_status_t st, const char *fmt, ...) {
 }
 
 kron_status_t cuda_fail(cudaError_t e, const char *what) {
-    return fail(KRON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return fail(KRON_ERR_CUDA, "%s (%s): %s", what, kron::launch_step(), cudaGetErrorString(e));
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }

@@ -8,6 +8,9 @@
 
 namespace kron {
 
+// Name of the host-side step that failed in the last launcher call on this thread.
+const char *&launch_step();
+
 struct Shape {
     int64_t N;
     int p, q, m1, m2, r;

@@ -6,9 +6,10 @@
 // as on the page "kronecker-layer-benchmark", section "1. Build W, then multiply".)
 //
 // Workspace layout per range g: ws[g*stride + ...] = [dC: r*p*q][dB: r*m1*m2][dbias: q*m2].
-// Each block owns 32 consecutive output columns; its 8 warps sum ranges g = w, w+8, ...
-// in double, then warp 0 adds the 8 warp sums in order w = 0..7.  The order depends
-// only on `parts`, so results are bitwise reproducible.
+// Each block owns 32 consecutive output columns (for dC: 32 (a,c) positions and all r
+// ranks).  Its 8 warps sum ranges g = w, w+8, ... in double with several independent
+// accumulators, which are then added in a fixed order.  The order depends only on
+// `parts`, so results are bitwise reproducible.
 #include "internal.h"
 
 #include <cuda_bf16.h>
@@ -19,22 +20,52 @@ namespace {
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-__device__ __forceinline__ double block_sum(const float *__restrict__ ws, int parts,
-                                            size_t stride, size_t off, bool valid,
-                                            double (*red)[33]) {
+// Sums over the row ranges of up to NC columns off[0..ncols): warp w adds ranges
+// g = w, w+8, ... into U independent accumulators per column (so U*ncols loads are in
+// flight per thread); then the accumulators and the 8 warp sums are added in a fixed
+// order.
+template <int U, int NC>
+__device__ __forceinline__ void col_sums(const float *__restrict__ ws, int parts, size_t stride,
+                                         const size_t *off, bool valid, int ncols,
+                                         double (*red)[33], double *out) {
     const int lane = threadIdx.x, w = threadIdx.y;
-    double acc = 0.0;
-    if (valid)
-        for (int g = w; g < parts; g += 8) acc += (double)ws[(size_t)g * stride + off];
-    red[w][lane] = acc;
-    __syncthreads();
-    double tot = 0.0;
-    if (w == 0)
+    double acc[NC][U];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) tot += red[t][lane];
-    __syncthreads();
-    return tot;
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int u = 0; u < U; ++u) acc[c][u] = 0.0;
+    if (valid) {
+        for (int g = w; g < parts; g += 8 * U) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int gg = g + 8 * u;
+                if (gg < parts) {
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+                        if (c < ncols) acc[c][u] += (double)ws[(size_t)gg * stride + off[c]];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if (c >= ncols) break;
+        double sum = 0.0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) sum += acc[c][u];
+        red[w][lane] = sum;
+        __syncthreads();
+        if (w == 0) {
+            double tot = 0.0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) tot += red[t][lane];
+            out[c] = tot;
+        }
+        __syncthreads();
+    }
 }
+
+constexpr int kMaxRanksPerPass = 8;
 
 template <typename TI>
 __global__ void __launch_bounds__(256)
@@ -49,32 +80,44 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
     const int lane = threadIdx.x;
     int blk = blockIdx.x;
     if (blk < blocks_dc) {
+        // dC for all ranks of columns (a,c) -> dA = dC (.) S, dS = sum_i dC_i (.) A_i
         const size_t col = (size_t)blk * 32 + lane;
-        const bool valid = col < pq;
+        const bool v = col < pq;
         double ds = 0.0;
-        for (int i = 0; i < s.r; ++i) {
-            const double dc = block_sum(ws, parts, stride, (size_t)i * pq + col, valid, red);
-            if (threadIdx.y == 0 && valid) {
-                dA[(size_t)i * pq + col] = (float)(dc * (double)to_f(S[col]));
-                ds += dc * (double)to_f(A[(size_t)i * pq + col]);
+        for (int i0 = 0; i0 < s.r; i0 += kMaxRanksPerPass) {
+            const int nr = s.r - i0 < kMaxRanksPerPass ? s.r - i0 : kMaxRanksPerPass;
+            size_t off[kMaxRanksPerPass];
+            double dc[kMaxRanksPerPass];
+            for (int ii = 0; ii < kMaxRanksPerPass; ++ii) off[ii] = (size_t)(i0 + ii) * pq + col;
+            col_sums<2, kMaxRanksPerPass>(ws, parts, stride, off, v, nr, red, dc);
+            if (threadIdx.y == 0 && v) {
+                for (int ii = 0; ii < nr; ++ii) {
+                    const size_t e = (size_t)(i0 + ii) * pq + col;
+                    dA[e] = (float)(dc[ii] * (double)to_f(S[col]));
+                    ds += dc[ii] * (double)to_f(A[e]);
+                }
             }
         }
-        if (threadIdx.y == 0 && valid) dS[col] = (float)ds;
+        if (threadIdx.y == 0 && v) dS[col] = (float)ds;
         return;
     }
     blk -= blocks_dc;
     if (blk < blocks_db) {
         const size_t col = (size_t)blk * 32 + lane;
-        const bool valid = col < n_db;
-        const double v = block_sum(ws, parts, stride, n_dc + col, valid, red);
-        if (threadIdx.y == 0 && valid) dB[col] = (float)v;
+        const size_t off = n_dc + col;
+        const bool v = col < n_db;
+        double out;
+        col_sums<8, 1>(ws, parts, stride, &off, v, 1, red, &out);
+        if (threadIdx.y == 0 && v) dB[col] = (float)out;
         return;
     }
     blk -= blocks_db;
     const size_t col = (size_t)blk * 32 + lane;
-    const bool valid = col < n_b;
-    const double v = block_sum(ws, parts, stride, n_dc + n_db + col, valid, red);
-    if (threadIdx.y == 0 && valid) dbias[col] = (float)v;
+    const size_t off = n_dc + n_db + col;
+    const bool v = col < n_b;
+    double out;
+    col_sums<8, 1>(ws, parts, stride, &off, v, 1, red, &out);
+    if (threadIdx.y == 0 && v) dbias[col] = (float)out;
 }
 
 }  // namespace
@@ -86,18 +129,17 @@ cudaError_t reduce_partials(const float *ws, int parts, const void *S, const voi
     const int blocks_dc = (int)((pq + 31) / 32);
     const int blocks_db = (int)(((size_t)s.r * s.m1 * s.m2 + 31) / 32);
     const int blocks_b = dbias ? (int)(((size_t)s.q * s.m2 + 31) / 32) : 0;
-    const dim3 block(32, 8);
-    const unsigned grid = (unsigned)(blocks_dc + blocks_db + blocks_b);
     const size_t stride = partial_stride(s);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(blocks_dc + blocks_db + blocks_b));
+    cfg.blockDim = dim3(32, 8);
+    cfg.stream = st;
     if (is_bf16)
-        kron_reduce_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
-            ws, parts, stride, (const __nv_bfloat16 *)S, (const __nv_bfloat16 *)A, dS, dA, dB,
-            dbias, s, blocks_dc, blocks_db);
-    else
-        kron_reduce_kernel<float><<<grid, block, 0, st>>>(ws, parts, stride, (const float *)S,
-                                                          (const float *)A, dS, dA, dB, dbias,
-                                                          s, blocks_dc, blocks_db);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, kron_reduce_kernel<__nv_bfloat16>, ws, parts, stride,
+                                  (const __nv_bfloat16 *)S, (const __nv_bfloat16 *)A, dS, dA, dB,
+                                  dbias, s, blocks_dc, blocks_db);
+    return cudaLaunchKernelEx(&cfg, kron_reduce_kernel<float>, ws, parts, stride, (const float *)S,
+                              (const float *)A, dS, dA, dB, dbias, s, blocks_dc, blocks_db);
 }
 
 }  // namespace kron

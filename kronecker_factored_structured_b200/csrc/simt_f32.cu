@@ -348,8 +348,14 @@ cudaError_t simt_forward(const float *x, const float *S, const float *A, const f
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (s.N + R - 1) / R;
-    kron_fwd_simt_kernel<<<(unsigned)tiles, kThreads, smem, st>>>(x, S, A, B, bias, y, s, L);
-    return cudaGetLastError();
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)tiles);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        return cudaLaunchKernelEx(&cfg, kron_fwd_simt_kernel, x, S, A, B, bias, y, s, L);
+    }
 }
 
 cudaError_t simt_backward(const float *x, const float *S, const float *A, const float *B,
@@ -361,9 +367,14 @@ cudaError_t simt_backward(const float *x, const float *S, const float *A, const 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t rows_per_part = (s.N + parts - 1) / parts;
-    kron_bwd_simt_kernel<<<parts, kThreads, smem, st>>>(x, S, A, B, dY, dX, ws, rows_per_part,
-                                                        partial_stride(s), s, L);
-    return cudaGetLastError();
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)parts);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        return cudaLaunchKernelEx(&cfg, kron_bwd_simt_kernel, x, S, A, B, dY, dX, ws, rows_per_part, partial_stride(s), s, L);
+    }
 }
 
 }  // namespace kron

@@ -2,29 +2,32 @@
 //
 // Gradients of L = <G, y> (G = dY), W = sum_i kron(C_i, B_i), C_i = S (.) A_i (page
 // "kronecker-layer-benchmark", section "1. Build W, then multiply"; the page leaves the
-// backward to autograd).  Per tile of NT = 128/m1 rows, with only K-major operands:
+// backward to autograd).  Per tile of NT = r rows (shapes with p = m2 = 128/r), every
+// contraction on the tensor cores with K-major operands and a TMEM accumulator:
 //
-//   T'[(i,j),(n,c)] = sum_k B_i[j,k] G[(n,c),k]          (G B_i^T, A = B' [(i,j)][k])
-//   U [(n,k),(i,a)] = sum_c G[(n,c),k] C_i[a,c]          (C_i G,   A = G^T [(n,k)][c])
-//   dX[(n,j),a]     = sum_(i,c) T'[n,c,i,j] C_i[a,c]     (A = T'1 [(n,j)][(i,c)])
-//   dC[(i,c),a]    += sum_(n,j) T'[n,c,i,j] X[(n,a),j]   (A = T'2 [(i,c)][(n,j)])
-//   dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X[(n,a),j]    (A = U2 [(i,k)][(n,a)], B = X^T)
-//   dbias[c*m2+k]  += sum_n G[(n,c),k]
+//   U  = C_i G_n     as Ua[(i,a),(n,k)] = sum_c C[(i,a),c] G^T[(n,k),c]
+//                    and Ub[(n,k),(i,a)] = sum_c G^T[(n,k),c] C[(i,a),c]
+//   T  = X_n B_i     as T[(n,a),(i,k)]  = sum_j X[(n,a),j] Bt[(i,k),j]
+//   dX[(n,a),j]   = sum_(i,k) U[n,a,i,k] B_i[j,k]           A = U1 [(n,a)][(i,k)]
+//   dC[(i,a),c]  += sum_(n,k) T[n,a,i,k] G[(n,c),k]          A = T2 [(i,a)][(n,k)]
+//   dB[(i,k),j]  += sum_(n,a) U[n,a,i,k] X[(n,a),j]          A = U2 [(i,k)][(n,a)], B = X^T
+//   dbias[c*m2+k] += sum_n G[(n,c),k]
 //
-// T' and U exist only in TMEM and shared memory.  The TMEM -> shared-memory epilogues
-// write them in the K-major swizzled layouts the next contraction reads (the permute
-// the page's loop-free version does in HBM).  dC and dB accumulate in TMEM over the
-// CTA's fixed, contiguous range of rows, then go to the workspace as this range's
-// partial sums; reduce.cu adds the partials in a fixed order, so results are
-// reproducible bit for bit.
+// U is computed in both orientations so that each TMEM lane holds a contiguous row of
+// the operand the next contraction reads; every TMEM -> shared-memory epilogue is then
+// a sequence of 16-byte stores into a K-major swizzled layout (the permute the page's
+// loop-free version does in HBM).  dC and dB accumulate in TMEM over the CTA's fixed,
+// contiguous range of rows and are written to the workspace as that range's partial
+// sums; reduce.cu adds the partials in a fixed order (bitwise reproducible).
 //
-// Shared memory holds two intermediate buffers: A (T'1, then U2) and B (T'2, then X^T).
+// Shared memory: factors C, Bt, Bdx; tiles G, X, G^T; two intermediate buffers:
+//   A: U1 (read by dX), then U2 (read by dB)       -- "A chain"
+//   B: T2 (read by dC), then X^T (read by dB)      -- "B chain"
 // Warp roles (448 threads, one CTA per SM):
-//   warp 0       TMA producer (G and X tiles, one buffer each)
-//   warp 1       TMEM allocator + single-thread MMA issuer
-//   warps 2-5    G^T and X^T transposes, dbias partial, dX epilogue (TMEM -> HBM)
-//   warps 6-13   T' epilogue (T'1 and T'2) and U epilogue (U2), 2 warps per TMEM quadrant
-// The issuer waits at few points per tile (each wait drains its queued MMAs).
+//   warp 0       TMA producer (G and X tiles)
+//   warp 1       TMEM allocator + MMA issuer
+//   warps 2-5    B chain: T2 epilogue, X^T; also G^T, dbias and the dX epilogue
+//   warps 6-13   A chain: U1 and U2 epilogues, 2 warps per TMEM lane quadrant
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -34,7 +37,6 @@ namespace kron {
 namespace tc {
 
 int *device_error_ptr();
-int num_sms();
 cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
                          uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw);
 
@@ -53,62 +55,58 @@ template <> struct BE<__nv_bfloat16> {
 };
 
 constexpr int imin(int a, int b) { return a < b ? a : b; }
-constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
 struct BwdCfg {
     using T = T_;
     static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_;
     static constexpr int E = BE<T>::bytes;
-    static constexpr int NT = 128 / M1;            // rows per tile
-    // swizzle widths of the K extents used below (bytes)
-    static constexpr int SWK = imin(128, M2 * E);  // K = k   (T' MMA: B', G)
-    static constexpr int SWC = imin(128, Q * E);   // K = c   (U MMA: G^T, C_stack)
-    static constexpr int SWQ = imin(128, Q * E);   // K = (i,c) chunks (dX: T'1, Cdx)
-    static constexpr int SWJ = imin(128, M1 * E);  // K = (n,j) chunks (dC: T'2, X)
-    static constexpr int SWA = imin(128, P * E);   // K = (n,a) chunks (dB: U2, X^T)
+    static constexpr int NT = R;                   // rows per tile
+    static constexpr int SWC = imin(128, Q * E);   // K = c       (Ua, Ub)
+    static constexpr int SWJ = imin(128, M1 * E);  // K = j       (T)
+    static constexpr int SW128 = 128;              // K = (i,k), (n,k), (n,a): 128 * E bytes
+    static constexpr int SWG = M2 * E;             // G tile rows (k) and dC's B chunks
     // region sizes (bytes)
-    static constexpr int F_BP = 128 * M2 * E;          // B'      [(i,j)][k]
-    static constexpr int F_CS = R * P * Q * E;         // C_stack [(i,a)][c]
-    static constexpr int F_CDX = P * R * Q * E;        // Cdx     [a][(i,c)]
-    static constexpr int TILE_G = NT * Q * M2 * E;     // G tile  [(n,c)][k]
-    static constexpr int TILE_X = NT * P * M1 * E;     // X tile  [(n,a)][j]
-    static constexpr int TILE_GT = TILE_G;             // G^T     [(n,k)][c]
-    static constexpr int BUF_A = imax(128 * R * Q * E, R * M2 * NT * P * E);  // T'1 | U2
-    static constexpr int BUF_B = imax(R * Q * NT * M1 * E, M1 * NT * P * E);  // T'2 | X^T
-    static constexpr int OFF_BP = 0;
-    static constexpr int OFF_CS = OFF_BP + F_BP;
-    static constexpr int OFF_CDX = OFF_CS + F_CS;
-    static constexpr int OFF_G = OFF_CDX + F_CDX;
-    static constexpr int OFF_X = OFF_G + TILE_G;
+    static constexpr int F_C = 128 * Q * E;        // C    [(i,a)][c]
+    static constexpr int F_BT = 128 * M1 * E;      // Bt   [(i,k)][j]
+    static constexpr int F_BD = M1 * 128 * E;      // Bdx  [j][(i,k)]
+    static constexpr int TILE_G = 128 * M2 * E;    // G    [(n,c)][k]   (NT*Q rows)
+    static constexpr int TILE_X = 128 * M1 * E;    // X    [(n,a)][j]   (NT*P = 128 rows)
+    static constexpr int TILE_GT = 128 * Q * E;    // G^T  [(n,k)][c]
+    static constexpr int BUF = 128 * 128 * E;      // U1 | U2 (A), T2 | X^T (B)
+    static constexpr int OFF_C = 0;
+    static constexpr int OFF_BT = OFF_C + F_C;
+    static constexpr int OFF_BD = OFF_BT + F_BT;
+    static constexpr int OFF_G = OFF_BD + F_BD;
+    static constexpr int OFF_X = OFF_G + NT * Q * M2 * E;
     static constexpr int OFF_GT = OFF_X + TILE_X;
     static constexpr int OFF_A = OFF_GT + TILE_GT;
-    static constexpr int OFF_B = OFF_A + BUF_A;
-    static constexpr int OFF_BAR = OFF_B + BUF_B;
+    static constexpr int OFF_B = OFF_A + BUF;
+    static constexpr int OFF_BAR = OFF_B + BUF;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
     // TMEM columns
-    static constexpr int TM_TP = 0;                    // T'  : lanes (i,j), NT*Q columns (n,c)
-    static constexpr int TM_U = TM_TP + NT * Q;        // U   : lanes (n,k), R*P columns (i,a)
-    static constexpr int TM_DX = TM_U + R * P;         // dX  : lanes (n,j), P columns (a)
-    static constexpr int TM_DC = TM_DX + P;            // dC  : lanes (i,c), P columns (a)
-    static constexpr int TM_DB = TM_DC + P;            // dB  : lanes (i,k), M1 columns (j)
+    static constexpr int TM_UA = 0;              // Ua : lanes (i,a), 128 columns (n,k)
+    static constexpr int TM_UB = 128;            // Ub : lanes (n,k), 128 columns (i,a)
+    static constexpr int TM_T = 256;             // T  : lanes (n,a), 128 columns (i,k)
+    static constexpr int TM_DX = 384;            // dX : lanes (n,a), M1 columns (j)
+    static constexpr int TM_DC = TM_DX + M1;     // dC : lanes (i,a), Q columns (c)
+    static constexpr int TM_DB = TM_DC + Q;      // dB : lanes (i,k), M1 columns (j)
     static constexpr int TM_USED = TM_DB + M1;
-    static constexpr int TM_COLS = TM_USED <= 128 ? 128 : TM_USED <= 256 ? 256 : 512;
-    static constexpr uint32_t ID_TP = idesc_f32acc(128, NT * Q, BE<T>::fmt);
-    static constexpr uint32_t ID_U = idesc_f32acc(128, R * P, BE<T>::fmt);
-    static constexpr uint32_t ID_DX = idesc_f32acc(128, P, BE<T>::fmt);
-    static constexpr uint32_t ID_DC = idesc_f32acc(128, P, BE<T>::fmt);
-    static constexpr uint32_t ID_DB = idesc_f32acc(128, M1, BE<T>::fmt);
+    static constexpr int TM_COLS = 512;
+    static constexpr uint32_t ID_128 = idesc_f32acc(128, 128, BE<T>::fmt);
+    static constexpr uint32_t ID_M1 = idesc_f32acc(128, M1, BE<T>::fmt);
+    static constexpr uint32_t ID_Q = idesc_f32acc(128, Q, BE<T>::fmt);
 
-    static_assert(R * M1 == 128 && M1 == M2 && Q == M1, "needs r*m1 = 128 and m1 = m2 = q");
-    static_assert(NT * M1 == 128 && NT * M2 == 128, "tile rows");
-    static_assert(P % 32 == 0 && P <= 64 && R * P <= 256, "p: multiple of 32, r*p <= 256");
-    static_assert(NT * Q <= 256 && NT * Q % 32 == 0, "T' columns");
-    static_assert(M1 % 32 == 0 && Q % 32 == 0, "32-column TMEM loads");
-    static_assert(M1 * E % 32 == 0 && M1 * E <= 128, "an x row block of m1 must fit one swizzle row");
-    static_assert(Q * E % 32 == 0 && (Q * E <= 128 || Q * E % 128 == 0), "q bytes");
-    static_assert(P * E % 32 == 0 && (P * E <= 128 || P * E % 128 == 0), "p bytes");
-    static_assert(TM_USED <= 512, "TMEM budget");
+    static_assert(R * P == 128 && R * M2 == 128, "needs p = m2 = 128 / r");
+    static_assert(M2 % 32 == 0 && P % 32 == 0, "a 32-column TMEM chunk maps to one operand row");
+    static_assert(NT * Q <= 256 && (NT * Q) % 8 == 0, "G tile rows (TMA box) at most 256");
+    static_assert(M2 * E <= 128 && P * E <= 128 && M1 * E <= 128,
+                  "a block of m2 (p, m1) values must fit one 128-byte swizzle row");
+    static_assert(SWG == 32 || SWG == 64 || SWG == 128, "G tile swizzle");
+    static_assert(M1 % 32 == 0 && Q % 32 == 0 && M1 <= 64 && Q <= 64, "m1, q in {32, 64}");
+    static_assert((M1 * E) % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
+    static_assert((Q * E) % 32 == 0 && (Q * E <= 128 || Q * E % 128 == 0), "q bytes");
+    static_assert(TM_USED <= TM_COLS, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -129,7 +127,7 @@ __device__ __forceinline__ float bld(const void *p, size_t i) {
     else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
 }
 
-// (row, kbyte) of a K-major swizzled operand region: K split in chunks of sw bytes
+// (row, kbyte) of a K-major swizzled operand region: K in chunks of sw bytes
 // (chunk-major), rows in 8-row atoms of 8*sw bytes.
 __device__ __forceinline__ uint32_t koff(int row, int kbyte, int rows, int sw) {
     const int chunk = kbyte / sw, inner = kbyte % sw;
@@ -149,29 +147,42 @@ __device__ __forceinline__ void st16v(uint32_t addr, const float *v) {
     }
 }
 
-// one operand element (as stored: tf32-rounded fp32 or bf16)
+// TMEM (32 columns of this thread's lane) -> one operand row of a 128B-swizzled K-major
+// region: the 32 values go to K bytes [kbyte0, kbyte0 + 32*E) of row `row` (kbyte0
+// 16-byte aligned, the run stays inside one 128-byte K-chunk).
 template <typename T>
-__device__ __forceinline__ void st1(uint32_t addr, float v) {
-    if constexpr (BE<T>::tf32) {
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(f32_to_tf32(v)) : "memory");
-    } else {
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-        asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr),
-                     "h"(*reinterpret_cast<const unsigned short *>(&h))
-                     : "memory");
+__device__ __forceinline__ void tmem_row_to_smem(uint32_t taddr, uint32_t region, int rows,
+                                                 int row, int kbyte0) {
+    constexpr int VPC = 16 / BE<T>::bytes;
+    uint32_t r[32];
+    tmem_load32(taddr, r);
+    const uint32_t base = sw128_row(region, rows, kbyte0 >> 7, row);
+    const int slot0 = (kbyte0 & 127) >> 4, x = row & 7;
+#pragma unroll
+    for (int g = 0; g < 32 / VPC; ++g) {
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < VPC; ++t) v[t] = __uint_as_float(r[g * VPC + t]);
+        st16v<T>(base + (uint32_t)(((slot0 + g) ^ x) << 4), v);
     }
 }
 
+// Transpose of 8 source rows x 16 bytes (VPC elements) held as in[8][4] words into VPC
+// output rows of 8 elements each: out row e = (in[0][e], ..., in[7][e]).  The
+// elements are already in operand format (raw fp32 is rounded to tf32 here).
 template <typename T>
-__device__ __forceinline__ float ld1(uint32_t addr) {
+__device__ __forceinline__ void store_transposed(const uint32_t (&in)[8][4], int e,
+                                                 uint32_t addr_lo, uint32_t addr_hi) {
     if constexpr (BE<T>::tf32) {
-        float v;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-        return v;
+        st_shared_v4(addr_lo, f32_to_tf32(__uint_as_float(in[0][e])), f32_to_tf32(__uint_as_float(in[1][e])),
+                     f32_to_tf32(__uint_as_float(in[2][e])), f32_to_tf32(__uint_as_float(in[3][e])));
+        st_shared_v4(addr_hi, f32_to_tf32(__uint_as_float(in[4][e])), f32_to_tf32(__uint_as_float(in[5][e])),
+                     f32_to_tf32(__uint_as_float(in[6][e])), f32_to_tf32(__uint_as_float(in[7][e])));
     } else {
-        unsigned short h;
-        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(h) : "r"(addr) : "memory");
-        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(&h));
+        const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
+        const int w = e >> 1;
+        st_shared_v4(addr_lo, __byte_perm(in[0][w], in[1][w], sel), __byte_perm(in[2][w], in[3][w], sel),
+                     __byte_perm(in[4][w], in[5][w], sel), __byte_perm(in[6][w], in[7][w], sel));
     }
 }
 
@@ -188,21 +199,24 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
-    const uint32_t sBP = sb + Cfg::OFF_BP, sCS = sb + Cfg::OFF_CS, sCDX = sb + Cfg::OFF_CDX;
+    const uint32_t sC = sb + Cfg::OFF_C, sBT = sb + Cfg::OFF_BT, sBD = sb + Cfg::OFF_BD;
     const uint32_t sG = sb + Cfg::OFF_G, sX = sb + Cfg::OFF_X, sGT = sb + Cfg::OFF_GT;
     const uint32_t sA = sb + Cfg::OFF_A, sBb = sb + Cfg::OFF_B;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     enum {
-        G_FULL, X_FULL,       // TMA landed
-        G_FREE, X_FREE,       // G / X tile may be overwritten
-        GT_FULL, GT_FREE,     // G^T written / consumed by the U MMA
-        TP_FULL,              // T' accumulator ready (read out before TT_FULL)
-        U_FULL,               // U accumulator ready (read out before UX_FULL)
-        TT_FULL,              // T'1 and T'2 written
-        AB_FREE1,             // dX + dC MMAs done: buffers A, B and the X tile (for dC) free
-        DX_FULL, DX_FREE,     // dX accumulator ready / read out
-        UX_FULL,              // U2 and X^T written
-        AB_FREE2,             // dB MMAs done: buffers A and B free
+        G_FULL, X_FULL,   // TMA landed
+        G_FREE,           // dC done with G and G^T/dbias read it (transposer arrives after X^T)
+        X_FREE,           // T done with X and X^T written
+        GT_FULL,          // G^T written
+        UT_FULL,          // Ua, Ub, T accumulators ready; G^T consumed
+        E1A_DONE,         // U1 written (buffer A)
+        E1B_DONE,         // T2 written (buffer B)
+        DX_FULL,          // dX accumulator ready; U1 consumed (buffer A free)
+        DX_FREE,          // dX accumulator read out
+        DC_DONE,          // dC MMAs done: T2 consumed (buffer B free), G consumed
+        U2_DONE,          // U2 written; Ua, Ub, T accumulators fully read out
+        XT_DONE,          // X^T written
+        DB_DONE,          // dB MMAs done: buffers A and B free
         DRAIN,
         NBARS
     };
@@ -215,18 +229,18 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
     if (threadIdx.x == 0) {
         mbar_init(bar(G_FULL), 1);
         mbar_init(bar(X_FULL), 1);
-        mbar_init(bar(G_FREE), 1 + 128);  // T' MMA commit + transpose warps
-        mbar_init(bar(X_FREE), 1 + 128);  // dC MMA commit + transpose warps (X^T written)
-        mbar_init(bar(GT_FULL), 128);
-        mbar_init(bar(GT_FREE), 1);
-        mbar_init(bar(TP_FULL), 1);
-        mbar_init(bar(U_FULL), 1);
-        mbar_init(bar(TT_FULL), 256);
-        mbar_init(bar(AB_FREE1), 1);
+        mbar_init(bar(G_FREE), 1 + 4);   // dC commit + B-chain warps
+        mbar_init(bar(X_FREE), 1 + 4);
+        mbar_init(bar(GT_FULL), 4);
+        mbar_init(bar(UT_FULL), 1);
+        mbar_init(bar(E1A_DONE), 8);     // A-chain warps
+        mbar_init(bar(E1B_DONE), 4);
         mbar_init(bar(DX_FULL), 1);
-        mbar_init(bar(DX_FREE), 128);
-        mbar_init(bar(UX_FULL), 256 + 128);
-        mbar_init(bar(AB_FREE2), 1);
+        mbar_init(bar(DX_FREE), 4);
+        mbar_init(bar(DC_DONE), 1);
+        mbar_init(bar(U2_DONE), 8);
+        mbar_init(bar(XT_DONE), 4);
+        mbar_init(bar(DB_DONE), 1);
         mbar_init(bar(DRAIN), 1);
         *ab.flag = 0;
         mbar_init_fence();
@@ -234,23 +248,31 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
         prefetch_tmap(&tmap_x);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
-    // factors: B'[(i,j)][k] = B_i[j][k]; C_stack[(i,a)][c] = C_i[a][c]; Cdx[a][(i,c)] = C_i[a][c]
-    for (int e = threadIdx.x; e < 128 * (M2 / VPC); e += blockDim.x) {
-        const int row = e / (M2 / VPC), k0 = (e % (M2 / VPC)) * VPC;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) v[t] = bld<T>(args.B, (size_t)row * M2 + k0 + t);
-        st16v<T>(sBP + koff(row, k0 * E, 128, Cfg::SWK), v);
-    }
-    for (int e = threadIdx.x; e < R * P * (Q / VPC); e += blockDim.x) {
-        const int row = e / (Q / VPC), c0 = (e % (Q / VPC)) * VPC;  // row = (i,a)
+    // factors: C[(i,a)][c] = S[a][c] A_i[a][c]; Bt[(i,k)][j] = B_i[j][k]; Bdx[j][(i,k)] = B_i[j][k]
+    for (int e = threadIdx.x; e < 128 * (Q / VPC); e += blockDim.x) {
+        const int row = e / (Q / VPC), c0 = (e % (Q / VPC)) * VPC;
         const int i = row / P, a = row % P;
         float v[8];
 #pragma unroll
         for (int t = 0; t < VPC; ++t)
             v[t] = bld<T>(args.S, (size_t)a * Q + c0 + t) * bld<T>(args.A, ((size_t)i * P + a) * Q + c0 + t);
-        st16v<T>(sCS + koff(row, c0 * E, R * P, Cfg::SWC), v);
-        st16v<T>(sCDX + koff(a, (i * Q + c0) * E, P, Cfg::SWQ), v);
+        st16v<T>(sC + koff(row, c0 * E, 128, Cfg::SWC), v);
+    }
+    for (int e = threadIdx.x; e < 128 * (M1 / VPC); e += blockDim.x) {
+        const int row = e / (M1 / VPC), j0 = (e % (M1 / VPC)) * VPC;
+        const int i = row / M2, k = row % M2;
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < VPC; ++t) v[t] = bld<T>(args.B, ((size_t)i * M1 + j0 + t) * M2 + k);
+        st16v<T>(sBT + koff(row, j0 * E, 128, Cfg::SWJ), v);
+    }
+    for (int e = threadIdx.x; e < M1 * (128 / VPC); e += blockDim.x) {
+        const int j = e / (128 / VPC), ik0 = (e % (128 / VPC)) * VPC;
+        const int i = ik0 / M2, k0 = ik0 % M2;
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < VPC; ++t) v[t] = bld<T>(args.B, ((size_t)i * M1 + j) * M2 + k0 + t);
+        st16v<T>(sBD + koff(j, ik0 * E, M1, Cfg::SW128), v);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -270,15 +292,11 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
                 const uint32_t ph = u & 1;
                 const int tile = t0 + u;
                 if (!mbar_wait(bar(G_FREE), ph ^ 1, ab)) break;
-                mbar_arrive_expect_tx(bar(G_FULL), Cfg::TILE_G);
-                for (int kc = 0; kc < M2 * E / Cfg::SWK; ++kc)
-                    tma_load_2d(sG + kc * NT * Q * Cfg::SWK, &tmap_g, kc * (Cfg::SWK / E),
-                                tile * NT * Q, bar(G_FULL));
+                mbar_arrive_expect_tx(bar(G_FULL), NT * Q * M2 * E);
+                tma_load_2d(sG, &tmap_g, 0, tile * NT * Q, bar(G_FULL));
                 if (!mbar_wait(bar(X_FREE), ph ^ 1, ab)) break;
                 mbar_arrive_expect_tx(bar(X_FULL), Cfg::TILE_X);
-                for (int kc = 0; kc < M1 * E / Cfg::SWJ; ++kc)
-                    tma_load_2d(sX + kc * NT * P * Cfg::SWJ, &tmap_x, kc * (Cfg::SWJ / E),
-                                tile * NT * P, bar(X_FULL));
+                tma_load_2d(sX, &tmap_x, 0, tile * NT * P, bar(X_FULL));
                 issued = u + 1;
             }
             if (issued > 0) {
@@ -289,93 +307,79 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-                mma_ss<BE<T>::tf32>(d, a, b, id, acc);
+            auto mma = [&](uint32_t d, uint32_t a, int swa, uint32_t b, int swb, uint32_t id, uint32_t acc) {
+                mma_ss<BE<T>::tf32>(d, sdesc_kmajor(a, swa), sdesc_kmajor(b, swb), id, acc);
             };
-            // T'(u): D[(i,j),(n,c)] = B'[(i,j)][k] . G[(n,c)][k]
-            auto issue_tp = [&]() {
-                for (int kb = 0; kb < M2 * E; kb += 32) {
-                    const int ch = kb / Cfg::SWK, in = kb % Cfg::SWK;
-                    mma(tmem + Cfg::TM_TP, sdesc_kmajor(sBP + ch * 128 * Cfg::SWK + in, Cfg::SWK),
-                        sdesc_kmajor(sG + ch * NT * Q * Cfg::SWK + in, Cfg::SWK), Cfg::ID_TP, kb > 0);
-                }
-            };
-            // U(u): D[(n,k),(i,a)] = G^T[(n,k)][c] . C_stack[(i,a)][c]
-            auto issue_u = [&]() {
+            // Ua, Ub and T of the current tile
+            auto issue_ut = [&]() {
                 for (int kb = 0; kb < Q * E; kb += 32) {
                     const int ch = kb / Cfg::SWC, in = kb % Cfg::SWC;
-                    mma(tmem + Cfg::TM_U, sdesc_kmajor(sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC),
-                        sdesc_kmajor(sCS + ch * R * P * Cfg::SWC + in, Cfg::SWC), Cfg::ID_U, kb > 0);
+                    mma(tmem + Cfg::TM_UA, sC + ch * 128 * Cfg::SWC + in, Cfg::SWC,
+                        sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC, Cfg::ID_128, kb > 0);
+                    mma(tmem + Cfg::TM_UB, sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC,
+                        sC + ch * 128 * Cfg::SWC + in, Cfg::SWC, Cfg::ID_128, kb > 0);
                 }
+                for (int kb = 0; kb < M1 * E; kb += 32) {
+                    const int ch = kb / Cfg::SWJ, in = kb % Cfg::SWJ;
+                    mma(tmem + Cfg::TM_T, sX + ch * 128 * Cfg::SWJ + in, Cfg::SWJ,
+                        sBT + ch * 128 * Cfg::SWJ + in, Cfg::SWJ, Cfg::ID_128, kb > 0);
+                }
+                mma_commit(bar(UT_FULL));
+                mma_commit(bar(X_FREE));
             };
             bool ok = true;
-            // prologue: T'(0) and U(0)
             if (nt > 0) {
-                ok = mbar_wait(bar(G_FULL), 0, ab) && mbar_wait(bar(GT_FULL), 0, ab);
+                ok = mbar_wait(bar(X_FULL), 0, ab) && mbar_wait(bar(GT_FULL), 0, ab);
                 if (ok) {
                     tc_fence_after();
-                    issue_tp();
-                    mma_commit(bar(TP_FULL));
-                    mma_commit(bar(G_FREE));
-                    issue_u();
-                    mma_commit(bar(U_FULL));
-                    mma_commit(bar(GT_FREE));
+                    issue_ut();
                 }
             }
             for (int u = 0; u < nt && ok; ++u) {
                 const uint32_t ph = u & 1;
-                // dX and dC of tile u
-                if (!mbar_wait(bar(TT_FULL), ph, ab) || !mbar_wait(bar(X_FULL), ph, ab) ||
-                    !mbar_wait(bar(DX_FREE), ph ^ 1, ab)) { ok = false; break; }
+                // dX(u) = U1 . Bdx^T  (K = (i,k)); dC(u) += T2 . G^T (K = (n,k))
+                if (!mbar_wait(bar(E1A_DONE), ph, ab) || !mbar_wait(bar(DX_FREE), ph ^ 1, ab)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < R * Q * E; kb += 32) {  // K = (i,c)
-                    const int ch = kb / Cfg::SWQ, in = kb % Cfg::SWQ;
-                    mma(tmem + Cfg::TM_DX, sdesc_kmajor(sA + ch * 128 * Cfg::SWQ + in, Cfg::SWQ),
-                        sdesc_kmajor(sCDX + ch * P * Cfg::SWQ + in, Cfg::SWQ), Cfg::ID_DX, kb > 0);
+                for (int kb = 0; kb < 128 * E; kb += 32) {
+                    const int ch = kb / 128, in = kb % 128;
+                    mma(tmem + Cfg::TM_DX, sA + ch * 128 * 128 + in, 128, sBD + ch * M1 * 128 + in, 128,
+                        Cfg::ID_M1, kb > 0);
                 }
                 mma_commit(bar(DX_FULL));
-                for (int kb = 0; kb < NT * M1 * E; kb += 32) {  // K = (n,j)
-                    const int ch = kb / Cfg::SWJ, in = kb % Cfg::SWJ;
-                    mma(tmem + Cfg::TM_DC, sdesc_kmajor(sBb + ch * 128 * Cfg::SWJ + in, Cfg::SWJ),
-                        sdesc_kmajor(sX + ch * P * Cfg::SWJ + in, Cfg::SWJ), Cfg::ID_DC,
-                        (u > 0 || kb > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(AB_FREE1));
-                mma_commit(bar(X_FREE));
-                // T' of tile u+1 (its accumulator was read out before TT_FULL(u))
-                if (u + 1 < nt) {
-                    if (!mbar_wait(bar(G_FULL), ph ^ 1, ab)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_tp();
-                    mma_commit(bar(TP_FULL));
-                    mma_commit(bar(G_FREE));
-                }
-                // dB of tile u
-                if (!mbar_wait(bar(UX_FULL), ph, ab)) { ok = false; break; }
+                if (!mbar_wait(bar(E1B_DONE), ph, ab)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < NT * P * E; kb += 32) {  // K = (n,a)
-                    const int ch = kb / Cfg::SWA, in = kb % Cfg::SWA;
-                    mma(tmem + Cfg::TM_DB, sdesc_kmajor(sA + ch * 128 * Cfg::SWA + in, Cfg::SWA),
-                        sdesc_kmajor(sBb + ch * M1 * Cfg::SWA + in, Cfg::SWA), Cfg::ID_DB,
-                        (u > 0 || kb > 0) ? 1u : 0u);
+                for (int kb = 0; kb < 128 * E; kb += 32) {
+                    const int ch = kb / 128, in = kb % 128;                // T2: 128-byte chunks
+                    const int chg = kb / Cfg::SWG, ing = kb % Cfg::SWG;    // G: one chunk per n
+                    mma(tmem + Cfg::TM_DC, sBb + ch * 128 * 128 + in, 128,
+                        sG + chg * Q * Cfg::SWG + ing, Cfg::SWG, Cfg::ID_Q, (u > 0 || kb > 0) ? 1u : 0u);
                 }
-                mma_commit(bar(AB_FREE2));
-                // U of tile u+1 (its accumulator was read out before UX_FULL(u))
+                mma_commit(bar(DC_DONE));
+                mma_commit(bar(G_FREE));
+                // dB(u) += U2 . X^T^T (K = (n,a)) once U2 and X^T are written
+                if (!mbar_wait(bar(U2_DONE), ph, ab) || !mbar_wait(bar(XT_DONE), ph, ab)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < 128 * E; kb += 32) {
+                    const int ch = kb / 128, in = kb % 128;
+                    mma(tmem + Cfg::TM_DB, sA + ch * 128 * 128 + in, 128, sBb + ch * M1 * 128 + in, 128,
+                        Cfg::ID_M1, (u > 0 || kb > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(DB_DONE));
+                // Ua, Ub, T of tile u+1 (their accumulators were read out before U2_DONE(u))
                 if (u + 1 < nt) {
-                    if (!mbar_wait(bar(GT_FULL), ph ^ 1, ab)) { ok = false; break; }
+                    if (!mbar_wait(bar(X_FULL), ph ^ 1, ab) || !mbar_wait(bar(GT_FULL), ph ^ 1, ab)) { ok = false; break; }
                     tc_fence_after();
-                    issue_u();
-                    mma_commit(bar(U_FULL));
-                    mma_commit(bar(GT_FREE));
+                    issue_ut();
                 }
             }
             mma_commit(bar(DRAIN));
             mbar_wait_drain(bar(DRAIN), 0);
         }
     } else if (warp < 6) {
-        // ---------------- transposes, dbias, dX epilogue (128 threads) ----------------
-        const int tid = threadIdx.x - 64;         // 0..127
+        // ---------------- B chain (128 threads) ----------------
+        const int tid = threadIdx.x - 64;
         const int quad = warp & 3;
+        const int L = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float dbias[Q * M2 / 128];
 #pragma unroll
@@ -383,165 +387,188 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
         for (int u = 0; u < nt; ++u) {
             const uint32_t ph = u & 1;
             const int64_t row0 = (int64_t)(t0 + u) * NT;
-            // G^T(u) and the dbias partial, once G(u) has landed and G^T(u-1) is consumed
-            if (!mbar_wait(bar(G_FULL), ph, ab) || !mbar_wait(bar(GT_FREE), ph ^ 1, ab)) break;
-            {
-                // thread (n,k) for two n per pass: reads G[(n,c)][k] for all c, writes row (n,k)
-                for (int rr = tid; rr < NT * M2; rr += 128) {
-                    const int n = rr / M2, k = rr % M2;
-                    for (int c0 = 0; c0 < Q; c0 += VPC) {
-                        float v[8];
+            // G^T(u) [(n,k)][c] from G(u) [(n,c)][k] (8-row register blocks), dbias partial.
+            // G^T(u-1) was consumed by the U MMAs of tile u-1 (UT_FULL(u-1) preceded E1B(u-1)).
+            if (!mbar_wait(bar(G_FULL), ph, ab)) break;
+            for (int blk = tid; blk < NT * (Q / 8) * (M2 / VPC); blk += 128) {
+                const int kb = blk % (M2 / VPC), cb = (blk / (M2 / VPC)) % (Q / 8), n = blk / ((M2 / VPC) * (Q / 8));
+                uint32_t in[8][4];
 #pragma unroll
-                        for (int t = 0; t < VPC; ++t)
-                            v[t] = ld1<T>(sG + koff(n * Q + c0 + t, k * E, NT * Q, Cfg::SWK));
-                        st16v<T>(sGT + koff(rr, c0 * E, NT * M2, Cfg::SWC), v);
-                    }
-                }
+                for (int t = 0; t < 8; ++t)
+                    ld_shared_v4(sG + koff(n * Q + cb * 8 + t, kb * 16, NT * Q, Cfg::SWG), in[t]);
 #pragma unroll
-                for (int e = 0; e < Q * M2 / 128; ++e) {
-                    const int o = tid + 128 * e, c = o / M2, k = o % M2;
-                    float s = 0.f;
-                    for (int n = 0; n < NT; ++n)
-                        if (row0 + n < args.N) s += ld1<T>(sG + koff(n * Q + c, k * E, NT * Q, Cfg::SWK));
-                    dbias[e] += s;
+                for (int e = 0; e < VPC; ++e) {
+                    const int row = n * M2 + kb * VPC + e;
+                    const uint32_t lo = sGT + koff(row, cb * 8 * E, 128, Cfg::SWC);
+                    store_transposed<T>(in, e, lo, lo ^ 16u);
                 }
             }
+#pragma unroll
+            for (int e = 0; e < Q * M2 / 128; ++e) {
+                const int o = tid + 128 * e, c = o / M2, k = o % M2;
+                float sacc = 0.f;
+                for (int n = 0; n < NT; ++n) {
+                    if (row0 + n < args.N) {
+                        const uint32_t a = sG + koff(n * Q + c, k * E, NT * Q, Cfg::SWG);
+                        if constexpr (BE<T>::tf32) {
+                            float v;
+                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+                            sacc += v;
+                        } else {
+                            unsigned short h;
+                            asm volatile("ld.shared.b16 %0, [%1];" : "=h"(h) : "r"(a) : "memory");
+                            sacc += __bfloat162float(*reinterpret_cast<__nv_bfloat16 *>(&h));
+                        }
+                    }
+                }
+                dbias[e] += sacc;
+            }
             fence_proxy_async();
-            mbar_arrive(bar(GT_FULL));
-            mbar_arrive(bar(G_FREE));
-            // dX(u): D[(n,j), a] -> dx[row n][a*m1 + j]
+            mbar_arrive_warp(bar(GT_FULL));
+            // T2(u) [(i,a)][(n,k)] <- T accumulator (lanes (n,a), columns (i,k)) into buffer B,
+            // once dB(u-1) has consumed X^T(u-1)
+            if (!mbar_wait(bar(UT_FULL), ph, ab) || !mbar_wait(bar(DB_DONE), ph ^ 1, ab)) break;
+            tc_fence_after();
+            {
+                const int n = L / P, a = L % P;
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {   // columns (i,k): i = c0 / M2
+                    const int i = c0 / M2, k0 = c0 % M2;
+                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_T + c0, sBb, 128, i * P + a,
+                                        (n * M2 + k0) * E);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async();
+            mbar_arrive_warp(bar(E1B_DONE));
+            // dX(u): lanes (n,a), columns j -> dx[row0 + n][a*m1 + j] (16-byte stores)
             if (!mbar_wait(bar(DX_FULL), ph, ab)) break;
             tc_fence_after();
             {
-                const int L = quad * 32 + lane, n = L / M1, j = L % M1;
+                const int n = L / P, a = L % P;
                 const int64_t row = row0 + n;
 #pragma unroll
-                for (int a0 = 0; a0 < P; a0 += 32) {
+                for (int j0 = 0; j0 < M1; j0 += 32) {
                     uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_DX + a0, r);
-                    if (a0 + 32 >= P) {
+                    tmem_load32(tmem + lane_addr + Cfg::TM_DX + j0, r);
+                    if (j0 + 32 >= M1) {
                         tc_fence_before();
-                        mbar_arrive(bar(DX_FREE));
+                        mbar_arrive_warp(bar(DX_FREE));
                     }
                     if (args.dX && row < args.N) {
+                        if constexpr (BE<T>::tf32) {
+                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(args.dX) +
+                                                                     (size_t)row * (P * M1) + (size_t)a * M1 + j0);
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) {
-                            const size_t o = (size_t)row * (P * M1) + (size_t)(a0 + t) * M1 + j;
-                            if constexpr (BE<T>::tf32) static_cast<float *>(args.dX)[o] = __uint_as_float(r[t]);
-                            else static_cast<__nv_bfloat16 *>(args.dX)[o] = __float2bfloat16_rn(__uint_as_float(r[t]));
+                            for (int q4 = 0; q4 < 8; ++q4)
+                                dst[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
+                                                      __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(args.dX) +
+                                                                   (size_t)row * (P * M1) + (size_t)a * M1 + j0);
+#pragma unroll
+                            for (int q8 = 0; q8 < 4; ++q8)
+                                dst[q8] = make_uint4(
+                                    pack_bf16x2(__uint_as_float(r[8 * q8]), __uint_as_float(r[8 * q8 + 1])),
+                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 2]), __uint_as_float(r[8 * q8 + 3])),
+                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 4]), __uint_as_float(r[8 * q8 + 5])),
+                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 6]), __uint_as_float(r[8 * q8 + 7])));
                         }
                     }
                 }
             }
-            // X^T(u) into buffer B once dC(u) has consumed T'2 (buffer B) and X(u) has landed
-            if (!mbar_wait(bar(AB_FREE1), ph, ab)) break;
-            for (int rr = tid; rr < NT * M1; rr += 128) {
-                const int n = rr / M1, j = rr % M1;  // reads X[(n,a)][j] for all a
-                for (int a0 = 0; a0 < P; a0 += VPC) {
-                    float v[8];
+            // X^T(u) [j][(n,a)] into buffer B once dC(u) has consumed T2(u)
+            if (!mbar_wait(bar(DC_DONE), ph, ab)) break;
+            for (int blk = tid; blk < NT * (P / 8) * (M1 / VPC); blk += 128) {
+                const int jb = blk % (M1 / VPC), ab8 = (blk / (M1 / VPC)) % (P / 8), n = blk / ((M1 / VPC) * (P / 8));
+                uint32_t in[8][4];
 #pragma unroll
-                    for (int t = 0; t < VPC; ++t)
-                        v[t] = ld1<T>(sX + koff(n * P + a0 + t, j * E, NT * P, Cfg::SWJ));
-                    st16v<T>(sBb + koff(j, (n * P + a0) * E, M1, Cfg::SWA), v);
+                for (int t = 0; t < 8; ++t)
+                    ld_shared_v4(sX + koff(n * P + ab8 * 8 + t, jb * 16, 128, Cfg::SWJ), in[t]);
+#pragma unroll
+                for (int e = 0; e < VPC; ++e) {
+                    const int j = jb * VPC + e;
+                    const uint32_t lo = sBb + koff(j, (n * P + ab8 * 8) * E, M1, 128);
+                    store_transposed<T>(in, e, lo, lo ^ 16u);
                 }
             }
             fence_proxy_async();
-            mbar_arrive(bar(UX_FULL));
-            mbar_arrive(bar(X_FREE));
+            mbar_arrive_warp(bar(XT_DONE));
+            mbar_arrive_warp(bar(X_FREE));
+            mbar_arrive_warp(bar(G_FREE));
         }
-        // dbias partial of this row range
         const size_t off = (size_t)R * P * Q + (size_t)R * M1 * M2;
         float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
 #pragma unroll
         for (int e = 0; e < Q * M2 / 128; ++e) part[off + tid + 128 * e] = dbias[e];
     } else {
-        // ---------------- T' and U epilogues (256 threads) ----------------
+        // ---------------- A chain (256 threads) ----------------
         const int half = (warp - 6) / 4;
         const int quad = warp & 3;
         const int L = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         for (int u = 0; u < nt; ++u) {
             const uint32_t ph = u & 1;
-            // T'(u): lanes (i,j), columns (n,c) -> T'1 [(n,j)][(i,c)] (buffer A) and
-            // T'2 [(i,c)][(n,j)] (buffer B), once dB(u-1) has released both buffers
-            if (!mbar_wait(bar(TP_FULL), ph, ab) || !mbar_wait(bar(AB_FREE2), ph ^ 1, ab)) break;
+            // U1(u) [(n,a)][(i,k)] <- Ua (lanes (i,a), columns (n,k)) into buffer A, once
+            // dB(u-1) has consumed U2(u-1)
+            if (!mbar_wait(bar(UT_FULL), ph, ab) || !mbar_wait(bar(DB_DONE), ph ^ 1, ab)) break;
             tc_fence_after();
             {
-                const int i = L / M1, j = L % M1;
-                constexpr int HC = NT * Q / 2;
-                for (int c0 = half * HC; c0 < (half + 1) * HC; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_TP + c0, r);
+                const int i = L / P, a = L % P;
 #pragma unroll
-                    for (int g = 0; g < 32 / VPC; ++g) {
-                        const int col = c0 + g * VPC, n = col / Q, c = col % Q;
-                        float v[8];
-#pragma unroll
-                        for (int t = 0; t < VPC; ++t) v[t] = __uint_as_float(r[g * VPC + t]);
-                        st16v<T>(sA + koff(n * M1 + j, (i * Q + c) * E, 128, Cfg::SWQ), v);
-#pragma unroll
-                        for (int t = 0; t < VPC; ++t)
-                            st1<T>(sBb + koff(i * Q + c + t, (n * M1 + j) * E, 128, Cfg::SWJ), v[t]);
-                    }
+                for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {   // columns (n,k)
+                    const int n = c0 / M2, k0 = c0 % M2;
+                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_UA + c0, sA, 128, n * P + a,
+                                        (i * M2 + k0) * E);
                 }
             }
             tc_fence_before();
             fence_proxy_async();
-            mbar_arrive(bar(TT_FULL));
-            // U(u): lanes (n,k), columns (i,a) -> U2 [(i,k)][(n,a)] (buffer A), once dX(u)
-            // has consumed T'1
-            if (!mbar_wait(bar(U_FULL), ph, ab) || !mbar_wait(bar(AB_FREE1), ph, ab)) break;
+            mbar_arrive_warp(bar(E1A_DONE));
+            // U2(u) [(i,k)][(n,a)] <- Ub (lanes (n,k), columns (i,a)) into buffer A, once
+            // dX(u) has consumed U1(u)
+            if (!mbar_wait(bar(DX_FULL), ph, ab)) break;
             tc_fence_after();
             {
                 const int n = L / M2, k = L % M2;
-                constexpr int HC = R * P / 2;
-                for (int c0 = half * HC; c0 < (half + 1) * HC; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_U + c0, r);
 #pragma unroll
-                    for (int g = 0; g < 32 / VPC; ++g) {
-                        const int col = c0 + g * VPC, i = col / P, a = col % P;
-                        float v[8];
-#pragma unroll
-                        for (int t = 0; t < VPC; ++t) v[t] = __uint_as_float(r[g * VPC + t]);
-                        st16v<T>(sA + koff(i * M2 + k, (n * P + a) * E, 128, Cfg::SWA), v);
-                    }
+                for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {   // columns (i,a)
+                    const int i = c0 / P, a0 = c0 % P;
+                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_UB + c0, sA, 128, i * M2 + k,
+                                        (n * P + a0) * E);
                 }
             }
             tc_fence_before();
             fence_proxy_async();
-            mbar_arrive(bar(UX_FULL));
+            mbar_arrive_warp(bar(U2_DONE));
         }
-        // dC and dB partials of this row range, once the last dB MMAs are done
-        if (nt > 0 && mbar_wait(bar(AB_FREE2), (nt - 1) & 1, ab)) {
+        // dC and dB partials of this row range, after the last dB MMAs
+        float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
+        if (nt > 0 && mbar_wait(bar(DB_DONE), (nt - 1) & 1, ab)) {
             tc_fence_after();
-            float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
-            const int cols = half == 0 ? 0 : 16;   // each half writes 16 of the 32 columns
-            {   // dC: lanes (i,c), columns a -> dC_i[a][c] at i*p*q + a*q + c
-                const int i = L / Q, c = L % Q;
-                for (int a0 = 0; a0 < P; a0 += 32) {
+            if (half == 0) {   // dC: lanes (i,a), columns c -> dC_i[a][c] (16-byte stores)
+                const int i = L / P, a = L % P;
+                for (int c0 = 0; c0 < Q; c0 += 32) {
                     uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_DC + a0, r);
+                    tmem_load32(tmem + lane_addr + Cfg::TM_DC + c0, r);
+                    float4 *dst = reinterpret_cast<float4 *>(part + (size_t)i * P * Q + (size_t)a * Q + c0);
 #pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if ((t >= cols) && (t < cols + 16))
-                            part[(size_t)i * P * Q + (size_t)(a0 + t) * Q + c] = __uint_as_float(r[t]);
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        dst[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
+                                              __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
                 }
-            }
-            {   // dB: lanes (i,k), columns j -> dB_i[j][k] at r*p*q + i*m1*m2 + j*m2 + k
+            } else {           // dB: lanes (i,k), columns j -> dB_i[j][k]
                 const int i = L / M2, k = L % M2;
                 for (int j0 = 0; j0 < M1; j0 += 32) {
                     uint32_t r[32];
                     tmem_load32(tmem + lane_addr + Cfg::TM_DB + j0, r);
 #pragma unroll
                     for (int t = 0; t < 32; ++t)
-                        if ((t >= cols) && (t < cols + 16))
-                            part[(size_t)R * P * Q + (size_t)i * M1 * M2 + (size_t)(j0 + t) * M2 + k] =
-                                __uint_as_float(r[t]);
+                        part[(size_t)R * P * Q + (size_t)i * M1 * M2 + (size_t)(j0 + t) * M2 + k] =
+                            __uint_as_float(r[t]);
                 }
             }
         } else if (nt == 0) {
-            float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
             for (int e = threadIdx.x - 192; e < R * P * Q + R * M1 * M2; e += 256) part[e] = 0.f;
         }
     }
@@ -560,15 +587,19 @@ cudaError_t launch_bwd(const void *x, const void *S, const void *A, const void *
     using T = typename Cfg::T;
     const bool bf16 = !BE<T>::tf32;
     CUtensorMap tg, tx;
-    cudaError_t e = make_tmap_2d(&tg, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2,
-                                 Cfg::SWK / Cfg::E, Cfg::NT * Cfg::Q, Cfg::SWK);
+    launch_step() = "tensor map of dY";
+    cudaError_t e = make_tmap_2d(&tg, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2,
+                                 Cfg::NT * Cfg::Q, Cfg::M2 * Cfg::E);
     if (e != cudaSuccess) return e;
+    launch_step() = "tensor map of x";
     e = make_tmap_2d(&tx, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::SWJ / Cfg::E,
                      Cfg::NT * Cfg::P, Cfg::SWJ);
     if (e != cudaSuccess) return e;
+    launch_step() = "shared-memory attribute";
     e = cudaFuncSetAttribute(kron_bwd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
     if (e != cudaSuccess) return e;
+    launch_step() = "kernel launch";
     BwdTcArgs a;
     a.S = S; a.A = A; a.B = B; a.dX = dX; a.ws = ws;
     a.ws_stride = partial_stride(s);
@@ -576,8 +607,14 @@ cudaError_t launch_bwd(const void *x, const void *S, const void *A, const void *
     a.num_tiles = (int)((s.N + Cfg::NT - 1) / Cfg::NT);
     a.tiles_per_part = (a.num_tiles + parts - 1) / parts;
     a.device_error = device_error_ptr();
-    kron_bwd_tc_kernel<Cfg><<<parts, 448, Cfg::SMEM, st>>>(tg, tx, a);
-    return cudaGetLastError();
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)parts);
+        cfg.blockDim = dim3(448);
+        cfg.dynamicSmemBytes = Cfg::SMEM;
+        cfg.stream = st;
+        return cudaLaunchKernelEx(&cfg, kron_bwd_tc_kernel<Cfg>, tg, tx, a);
+    }
 }
 
 using BwdFn = cudaError_t (*)(const void *, const void *, const void *, const void *,
@@ -604,7 +641,7 @@ BwdFn find_bwd(const Shape &s, bool bf16) {
 
 bool tc_backward_supported(const Shape &s, bool bf16) { return tc::find_bwd(s, bf16) != nullptr; }
 
-int tc_backward_tile_rows(const Shape &s) { return 128 / s.m1; }
+int tc_backward_tile_rows(const Shape &s) { return s.r; }
 
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,

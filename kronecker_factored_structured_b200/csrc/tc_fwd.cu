@@ -93,6 +93,8 @@ struct FwdCfg {
     static_assert(M1 * E % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
     static_assert(K2B % 32 == 0 && (K2B <= 128 || K2B % 128 == 0), "r*p bytes");
     static_assert((P * E) % 16 == 0, "p*elt must be a multiple of 16 bytes");
+    static_assert(P % 32 == 0 && (32 * E) <= SW2 && SW2 == 128,
+                  "a 32-column TMEM chunk maps to one 128B-swizzled row of T");
     static_assert(TM_COLS_USED <= 512, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -166,13 +168,13 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         }
         for (int b = 0; b < D1S; ++b) {
             mbar_init(bar(B_D1FULL + b), 1);
-            mbar_init(bar(B_D1EMPTY + b), 256);
+            mbar_init(bar(B_D1EMPTY + b), 8);   // epilogue-1 warps
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(B_TFULL + b), 256);
+            mbar_init(bar(B_TFULL + b), 8);
             mbar_init(bar(B_TEMPTY + b), 1);
             mbar_init(bar(B_D2FULL + b), 1);
-            mbar_init(bar(B_D2EMPTY + b), 128);
+            mbar_init(bar(B_D2EMPTY + b), 4);    // epilogue-2 warps
             mbar_init(bar(B_DRAIN + b), 1);
         }
         *abort_flag.flag = 0;
@@ -305,20 +307,24 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
                 tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1 + c0, r);
                 if (c0 + 32 >= (half + 1) * HC) {  // this thread's columns of the slot are read
                     tc_fence_before();
-                    mbar_arrive(bar(B_D1EMPTY + d1));
+                    mbar_arrive_warp(bar(B_D1EMPTY + d1));
                 }
+                // 32 columns (n, a0..a0+31) -> row (n,k) of T, K bytes (i*p + a0)*E onward
+                const int n = c0 / P, a0 = c0 % P, row = n * M2 + k;
+                const int kbyte0 = (i * P + a0) * E;
+                const uint32_t base = tb + (uint32_t)(kbyte0 / Cfg::SW2) * 128 * Cfg::SW2 +
+                                      (uint32_t)(row >> 3) * 8 * Cfg::SW2 + (uint32_t)(row & 7) * Cfg::SW2;
+                const int slot0 = (kbyte0 % Cfg::SW2) >> 4, xr = (row & 7) & (Cfg::SW2 / 16 - 1);
 #pragma unroll
                 for (int g = 0; g < 32 / VPC; ++g) {
-                    const int col = c0 + g * VPC;   // (n,a) of the first value
-                    const int n = col / P, a = col % P;
                     float v[8];
 #pragma unroll
                     for (int u = 0; u < VPC; ++u) v[u] = __uint_as_float(r[g * VPC + u]);
-                    st16<T>(tb + kmajor_off(n * M2 + k, (i * P + a) * E, 128, Cfg::SW2), v);
+                    st16<T>(base + (uint32_t)(((slot0 + g) ^ xr) << 4), v);
                 }
             }
             fence_proxy_async();
-            mbar_arrive(bar(B_TFULL + b));
+            mbar_arrive_warp(bar(B_TFULL + b));
         }
     } else {
         // ---------------- epilogue 2: D2 (lanes (n,k), columns c) + bias -> y ----------------
@@ -346,7 +352,7 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
                 }
                 if (c0 + 32 >= Q) {
                     tc_fence_before();
-                    mbar_arrive(bar(B_D2EMPTY + b));
+                    mbar_arrive_warp(bar(B_D2EMPTY + b));
                 }
                 if (row < args.N) {
 #pragma unroll
@@ -390,6 +396,12 @@ cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t
                          uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw) {
     auto enc = get_encode();
     if (!enc) return cudaErrorNotSupported;
+    // The encoder is a driver-API call: make the current device's primary context current
+    // on this host thread first (a thread whose first CUDA call this is has none bound).
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce == cudaSuccess) ce = cudaSetDevice(dev);
+    if (ce != cudaSuccess) return ce;
     const int E = bf16 ? 2 : 4;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * E};
@@ -431,16 +443,25 @@ cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *
     using T = typename Cfg::T;
     const bool bf16 = !Elt<T>::tf32;
     CUtensorMap tm;
+    launch_step() = "tensor map of x";
     cudaError_t e = make_tmap_2d(&tm, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1,
                                  Cfg::SW1 / Cfg::E, Cfg::N1, Cfg::SW1);
     if (e != cudaSuccess) return e;
+    launch_step() = "shared-memory attribute";
     e = cudaFuncSetAttribute(kron_fwd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
     if (e != cudaSuccess) return e;
+    launch_step() = "kernel launch";
     FwdArgs a{S, A, B, bias, y, s.N, (int)((s.N + Cfg::NT - 1) / Cfg::NT), device_error_ptr()};
     const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-    kron_fwd_tc_kernel<Cfg><<<grid, 480, Cfg::SMEM, st>>>(tm, a);
-    return cudaGetLastError();
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(480);
+        cfg.dynamicSmemBytes = Cfg::SMEM;
+        cfg.stream = st;
+        return cudaLaunchKernelEx(&cfg, kron_fwd_tc_kernel<Cfg>, tm, a);
+    }
 }
 
 using FwdFn = cudaError_t (*)(const void *, const void *, const void *, const void *,

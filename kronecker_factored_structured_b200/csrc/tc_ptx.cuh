@@ -36,6 +36,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One arrival per warp: every lane has already fenced its own writes; __syncwarp orders
+// them before lane 0's arrival (a 32-lane arrive on one barrier would serialise).
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
@@ -216,6 +223,21 @@ __device__ __forceinline__ uint32_t f32_to_tf32(float v) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Base address of row `row` of a 128B-swizzled K-major region (rows `rows`, K in
+// 128-byte chunks) at K-chunk `kchunk`: 16-byte slot j of that 128-byte row is at
+// base + ((j ^ (row & 7)) << 4).
+__device__ __forceinline__ uint32_t sw128_row(uint32_t region, int rows, int kchunk, int row) {
+    return region + (uint32_t)kchunk * rows * 128 + (uint32_t)(row >> 3) * 1024 +
+           (uint32_t)(row & 7) * 128;
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&v)[4]) {
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(addr)
+                 : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
