@@ -115,6 +115,33 @@ KRON_API kron_status_t kron_linear_backward(const void *x, const void *S, const 
                                    kron_dtype_t dtype, unsigned flags,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Backward without a caller-provided workspace.  (An addition of this library: the
+ * paper has no counterpart.)
+ *
+ * Some callers cannot allocate device memory at the moment they run the backward: a
+ * real-time loop in which cudaMalloc's device-wide synchronisation is not acceptable,
+ * a host whose device memory is entirely owned by another allocator, or plain C code
+ * with no allocator of its own.  This entry point takes the same arguments as
+ * kron_linear_backward without the workspace and uses instead a fixed scratch array
+ * of KRON_NOALLOC_SCRATCH_BYTES compiled into the library; it allocates nothing.
+ *   - Every GPU that loads the library holds that array until the process exits.
+ *   - Problems whose kron_linear_workspace_size exceeds KRON_NOALLOC_SCRATCH_BYTES are
+ *     rejected with KRON_ERR_WORKSPACE before anything is launched.
+ *   - All calls share the one array per device: calls that overlap on the GPU (for
+ *     example on two streams) race on it and must be serialised by the caller.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ * Results are the same as kron_linear_backward's.
+ */
+#define KRON_NOALLOC_SCRATCH_BYTES (8u << 20)
+KRON_API kron_status_t kron_linear_backward_noalloc(const void *x, const void *S, const void *A,
+                                                    const void *B, const void *dY, void *dX,
+                                                    void *dS, void *dA, void *dB, void *dbias,
+                                                    int64_t N, int p, int q, int m1, int m2, int r,
+                                                    kron_dtype_t dtype, unsigned flags,
+                                                    void *stream);
+
 /* Bytes of device workspace kron_linear_backward needs for this problem (0 if the
  * arguments are invalid).  Depends only on the arguments, not on the device. */
 KRON_API size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r,

@@ -69,6 +69,11 @@ int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
 
 }  // namespace
 
+namespace kron {
+// Records a failure in this thread's last-error string (for entry points in other files).
+kron_status_t report_failure(kron_status_t st, const char *msg) { return fail(st, "%s", msg); }
+}  // namespace kron
+
 extern "C" {
 
 int kron_linear_abi_version(void) { return KRON_LINEAR_ABI_VERSION; }

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libkronlinear.so")
 KRON_F32, KRON_TF32, KRON_BF16 = 0, 1, 2
 DTYPES = {"f32": KRON_F32, "tf32": KRON_TF32, "bf16": KRON_BF16}
 KRON_FLAG_SKIP_ZERO_BLOCKS = 1
+KRON_NOALLOC_SCRATCH_BYTES = 8 << 20   # fixed scratch of kron_linear_backward_noalloc
 
 # Paths whose kernels are built into the library.
 IMPLEMENTED_PATHS = ("f32", "tf32", "bf16")
@@ -27,7 +28,8 @@ STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
           6: "KRON_ERR_TIMEOUT"}
 
 # Every symbol include/kron_linear.h declares.
-EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_workspace_size",
+EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_noalloc",
+           "kron_linear_workspace_size",
            "kron_status_string", "kron_last_error", "kron_linear_device_error",
            "kron_linear_abi_version")
 
@@ -57,6 +59,9 @@ def load(path: str = LIB_PATH):
     lib.kron_linear_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                          i64, I, I, I, I, I, I, U, vp, sz, vp]
     lib.kron_linear_backward.restype = I
+    lib.kron_linear_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                 i64, I, I, I, I, I, I, U, vp]
+    lib.kron_linear_backward_noalloc.restype = I
     lib.kron_linear_workspace_size.argtypes = [i64, I, I, I, I, I, I]
     lib.kron_linear_workspace_size.restype = sz
     lib.kron_status_string.argtypes = [I]
