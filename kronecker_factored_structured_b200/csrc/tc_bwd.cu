@@ -25,7 +25,8 @@
 //   B: T2 (read by dC), then X^T (read by dB)      -- "B chain"
 // Warp roles (448 threads, one CTA per SM):
 //   warp 0       TMA producer (G and X tiles)
-//   warp 1       TMEM allocator + MMA issuer
+//   warp 1       TMEM allocator + MMA issuer (the whole warp runs the issue loop, one
+//                elected lane issues each burst)
 //   warps 2-5    B chain: T2 epilogue, X^T; also G^T, dbias and the dX epilogue
 //   warps 6-13   A chain: U1 and U2 epilogues, 2 warps per TMEM lane quadrant
 #include "internal.h"
@@ -160,24 +161,29 @@ __device__ __forceinline__ void tmem_row_to_smem(uint32_t taddr, uint32_t region
     const int slot0 = (kbyte0 & 127) >> 4, x = row & 7;
 #pragma unroll
     for (int g = 0; g < 32 / VPC; ++g) {
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) v[t] = __uint_as_float(r[g * VPC + t]);
-        st16v<T>(base + (uint32_t)(((slot0 + g) ^ x) << 4), v);
+        const uint32_t addr = base + (uint32_t)(((slot0 + g) ^ x) << 4);
+        if constexpr (BE<T>::tf32) {
+            // fp32 bits as they are: the TF32 MMA reads the top 19 bits of each operand
+            st_shared_v4(addr, r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+        } else {
+            st_shared_v4(addr, pack_bf16x2(__uint_as_float(r[8 * g]), __uint_as_float(r[8 * g + 1])),
+                         pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3])),
+                         pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5])),
+                         pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7])));
+        }
     }
 }
 
 // Transpose of 8 source rows x 16 bytes (VPC elements) held as in[8][4] words into VPC
 // output rows of 8 elements each: out row e = (in[0][e], ..., in[7][e]).  The
-// elements are already in operand format (raw fp32 is rounded to tf32 here).
+// elements are copied as they are (fp32 bits for TF32: the MMA reads the top 19 bits,
+// as it does for the tiles TMA brings in).
 template <typename T>
 __device__ __forceinline__ void store_transposed(const uint32_t (&in)[8][4], int e,
                                                  uint32_t addr_lo, uint32_t addr_hi) {
     if constexpr (BE<T>::tf32) {
-        st_shared_v4(addr_lo, f32_to_tf32(__uint_as_float(in[0][e])), f32_to_tf32(__uint_as_float(in[1][e])),
-                     f32_to_tf32(__uint_as_float(in[2][e])), f32_to_tf32(__uint_as_float(in[3][e])));
-        st_shared_v4(addr_hi, f32_to_tf32(__uint_as_float(in[4][e])), f32_to_tf32(__uint_as_float(in[5][e])),
-                     f32_to_tf32(__uint_as_float(in[6][e])), f32_to_tf32(__uint_as_float(in[7][e])));
+        st_shared_v4(addr_lo, in[0][e], in[1][e], in[2][e], in[3][e]);
+        st_shared_v4(addr_hi, in[4][e], in[5][e], in[6][e], in[7][e]);
     } else {
         const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
         const int w = e >> 1;
@@ -305,13 +311,14 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            auto mma = [&](uint32_t d, uint32_t a, int swa, uint32_t b, int swb, uint32_t id, uint32_t acc) {
-                mma_ss<BE<T>::tf32>(d, sdesc_kmajor(a, swa), sdesc_kmajor(b, swb), id, acc);
-            };
-            // Ua, Ub and T of the current tile
-            auto issue_ut = [&]() {
+        // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+        auto mma = [&](uint32_t d, uint32_t a, int swa, uint32_t b, int swb, uint32_t id, uint32_t acc) {
+            mma_ss<BE<T>::tf32>(d, sdesc_kmajor(a, swa), sdesc_kmajor(b, swb), id, acc);
+        };
+        // Ua, Ub and T of the current tile
+        auto issue_ut = [&]() {
+            if (elect_one()) {
+#pragma unroll
                 for (int kb = 0; kb < Q * E; kb += 32) {
                     const int ch = kb / Cfg::SWC, in = kb % Cfg::SWC;
                     mma(tmem + Cfg::TM_UA, sC + ch * 128 * Cfg::SWC + in, Cfg::SWC,
@@ -319,6 +326,7 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
                     mma(tmem + Cfg::TM_UB, sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC,
                         sC + ch * 128 * Cfg::SWC + in, Cfg::SWC, Cfg::ID_128, kb > 0);
                 }
+#pragma unroll
                 for (int kb = 0; kb < M1 * E; kb += 32) {
                     const int ch = kb / Cfg::SWJ, in = kb % Cfg::SWJ;
                     mma(tmem + Cfg::TM_T, sX + ch * 128 * Cfg::SWJ + in, Cfg::SWJ,
@@ -326,28 +334,36 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
                 }
                 mma_commit(bar(UT_FULL));
                 mma_commit(bar(X_FREE));
-            };
-            bool ok = true;
-            if (nt > 0) {
-                ok = mbar_wait(bar(X_FULL), 0, ab) && mbar_wait(bar(GT_FULL), 0, ab);
-                if (ok) {
-                    tc_fence_after();
-                    issue_ut();
-                }
             }
-            for (int u = 0; u < nt && ok; ++u) {
-                const uint32_t ph = u & 1;
-                // dX(u) = U1 . Bdx^T  (K = (i,k)); dC(u) += T2 . G^T (K = (n,k))
-                if (!mbar_wait(bar(E1A_DONE), ph, ab) || !mbar_wait(bar(DX_FREE), ph ^ 1, ab)) { ok = false; break; }
+            __syncwarp();
+        };
+        bool ok = true;
+        if (nt > 0) {
+            ok = warp_wait(bar(X_FULL), 0, ab) && warp_wait(bar(GT_FULL), 0, ab);
+            if (ok) {
                 tc_fence_after();
+                issue_ut();
+            }
+        }
+        for (int u = 0; u < nt && ok; ++u) {
+            const uint32_t ph = u & 1;
+            // dX(u) = U1 . Bdx^T  (K = (i,k)); dC(u) += T2 . G^T (K = (n,k))
+            if (!warp_wait(bar(E1A_DONE), ph, ab) || !warp_wait(bar(DX_FREE), ph ^ 1, ab)) break;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
                 for (int kb = 0; kb < 128 * E; kb += 32) {
                     const int ch = kb / 128, in = kb % 128;
                     mma(tmem + Cfg::TM_DX, sA + ch * 128 * 128 + in, 128, sBD + ch * M1 * 128 + in, 128,
                         Cfg::ID_M1, kb > 0);
                 }
                 mma_commit(bar(DX_FULL));
-                if (!mbar_wait(bar(E1B_DONE), ph, ab)) { ok = false; break; }
-                tc_fence_after();
+            }
+            __syncwarp();
+            if (!warp_wait(bar(E1B_DONE), ph, ab)) break;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
                 for (int kb = 0; kb < 128 * E; kb += 32) {
                     const int ch = kb / 128, in = kb % 128;                // T2: 128-byte chunks
                     const int chg = kb / Cfg::SWG, ing = kb % Cfg::SWG;    // G: one chunk per n
@@ -356,25 +372,32 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
                 }
                 mma_commit(bar(DC_DONE));
                 mma_commit(bar(G_FREE));
-                // dB(u) += U2 . X^T^T (K = (n,a)) once U2 and X^T are written
-                if (!mbar_wait(bar(U2_DONE), ph, ab) || !mbar_wait(bar(XT_DONE), ph, ab)) { ok = false; break; }
-                tc_fence_after();
+            }
+            __syncwarp();
+            // dB(u) += U2 . X^T^T (K = (n,a)) once U2 and X^T are written
+            if (!warp_wait(bar(U2_DONE), ph, ab) || !warp_wait(bar(XT_DONE), ph, ab)) break;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
                 for (int kb = 0; kb < 128 * E; kb += 32) {
                     const int ch = kb / 128, in = kb % 128;
                     mma(tmem + Cfg::TM_DB, sA + ch * 128 * 128 + in, 128, sBb + ch * M1 * 128 + in, 128,
                         Cfg::ID_M1, (u > 0 || kb > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(DB_DONE));
-                // Ua, Ub, T of tile u+1 (their accumulators were read out before U2_DONE(u))
-                if (u + 1 < nt) {
-                    if (!mbar_wait(bar(X_FULL), ph ^ 1, ab) || !mbar_wait(bar(GT_FULL), ph ^ 1, ab)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_ut();
-                }
             }
-            mma_commit(bar(DRAIN));
-            mbar_wait_drain(bar(DRAIN), 0);
+            __syncwarp();
+            // Ua, Ub, T of tile u+1 (their accumulators were read out before U2_DONE(u))
+            if (u + 1 < nt) {
+                if (!warp_wait(bar(X_FULL), ph ^ 1, ab) || !warp_wait(bar(GT_FULL), ph ^ 1, ab)) break;
+                tc_fence_after();
+                issue_ut();
+            }
         }
+        if (elect_one()) mma_commit(bar(DRAIN));
+        __syncwarp();
+        if (lane == 0) mbar_wait_drain(bar(DRAIN), 0);
+        __syncwarp();
     } else if (warp < 6) {
         // ---------------- B chain (128 threads) ----------------
         const int tid = threadIdx.x - 64;

@@ -10,23 +10,23 @@
 // Stage 1 is computed transposed, so each accumulator lane (i,k) holds a whole row of
 // stage 2's A operand: the epilogue moves it TMEM -> registers -> shared memory with
 // 16-byte stores straight into the K-major swizzled layout stage 2 reads.  That is the
-// page's permute of Z, done on chip; T never reaches HBM.
+// page's permute of Z, done on chip; T never reaches HBM.  Stage 1's A operand, B_all^T,
+// stays in TMEM for the whole kernel.
 //
-// Warp roles (480 threads, one CTA per SM, persistent over tiles):
+// Warp roles (736 threads, one CTA per SM, persistent over tiles):
 //   warp 0       TMA producer: x tiles into an S-stage ring (128B-swizzled)
-//   warps 1, 2   MMA issuers for even / odd tiles (warp 1 also owns the TMEM allocation)
-//   warps 3-10   epilogue 1: stage-1 accumulator -> T in shared memory (stage 2's A
-//                operand); every tile is handled by all 8 warps, two per TMEM lane
-//                quadrant, each taking half of the columns
-//   warps 11-14  epilogue 2: stage-2 accumulator + bias -> y in HBM (coalesced rows)
-// Any shared-memory access by an MMA-issuing thread (an mbarrier wait included) first
-// drains that thread's queued MMAs, leaving the tensor pipe idle.  So each issuer
-// synchronises once per tile -- round k waits for everything it needs, then issues
-// stage 2 of tile k and stage 1 of tile k+2 in one burst -- and two issuers own
-// alternate tiles, so while one drains at its sync point the other keeps the tensor
-// core busy.  Stage-1 accumulators are triple-buffered; T and the stage-2 accumulator
-// are one per tile parity.  The epilogues take the tiles strictly in order, which keeps
-// every mbarrier's phases in order (a consumer can never test a phase two ahead).
+//   warp 1       stage-1 MMA issuer (also owns the TMEM allocation)
+//   warp 2       stage-2 MMA issuer
+//   warps 3-18   epilogue 1: stage-1 accumulator -> T in shared memory; every tile is
+//                handled by all 16 warps, four per TMEM lane quadrant, 32 columns each
+//   warps 19-22  epilogue 2: stage-2 accumulator + bias -> y in HBM (coalesced rows)
+// Both issuers run their loops as whole warps (waits and descriptors warp-uniform) and
+// let one elected lane issue each burst of MMAs: a loop run by a single lane issues
+// several times slower.  Each issuer waits once per tile; while one waits, the other's
+// MMAs keep the tensor pipe busy.  Both accumulators are triple-buffered in TMEM; T
+// rotates over TB shared-memory buffers (as many as fit beside a deep x ring), which
+// sets how far epilogue 1 can run ahead of stage 2.  Every consumer takes the tiles in
+// order, which keeps each mbarrier's phases in order (no test of a phase two ahead).
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -53,6 +53,8 @@ template <> struct Elt<__nv_bfloat16> {
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
+constexpr int kFwdThreads = 736;
+
 template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
 struct FwdCfg {
     using T = T_;
@@ -61,26 +63,31 @@ struct FwdCfg {
     static constexpr int NT = 128 / M2;        // rows of x per tile
     static constexpr int N1 = NT * P;          // stage-1 N: (n,a)
     static constexpr int SW1 = cmin(128, M1 * E);
-    static constexpr int KC1 = M1 * E / SW1;   // 128B K-chunks along j
+    static constexpr int KC1 = M1 * E / SW1;   // K-chunks of SW1 bytes along j
     static constexpr int K2B = R * P * E;      // stage-2 K in bytes: (i,a)
     static constexpr int SW2 = cmin(128, K2B);
-    static constexpr int KC2 = K2B / SW2;
-    static constexpr int STAGES = 3;
-    // shared-memory regions (bytes, each 1024-aligned)
-    static constexpr int A1_BYTES = 128 * M1 * E;      // B_all^T [(i,k)][j]
-    static constexpr int B2_BYTES = Q * K2B;           // C'      [c][(i,a)]
-    static constexpr int X_BYTES = N1 * M1 * E;        // x tile  [(n,a)][j]
-    static constexpr int T_BYTES = 128 * K2B;          // T       [(n,k)][(i,a)]
-    static constexpr int OFF_A1 = 0;
-    static constexpr int OFF_B2 = OFF_A1 + A1_BYTES;
-    static constexpr int OFF_X = OFF_B2 + B2_BYTES;
-    static constexpr int OFF_T = OFF_X + STAGES * X_BYTES;
-    static constexpr int OFF_BAR = OFF_T + 2 * T_BYTES;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + alignment slack
-    // TMEM columns: D1[3] (N1 each; stage 1 runs two tiles ahead), D2[2] (Q each)
-    static constexpr int D1_SLOTS = 3;
-    static constexpr int TM_D1 = 0, TM_D2 = D1_SLOTS * N1;
-    static constexpr int TM_COLS_USED = D1_SLOTS * N1 + 2 * Q;
+    // shared memory (bytes, each region 1024-aligned)
+    static constexpr int B2_BYTES = Q * K2B;             // C'      [c][(i,a)]
+    static constexpr int X_BYTES = N1 * M1 * E;          // x tile  [(n,a)][j]
+    static constexpr int T_BYTES = 128 * K2B;            // T       [(n,k)][(i,a)]
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM_MAX = 232448;
+    static constexpr int FIXED = 1024 + BAR_BYTES + B2_BYTES;
+    // T buffers: as many as leave room for at least 6 x stages (at most 4)
+    static constexpr int TB = (SMEM_MAX - FIXED - 4 * T_BYTES) / X_BYTES >= 6 ? 4
+                            : (SMEM_MAX - FIXED - 3 * T_BYTES) / X_BYTES >= 6 ? 3 : 2;
+    static constexpr int STAGES = cmin(8, (SMEM_MAX - FIXED - TB * T_BYTES) / X_BYTES);
+    static constexpr int OFF_B2 = 0;
+    static constexpr int OFF_T = OFF_B2 + B2_BYTES;
+    static constexpr int OFF_X = OFF_T + TB * T_BYTES;
+    static constexpr int OFF_BAR = OFF_X + STAGES * X_BYTES;
+    static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // barriers + alignment slack
+    // TMEM columns: D1[3] (N1 each), D2[3] (Q each), stage 1's A operand B_all^T
+    // [(i,k)][j] (M1 values per lane, two per column for BF16)
+    static constexpr int D1_SLOTS = 3, D2_SLOTS = 3;
+    static constexpr int TM_D1 = 0, TM_D2 = D1_SLOTS * N1, TM_A1 = TM_D2 + D2_SLOTS * Q;
+    static constexpr int A1_COLS = M1 * E / 4;
+    static constexpr int TM_COLS_USED = TM_A1 + A1_COLS;
     static constexpr int TM_COLS = TM_COLS_USED <= 32 ? 32 : TM_COLS_USED <= 64 ? 64
                                  : TM_COLS_USED <= 128 ? 128 : TM_COLS_USED <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC1 = idesc_f32acc(128, N1, Elt<T>::fmt);
@@ -88,15 +95,18 @@ struct FwdCfg {
 
     static_assert(R * M2 == 128, "stage-1 M = r*m2 must be 128");
     static_assert(128 % M2 == 0, "m2 must divide 128");
-    static_assert(N1 % 64 == 0 && N1 <= 256, "stage-1 N = (128/m2)*p: multiple of 64, at most 256");
+    static_assert(N1 == 128, "stage-1 N = (128/m2)*p: 128 (four 32-column epilogue chunks)");
     static_assert(Q % 32 == 0 && Q <= 256, "q must be a multiple of 32, at most 256");
     static_assert(M1 * E % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
+    static_assert(A1_COLS % 8 == 0, "stage-1 A operand: whole 8-column groups");
     static_assert(K2B % 32 == 0 && (K2B <= 128 || K2B % 128 == 0), "r*p bytes");
-    static_assert((P * E) % 16 == 0, "p*elt must be a multiple of 16 bytes");
     static_assert(P % 32 == 0 && (32 * E) <= SW2 && SW2 == 128,
                   "a 32-column TMEM chunk maps to one 128B-swizzled row of T");
+    static_assert(STAGES >= 3, "x ring");
+    static_assert(2 * STAGES + 2 * D1_SLOTS + 2 * TB + 2 * D2_SLOTS + 2 + 2 <= BAR_BYTES / 8,
+                  "barrier region");
     static_assert(TM_COLS_USED <= 512, "TMEM budget");
-    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
 
 struct FwdArgs {
@@ -135,25 +145,24 @@ __device__ __forceinline__ void st16(uint32_t addr, const float *v) {
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(480, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     using T = typename Cfg::T;
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
-    constexpr int NT = Cfg::NT, N1 = Cfg::N1, S = Cfg::STAGES;
+    constexpr int NT = Cfg::NT, N1 = Cfg::N1, S = Cfg::STAGES, TB = Cfg::TB;
+    constexpr int D1S = Cfg::D1_SLOTS, D2S = Cfg::D2_SLOTS;
     constexpr int VPC = 16 / E;  // values per 16-byte chunk
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sA1 = sbase + Cfg::OFF_A1, sB2 = sbase + Cfg::OFF_B2;
-    const uint32_t sX = sbase + Cfg::OFF_X, sT = sbase + Cfg::OFF_T;
+    const uint32_t sB2 = sbase + Cfg::OFF_B2, sX = sbase + Cfg::OFF_X, sT = sbase + Cfg::OFF_T;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     // barrier indices
-    constexpr int D1S = Cfg::D1_SLOTS;
     constexpr int B_XFULL = 0, B_XEMPTY = S, B_D1FULL = 2 * S, B_D1EMPTY = 2 * S + D1S,
-                  B_TFULL = 2 * S + 2 * D1S, B_TEMPTY = B_TFULL + 2, B_D2FULL = B_TFULL + 4,
-                  B_D2EMPTY = B_TFULL + 6, B_DRAIN = B_TFULL + 8, NBARS = B_TFULL + 10;
+                  B_TFULL = 2 * S + 2 * D1S, B_TEMPTY = B_TFULL + TB, B_D2FULL = B_TFULL + 2 * TB,
+                  B_D2EMPTY = B_D2FULL + D2S, B_DRAIN = B_D2FULL + 2 * D2S, NBARS = B_DRAIN + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
     const Abort abort_flag{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
     auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -168,30 +177,24 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         }
         for (int b = 0; b < D1S; ++b) {
             mbar_init(bar(B_D1FULL + b), 1);
-            mbar_init(bar(B_D1EMPTY + b), 8);   // epilogue-1 warps
+            mbar_init(bar(B_D1EMPTY + b), 16);  // epilogue-1 warps
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(B_TFULL + b), 8);
+        for (int b = 0; b < TB; ++b) {
+            mbar_init(bar(B_TFULL + b), 16);
             mbar_init(bar(B_TEMPTY + b), 1);
-            mbar_init(bar(B_D2FULL + b), 1);
-            mbar_init(bar(B_D2EMPTY + b), 4);    // epilogue-2 warps
-            mbar_init(bar(B_DRAIN + b), 1);
         }
+        for (int b = 0; b < D2S; ++b) {
+            mbar_init(bar(B_D2FULL + b), 1);
+            mbar_init(bar(B_D2EMPTY + b), 4);   // epilogue-2 warps
+        }
+        mbar_init(bar(B_DRAIN + 0), 1);
+        mbar_init(bar(B_DRAIN + 1), 1);
         *abort_flag.flag = 0;
         mbar_init_fence();
         prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
-    }
-    // stage-1 A operand: B_all^T[(i,k)][j] = B_i[j][k]
-    for (int e = threadIdx.x; e < 128 * (M1 / VPC); e += blockDim.x) {
-        const int row = e / (M1 / VPC), j0 = (e % (M1 / VPC)) * VPC;
-        const int i = row / M2, k = row % M2;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) v[t] = ldf<T>(args.B, ((size_t)i * M1 + j0 + t) * M2 + k);
-        st16<T>(sA1 + kmajor_off(row, j0 * E, 128, Cfg::SW1), v);
     }
     // stage-2 B operand: C'[c][(i,a)] = S[a][c] * A_i[a][c]
     for (int e = threadIdx.x; e < Q * (R * P / VPC); e += blockDim.x) {
@@ -209,6 +212,29 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // stage-1 A operand in TMEM: lane (i,k) holds B_all^T[(i,k)][j] = B_i[j][k] along j
+    if (warp >= 4 && warp < 8) {
+        const int L = (warp & 3) * 32 + lane, i = L / M2, k = L % M2;
+        const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + Cfg::TM_A1;
+#pragma unroll
+        for (int c0 = 0; c0 < Cfg::A1_COLS; c0 += 8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if constexpr (Elt<T>::tf32) {
+                    w[u] = f32_to_tf32(ldf<T>(args.B, ((size_t)i * M1 + c0 + u) * M2 + k));
+                } else {
+                    const int j = 2 * (c0 + u);
+                    w[u] = pack_bf16x2(ldf<T>(args.B, ((size_t)i * M1 + j) * M2 + k),
+                                       ldf<T>(args.B, ((size_t)i * M1 + j + 1) * M2 + k));
+                }
+            }
+            tmem_store8(ta + c0, w);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     const int my_tiles = (args.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
@@ -232,45 +258,43 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             for (int t = (issued > S ? issued - S : 0); t < issued; ++t)
                 mbar_wait_drain(bar(B_XFULL + t % S), (t / S) & 1);
         }
-    } else if (warp == 1 || warp == 2) {
-        // ---------------- MMA issuers: warp 1 even tiles, warp 2 odd tiles ----------------
-        const int par = warp - 1;
-        if (lane == 0) {
-            // stage 1 of tile u into D1 slot u % 3 (its waits already done)
-            auto issue_stage1 = [&](int u) {
-                const int s = u % S, d1 = u % D1S;
+    } else if (warp == 1) {
+        // ---------------- stage-1 issuer: D1[(i,k)][(n,a)] = B_all^T (TMEM) . x tile ----------------
+        for (int t = 0; t < my_tiles; ++t) {
+            const int s = t % S, d1 = t % D1S;
+            if (!warp_wait(bar(B_XFULL + s), (t / S) & 1, abort_flag) ||
+                !warp_wait(bar(B_D1EMPTY + d1), ((t / D1S) & 1) ^ 1, abort_flag))
+                break;
+            tc_fence_after();
+            if (elect_one()) {
                 const uint32_t d = tmem + Cfg::TM_D1 + d1 * N1;
 #pragma unroll
                 for (int kk = 0; kk < M1 * E / 32; ++kk) {
                     const int kb = kk * 32, ch = kb / Cfg::SW1, in = kb % Cfg::SW1;
-                    const uint64_t ad = sdesc_kmajor(sA1 + ch * 128 * Cfg::SW1 + in, Cfg::SW1);
                     const uint64_t bd = sdesc_kmajor(sX + s * Cfg::X_BYTES + ch * N1 * Cfg::SW1 + in, Cfg::SW1);
-                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC1, kk > 0);
+                    mma_ts<Elt<T>::tf32>(d, tmem + Cfg::TM_A1 + kk * 8, bd, Cfg::IDESC1, kk > 0);
                 }
                 mma_commit(bar(B_XEMPTY + s));
                 mma_commit(bar(B_D1FULL + d1));
-            };
-            auto wait_stage1 = [&](int u) -> bool {
-                return mbar_wait(bar(B_XFULL + u % S), (u / S) & 1, abort_flag) &&
-                       mbar_wait(bar(B_D1EMPTY + u % D1S), ((u / D1S) & 1) ^ 1, abort_flag);
-            };
-            bool ok = true;
-            if (par < my_tiles) {  // prologue: stage 1 of this issuer's first tile
-                ok = wait_stage1(par);
-                if (ok) {
-                    tc_fence_after();
-                    issue_stage1(par);
-                }
             }
-            const uint32_t d = tmem + Cfg::TM_D2 + par * Q;
-            const uint32_t tb = sT + par * Cfg::T_BYTES;
-            for (int k = par; k < my_tiles && ok; k += 2) {
-                const uint32_t pb = (k >> 1) & 1;
-                // one synchronisation point per round
-                if (!mbar_wait(bar(B_TFULL + par), pb, abort_flag)) break;
-                if (!mbar_wait(bar(B_D2EMPTY + par), pb ^ 1, abort_flag)) break;
-                if (k + 2 < my_tiles && !wait_stage1(k + 2)) break;
-                tc_fence_after();
+            __syncwarp();
+        }
+        // every MMA of this issuer has completed before TMEM can be released
+        if (elect_one()) mma_commit(bar(B_DRAIN + 0));
+        __syncwarp();
+        if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 0), 0);
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- stage-2 issuer: D2[(n,k)][c] = T . C' ----------------
+        for (int t = 0; t < my_tiles; ++t) {
+            const int b = t % TB, d2 = t % D2S;
+            if (!warp_wait(bar(B_D2EMPTY + d2), ((t / D2S) & 1) ^ 1, abort_flag) ||
+                !warp_wait(bar(B_TFULL + b), (t / TB) & 1, abort_flag))
+                break;
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t d = tmem + Cfg::TM_D2 + d2 * Q;
+                const uint32_t tb = sT + b * Cfg::T_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
                     const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
@@ -278,49 +302,50 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
                     const uint64_t bd = sdesc_kmajor(sB2 + ch * Q * Cfg::SW2 + in, Cfg::SW2);
                     mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC2, kk > 0);
                 }
-                mma_commit(bar(B_TEMPTY + par));
-                mma_commit(bar(B_D2FULL + par));
-                if (k + 2 < my_tiles) issue_stage1(k + 2);
+                mma_commit(bar(B_TEMPTY + b));
+                mma_commit(bar(B_D2FULL + d2));
             }
-            // every MMA of this issuer has completed before TMEM can be released
-            mma_commit(bar(B_DRAIN + par));
-            mbar_wait_drain(bar(B_DRAIN + par), 0);
+            __syncwarp();
         }
-    } else if (warp < 11) {
+        if (elect_one()) mma_commit(bar(B_DRAIN + 1));
+        __syncwarp();
+        if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 1), 0);
+        __syncwarp();
+    } else if (warp < 19) {
         // ---------------- epilogue 1: D1 (lanes (i,k), columns (n,a)) -> T smem ----------------
-        const int half = (warp - 3) / 4;          // which half of the columns
-        const int quad = warp & 3;
+        const int quad = warp & 3, part = (warp - 3) >> 2;
         const int L = quad * 32 + lane;  // (i,k)
         const int i = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        constexpr int HC = N1 / 2;                // columns per warp
+        const int c0 = part * 32;        // this warp's 32 columns (n, a0 .. a0+31)
+        const int n = c0 / P, a0 = c0 % P, row = n * M2 + k;
+        const int kbyte0 = (i * P + a0) * E;
+        const uint32_t roff = (uint32_t)(kbyte0 / Cfg::SW2) * 128 * Cfg::SW2 +
+                              (uint32_t)(row >> 3) * 8 * Cfg::SW2 + (uint32_t)(row & 7) * Cfg::SW2;
+        const int slot0 = (kbyte0 % Cfg::SW2) >> 4, xr = (row & 7) & (Cfg::SW2 / 16 - 1);
         for (int t = 0; t < my_tiles; ++t) {
-            const int b = t & 1, d1 = t % D1S;
-            const uint32_t pb = (t >> 1) & 1;
+            const int b = t % TB, d1 = t % D1S;
             if (!mbar_wait(bar(B_D1FULL + d1), (t / D1S) & 1, abort_flag)) break;
-            if (!mbar_wait(bar(B_TEMPTY + b), pb ^ 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t tb = sT + b * Cfg::T_BYTES;
-#pragma unroll 1
-            for (int c0 = half * HC; c0 < (half + 1) * HC; c0 += 32) {
-                uint32_t r[32];
-                tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1 + c0, r);
-                if (c0 + 32 >= (half + 1) * HC) {  // this thread's columns of the slot are read
-                    tc_fence_before();
-                    mbar_arrive_warp(bar(B_D1EMPTY + d1));
-                }
-                // 32 columns (n, a0..a0+31) -> row (n,k) of T, K bytes (i*p + a0)*E onward
-                const int n = c0 / P, a0 = c0 % P, row = n * M2 + k;
-                const int kbyte0 = (i * P + a0) * E;
-                const uint32_t base = tb + (uint32_t)(kbyte0 / Cfg::SW2) * 128 * Cfg::SW2 +
-                                      (uint32_t)(row >> 3) * 8 * Cfg::SW2 + (uint32_t)(row & 7) * Cfg::SW2;
-                const int slot0 = (kbyte0 % Cfg::SW2) >> 4, xr = (row & 7) & (Cfg::SW2 / 16 - 1);
+            uint32_t r[32];
+            tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1 + c0, r);
+            tc_fence_before();
+            mbar_arrive_warp(bar(B_D1EMPTY + d1));
+            // 32 columns (n, a0..a0+31) -> row (n,k) of T, K bytes (i*p + a0)*E onward
+            if (!mbar_wait(bar(B_TEMPTY + b), ((t / TB) & 1) ^ 1, abort_flag)) break;
+            const uint32_t base = sT + b * Cfg::T_BYTES + roff;
 #pragma unroll
-                for (int g = 0; g < 32 / VPC; ++g) {
-                    float v[8];
-#pragma unroll
-                    for (int u = 0; u < VPC; ++u) v[u] = __uint_as_float(r[g * VPC + u]);
-                    st16<T>(base + (uint32_t)(((slot0 + g) ^ xr) << 4), v);
+            for (int g = 0; g < 32 / VPC; ++g) {
+                const uint32_t addr = base + (uint32_t)(((slot0 + g) ^ xr) << 4);
+                if constexpr (Elt<T>::tf32) {
+                    // fp32 bits as they are: the TF32 MMA reads the top 19 bits of each
+                    // operand (as it does for the x tile, which TMA copies unchanged)
+                    st_shared_v4(addr, r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+                } else {
+                    st_shared_v4(addr, pack_bf16x2(__uint_as_float(r[8 * g]), __uint_as_float(r[8 * g + 1])),
+                                 pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3])),
+                                 pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5])),
+                                 pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7])));
                 }
             }
             fence_proxy_async();
@@ -332,32 +357,26 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         const int L = quad * 32 + lane;  // (n,k)
         const int n = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        float bias[Q];
+        float bias[Q];  // this lane's bias values, kept in registers
 #pragma unroll
         for (int c = 0; c < Q; ++c) bias[c] = args.bias ? ldf<T>(args.bias, (size_t)c * M2 + k) : 0.f;
         for (int t = 0; t < my_tiles; ++t) {
-            const int b = t & 1;
-            const uint32_t pb = (t >> 1) & 1;
-            if (!mbar_wait(bar(B_D2FULL + b), pb, abort_flag)) break;
+            const int d2 = t % D2S;
+            if (!mbar_wait(bar(B_D2FULL + d2), (t / D2S) & 1, abort_flag)) break;
             tc_fence_after();
             const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
 #pragma unroll
             for (int c0 = 0; c0 < Q; c0 += 32) {
-                float acc[32];
-                {
-                    uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_D2 + b * Q + c0, r);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) acc[u] = __uint_as_float(r[u]);
-                }
+                uint32_t r[32];
+                tmem_load32(tmem + lane_addr + Cfg::TM_D2 + d2 * Q + c0, r);
                 if (c0 + 32 >= Q) {
                     tc_fence_before();
-                    mbar_arrive_warp(bar(B_D2EMPTY + b));
+                    mbar_arrive_warp(bar(B_D2EMPTY + d2));
                 }
                 if (row < args.N) {
 #pragma unroll
-                    for (int u = 0; u < 32 && c0 + u < Q; ++u) {
-                        const float v = acc[u] + bias[c0 + u];
+                    for (int u = 0; u < 32; ++u) {
+                        const float v = __uint_as_float(r[u]) + bias[c0 + u];
                         const size_t o = (size_t)row * (Q * M2) + (size_t)(c0 + u) * M2 + k;
                         if constexpr (Elt<T>::tf32) static_cast<float *>(args.y)[o] = v;
                         else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
@@ -457,7 +476,7 @@ cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *
     {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
-        cfg.blockDim = dim3(480);
+        cfg.blockDim = dim3(kFwdThreads);
         cfg.dynamicSmemBytes = Cfg::SMEM;
         cfg.stream = st;
         return cudaLaunchKernelEx(&cfg, kron_fwd_tc_kernel<Cfg>, tm, a);
