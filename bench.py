@@ -179,6 +179,7 @@ def main():
 
     import kronecker_factored_structured_b200 as kfs
     from kronecker_factored_structured_b200 import accounting as acc
+    from kronecker_factored_structured_b200 import dp
 
     path = args.path or ("tf32" if "tf32" in kfs.native.IMPLEMENTED_PATHS else "f32")
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -198,21 +199,18 @@ def main():
     fac = {k: v.to(dev) for k, v in kw.factors(w).items()}
     sets = []
     for s in range(ROTATE):
-        ws = dataclasses.replace(w, seed=w.seed + 1000 * s) if s else w
+        # each rank holds its own rows (weak scaling): a rank- and set-specific seed
+        ws = dataclasses.replace(w, seed=w.seed + 1000 * s + 100000 * rank) if (s or rank) else w
         sets.append((kw.rows(ws, "x").to(dev), kw.rows(ws, "G").to(dev)))
     p, q, m1, m2, r, N = w.p, w.q, w.m1, w.m2, w.r, w.N
     t_io = kfs.native.io_dtype(path)
     elt = 2 if path == "bf16" else 4
     y = torch.empty(N, q * m2, dtype=t_io, device=dev)
     grads = {"dX": torch.empty(N, p * m1, dtype=t_io, device=dev)}
-    flat = torch.empty(p * q + r * p * q + r * m1 * m2 + q * m2, dtype=torch.float32, device=dev)
-    o = 0
-    for k, shp in (("dS", (p, q)), ("dA", (r, p, q)), ("dB", (r, m1, m2)), ("dbias", (q * m2,))):
-        n = 1
-        for d in shp:
-            n *= d
-        grads[k] = flat[o:o + n].view(*shp)
-        o += n
+    # parameter gradients as views of one flat buffer: the one exchange of the data-parallel
+    # backward is a single all-reduce of it
+    flat, views = dp.flat_grad_buffer(p, q, m1, m2, r, device=dev)
+    grads.update(views)
     wsb = torch.empty(max(kfs.workspace_size(N, p, q, m1, m2, r, path), 1), dtype=torch.uint8,
                       device=dev)
     stream = torch.cuda.current_stream()
@@ -229,7 +227,7 @@ def main():
         if timing is not None:
             timing[2].record(stream)
         if world > 1:
-            dist.all_reduce(flat)
+            dp.allreduce_grads(flat)
 
     for i in range(args.warmup):
         step(i)
@@ -274,7 +272,7 @@ def main():
         kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, out=y)
         kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, workspace=wsb, grads=grads)
         if world > 1:
-            dist.all_reduce(flat)
+            dp.allreduce_grads(flat)
         yh.copy_(y, non_blocking=True)
         dxh.copy_(grads["dX"], non_blocking=True)
         fh.copy_(flat, non_blocking=True)

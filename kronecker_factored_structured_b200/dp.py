@@ -1,0 +1,53 @@
+"""Data-parallel plumbing for the Kronecker layer: row sharding and the one gradient exchange.
+
+Rows are independent (page "kronecker-layer-benchmark", section "Setup": a batch is just rows
+fed to the layer), so N rows split into contiguous per-rank ranges and the forward needs no
+communication.  The backward's only exchange is the sum over ranks of the parameter gradients
+dS, dA, dB and dbias; they live as views of one flat fp32 buffer so that a single all-reduce
+moves them all (dX stays sharded like x).
+"""
+from __future__ import annotations
+
+from typing import Dict, Tuple
+
+import torch
+
+
+def shard_rows(n_rows: int, world: int, rank: int) -> Tuple[int, int]:
+    """Contiguous row range (start, count) of `rank`: the first n_rows % world ranks take one
+    extra row; every row belongs to exactly one rank."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside a world of {world}")
+    if n_rows < 0:
+        raise ValueError("n_rows must be non-negative")
+    base, extra = divmod(n_rows, world)
+    start = rank * base + min(rank, extra)
+    return start, base + (1 if rank < extra else 0)
+
+
+def param_grad_sizes(p: int, q: int, m1: int, m2: int, r: int) -> Dict[str, tuple]:
+    """Shapes of the parameter gradients, in the order they sit in the flat buffer."""
+    return {"dS": (p, q), "dA": (r, p, q), "dB": (r, m1, m2), "dbias": (q * m2,)}
+
+
+def flat_grad_buffer(p: int, q: int, m1: int, m2: int, r: int,
+                     device="cpu") -> Tuple[torch.Tensor, Dict[str, torch.Tensor]]:
+    """One fp32 buffer holding dS, dA, dB, dbias back to back, and a view of it per gradient
+    (the layout the backward call writes into through `grads=`)."""
+    shapes = param_grad_sizes(p, q, m1, m2, r)
+    total = sum(int(torch.Size(s).numel()) for s in shapes.values())
+    flat = torch.zeros(total, dtype=torch.float32, device=device)
+    views, o = {}, 0
+    for k, s in shapes.items():
+        n = int(torch.Size(s).numel())
+        views[k] = flat[o:o + n].view(*s)
+        o += n
+    return flat, views
+
+
+def allreduce_grads(flat: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum the flat parameter-gradient buffer over the ranks of `group` (in place)."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    return flat
