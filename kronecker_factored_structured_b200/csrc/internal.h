@@ -45,6 +45,10 @@ cudaError_t simt_backward(const float *x, const float *S, const float *A, const 
 bool tc_forward_supported(const Shape &s, bool bf16);
 cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
                        const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st);
+// dX = dY W^T by the forward kernel with transposed factors (s is the layer's shape).
+bool tc_dx_supported(const Shape &s, bool bf16);
+cudaError_t tc_dx(const void *dY, const void *S, const void *A, const void *B, void *dX,
+                  const Shape &s, bool bf16, cudaStream_t st);
 bool tc_backward_supported(const Shape &s, bool bf16);
 int tc_backward_tile_rows(const Shape &s);
 // Writes dX (if non-null) and the per-range partials (parts x partial_stride floats).

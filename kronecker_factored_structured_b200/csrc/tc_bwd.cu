@@ -2,33 +2,36 @@
 //
 // Gradients of L = <G, y> (G = dY), W = sum_i kron(C_i, B_i), C_i = S (.) A_i (page
 // "kronecker-layer-benchmark", section "1. Build W, then multiply"; the page leaves the
-// backward to autograd).  Per tile of NT = r rows (shapes with p = m2 = 128/r), every
-// contraction on the tensor cores with K-major operands and a TMEM accumulator:
+// backward to autograd).  Two kernels:
 //
-//   U  = C_i G_n     as Ua[(i,a),(n,k)] = sum_c C[(i,a),c] G^T[(n,k),c]
-//                    and Ub[(n,k),(i,a)] = sum_c G^T[(n,k),c] C[(i,a),c]
-//   T  = X_n B_i     as T[(n,a),(i,k)]  = sum_j X[(n,a),j] Bt[(i,k),j]
-//   dX[(n,a),j]   = sum_(i,k) U[n,a,i,k] B_i[j,k]           A = U1 [(n,a)][(i,k)]
-//   dC[(i,a),c]  += sum_(n,k) T[n,a,i,k] G[(n,c),k]          A = T2 [(i,a)][(n,k)]
-//   dB[(i,k),j]  += sum_(n,a) U[n,a,i,k] X[(n,a),j]          A = U2 [(i,k)][(n,a)], B = X^T
-//   dbias[c*m2+k] += sum_n G[(n,c),k]
+//   dX_n = sum_i C_i G_n B_i^T        the forward's vec trick with C_i^T and B_i^T: the
+//                                     forward kernel in its transposed mode (tc_fwd.cu)
+//   parameter gradients (this file), per tile of NT = 2 rows, all on the tensor cores:
+//     T [(i,k),(n,a)] = sum_j  B_i[j,k] X_n[a,j]      A = B_all^T (TMEM), B = x tile
+//     U [(i,a),(n,k)] = sum_c  C_i[a,c] G_n[c,k]      A = C_stack (TMEM), B = G tile MN-major
+//     dC[(i,a),c]    += sum_(n,k) T[n,a,i,k] G_n[c,k]  A = T2 [(i,a)][(n,k)], B = G tile
+//     dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]  A = U2 [(i,k)][(n,a)], B = x tile MN-major
+//     dbias[c*m2+k]  += sum_n G_n[c,k]
+//   dC and dB accumulate in TMEM over the CTA's fixed, contiguous range of rows and are
+//   written to the workspace as that range's partials; reduce.cu adds the partials in a
+//   fixed order and forms dA = dC (.) S and dS = sum_i dC_i (.) A_i (bitwise reproducible).
 //
-// U is computed in both orientations so that each TMEM lane holds a contiguous row of
-// the operand the next contraction reads; every TMEM -> shared-memory epilogue is then
-// a sequence of 16-byte stores into a K-major swizzled layout (the permute the page's
-// loop-free version does in HBM).  dC and dB accumulate in TMEM over the CTA's fixed,
-// contiguous range of rows and are written to the workspace as that range's partial
-// sums; reduce.cu adds the partials in a fixed order (bitwise reproducible).
+// The x and G tiles serve as K-major operands (T, dC) and as MN-major ones (U, dB): TMA
+// brings each in both shared-memory layouts for TF32 (whose MN-major layout is the 128-byte
+// swizzle with 32-byte atoms), once for BF16 (one swizzled tile is valid both ways).  So no
+// thread ever transposes an input; the only permutes are the two epilogues, which move the
+// T and U accumulators (TMEM -> registers) into the K-major layouts dC and dB read, one
+// 128-byte row segment per warp store.
 //
-// Shared memory: factors C, Bt, Bdx; tiles G, X, G^T; two intermediate buffers:
-//   A: U1 (read by dX), then U2 (read by dB)       -- "A chain"
-//   B: T2 (read by dC), then X^T (read by dB)      -- "B chain"
-// Warp roles (448 threads, one CTA per SM):
-//   warp 0       TMA producer (G and X tiles)
-//   warp 1       TMEM allocator + MMA issuer (the whole warp runs the issue loop, one
-//                elected lane issues each burst)
-//   warps 2-5    B chain: T2 epilogue, X^T; also G^T, dbias and the dX epilogue
-//   warps 6-13   A chain: U1 and U2 epilogues, 2 warps per TMEM lane quadrant
+// Warp roles (480 threads, one CTA per SM, tiles of the CTA's row range in order):
+//   warp 0       TMA producer: an SI-deep ring of input sets (x and G tiles)
+//   warp 1       issuer A: T and U of tile t into TMEM (two accumulator slots); owns TMEM
+//   warp 2       issuer B: dC and dB of tile t from T2/U2 (an SB-deep ring in shared memory)
+//   warps 3-6    epilogue T -> T2 (one warp per TMEM lane quadrant)
+//   warps 7-10   epilogue U -> U2
+//   warps 11-14  dbias column sums of the G tiles
+// Issuers run their loops as whole warps and let one elected lane issue each burst; every
+// consumer takes the tiles in order, so no mbarrier phase can be mistaken for another.
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -39,7 +42,8 @@ namespace tc {
 
 int *device_error_ptr();
 cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
-                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw);
+                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw,
+                         bool atom32);
 
 namespace {
 
@@ -56,67 +60,70 @@ template <> struct BE<__nv_bfloat16> {
 };
 
 constexpr int imin(int a, int b) { return a < b ? a : b; }
+constexpr int kPgThreads = 480;
 
 template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
-struct BwdCfg {
+struct PgCfg {
     using T = T_;
     static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_;
     static constexpr int E = BE<T>::bytes;
-    static constexpr int NT = R;                   // rows per tile
-    static constexpr int SWC = imin(128, Q * E);   // K = c       (Ua, Ub)
-    static constexpr int SWJ = imin(128, M1 * E);  // K = j       (T)
-    static constexpr int SW128 = 128;              // K = (i,k), (n,k), (n,a): 128 * E bytes
-    static constexpr int SWG = M2 * E;             // G tile rows (k) and dC's B chunks
-    // region sizes (bytes)
-    static constexpr int F_C = 128 * Q * E;        // C    [(i,a)][c]
-    static constexpr int F_BT = 128 * M1 * E;      // Bt   [(i,k)][j]
-    static constexpr int F_BD = M1 * 128 * E;      // Bdx  [j][(i,k)]
-    static constexpr int TILE_G = 128 * M2 * E;    // G    [(n,c)][k]   (NT*Q rows)
-    static constexpr int TILE_X = 128 * M1 * E;    // X    [(n,a)][j]   (NT*P = 128 rows)
-    static constexpr int TILE_GT = 128 * Q * E;    // G^T  [(n,k)][c]
-    static constexpr int BUF = 128 * 128 * E;      // U1 | U2 (A), T2 | X^T (B)
-    static constexpr int OFF_C = 0;
-    static constexpr int OFF_BT = OFF_C + F_C;
-    static constexpr int OFF_BD = OFF_BT + F_BT;
-    static constexpr int OFF_G = OFF_BD + F_BD;
-    static constexpr int OFF_X = OFF_G + NT * Q * M2 * E;
-    static constexpr int OFF_GT = OFF_X + TILE_X;
-    static constexpr int OFF_A = OFF_GT + TILE_GT;
-    static constexpr int OFF_B = OFF_A + BUF;
-    static constexpr int OFF_BAR = OFF_B + BUF;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static constexpr bool TWO = BE<T>::tf32;       // TF32: inputs in two layouts
+    static constexpr int NT = 2;                   // rows per tile
+    static constexpr int XR = NT * P, GR = NT * Q; // tile rows: (n,a) and (n,c)
+    static constexpr int XRB = M1 * E, GRB = M2 * E;  // tile row bytes = their swizzle width
+    static constexpr int X_BYTES = XR * XRB, G_BYTES = GR * GRB;
+    // one input set: x (K-major), G (K-major) [, x MN-major, G MN-major]
+    static constexpr int OFF_XK = 0, OFF_GK = X_BYTES;
+    static constexpr int OFF_XM = TWO ? X_BYTES + G_BYTES : OFF_XK;
+    static constexpr int OFF_GM = TWO ? 2 * X_BYTES + G_BYTES : OFF_GK;
+    static constexpr int IN_BYTES = (X_BYTES + G_BYTES) * (TWO ? 2 : 1);
+    // intermediates: T2 [(i,a)][(n,k)] and U2 [(i,k)][(n,a)], 128 rows, K-major, SW128
+    static constexpr int T2K = NT * M2, U2K = NT * P;          // K extents (elements)
+    static constexpr int T2_BYTES = 128 * T2K * E, U2_BYTES = 128 * U2K * E;
+    static constexpr int IB = T2_BYTES + U2_BYTES;
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM_MAX = 232448;
+    static constexpr int FREE = SMEM_MAX - 1024 - BAR_BYTES;
+    static constexpr int SB = FREE - 4 * IB >= 4 * IN_BYTES ? 4 : FREE - 3 * IB >= 3 * IN_BYTES ? 3 : 2;
+    static constexpr int SI = imin(4, (FREE - SB * IB) / IN_BYTES);
+    static constexpr int OFF_IN = 0;
+    static constexpr int OFF_I = SI * IN_BYTES;
+    static constexpr int OFF_BAR = OFF_I + SB * IB;
+    static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
     // TMEM columns
-    static constexpr int TM_UA = 0;              // Ua : lanes (i,a), 128 columns (n,k)
-    static constexpr int TM_UB = 128;            // Ub : lanes (n,k), 128 columns (i,a)
-    static constexpr int TM_T = 256;             // T  : lanes (n,a), 128 columns (i,k)
-    static constexpr int TM_DX = 384;            // dX : lanes (n,a), M1 columns (j)
-    static constexpr int TM_DC = TM_DX + M1;     // dC : lanes (i,a), Q columns (c)
-    static constexpr int TM_DB = TM_DC + Q;      // dB : lanes (i,k), M1 columns (j)
+    static constexpr int TM_BT = 0;                          // B_all^T: lanes (i,k), K = j
+    static constexpr int TM_C = TM_BT + M1 * E / 4;          // C_stack: lanes (i,a), K = c
+    static constexpr int TM_DT = TM_C + Q * E / 4;           // T: 2 slots of XR columns
+    static constexpr int TM_DU = TM_DT + 2 * XR;             // U: 2 slots of NT*M2 columns
+    static constexpr int TM_DC = TM_DU + 2 * NT * M2;        // dC: lanes (i,a), Q columns
+    static constexpr int TM_DB = TM_DC + Q;                  // dB: lanes (i,k), M1 columns
     static constexpr int TM_USED = TM_DB + M1;
     static constexpr int TM_COLS = 512;
-    static constexpr uint32_t ID_128 = idesc_f32acc(128, 128, BE<T>::fmt);
-    static constexpr uint32_t ID_M1 = idesc_f32acc(128, M1, BE<T>::fmt);
-    static constexpr uint32_t ID_Q = idesc_f32acc(128, Q, BE<T>::fmt);
+    static constexpr uint32_t ID_T = idesc_f32acc(128, XR, BE<T>::fmt);
+    static constexpr uint32_t ID_U = idesc_f32acc(128, NT * M2, BE<T>::fmt) | kBMajorMN;
+    static constexpr uint32_t ID_DC = idesc_f32acc(128, Q, BE<T>::fmt);
+    static constexpr uint32_t ID_DB = idesc_f32acc(128, M1, BE<T>::fmt) | kBMajorMN;
+    // MN-major layouts of the input tiles: TF32 128-byte rows with 32-byte atoms (4-row
+    // groups), BF16 the tile's own swizzle (8-row groups); both put 1 KB per 32-byte K step
+    static constexpr uint32_t MN_LAYOUT = TWO ? kLayoutSw128Atom32 : layout_type(XRB);
+    static constexpr uint32_t MN_SBO = TWO ? 4 * 128 : 8 * XRB;
 
-    static_assert(R * P == 128 && R * M2 == 128, "needs p = m2 = 128 / r");
-    static_assert(M2 % 32 == 0 && P % 32 == 0, "a 32-column TMEM chunk maps to one operand row");
-    static_assert(NT * Q <= 256 && (NT * Q) % 8 == 0, "G tile rows (TMA box) at most 256");
-    static_assert(M2 * E <= 128 && P * E <= 128 && M1 * E <= 128,
-                  "a block of m2 (p, m1) values must fit one 128-byte swizzle row");
-    static_assert(SWG == 32 || SWG == 64 || SWG == 128, "G tile swizzle");
-    static_assert(M1 % 32 == 0 && Q % 32 == 0 && M1 <= 64 && Q <= 64, "m1, q in {32, 64}");
-    static_assert((M1 * E) % 32 == 0 && (M1 * E <= 128 || M1 * E % 128 == 0), "m1 bytes");
-    static_assert((Q * E) % 32 == 0 && (Q * E <= 128 || Q * E % 128 == 0), "q bytes");
+    static_assert(R * P == 128 && R * M2 == 128, "T2/U2 rows and the U/T accumulators: M = 128");
+    static_assert(XR % 32 == 0 && XR <= 256 && (NT * M2) % 32 == 0 && NT * M2 <= 256, "N of T and U");
+    static_assert(XRB == GRB && (XRB == 128 || (!TWO && XRB == 64)),
+                  "tile rows of 128 bytes (TF32) or 64/128 bytes (BF16)");
+    static_assert(Q % 32 == 0 && M1 % 32 == 0 && Q <= 256 && M1 <= 256, "N of dC and dB");
+    static_assert((T2K * E) % 128 == 0 && (U2K * E) % 128 == 0, "T2/U2 rows: whole 128-byte chunks");
+    static_assert(P == 32 && M2 == 32, "epilogue: one 32-column TMEM load per (n, block)");
+    static_assert(SI >= 2 && SB >= 2, "rings");
     static_assert(TM_USED <= TM_COLS, "TMEM budget");
-    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
 
-struct BwdTcArgs {
+struct PgArgs {
     const void *S, *A, *B;
-    void *dX;
     float *ws;
     size_t ws_stride;
-    int64_t N;
     int num_tiles;
     int tiles_per_part;
     int *device_error;
@@ -128,8 +135,8 @@ __device__ __forceinline__ float bld(const void *p, size_t i) {
     else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
 }
 
-// (row, kbyte) of a K-major swizzled operand region: K in chunks of sw bytes
-// (chunk-major), rows in 8-row atoms of 8*sw bytes.
+// Byte offset of element (row, kbyte) of a K-major swizzled operand region: K in chunks of
+// sw bytes (chunk-major), rows in 8-row atoms of 8*sw bytes.
 __device__ __forceinline__ uint32_t koff(int row, int kbyte, int rows, int sw) {
     const int chunk = kbyte / sw, inner = kbyte % sw;
     return swz((uint32_t)chunk * rows * sw + (uint32_t)(row >> 3) * 8 * sw +
@@ -137,154 +144,94 @@ __device__ __forceinline__ uint32_t koff(int row, int kbyte, int rows, int sw) {
                sw);
 }
 
+// One accumulator value as an operand element of a K-major region (fp32 bits for TF32: the
+// MMA reads the top 19 bits of each operand).
 template <typename T>
-__device__ __forceinline__ void st16v(uint32_t addr, const float *v) {
-    if constexpr (BE<T>::tf32) {
-        st_shared_v4(addr, f32_to_tf32(v[0]), f32_to_tf32(v[1]), f32_to_tf32(v[2]),
-                     f32_to_tf32(v[3]));
-    } else {
-        st_shared_v4(addr, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-    }
-}
-
-// TMEM (32 columns of this thread's lane) -> one operand row of a 128B-swizzled K-major
-// region: the 32 values go to K bytes [kbyte0, kbyte0 + 32*E) of row `row` (kbyte0
-// 16-byte aligned, the run stays inside one 128-byte K-chunk).
-template <typename T>
-__device__ __forceinline__ void tmem_row_to_smem(uint32_t taddr, uint32_t region, int rows,
-                                                 int row, int kbyte0) {
-    constexpr int VPC = 16 / BE<T>::bytes;
-    uint32_t r[32];
-    tmem_load32(taddr, r);
-    const uint32_t base = sw128_row(region, rows, kbyte0 >> 7, row);
-    const int slot0 = (kbyte0 & 127) >> 4, x = row & 7;
-#pragma unroll
-    for (int g = 0; g < 32 / VPC; ++g) {
-        const uint32_t addr = base + (uint32_t)(((slot0 + g) ^ x) << 4);
-        if constexpr (BE<T>::tf32) {
-            // fp32 bits as they are: the TF32 MMA reads the top 19 bits of each operand
-            st_shared_v4(addr, r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-        } else {
-            st_shared_v4(addr, pack_bf16x2(__uint_as_float(r[8 * g]), __uint_as_float(r[8 * g + 1])),
-                         pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3])),
-                         pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5])),
-                         pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7])));
-        }
-    }
-}
-
-// Transpose of 8 source rows x 16 bytes (VPC elements) held as in[8][4] words into VPC
-// output rows of 8 elements each: out row e = (in[0][e], ..., in[7][e]).  The
-// elements are copied as they are (fp32 bits for TF32: the MMA reads the top 19 bits,
-// as it does for the tiles TMA brings in).
-template <typename T>
-__device__ __forceinline__ void store_transposed(const uint32_t (&in)[8][4], int e,
-                                                 uint32_t addr_lo, uint32_t addr_hi) {
-    if constexpr (BE<T>::tf32) {
-        st_shared_v4(addr_lo, in[0][e], in[1][e], in[2][e], in[3][e]);
-        st_shared_v4(addr_hi, in[4][e], in[5][e], in[6][e], in[7][e]);
-    } else {
-        const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
-        const int w = e >> 1;
-        st_shared_v4(addr_lo, __byte_perm(in[0][w], in[1][w], sel), __byte_perm(in[2][w], in[3][w], sel),
-                     __byte_perm(in[4][w], in[5][w], sel), __byte_perm(in[6][w], in[7][w], sel));
-    }
+__device__ __forceinline__ void st_elem(uint32_t addr, uint32_t v) {
+    if constexpr (BE<T>::tf32) st_shared_u32(addr, v);
+    else st_shared_u16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v))));
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(448, 1)
-kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
-                   const __grid_constant__ CUtensorMap tmap_x, BwdTcArgs args) {
+__global__ void __launch_bounds__(kPgThreads, 1)
+kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_constant__ CUtensorMap tm_gk,
+                     const __grid_constant__ CUtensorMap tm_xm, const __grid_constant__ CUtensorMap tm_gm,
+                     PgArgs args) {
     using T = typename Cfg::T;
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
-    constexpr int NT = Cfg::NT;
-    constexpr int VPC = 16 / E;
+    constexpr int NT = Cfg::NT, XR = Cfg::XR, GR = Cfg::GR, SI = Cfg::SI, SB = Cfg::SB;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
-    const uint32_t sC = sb + Cfg::OFF_C, sBT = sb + Cfg::OFF_BT, sBD = sb + Cfg::OFF_BD;
-    const uint32_t sG = sb + Cfg::OFF_G, sX = sb + Cfg::OFF_X, sGT = sb + Cfg::OFF_GT;
-    const uint32_t sA = sb + Cfg::OFF_A, sBb = sb + Cfg::OFF_B;
+    const uint32_t sIn = sb + Cfg::OFF_IN, sI = sb + Cfg::OFF_I;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-    enum {
-        G_FULL, X_FULL,   // TMA landed
-        G_FREE,           // dC done with G and G^T/dbias read it (transposer arrives after X^T)
-        X_FREE,           // T done with X and X^T written
-        GT_FULL,          // G^T written
-        UT_FULL,          // Ua, Ub, T accumulators ready; G^T consumed
-        E1A_DONE,         // U1 written (buffer A)
-        E1B_DONE,         // T2 written (buffer B)
-        DX_FULL,          // dX accumulator ready; U1 consumed (buffer A free)
-        DX_FREE,          // dX accumulator read out
-        DC_DONE,          // dC MMAs done: T2 consumed (buffer B free), G consumed
-        U2_DONE,          // U2 written; Ua, Ub, T accumulators fully read out
-        XT_DONE,          // X^T written
-        DB_DONE,          // dB MMAs done: buffers A and B free
-        DRAIN,
-        NBARS
-    };
+    // barrier indices
+    constexpr int IN_FULL = 0, IN_FREE = SI, D_FULL = 2 * SI, D_EMPTY = 2 * SI + 2,
+                  I_FULL = 2 * SI + 4, I_EMPTY = I_FULL + SB, DONE = I_FULL + 2 * SB,
+                  DRAIN = DONE + 1, NBARS = DRAIN + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
     const Abort ab{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-    // ---------------- set-up ----------------
+    // ---------------- set-up: barriers, TMEM, factors into TMEM ----------------
     if (threadIdx.x == 0) {
-        mbar_init(bar(G_FULL), 1);
-        mbar_init(bar(X_FULL), 1);
-        mbar_init(bar(G_FREE), 1 + 4);   // dC commit + B-chain warps
-        mbar_init(bar(X_FREE), 1 + 4);
-        mbar_init(bar(GT_FULL), 4);
-        mbar_init(bar(UT_FULL), 1);
-        mbar_init(bar(E1A_DONE), 8);     // A-chain warps
-        mbar_init(bar(E1B_DONE), 4);
-        mbar_init(bar(DX_FULL), 1);
-        mbar_init(bar(DX_FREE), 4);
-        mbar_init(bar(DC_DONE), 1);
-        mbar_init(bar(U2_DONE), 8);
-        mbar_init(bar(XT_DONE), 4);
-        mbar_init(bar(DB_DONE), 1);
+        for (int s = 0; s < SI; ++s) {
+            mbar_init(bar(IN_FULL + s), 1);
+            mbar_init(bar(IN_FREE + s), 1 + 1 + 4);  // issuer A, issuer B, dbias warps
+        }
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(bar(D_FULL + d), 1);
+            mbar_init(bar(D_EMPTY + d), 8);          // both epilogues
+        }
+        for (int b = 0; b < SB; ++b) {
+            mbar_init(bar(I_FULL + b), 8);
+            mbar_init(bar(I_EMPTY + b), 1);
+        }
+        mbar_init(bar(DONE), 1);
         mbar_init(bar(DRAIN), 1);
         *ab.flag = 0;
         mbar_init_fence();
-        prefetch_tmap(&tmap_g);
-        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tm_xk);
+        prefetch_tmap(&tm_gk);
+        if (Cfg::TWO) {
+            prefetch_tmap(&tm_xm);
+            prefetch_tmap(&tm_gm);
+        }
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
-    // factors: C[(i,a)][c] = S[a][c] A_i[a][c]; Bt[(i,k)][j] = B_i[j][k]; Bdx[j][(i,k)] = B_i[j][k]
-    for (int e = threadIdx.x; e < 128 * (Q / VPC); e += blockDim.x) {
-        const int row = e / (Q / VPC), c0 = (e % (Q / VPC)) * VPC;
-        const int i = row / P, a = row % P;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t)
-            v[t] = bld<T>(args.S, (size_t)a * Q + c0 + t) * bld<T>(args.A, ((size_t)i * P + a) * Q + c0 + t);
-        st16v<T>(sC + koff(row, c0 * E, 128, Cfg::SWC), v);
-    }
-    for (int e = threadIdx.x; e < 128 * (M1 / VPC); e += blockDim.x) {
-        const int row = e / (M1 / VPC), j0 = (e % (M1 / VPC)) * VPC;
-        const int i = row / M2, k = row % M2;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) v[t] = bld<T>(args.B, ((size_t)i * M1 + j0 + t) * M2 + k);
-        st16v<T>(sBT + koff(row, j0 * E, 128, Cfg::SWJ), v);
-    }
-    for (int e = threadIdx.x; e < M1 * (128 / VPC); e += blockDim.x) {
-        const int j = e / (128 / VPC), ik0 = (e % (128 / VPC)) * VPC;
-        const int i = ik0 / M2, k0 = ik0 % M2;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) v[t] = bld<T>(args.B, ((size_t)i * M1 + j) * M2 + k0 + t);
-        st16v<T>(sBD + koff(j, ik0 * E, M1, Cfg::SW128), v);
-    }
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // A operands in TMEM, one lane per row (two BF16 values per column):
+    //   B_all^T: lane (i,k), column j -> B_i[j][k];   C_stack: lane (i,a), column c -> C_i[a][c]
+    if (warp >= 3 && warp < 11) {
+        const int qd = warp & 3, L = qd * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+        const bool is_c = warp >= 7;
+        const int i = is_c ? L / P : L / M2, o = is_c ? L % P : L % M2;  // o = a or k
+        const int K = is_c ? Q : M1;
+        auto val = [&](int j) {
+            return is_c ? bld<T>(args.S, (size_t)o * Q + j) * bld<T>(args.A, ((size_t)i * P + o) * Q + j)
+                        : bld<T>(args.B, ((size_t)i * M1 + j) * M2 + o);
+        };
+        const uint32_t base = tmem + lane_addr + (is_c ? Cfg::TM_C : Cfg::TM_BT);
+        for (int c0 = 0; c0 < K * E / 4; c0 += 8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if constexpr (BE<T>::tf32) w[u] = f32_to_tf32(val(c0 + u));
+                else w[u] = pack_bf16x2(val(2 * (c0 + u)), val(2 * (c0 + u) + 1));
+            }
+            tmem_store8(base + c0, w);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     const int t0 = blockIdx.x * args.tiles_per_part;
     const int t1 = imin(t0 + args.tiles_per_part, args.num_tiles);
@@ -295,307 +242,184 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
         if (lane == 0) {
             int issued = 0;
             for (int u = 0; u < nt; ++u) {
-                const uint32_t ph = u & 1;
+                const int s = u % SI;
+                if (!mbar_wait(bar(IN_FREE + s), ((u / SI) & 1) ^ 1, ab)) break;
+                const uint32_t dst = sIn + s * Cfg::IN_BYTES;
                 const int tile = t0 + u;
-                if (!mbar_wait(bar(G_FREE), ph ^ 1, ab)) break;
-                mbar_arrive_expect_tx(bar(G_FULL), NT * Q * M2 * E);
-                tma_load_2d(sG, &tmap_g, 0, tile * NT * Q, bar(G_FULL));
-                if (!mbar_wait(bar(X_FREE), ph ^ 1, ab)) break;
-                mbar_arrive_expect_tx(bar(X_FULL), Cfg::TILE_X);
-                tma_load_2d(sX, &tmap_x, 0, tile * NT * P, bar(X_FULL));
+                mbar_arrive_expect_tx(bar(IN_FULL + s), Cfg::IN_BYTES);
+                tma_load_2d(dst + Cfg::OFF_XK, &tm_xk, 0, tile * XR, bar(IN_FULL + s));
+                tma_load_2d(dst + Cfg::OFF_GK, &tm_gk, 0, tile * GR, bar(IN_FULL + s));
+                if (Cfg::TWO) {
+                    tma_load_2d(dst + Cfg::OFF_XM, &tm_xm, 0, tile * XR, bar(IN_FULL + s));
+                    tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * GR, bar(IN_FULL + s));
+                }
                 issued = u + 1;
             }
-            if (issued > 0) {
-                mbar_wait_drain(bar(G_FULL), (issued - 1) & 1);
-                mbar_wait_drain(bar(X_FULL), (issued - 1) & 1);
-            }
+            for (int u = (issued > SI ? issued - SI : 0); u < issued; ++u)
+                mbar_wait_drain(bar(IN_FULL + u % SI), (u / SI) & 1);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
-        auto mma = [&](uint32_t d, uint32_t a, int swa, uint32_t b, int swb, uint32_t id, uint32_t acc) {
-            mma_ss<BE<T>::tf32>(d, sdesc_kmajor(a, swa), sdesc_kmajor(b, swb), id, acc);
-        };
-        // Ua, Ub and T of the current tile
-        auto issue_ut = [&]() {
-            if (elect_one()) {
-#pragma unroll
-                for (int kb = 0; kb < Q * E; kb += 32) {
-                    const int ch = kb / Cfg::SWC, in = kb % Cfg::SWC;
-                    mma(tmem + Cfg::TM_UA, sC + ch * 128 * Cfg::SWC + in, Cfg::SWC,
-                        sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC, Cfg::ID_128, kb > 0);
-                    mma(tmem + Cfg::TM_UB, sGT + ch * 128 * Cfg::SWC + in, Cfg::SWC,
-                        sC + ch * 128 * Cfg::SWC + in, Cfg::SWC, Cfg::ID_128, kb > 0);
-                }
-#pragma unroll
-                for (int kb = 0; kb < M1 * E; kb += 32) {
-                    const int ch = kb / Cfg::SWJ, in = kb % Cfg::SWJ;
-                    mma(tmem + Cfg::TM_T, sX + ch * 128 * Cfg::SWJ + in, Cfg::SWJ,
-                        sBT + ch * 128 * Cfg::SWJ + in, Cfg::SWJ, Cfg::ID_128, kb > 0);
-                }
-                mma_commit(bar(UT_FULL));
-                mma_commit(bar(X_FREE));
-            }
-            __syncwarp();
-        };
-        bool ok = true;
-        if (nt > 0) {
-            ok = warp_wait(bar(X_FULL), 0, ab) && warp_wait(bar(GT_FULL), 0, ab);
-            if (ok) {
-                tc_fence_after();
-                issue_ut();
-            }
-        }
-        for (int u = 0; u < nt && ok; ++u) {
-            const uint32_t ph = u & 1;
-            // dX(u) = U1 . Bdx^T  (K = (i,k)); dC(u) += T2 . G^T (K = (n,k))
-            if (!warp_wait(bar(E1A_DONE), ph, ab) || !warp_wait(bar(DX_FREE), ph ^ 1, ab)) break;
+        // ---------------- issuer A: T and U of each tile ----------------
+        for (int u = 0; u < nt; ++u) {
+            const int s = u % SI, d = u & 1;
+            if (!warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab) ||
+                !warp_wait(bar(D_EMPTY + d), ((u >> 1) & 1) ^ 1, ab))
+                break;
             tc_fence_after();
             if (elect_one()) {
+                const uint32_t in = sIn + s * Cfg::IN_BYTES;
 #pragma unroll
-                for (int kb = 0; kb < 128 * E; kb += 32) {
-                    const int ch = kb / 128, in = kb % 128;
-                    mma(tmem + Cfg::TM_DX, sA + ch * 128 * 128 + in, 128, sBD + ch * M1 * 128 + in, 128,
-                        Cfg::ID_M1, kb > 0);
-                }
-                mma_commit(bar(DX_FULL));
+                for (int kk = 0; kk < M1 * E / 32; ++kk)   // T[(i,k)][(n,a)], K = j
+                    mma_ts<BE<T>::tf32>(tmem + Cfg::TM_DT + d * XR, tmem + Cfg::TM_BT + kk * 8,
+                                        sdesc_kmajor(in + Cfg::OFF_XK + kk * 32, Cfg::XRB), Cfg::ID_T,
+                                        kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < Q * E / 32; ++kk)    // U[(i,a)][(n,k)], K = c, G MN-major
+                    mma_ts<BE<T>::tf32>(tmem + Cfg::TM_DU + d * NT * M2, tmem + Cfg::TM_C + kk * 8,
+                                        sdesc_mn(in + Cfg::OFF_GM + kk * 1024, Cfg::MN_LAYOUT,
+                                                 Q * Cfg::GRB, Cfg::MN_SBO),
+                                        Cfg::ID_U, kk > 0);
+                mma_commit(bar(D_FULL + d));
+                mma_commit(bar(IN_FREE + s));
             }
             __syncwarp();
-            if (!warp_wait(bar(E1B_DONE), ph, ab)) break;
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int kb = 0; kb < 128 * E; kb += 32) {
-                    const int ch = kb / 128, in = kb % 128;                // T2: 128-byte chunks
-                    const int chg = kb / Cfg::SWG, ing = kb % Cfg::SWG;    // G: one chunk per n
-                    mma(tmem + Cfg::TM_DC, sBb + ch * 128 * 128 + in, 128,
-                        sG + chg * Q * Cfg::SWG + ing, Cfg::SWG, Cfg::ID_Q, (u > 0 || kb > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(DC_DONE));
-                mma_commit(bar(G_FREE));
-            }
-            __syncwarp();
-            // dB(u) += U2 . X^T^T (K = (n,a)) once U2 and X^T are written
-            if (!warp_wait(bar(U2_DONE), ph, ab) || !warp_wait(bar(XT_DONE), ph, ab)) break;
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int kb = 0; kb < 128 * E; kb += 32) {
-                    const int ch = kb / 128, in = kb % 128;
-                    mma(tmem + Cfg::TM_DB, sA + ch * 128 * 128 + in, 128, sBb + ch * M1 * 128 + in, 128,
-                        Cfg::ID_M1, (u > 0 || kb > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(DB_DONE));
-            }
-            __syncwarp();
-            // Ua, Ub, T of tile u+1 (their accumulators were read out before U2_DONE(u))
-            if (u + 1 < nt) {
-                if (!warp_wait(bar(X_FULL), ph ^ 1, ab) || !warp_wait(bar(GT_FULL), ph ^ 1, ab)) break;
-                tc_fence_after();
-                issue_ut();
-            }
         }
         if (elect_one()) mma_commit(bar(DRAIN));
         __syncwarp();
         if (lane == 0) mbar_wait_drain(bar(DRAIN), 0);
         __syncwarp();
-    } else if (warp < 6) {
-        // ---------------- B chain (128 threads) ----------------
-        const int tid = threadIdx.x - 64;
-        const int quad = warp & 3;
-        const int L = quad * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        float dbias[Q * M2 / 128];
-#pragma unroll
-        for (int e = 0; e < Q * M2 / 128; ++e) dbias[e] = 0.f;
+    } else if (warp == 2) {
+        // ---------------- issuer B: dC and dB of each tile ----------------
         for (int u = 0; u < nt; ++u) {
-            const uint32_t ph = u & 1;
-            const int64_t row0 = (int64_t)(t0 + u) * NT;
-            // G^T(u) [(n,k)][c] from G(u) [(n,c)][k] (8-row register blocks), dbias partial.
-            // G^T(u-1) was consumed by the U MMAs of tile u-1 (UT_FULL(u-1) preceded E1B(u-1)).
-            if (!mbar_wait(bar(G_FULL), ph, ab)) break;
-            for (int blk = tid; blk < NT * (Q / 8) * (M2 / VPC); blk += 128) {
-                const int kb = blk % (M2 / VPC), cb = (blk / (M2 / VPC)) % (Q / 8), n = blk / ((M2 / VPC) * (Q / 8));
-                uint32_t in[8][4];
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    ld_shared_v4(sG + koff(n * Q + cb * 8 + t, kb * 16, NT * Q, Cfg::SWG), in[t]);
-#pragma unroll
-                for (int e = 0; e < VPC; ++e) {
-                    const int row = n * M2 + kb * VPC + e;
-                    const uint32_t lo = sGT + koff(row, cb * 8 * E, 128, Cfg::SWC);
-                    store_transposed<T>(in, e, lo, lo ^ 16u);
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < Q * M2 / 128; ++e) {
-                const int o = tid + 128 * e, c = o / M2, k = o % M2;
-                float sacc = 0.f;
-                for (int n = 0; n < NT; ++n) {
-                    if (row0 + n < args.N) {
-                        const uint32_t a = sG + koff(n * Q + c, k * E, NT * Q, Cfg::SWG);
-                        if constexpr (BE<T>::tf32) {
-                            float v;
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-                            sacc += v;
-                        } else {
-                            unsigned short h;
-                            asm volatile("ld.shared.b16 %0, [%1];" : "=h"(h) : "r"(a) : "memory");
-                            sacc += __bfloat162float(*reinterpret_cast<__nv_bfloat16 *>(&h));
-                        }
-                    }
-                }
-                dbias[e] += sacc;
-            }
-            fence_proxy_async();
-            mbar_arrive_warp(bar(GT_FULL));
-            // T2(u) [(i,a)][(n,k)] <- T accumulator (lanes (n,a), columns (i,k)) into buffer B,
-            // once dB(u-1) has consumed X^T(u-1)
-            if (!mbar_wait(bar(UT_FULL), ph, ab) || !mbar_wait(bar(DB_DONE), ph ^ 1, ab)) break;
+            const int s = u % SI, b = u % SB;
+            if (!warp_wait(bar(I_FULL + b), (u / SB) & 1, ab) ||
+                !warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab))
+                break;
             tc_fence_after();
-            {
-                const int n = L / P, a = L % P;
+            if (elect_one()) {
+                const uint32_t in = sIn + s * Cfg::IN_BYTES;
+                const uint32_t t2 = sI + b * Cfg::IB, u2 = t2 + Cfg::T2_BYTES;
 #pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {   // columns (i,k): i = c0 / M2
-                    const int i = c0 / M2, k0 = c0 % M2;
-                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_T + c0, sBb, 128, i * P + a,
-                                        (n * M2 + k0) * E);
+                for (int kk = 0; kk < Cfg::T2K * E / 32; ++kk) {   // dC, K = (n,k)
+                    const int kb = kk * 32, n = kb / Cfg::GRB, ing = kb % Cfg::GRB;
+                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DC,
+                                        sdesc_kmajor(t2 + (kb / 128) * 128 * 128 + kb % 128, 128),
+                                        sdesc_kmajor(in + Cfg::OFF_GK + n * Q * Cfg::GRB + ing, Cfg::GRB),
+                                        Cfg::ID_DC, (u > 0 || kk > 0) ? 1u : 0u);
                 }
-            }
-            tc_fence_before();
-            fence_proxy_async();
-            mbar_arrive_warp(bar(E1B_DONE));
-            // dX(u): lanes (n,a), columns j -> dx[row0 + n][a*m1 + j] (16-byte stores)
-            if (!mbar_wait(bar(DX_FULL), ph, ab)) break;
-            tc_fence_after();
-            {
-                const int n = L / P, a = L % P;
-                const int64_t row = row0 + n;
 #pragma unroll
-                for (int j0 = 0; j0 < M1; j0 += 32) {
-                    uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_DX + j0, r);
-                    if (j0 + 32 >= M1) {
-                        tc_fence_before();
-                        mbar_arrive_warp(bar(DX_FREE));
-                    }
-                    if (args.dX && row < args.N) {
-                        if constexpr (BE<T>::tf32) {
-                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(args.dX) +
-                                                                     (size_t)row * (P * M1) + (size_t)a * M1 + j0);
-#pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4)
-                                dst[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
-                                                      __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
-                        } else {
-                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(args.dX) +
-                                                                   (size_t)row * (P * M1) + (size_t)a * M1 + j0);
-#pragma unroll
-                            for (int q8 = 0; q8 < 4; ++q8)
-                                dst[q8] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(r[8 * q8]), __uint_as_float(r[8 * q8 + 1])),
-                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 2]), __uint_as_float(r[8 * q8 + 3])),
-                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 4]), __uint_as_float(r[8 * q8 + 5])),
-                                    pack_bf16x2(__uint_as_float(r[8 * q8 + 6]), __uint_as_float(r[8 * q8 + 7])));
-                        }
-                    }
+                for (int kk = 0; kk < Cfg::U2K * E / 32; ++kk) {   // dB, K = (n,a), x MN-major
+                    const int kb = kk * 32;
+                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DB,
+                                        sdesc_kmajor(u2 + (kb / 128) * 128 * 128 + kb % 128, 128),
+                                        sdesc_mn(in + Cfg::OFF_XM + kk * 1024, Cfg::MN_LAYOUT,
+                                                 Cfg::X_BYTES, Cfg::MN_SBO),
+                                        Cfg::ID_DB, (u > 0 || kk > 0) ? 1u : 0u);
                 }
+                mma_commit(bar(I_EMPTY + b));
+                mma_commit(bar(IN_FREE + s));
             }
-            // X^T(u) [j][(n,a)] into buffer B once dC(u) has consumed T2(u)
-            if (!mbar_wait(bar(DC_DONE), ph, ab)) break;
-            for (int blk = tid; blk < NT * (P / 8) * (M1 / VPC); blk += 128) {
-                const int jb = blk % (M1 / VPC), ab8 = (blk / (M1 / VPC)) % (P / 8), n = blk / ((M1 / VPC) * (P / 8));
-                uint32_t in[8][4];
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    ld_shared_v4(sX + koff(n * P + ab8 * 8 + t, jb * 16, 128, Cfg::SWJ), in[t]);
-#pragma unroll
-                for (int e = 0; e < VPC; ++e) {
-                    const int j = jb * VPC + e;
-                    const uint32_t lo = sBb + koff(j, (n * P + ab8 * 8) * E, M1, 128);
-                    store_transposed<T>(in, e, lo, lo ^ 16u);
-                }
-            }
-            fence_proxy_async();
-            mbar_arrive_warp(bar(XT_DONE));
-            mbar_arrive_warp(bar(X_FREE));
-            mbar_arrive_warp(bar(G_FREE));
+            __syncwarp();
         }
-        const size_t off = (size_t)R * P * Q + (size_t)R * M1 * M2;
-        float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
-#pragma unroll
-        for (int e = 0; e < Q * M2 / 128; ++e) part[off + tid + 128 * e] = dbias[e];
-    } else {
-        // ---------------- A chain (256 threads) ----------------
-        const int half = (warp - 6) / 4;
-        const int quad = warp & 3;
-        const int L = quad * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        // every dC/dB MMA is complete before the epilogue reads the sums (and before TMEM goes)
+        if (elect_one()) mma_commit(bar(DONE));
+        __syncwarp();
+        if (lane == 0) mbar_wait_drain(bar(DONE), 0);
+        __syncwarp();
+    } else if (warp < 11) {
+        // ---------------- epilogues: T -> T2 (warps 3-6), U -> U2 (warps 7-10) ----------------
+        const bool is_u = warp >= 7;
+        const int qd = warp & 3, L = qd * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+        // T lane (i,k), columns (n,a) -> T2 row (i,a), K (n,k);
+        // U lane (i,a), columns (n,k) -> U2 row (i,k), K (n,a)
+        const int i = L / 32, o = L % 32;   // o = k (T) or a (U); p = m2 = 32
+        bool ok = true;
         for (int u = 0; u < nt; ++u) {
-            const uint32_t ph = u & 1;
-            // U1(u) [(n,a)][(i,k)] <- Ua (lanes (i,a), columns (n,k)) into buffer A, once
-            // dB(u-1) has consumed U2(u-1)
-            if (!mbar_wait(bar(UT_FULL), ph, ab) || !mbar_wait(bar(DB_DONE), ph ^ 1, ab)) break;
+            const int d = u & 1, b = u % SB;
+            if (!mbar_wait(bar(D_FULL + d), (u >> 1) & 1, ab)) { ok = false; break; }
             tc_fence_after();
-            {
-                const int i = L / P, a = L % P;
-#pragma unroll
-                for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {   // columns (n,k)
-                    const int n = c0 / M2, k0 = c0 % M2;
-                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_UA + c0, sA, 128, n * P + a,
-                                        (i * M2 + k0) * E);
-                }
-            }
+            uint32_t r[64];
+            const uint32_t src = tmem + lane_addr + (is_u ? Cfg::TM_DU + d * NT * M2 : Cfg::TM_DT + d * XR);
+            tmem_load32(src, *reinterpret_cast<uint32_t(*)[32]>(r));
+            tmem_load32(src + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
             tc_fence_before();
-            fence_proxy_async();
-            mbar_arrive_warp(bar(E1A_DONE));
-            // U2(u) [(i,k)][(n,a)] <- Ub (lanes (n,k), columns (i,a)) into buffer A, once
-            // dX(u) has consumed U1(u)
-            if (!mbar_wait(bar(DX_FULL), ph, ab)) break;
-            tc_fence_after();
-            {
-                const int n = L / M2, k = L % M2;
+            mbar_arrive_warp(bar(D_EMPTY + d));
+            if (!mbar_wait(bar(I_EMPTY + b), ((u / SB) & 1) ^ 1, ab)) { ok = false; break; }
+            const uint32_t dst = sI + b * Cfg::IB + (is_u ? Cfg::T2_BYTES : 0);
 #pragma unroll
-                for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {   // columns (i,a)
-                    const int i = c0 / P, a0 = c0 % P;
-                    tmem_row_to_smem<T>(tmem + lane_addr + Cfg::TM_UB + c0, sA, 128, i * M2 + k,
-                                        (n * P + a0) * E);
-                }
+            for (int c = 0; c < 64; ++c) {
+                const int n = c / 32, w = c % 32;   // column (n, w): w = a (T) or k (U)
+                const int row = i * 32 + w, kidx = n * 32 + o;
+                st_elem<T>(dst + koff(row, kidx * E, 128, 128), r[c]);
             }
-            tc_fence_before();
             fence_proxy_async();
-            mbar_arrive_warp(bar(U2_DONE));
+            mbar_arrive_warp(bar(I_FULL + b));
         }
-        // dC and dB partials of this row range, after the last dB MMAs
+        // this range's partial dC (T warps) or dB (U warps), after the last MMAs
         float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
-        if (nt > 0 && mbar_wait(bar(DB_DONE), (nt - 1) & 1, ab)) {
+        if (ok && nt > 0 && mbar_wait(bar(DONE), 0, ab)) {
             tc_fence_after();
-            if (half == 0) {   // dC: lanes (i,a), columns c -> dC_i[a][c] (16-byte stores)
-                const int i = L / P, a = L % P;
+            if (!is_u) {   // dC: lane (i,a), columns c -> dC_i[a][c]
                 for (int c0 = 0; c0 < Q; c0 += 32) {
                     uint32_t r[32];
                     tmem_load32(tmem + lane_addr + Cfg::TM_DC + c0, r);
-                    float4 *dst = reinterpret_cast<float4 *>(part + (size_t)i * P * Q + (size_t)a * Q + c0);
+                    float4 *dstp = reinterpret_cast<float4 *>(part + (size_t)i * P * Q + (size_t)o * Q + c0);
 #pragma unroll
                     for (int q4 = 0; q4 < 8; ++q4)
-                        dst[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
-                                              __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
+                        dstp[q4] = make_float4(__uint_as_float(r[4 * q4]), __uint_as_float(r[4 * q4 + 1]),
+                                               __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3]));
                 }
-            } else {           // dB: lanes (i,k), columns j -> dB_i[j][k]
-                const int i = L / M2, k = L % M2;
+            } else {       // dB: lane (i,k), columns j -> dB_i[j][k]
                 for (int j0 = 0; j0 < M1; j0 += 32) {
                     uint32_t r[32];
                     tmem_load32(tmem + lane_addr + Cfg::TM_DB + j0, r);
 #pragma unroll
                     for (int t = 0; t < 32; ++t)
-                        part[(size_t)R * P * Q + (size_t)i * M1 * M2 + (size_t)(j0 + t) * M2 + k] =
+                        part[(size_t)R * P * Q + (size_t)i * M1 * M2 + (size_t)(j0 + t) * M2 + o] =
                             __uint_as_float(r[t]);
                 }
             }
         } else if (nt == 0) {
-            for (int e = threadIdx.x - 192; e < R * P * Q + R * M1 * M2; e += 256) part[e] = 0.f;
+            const size_t n0 = is_u ? (size_t)R * P * Q : 0, n1 = is_u ? (size_t)R * (P * Q + M1 * M2) : (size_t)R * P * Q;
+            for (size_t e = n0 + (size_t)(threadIdx.x - (is_u ? 224 : 96)); e < n1; e += 128) part[e] = 0.f;
         }
+    } else {
+        // ---------------- dbias: column sums of the G tiles (zero rows past N come from TMA) ----------------
+        const int tid = threadIdx.x - 352;
+        constexpr int PER = Q * M2 / 128;
+        float acc[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+        for (int u = 0; u < nt; ++u) {
+            const int s = u % SI;
+            if (!mbar_wait(bar(IN_FULL + s), (u / SI) & 1, ab)) break;
+            const uint32_t g = sIn + s * Cfg::IN_BYTES + Cfg::OFF_GK;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) {
+                const int idx = tid + 128 * e, c = idx / M2, k = idx % M2;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const uint32_t a = g + koff(n * Q + c, k * E, GR, Cfg::GRB);
+                    if constexpr (BE<T>::tf32) {
+                        float v;
+                        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+                        acc[e] += v;
+                    } else {
+                        unsigned short h;
+                        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(h) : "r"(a) : "memory");
+                        acc[e] += __bfloat162float(__ushort_as_bfloat16(h));
+                    }
+                }
+            }
+            mbar_arrive_warp(bar(IN_FREE + s));
+        }
+        float *part = args.ws + (size_t)blockIdx.x * args.ws_stride + (size_t)R * (P * Q + M1 * M2);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) part[tid + 128 * e] = acc[e];
     }
 
+    // ---------------- teardown ----------------
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -605,55 +429,61 @@ kron_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_g,
 }
 
 template <class Cfg>
-cudaError_t launch_bwd(const void *x, const void *S, const void *A, const void *B, const void *dY,
-                       void *dX, float *ws, int parts, const Shape &s, cudaStream_t st) {
+cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void *B, const void *dY,
+                         float *ws, int parts, const Shape &s, cudaStream_t st) {
     using T = typename Cfg::T;
     const bool bf16 = !BE<T>::tf32;
-    CUtensorMap tg, tx;
-    launch_step() = "tensor map of dY";
-    cudaError_t e = make_tmap_2d(&tg, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2,
-                                 Cfg::NT * Cfg::Q, Cfg::M2 * Cfg::E);
-    if (e != cudaSuccess) return e;
+    CUtensorMap txk, tgk, txm, tgm;
     launch_step() = "tensor map of x";
-    e = make_tmap_2d(&tx, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::SWJ / Cfg::E,
-                     Cfg::NT * Cfg::P, Cfg::SWJ);
+    cudaError_t e = make_tmap_2d(&txk, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::M1, Cfg::XR,
+                                 Cfg::XRB, false);
     if (e != cudaSuccess) return e;
+    launch_step() = "tensor map of dY";
+    e = make_tmap_2d(&tgk, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GR, Cfg::GRB, false);
+    if (e != cudaSuccess) return e;
+    txm = txk;
+    tgm = tgk;
+    if (Cfg::TWO) {
+        launch_step() = "MN-major tensor map of x";
+        e = make_tmap_2d(&txm, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::M1, Cfg::XR, 128, true);
+        if (e != cudaSuccess) return e;
+        launch_step() = "MN-major tensor map of dY";
+        e = make_tmap_2d(&tgm, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GR, 128, true);
+        if (e != cudaSuccess) return e;
+    }
     launch_step() = "shared-memory attribute";
-    e = cudaFuncSetAttribute(kron_bwd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(kron_pgrad_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
     if (e != cudaSuccess) return e;
     launch_step() = "kernel launch";
-    BwdTcArgs a;
-    a.S = S; a.A = A; a.B = B; a.dX = dX; a.ws = ws;
+    PgArgs a;
+    a.S = S; a.A = A; a.B = B; a.ws = ws;
     a.ws_stride = partial_stride(s);
-    a.N = s.N;
     a.num_tiles = (int)((s.N + Cfg::NT - 1) / Cfg::NT);
     a.tiles_per_part = (a.num_tiles + parts - 1) / parts;
     a.device_error = device_error_ptr();
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)parts);
-        cfg.blockDim = dim3(448);
-        cfg.dynamicSmemBytes = Cfg::SMEM;
-        cfg.stream = st;
-        return cudaLaunchKernelEx(&cfg, kron_bwd_tc_kernel<Cfg>, tg, tx, a);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)parts);
+    cfg.blockDim = dim3(kPgThreads);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, kron_pgrad_tc_kernel<Cfg>, txk, tgk, txm, tgm, a);
 }
 
-using BwdFn = cudaError_t (*)(const void *, const void *, const void *, const void *,
-                              const void *, void *, float *, int, const Shape &, cudaStream_t);
-struct BwdEntry {
+using PgFn = cudaError_t (*)(const void *, const void *, const void *, const void *, const void *,
+                             float *, int, const Shape &, cudaStream_t);
+struct PgEntry {
     int p, q, m1, m2, r;
     bool bf16;
-    BwdFn fn;
+    PgFn fn;
 };
-const BwdEntry kBwdTable[] = {
-    {32, 32, 32, 32, 4, false, &launch_bwd<BwdCfg<32, 32, 32, 32, 4, float>>},
-    {32, 32, 32, 32, 4, true, &launch_bwd<BwdCfg<32, 32, 32, 32, 4, __nv_bfloat16>>},
+const PgEntry kPgTable[] = {
+    {32, 32, 32, 32, 4, false, &launch_pgrad<PgCfg<32, 32, 32, 32, 4, float>>},
+    {32, 32, 32, 32, 4, true, &launch_pgrad<PgCfg<32, 32, 32, 32, 4, __nv_bfloat16>>},
 };
 
-BwdFn find_bwd(const Shape &s, bool bf16) {
-    for (const auto &f : kBwdTable)
+PgFn find_pg(const Shape &s, bool bf16) {
+    for (const auto &f : kPgTable)
         if (f.p == s.p && f.q == s.q && f.m1 == s.m1 && f.m2 == s.m2 && f.r == s.r && f.bf16 == bf16)
             return f.fn;
     return nullptr;
@@ -662,16 +492,22 @@ BwdFn find_bwd(const Shape &s, bool bf16) {
 }  // namespace
 }  // namespace tc
 
-bool tc_backward_supported(const Shape &s, bool bf16) { return tc::find_bwd(s, bf16) != nullptr; }
+bool tc_backward_supported(const Shape &s, bool bf16) {
+    return tc::find_pg(s, bf16) != nullptr && tc_dx_supported(s, bf16);
+}
 
-int tc_backward_tile_rows(const Shape &s) { return s.r; }
+int tc_backward_tile_rows(const Shape &) { return 2; }
 
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,
                         bool bf16, cudaStream_t st) {
-    tc::BwdFn fn = tc::find_bwd(s, bf16);
+    tc::PgFn fn = tc::find_pg(s, bf16);
     if (!fn) return cudaErrorNotSupported;
-    return fn(x, S, A, B, dY, dX, ws, parts, s, st);
+    if (dX) {
+        const cudaError_t e = tc_dx(dY, S, A, B, dX, s, bf16, st);
+        if (e != cudaSuccess) return e;
+    }
+    return fn(x, S, A, B, dY, ws, parts, s, st);
 }
 
 }  // namespace kron

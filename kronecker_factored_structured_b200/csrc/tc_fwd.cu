@@ -144,7 +144,11 @@ __device__ __forceinline__ void st16(uint32_t addr, const float *v) {
     }
 }
 
-template <class Cfg>
+// TR = false: the layer's forward, y = x W + bias.
+// TR = true:  dX = dY W^T, the same vec trick with C_i^T and B_i^T (dX_n = sum_i C_i G_n B_i^T):
+//             the kernel's (p, q, m1, m2) are the layer's (q, p, m2, m1), x is dY, y is dX,
+//             and the factors are read transposed while they are packed.
+template <class Cfg, bool TR>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     using T = typename Cfg::T;
@@ -203,7 +207,10 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
 #pragma unroll
         for (int t = 0; t < VPC; ++t) {
             const int ia = ia0 + t, i = ia / P, a = ia % P;
-            v[t] = ldf<T>(args.S, (size_t)a * Q + c) * ldf<T>(args.A, ((size_t)i * P + a) * Q + c);
+            // C'_i[a][c] = S[a][c] A_i[a][c]; transposed: the layer's C_i[c][a] (S is q' x p')
+            const size_t sa = TR ? (size_t)c * P + a : (size_t)a * Q + c;
+            const size_t aa = TR ? ((size_t)i * Q + c) * P + a : ((size_t)i * P + a) * Q + c;
+            v[t] = ldf<T>(args.S, sa) * ldf<T>(args.A, aa);
         }
         st16<T>(sB2 + kmajor_off(c, ia0 * E, Q, Cfg::SW2), v);
     }
@@ -221,12 +228,15 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             uint32_t w[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
+                // B'_i[j][k]; transposed: the layer's B_i[k][j] (B_i is m2' x m1')
+                auto bidx = [&](int j) {
+                    return TR ? ((size_t)i * M2 + k) * M1 + j : ((size_t)i * M1 + j) * M2 + k;
+                };
                 if constexpr (Elt<T>::tf32) {
-                    w[u] = f32_to_tf32(ldf<T>(args.B, ((size_t)i * M1 + c0 + u) * M2 + k));
+                    w[u] = f32_to_tf32(ldf<T>(args.B, bidx(c0 + u)));
                 } else {
                     const int j = 2 * (c0 + u);
-                    w[u] = pack_bf16x2(ldf<T>(args.B, ((size_t)i * M1 + j) * M2 + k),
-                                       ldf<T>(args.B, ((size_t)i * M1 + j + 1) * M2 + k));
+                    w[u] = pack_bf16x2(ldf<T>(args.B, bidx(j)), ldf<T>(args.B, bidx(j + 1)));
                 }
             }
             tmem_store8(ta + c0, w);
@@ -410,9 +420,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 2-D tensor map of a row-major [rows][cols] matrix, box = box_cols x box_rows, swizzled.
+// 2-D tensor map of a row-major [rows][cols] matrix, box = box_cols x box_rows, swizzled
+// by sw bytes (128, 64, 32 or 0); atom32 selects the 128-byte swizzle with 32-byte atoms
+// (the shared-memory layout of MN-major TF32 MMA operands).
 cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
-                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw) {
+                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw,
+                         bool atom32) {
     auto enc = get_encode();
     if (!enc) return cudaErrorNotSupported;
     // The encoder is a driver-API call: make the current device's primary context current
@@ -426,7 +439,8 @@ cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t
     cuuint64_t strides[1] = {cols * E};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUtensorMapSwizzle swm = sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+    CUtensorMapSwizzle swm = atom32      ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                           : sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                            : sw == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
                            : sw == 32  ? CU_TENSOR_MAP_SWIZZLE_32B
                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -456,7 +470,7 @@ int num_sms() {
     return n > 0 ? n : 148;
 }
 
-template <class Cfg>
+template <class Cfg, bool TR>
 cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *B,
                        const void *bias, void *y, const Shape &s, cudaStream_t st) {
     using T = typename Cfg::T;
@@ -464,10 +478,10 @@ cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *
     CUtensorMap tm;
     launch_step() = "tensor map of x";
     cudaError_t e = make_tmap_2d(&tm, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1,
-                                 Cfg::SW1 / Cfg::E, Cfg::N1, Cfg::SW1);
+                                 Cfg::SW1 / Cfg::E, Cfg::N1, Cfg::SW1, false);
     if (e != cudaSuccess) return e;
     launch_step() = "shared-memory attribute";
-    e = cudaFuncSetAttribute(kron_fwd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(kron_fwd_tc_kernel<Cfg, TR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
     if (e != cudaSuccess) return e;
     launch_step() = "kernel launch";
@@ -479,7 +493,7 @@ cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *
         cfg.blockDim = dim3(kFwdThreads);
         cfg.dynamicSmemBytes = Cfg::SMEM;
         cfg.stream = st;
-        return cudaLaunchKernelEx(&cfg, kron_fwd_tc_kernel<Cfg>, tm, a);
+        return cudaLaunchKernelEx(&cfg, kron_fwd_tc_kernel<Cfg, TR>, tm, a);
     }
 }
 
@@ -487,33 +501,53 @@ using FwdFn = cudaError_t (*)(const void *, const void *, const void *, const vo
                               const void *, void *, const Shape &, cudaStream_t);
 
 struct FwdEntry {
-    int p, q, m1, m2, r;
-    bool bf16;
+    int p, q, m1, m2, r;  // the kernel's shape (for TR, the layer's q, p, m2, m1)
+    bool bf16, tr;
     FwdFn fn;
 };
 
-// Shapes with a compiled tensor-core forward.
+// Shapes with a compiled tensor-core forward (tr = false) and dX kernel (tr = true).
 const FwdEntry kFwdTable[] = {
-    {32, 32, 32, 32, 4, false, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, float>>},
-    {32, 32, 32, 32, 4, true, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, __nv_bfloat16>>},
+    {32, 32, 32, 32, 4, false, false, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, float>, false>},
+    {32, 32, 32, 32, 4, true, false, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, __nv_bfloat16>, false>},
+    {32, 32, 32, 32, 4, false, true, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, float>, true>},
+    {32, 32, 32, 32, 4, true, true, &launch_fwd<FwdCfg<32, 32, 32, 32, 4, __nv_bfloat16>, true>},
 };
 
-FwdFn find_fwd(const Shape &s, bool bf16) {
+FwdFn find_fwd(const Shape &s, bool bf16, bool tr) {
     for (const auto &f : kFwdTable)
-        if (f.p == s.p && f.q == s.q && f.m1 == s.m1 && f.m2 == s.m2 && f.r == s.r && f.bf16 == bf16)
+        if (f.p == s.p && f.q == s.q && f.m1 == s.m1 && f.m2 == s.m2 && f.r == s.r &&
+            f.bf16 == bf16 && f.tr == tr)
             return f.fn;
     return nullptr;
 }
 
+// The kernel shape of dX = dY W^T: the layer's shape with (p, q) and (m1, m2) swapped.
+Shape transposed(const Shape &s) { return Shape{s.N, s.q, s.p, s.m2, s.m1, s.r}; }
+
 }  // namespace tc
 
-bool tc_forward_supported(const Shape &s, bool bf16) { return tc::find_fwd(s, bf16) != nullptr; }
+bool tc_forward_supported(const Shape &s, bool bf16) {
+    return tc::find_fwd(s, bf16, false) != nullptr;
+}
 
 cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
                        const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st) {
-    tc::FwdFn fn = tc::find_fwd(s, bf16);
+    tc::FwdFn fn = tc::find_fwd(s, bf16, false);
     if (!fn) return cudaErrorNotSupported;
     return fn(x, S, A, B, bias, y, s, st);
+}
+
+bool tc_dx_supported(const Shape &s, bool bf16) {
+    return tc::find_fwd(tc::transposed(s), bf16, true) != nullptr;
+}
+
+cudaError_t tc_dx(const void *dY, const void *S, const void *A, const void *B, void *dX,
+                  const Shape &s, bool bf16, cudaStream_t st) {
+    const Shape t = tc::transposed(s);
+    tc::FwdFn fn = tc::find_fwd(t, bf16, true);
+    if (!fn) return cudaErrorNotSupported;
+    return fn(dY, S, A, B, nullptr, dX, t, st);
 }
 
 int tc_read_device_error(bool clear) {

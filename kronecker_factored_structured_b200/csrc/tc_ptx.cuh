@@ -328,12 +328,29 @@ __device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr, int sw) {
     return d;
 }
 
+// MN-major operand tile: the M (or N) dimension runs along rows of 128 B (TF32, layout
+// type 1 = 128-byte swizzle with 32-byte atoms, 4-row K groups) or of `sw` bytes (16-bit
+// types, the ordinary swizzles, 8-row K groups); `lbo` = byte stride between successive
+// MN blocks of one row width, `sbo` = byte stride between successive K groups.
+__device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr, uint32_t layout, uint32_t lbo,
+                                             uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+constexpr uint32_t kLayoutSw128Atom32 = 1u;  // the only MN-major layout for TF32 operands
+
 // Instruction descriptor: FP32 accumulator, A/B of format fmt (1 = BF16, 2 = TF32), both
-// K-major, shape M x N.
+// K-major, shape M x N.  OR in kBMajorMN when B is MN-major.
 __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t fmt) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
+constexpr uint32_t kBMajorMN = 1u << 16;
 
 // Byte offset of (row, byte-in-row) inside a K-major swizzled region whose rows are `sw`
 // bytes, with 1024-byte-aligned base: the 16-byte chunk index is XORed with address
