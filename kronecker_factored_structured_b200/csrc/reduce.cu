@@ -7,9 +7,10 @@
 //
 // Workspace layout per range g: ws[g*stride + ...] = [dC: r*p*q][dB: r*m1*m2][dbias: q*m2].
 // Each block owns 32 consecutive output columns (for dC: 32 (a,c) positions and all r
-// ranks).  Its 8 warps sum ranges g = w, w+8, ... in double with several independent
-// accumulators, which are then added in a fixed order.  The order depends only on
-// `parts`, so results are bitwise reproducible.
+// ranks).  Its kWarps warps sum ranges g = w, w+kWarps, ... in double with several
+// independent accumulators, which are then added in a fixed order.  The order depends only
+// on `parts`, so results are bitwise reproducible.  Many warps per column keep each
+// thread's chain of dependent loads short: the kernel is latency-bound, not byte-bound.
 #include "internal.h"
 
 #include <cuda_bf16.h>
@@ -20,10 +21,12 @@ namespace {
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
+constexpr int kWarps = 32;
+
 // Sums over the row ranges of up to NC columns off[0..ncols): warp w adds ranges
-// g = w, w+8, ... into U independent accumulators per column (so U*ncols loads are in
-// flight per thread); then the accumulators and the 8 warp sums are added in a fixed
-// order.
+// g = w, w+kWarps, ... into U independent accumulators per column (so U*ncols loads are
+// in flight per thread); then the accumulators and the kWarps warp sums are added in a
+// fixed order.
 template <int U, int NC>
 __device__ __forceinline__ void col_sums(const float *__restrict__ ws, int parts, size_t stride,
                                          const size_t *off, bool valid, int ncols,
@@ -35,10 +38,10 @@ __device__ __forceinline__ void col_sums(const float *__restrict__ ws, int parts
 #pragma unroll
         for (int u = 0; u < U; ++u) acc[c][u] = 0.0;
     if (valid) {
-        for (int g = w; g < parts; g += 8 * U) {
+        for (int g = w; g < parts; g += kWarps * U) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int gg = g + 8 * u;
+                const int gg = g + kWarps * u;
                 if (gg < parts) {
 #pragma unroll
                     for (int c = 0; c < NC; ++c)
@@ -58,7 +61,7 @@ __device__ __forceinline__ void col_sums(const float *__restrict__ ws, int parts
         if (w == 0) {
             double tot = 0.0;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) tot += red[t][lane];
+            for (int t = 0; t < kWarps; ++t) tot += red[t][lane];
             out[c] = tot;
         }
         __syncthreads();
@@ -68,12 +71,12 @@ __device__ __forceinline__ void col_sums(const float *__restrict__ ws, int parts
 constexpr int kMaxRanksPerPass = 8;
 
 template <typename TI>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kWarps)
 kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
                    const TI *__restrict__ S, const TI *__restrict__ A, float *__restrict__ dS,
                    float *__restrict__ dA, float *__restrict__ dB, float *__restrict__ dbias,
                    Shape s, int blocks_dc, int blocks_db) {
-    __shared__ double red[8][33];
+    __shared__ double red[kWarps][33];
     const size_t pq = (size_t)s.p * s.q;
     const size_t n_dc = (size_t)s.r * pq, n_db = (size_t)s.r * s.m1 * s.m2;
     const size_t n_b = (size_t)s.q * s.m2;
@@ -89,7 +92,7 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
             size_t off[kMaxRanksPerPass];
             double dc[kMaxRanksPerPass];
             for (int ii = 0; ii < kMaxRanksPerPass; ++ii) off[ii] = (size_t)(i0 + ii) * pq + col;
-            col_sums<2, kMaxRanksPerPass>(ws, parts, stride, off, v, nr, red, dc);
+            col_sums<1, kMaxRanksPerPass>(ws, parts, stride, off, v, nr, red, dc);
             if (threadIdx.y == 0 && v) {
                 for (int ii = 0; ii < nr; ++ii) {
                     const size_t e = (size_t)(i0 + ii) * pq + col;
@@ -107,7 +110,7 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
         const size_t off = n_dc + col;
         const bool v = col < n_db;
         double out;
-        col_sums<8, 1>(ws, parts, stride, &off, v, 1, red, &out);
+        col_sums<4, 1>(ws, parts, stride, &off, v, 1, red, &out);
         if (threadIdx.y == 0 && v) dB[col] = (float)out;
         return;
     }
@@ -116,7 +119,7 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
     const size_t off = n_dc + n_db + col;
     const bool v = col < n_b;
     double out;
-    col_sums<8, 1>(ws, parts, stride, &off, v, 1, red, &out);
+    col_sums<4, 1>(ws, parts, stride, &off, v, 1, red, &out);
     if (threadIdx.y == 0 && v) dbias[col] = (float)out;
 }
 
@@ -132,7 +135,7 @@ cudaError_t reduce_partials(const float *ws, int parts, const void *S, const voi
     const size_t stride = partial_stride(s);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(blocks_dc + blocks_db + blocks_b));
-    cfg.blockDim = dim3(32, 8);
+    cfg.blockDim = dim3(32, kWarps);
     cfg.stream = st;
     if (is_bf16)
         return cudaLaunchKernelEx(&cfg, kron_reduce_kernel<__nv_bfloat16>, ws, parts, stride,

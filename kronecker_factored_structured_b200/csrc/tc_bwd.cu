@@ -23,13 +23,14 @@
 // T and U accumulators (TMEM -> registers) into the K-major layouts dC and dB read, one
 // 128-byte row segment per warp store.
 //
-// Warp roles (480 threads, one CTA per SM, tiles of the CTA's row range in order):
+// Warp roles (736 threads, one CTA per SM, tiles of the CTA's row range in order):
 //   warp 0       TMA producer: an SI-deep ring of input sets (x and G tiles)
 //   warp 1       issuer A: T and U of tile t into TMEM (two accumulator slots); owns TMEM
 //   warp 2       issuer B: dC and dB of tile t from T2/U2 (an SB-deep ring in shared memory)
-//   warps 3-6    epilogue T -> T2 (one warp per TMEM lane quadrant)
-//   warps 7-10   epilogue U -> U2
-//   warps 11-14  dbias column sums of the G tiles
+//   warps 3-18   epilogues in two teams taking alternate tiles (team = tile parity, which
+//                is also its TMEM slot and its T2/U2 buffers): per team, one warp per
+//                TMEM lane quadrant for T -> T2 and one for U -> U2
+//   warps 19-22  dbias column sums of the G tiles
 // Issuers run their loops as whole warps and let one elected lane issue each burst; every
 // consumer takes the tiles in order, so no mbarrier phase can be mistaken for another.
 #include "internal.h"
@@ -60,7 +61,7 @@ template <> struct BE<__nv_bfloat16> {
 };
 
 constexpr int imin(int a, int b) { return a < b ? a : b; }
-constexpr int kPgThreads = 480;
+constexpr int kPgThreads = 736;
 
 template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
 struct PgCfg {
@@ -84,8 +85,10 @@ struct PgCfg {
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_MAX = 232448;
     static constexpr int FREE = SMEM_MAX - 1024 - BAR_BYTES;
-    static constexpr int SB = FREE - 4 * IB >= 4 * IN_BYTES ? 4 : FREE - 3 * IB >= 3 * IN_BYTES ? 3 : 2;
-    static constexpr int SI = imin(4, (FREE - SB * IB) / IN_BYTES);
+    // the input ring holds a set from its load until dC/dB of that tile are done (the
+    // longest lifetime in the pipeline), so it gets every byte the intermediates leave
+    static constexpr int SB = FREE - 4 * IB >= 8 * IN_BYTES ? 4 : 2;  // even: two teams
+    static constexpr int SI = imin(12, (FREE - SB * IB) / IN_BYTES);
     static constexpr int OFF_IN = 0;
     static constexpr int OFF_I = SI * IN_BYTES;
     static constexpr int OFF_BAR = OFF_I + SB * IB;
@@ -116,6 +119,7 @@ struct PgCfg {
     static_assert((T2K * E) % 128 == 0 && (U2K * E) % 128 == 0, "T2/U2 rows: whole 128-byte chunks");
     static_assert(P == 32 && M2 == 32, "epilogue: one 32-column TMEM load per (n, block)");
     static_assert(SI >= 2 && SB >= 2, "rings");
+    static_assert(2 * SI + 4 + 2 * SB + 2 + 2 <= BAR_BYTES / 8, "barrier region");
     static_assert(TM_USED <= TM_COLS, "TMEM budget");
     static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -184,7 +188,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(bar(D_FULL + d), 1);
-            mbar_init(bar(D_EMPTY + d), 8);          // both epilogues
+            mbar_init(bar(D_EMPTY + d), 8);          // the slot's epilogue team
         }
         for (int b = 0; b < SB; ++b) {
             mbar_init(bar(I_FULL + b), 8);
@@ -208,7 +212,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     const uint32_t tmem = *tmem_slot;
     // A operands in TMEM, one lane per row (two BF16 values per column):
     //   B_all^T: lane (i,k), column j -> B_i[j][k];   C_stack: lane (i,a), column c -> C_i[a][c]
-    if (warp >= 3 && warp < 11) {
+    if (warp >= 3 && warp < 11) {   // team 0 loads the A operands
         const int qd = warp & 3, L = qd * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         const bool is_c = warp >= 7;
@@ -326,39 +330,43 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         __syncwarp();
         if (lane == 0) mbar_wait_drain(bar(DONE), 0);
         __syncwarp();
-    } else if (warp < 11) {
-        // ---------------- epilogues: T -> T2 (warps 3-6), U -> U2 (warps 7-10) ----------------
-        const bool is_u = warp >= 7;
+    } else if (warp < 19) {
+        // ---------------- epilogues: T -> T2 and U -> U2, two teams on alternate tiles ----------------
+        const int team = (warp - 3) >> 3;
+        const bool is_u = ((warp - 3) >> 2) & 1;
         const int qd = warp & 3, L = qd * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         // T lane (i,k), columns (n,a) -> T2 row (i,a), K (n,k);
         // U lane (i,a), columns (n,k) -> U2 row (i,k), K (n,a)
         const int i = L / 32, o = L % 32;   // o = k (T) or a (U); p = m2 = 32
         bool ok = true;
-        for (int u = 0; u < nt; ++u) {
+        for (int u = team; u < nt; u += 2) {
             const int d = u & 1, b = u % SB;
-            if (!mbar_wait(bar(D_FULL + d), (u >> 1) & 1, ab)) { ok = false; break; }
+            if (!mbar_wait(bar(D_FULL + d), (u >> 1) & 1, ab) ||
+                !mbar_wait(bar(I_EMPTY + b), ((u / SB) & 1) ^ 1, ab)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            uint32_t r[64];
             const uint32_t src = tmem + lane_addr + (is_u ? Cfg::TM_DU + d * NT * M2 : Cfg::TM_DT + d * XR);
-            tmem_load32(src, *reinterpret_cast<uint32_t(*)[32]>(r));
-            tmem_load32(src + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-            tc_fence_before();
-            mbar_arrive_warp(bar(D_EMPTY + d));
-            if (!mbar_wait(bar(I_EMPTY + b), ((u / SB) & 1) ^ 1, ab)) { ok = false; break; }
             const uint32_t dst = sI + b * Cfg::IB + (is_u ? Cfg::T2_BYTES : 0);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const int n = c / 32, w = c % 32;   // column (n, w): w = a (T) or k (U)
-                const int row = i * 32 + w, kidx = n * 32 + o;
-                st_elem<T>(dst + koff(row, kidx * E, 128, 128), r[c]);
+            for (int n = 0; n < NT; ++n) {   // column block (n, w), w = a (T) or k (U)
+                uint32_t r[32];
+                tmem_load32(src + n * 32, r);
+#pragma unroll
+                for (int w = 0; w < 32; ++w)
+                    st_elem<T>(dst + koff(i * 32 + w, (n * 32 + o) * E, 128, 128), r[w]);
             }
+            tc_fence_before();
+            mbar_arrive_warp(bar(D_EMPTY + d));
             fence_proxy_async();
             mbar_arrive_warp(bar(I_FULL + b));
         }
-        // this range's partial dC (T warps) or dB (U warps), after the last MMAs
+        // this range's partial dC (team 0's T warps) or dB (team 0's U warps), after the last MMAs
         float *part = args.ws + (size_t)blockIdx.x * args.ws_stride;
-        if (ok && nt > 0 && mbar_wait(bar(DONE), 0, ab)) {
+        const bool ok_all = named_bar_and(1, 512, ok);
+        if (team == 0 && ok_all && nt > 0 && mbar_wait(bar(DONE), 0, ab)) {
             tc_fence_after();
             if (!is_u) {   // dC: lane (i,a), columns c -> dC_i[a][c]
                 for (int c0 = 0; c0 < Q; c0 += 32) {
@@ -380,13 +388,13 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
                             __uint_as_float(r[t]);
                 }
             }
-        } else if (nt == 0) {
+        } else if (team == 0 && nt == 0) {
             const size_t n0 = is_u ? (size_t)R * P * Q : 0, n1 = is_u ? (size_t)R * (P * Q + M1 * M2) : (size_t)R * P * Q;
             for (size_t e = n0 + (size_t)(threadIdx.x - (is_u ? 224 : 96)); e < n1; e += 128) part[e] = 0.f;
         }
     } else {
         // ---------------- dbias: column sums of the G tiles (zero rows past N come from TMA) ----------------
-        const int tid = threadIdx.x - 352;
+        const int tid = threadIdx.x - 608;
         constexpr int PER = Q * M2 / 128;
         float acc[PER];
 #pragma unroll
