@@ -98,7 +98,9 @@ size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r
     if (check_shape(N, p, q, m1, m2, r, dtype, 0) != KRON_OK) return 0;
     const kron::Shape s{N, p, q, m1, m2, r};
     const int parts = backward_parts(s, dtype);
-    return (size_t)parts * kron::partial_stride(s) * sizeof(float);
+    if (parts <= 0) return 0;
+    return (size_t)parts * kron::partial_stride(s) * sizeof(float) +
+           (dtype == KRON_F32 ? 0 : kron::tc_backward_workspace_extra);
 }
 
 kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, const void *B,
@@ -197,10 +199,9 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
                 return fail(KRON_ERR_UNSUPPORTED,
                             "no tensor-core backward for p=%d q=%d m1=%d m2=%d r=%d (%s)", p, q,
                             m1, m2, r, bf16 ? "bf16" : "tf32");
-            e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16, cs);
+            e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, (float *)dS,
+                                  (float *)dA, (float *)dB, (float *)dbias, bf16, cs);
             if (e != cudaSuccess) return cuda_fail(e, "backward launch");
-            e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
-                                      (float *)dA, (float *)dB, (float *)dbias, s, cs);
             break;
         }
         default:

@@ -51,10 +51,14 @@ cudaError_t tc_dx(const void *dY, const void *S, const void *A, const void *B, v
                   const Shape &s, bool bf16, cudaStream_t st);
 bool tc_backward_supported(const Shape &s, bool bf16);
 int tc_backward_tile_rows(const Shape &s);
-// Writes dX (if non-null) and the per-range partials (parts x partial_stride floats).
+// Writes dX (if non-null) and the final dS, dA, dB, dbias (dbias may be null).  ws holds
+// parts x partial_stride floats of row-range partials followed by one grid-barrier word
+// (tc_backward_workspace_extra bytes).
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                        bool bf16, cudaStream_t st);
+                        float *dS, float *dA, float *dB, float *dbias, bool bf16,
+                        cudaStream_t st);
+constexpr size_t tc_backward_workspace_extra = 256;
 // Device error word of the tensor-core kernels (bounded waits); -1 if unreadable.
 int tc_read_device_error(bool clear);
 

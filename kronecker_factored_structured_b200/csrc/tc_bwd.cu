@@ -13,8 +13,9 @@
 //     dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]  A = U2 [(i,k)][(n,a)], B = x tile MN-major
 //     dbias[c*m2+k]  += sum_n G_n[c,k]
 //   dC and dB accumulate in TMEM over the CTA's fixed, contiguous range of rows and are
-//   written to the workspace as that range's partials; reduce.cu adds the partials in a
-//   fixed order and forms dA = dC (.) S and dS = sum_i dC_i (.) A_i (bitwise reproducible).
+//   written to the workspace as that range's partials; after a grid barrier (cooperative
+//   launch) the same kernel adds the partials in a fixed order and forms dA = dC (.) S and
+//   dS = sum_i dC_i (.) A_i (bitwise reproducible, no separate reduction launch).
 //
 // The x and G tiles serve as K-major operands (T, dC) and as MN-major ones (U, dB): TMA
 // brings each in both shared-memory layouts for TF32 (whose MN-major layout is the 128-byte
@@ -62,6 +63,13 @@ template <> struct BE<__nv_bfloat16> {
 
 constexpr int imin(int a, int b) { return a < b ? a : b; }
 constexpr int kPgThreads = 736;
+
+template <typename T>
+__device__ __forceinline__ float bld(const void *p, size_t i) {
+    if constexpr (BE<T>::tf32) return static_cast<const float *>(p)[i];
+    else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
 
 template <int P_, int Q_, int M1_, int M2_, int R_, typename T_>
 struct PgCfg {
@@ -131,12 +139,83 @@ struct PgArgs {
     int num_tiles;
     int tiles_per_part;
     int *device_error;
+    unsigned *arrived;     // grid barrier counter (zeroed by the host before the launch)
+    float *dS, *dA, *dB, *dbias;
 };
 
-template <typename T>
-__device__ __forceinline__ float bld(const void *p, size_t i) {
-    if constexpr (BE<T>::tf32) return static_cast<const float *>(p)[i];
-    else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Fixed-order reduction of every range's partials, run by the whole grid once all of them
+// are written.  The partial columns are visited as virtual columns: dC ordered (position
+// (a,c), rank i) so that the r ranks of a position are adjacent, then dB, then dbias.  CTA
+// g owns a run of virtual columns (a multiple of r long); within a pass of CW columns,
+// GS groups of threads each sum the ranges g' = ps, ps + GS, ... of one column in double
+// with four accumulators, and the GS group sums are added in a fixed order.  Only `parts`
+// decides the order, so the results are bitwise reproducible.  The epilogue forms
+// dA_i = dC_i (.) S and dS = sum_i dC_i (.) A_i (C_i = S (.) A_i, product rule) and writes
+// dB and dbias.
+template <class Cfg>
+__device__ void reduce_ranges(const PgArgs &args, int parts, double *red, double *vals) {
+    using T = typename Cfg::T;
+    constexpr int P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
+    constexpr int NDC = R * P * Q, NDB = R * M1 * M2, NB = Q * M2;
+    constexpr int NCOL = NDC + NDB + NB;
+    constexpr int CW = (64 / R) * R;                 // columns per pass (whole rank groups)
+    constexpr int GS = kPgThreads / CW;              // thread groups splitting the ranges
+    static_assert(64 % R == 0 || R <= 64, "rank groups within one pass");
+    const int per = ((NCOL + (int)gridDim.x * R - 1) / ((int)gridDim.x * R)) * R;
+    const int v0 = (int)blockIdx.x * per, v1 = imin(v0 + per, NCOL);
+    const int cs = threadIdx.x % CW, ps = threadIdx.x / CW;
+    for (int c0 = v0; c0 < v1; c0 += CW) {
+        const int v = c0 + cs;
+        if (ps < GS) {
+            double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+            if (v < v1) {
+                const size_t col = v < NDC ? (size_t)(v % R) * P * Q + (size_t)(v / R) : (size_t)v;
+                const float *src = args.ws + col;
+                int g = ps;
+                for (; g + 3 * GS < parts; g += 4 * GS) {
+                    a0 += (double)__ldcg(src + (size_t)g * args.ws_stride);
+                    a1 += (double)__ldcg(src + (size_t)(g + GS) * args.ws_stride);
+                    a2 += (double)__ldcg(src + (size_t)(g + 2 * GS) * args.ws_stride);
+                    a3 += (double)__ldcg(src + (size_t)(g + 3 * GS) * args.ws_stride);
+                }
+                for (; g < parts; g += GS) a0 += (double)__ldcg(src + (size_t)g * args.ws_stride);
+            }
+            red[ps * CW + cs] = (a0 + a1) + (a2 + a3);
+        }
+        __syncthreads();
+        if (threadIdx.x < CW) {
+            double tot = 0.0;
+            for (int k = 0; k < GS; ++k) tot += red[k * CW + threadIdx.x];
+            vals[threadIdx.x] = tot;
+        }
+        __syncthreads();
+        if (threadIdx.x < CW && v < v1) {
+            if (v < NDC) {
+                if (v % R == 0) {   // the rank group of position (a,c) = v / R
+                    const int pos = v / R;
+                    const double sv = (double)bld<T>(args.S, pos);
+                    double ds = 0.0;
+                    for (int i = 0; i < R; ++i) {
+                        const double dc = vals[threadIdx.x + i];
+                        args.dA[(size_t)i * P * Q + pos] = (float)(dc * sv);
+                        ds += dc * (double)bld<T>(args.A, (size_t)i * P * Q + pos);
+                    }
+                    args.dS[pos] = (float)ds;
+                }
+            } else if (v < NDC + NDB) {
+                args.dB[v - NDC] = (float)vals[threadIdx.x];
+            } else if (args.dbias) {
+                args.dbias[v - NDC - NDB] = (float)vals[threadIdx.x];
+            }
+        }
+        __syncthreads();
+    }
 }
 
 // Byte offset of element (row, kbyte) of a K-major swizzled operand region: K in chunks of
@@ -427,18 +506,46 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         for (int e = 0; e < PER; ++e) part[tid + 128 * e] = acc[e];
     }
 
-    // ---------------- teardown ----------------
+    // ---------------- teardown of the tensor-core state ----------------
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::TM_COLS);
     }
+
+    // ---------------- grid barrier, then the fixed-order reduction ----------------
+    // Every CTA arrives (also after an abort, so none waits forever); the launch is
+    // cooperative, so all CTAs are resident.  The wait is bounded like every other.
+    volatile int *grid_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(args.arrived, 1u);
+        const uint64_t w0 = globaltimer();
+        int okb = 1;
+        while (ld_acquire_gpu(args.arrived) < gridDim.x) {
+            if (globaltimer() - w0 > kWaitTimeoutNs) {
+                okb = 0;
+                if (args.device_error) atomicOr(args.device_error, 2);
+                break;
+            }
+            __nanosleep(128);
+        }
+        *grid_ok = okb && !*ab.flag;
+    }
+    __syncthreads();
+    if (*grid_ok) {
+        double *red = reinterpret_cast<double *>(smem);            // input ring: idle now
+        double *vals = red + kPgThreads + 64;
+        reduce_ranges<Cfg>(args, (int)gridDim.x, red, vals);
+    }
 }
 
 template <class Cfg>
 cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void *B, const void *dY,
-                         float *ws, int parts, const Shape &s, cudaStream_t st) {
+                         float *ws, int parts, const Shape &s, float *dS, float *dA, float *dB,
+                         float *dbias, cudaStream_t st) {
     using T = typename Cfg::T;
     const bool bf16 = !BE<T>::tf32;
     CUtensorMap txk, tgk, txm, tgm;
@@ -463,23 +570,34 @@ cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void
     e = cudaFuncSetAttribute(kron_pgrad_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    launch_step() = "kernel launch";
     PgArgs a;
     a.S = S; a.A = A; a.B = B; a.ws = ws;
     a.ws_stride = partial_stride(s);
     a.num_tiles = (int)((s.N + Cfg::NT - 1) / Cfg::NT);
     a.tiles_per_part = (a.num_tiles + parts - 1) / parts;
     a.device_error = device_error_ptr();
+    a.arrived = reinterpret_cast<unsigned *>(ws + (size_t)parts * a.ws_stride);
+    a.dS = dS; a.dA = dA; a.dB = dB; a.dbias = dbias;
+    launch_step() = "grid barrier reset";
+    e = cudaMemsetAsync(a.arrived, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return e;
+    launch_step() = "kernel launch (cooperative)";
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)parts);
     cfg.blockDim = dim3(kPgThreads);
     cfg.dynamicSmemBytes = Cfg::SMEM;
     cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kron_pgrad_tc_kernel<Cfg>, txk, tgk, txm, tgm, a);
 }
 
 using PgFn = cudaError_t (*)(const void *, const void *, const void *, const void *, const void *,
-                             float *, int, const Shape &, cudaStream_t);
+                             float *, int, const Shape &, float *, float *, float *, float *,
+                             cudaStream_t);
 struct PgEntry {
     int p, q, m1, m2, r;
     bool bf16;
@@ -508,14 +626,15 @@ int tc_backward_tile_rows(const Shape &) { return 2; }
 
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                        bool bf16, cudaStream_t st) {
+                        float *dS, float *dA, float *dB, float *dbias, bool bf16,
+                        cudaStream_t st) {
     tc::PgFn fn = tc::find_pg(s, bf16);
     if (!fn) return cudaErrorNotSupported;
     if (dX) {
         const cudaError_t e = tc_dx(dY, S, A, B, dX, s, bf16, st);
         if (e != cudaSuccess) return e;
     }
-    return fn(x, S, A, B, dY, ws, parts, s, st);
+    return fn(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, st);
 }
 
 }  // namespace kron
