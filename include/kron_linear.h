@@ -24,6 +24,9 @@
  *              cores with TF32 operands and FP32 accumulation.
  *   KRON_BF16  x, y, dY, dX, S, A, B and bias are bfloat16; dS, dA, dB and dbias are
  *              float32.  tcgen05 tensor cores with BF16 operands, FP32 accumulation.
+ *   The tensor-core kernels are compiled for p = q = m1 = m2 = 32, r = 4.  A TF32 or
+ *   BF16 call of any other shape runs the exact-FP32 CUDA-core kernels with the same
+ *   element types at the boundary (FP32 arithmetic: at least as accurate, slower).
  *
  * Ownership and synchronisation: every pointer except `stream` is a DEVICE pointer
  * owned by the caller.  The library allocates no memory, keeps no state between
@@ -32,8 +35,8 @@
  *
  * Errors: arguments, shapes, alignment and workspace size are checked on the host
  * before anything is launched; a failing check returns its status and launches
- * nothing.  Shapes a path does not cover return KRON_ERR_UNSUPPORTED (there is no
- * fallback to another path or to the CPU).  A failed launch returns KRON_ERR_CUDA;
+ * nothing.  Shapes no kernel covers (an FP32 tile larger than shared memory) return
+ * KRON_ERR_UNSUPPORTED; nothing ever falls back to the CPU.  A failed launch returns KRON_ERR_CUDA;
  * faults during execution surface at the caller's next synchronisation.
  * kron_last_error() gives a one-line description of the last failure on the
  * calling host thread.

@@ -55,10 +55,15 @@ kron_status_t check_shape(int64_t N, int p, int q, int m1, int m2, int r, kron_d
 
 // Number of contiguous row ranges of the backward: at most kRowParts, none empty.  A
 // function of the shape and path only, so the summation order is fixed.
+// True when the backward of this shape and dtype runs on the tensor-core kernels.
+bool tc_backward_path(const kron::Shape &s, kron_dtype_t dtype) {
+    return dtype != KRON_F32 && kron::tc_backward_supported(s, dtype == KRON_BF16);
+}
+
 int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
     int rows_per_tile = 0;
-    if (dtype == KRON_F32) rows_per_tile = kron::simt_backward_rows(s);
-    else if (kron::tc_backward_supported(s, dtype == KRON_BF16)) rows_per_tile = kron::tc_backward_tile_rows(s);
+    if (tc_backward_path(s, dtype)) rows_per_tile = kron::tc_backward_tile_rows(s);
+    else rows_per_tile = kron::simt_backward_rows(s);
     if (rows_per_tile <= 0) return 0;
     int64_t tiles = (s.N + rows_per_tile - 1) / rows_per_tile;
     if (tiles < 1) tiles = 1;
@@ -100,7 +105,7 @@ size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r
     const int parts = backward_parts(s, dtype);
     if (parts <= 0) return 0;
     return (size_t)parts * kron::partial_stride(s) * sizeof(float) +
-           (dtype == KRON_F32 ? 0 : kron::tc_backward_workspace_extra);
+           (tc_backward_path(s, dtype) ? kron::tc_backward_workspace_extra : 0);
 }
 
 kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, const void *B,
@@ -121,19 +126,20 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
     cudaError_t e = cudaSuccess;
     switch (dtype) {
         case KRON_F32:
-            if (kron::simt_forward_rows(s) <= 0)
-                return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
-            e = kron::simt_forward((const float *)x, (const float *)S, (const float *)A,
-                                   (const float *)B, (const float *)bias, (float *)y, s, cs);
-            break;
         case KRON_TF32:
         case KRON_BF16: {
             const bool bf16 = dtype == KRON_BF16;
-            if (!kron::tc_forward_supported(s, bf16))
+            if (dtype != KRON_F32 && kron::tc_forward_supported(s, bf16)) {
+                e = kron::tc_forward(x, S, A, B, bias, y, s, bf16, cs);
+                break;
+            }
+            // exact-FP32 CUDA-core kernels: every KRON_F32 call, and TF32/BF16 shapes with no
+            // compiled tensor-core kernel (fp32 arithmetic, I/O in the caller's dtype)
+            if (kron::simt_forward_rows(s) <= 0)
                 return fail(KRON_ERR_UNSUPPORTED,
-                            "no tensor-core forward for p=%d q=%d m1=%d m2=%d r=%d (%s)", p, q, m1,
-                            m2, r, bf16 ? "bf16" : "tf32");
-            e = kron::tc_forward(x, S, A, B, bias, y, s, bf16, cs);
+                            "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not "
+                            "fit shared memory", p, q, m1, m2, r);
+            e = kron::simt_forward(x, S, A, B, bias, y, s, bf16, cs);
             break;
         }
         default:
@@ -168,11 +174,11 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
             e = cudaMemsetAsync(dbias, 0, (size_t)q * m2 * sizeof(float), cs);
         return e == cudaSuccess ? KRON_OK : cuda_fail(e, "zero gradients");
     }
-    if (dtype != KRON_F32 && !kron::tc_backward_supported(s, dtype == KRON_BF16))
-        return fail(KRON_ERR_UNSUPPORTED, "no tensor-core backward for p=%d q=%d m1=%d m2=%d r=%d",
-                    p, q, m1, m2, r);
-    if (dtype == KRON_F32 && kron::simt_backward_rows(s) <= 0)
-        return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
+    const bool on_tc = tc_backward_path(s, dtype);
+    if (!on_tc && kron::simt_backward_rows(s) <= 0)
+        return fail(KRON_ERR_UNSUPPORTED,
+                    "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not fit shared "
+                    "memory", p, q, m1, m2, r);
     const size_t need = kron_linear_workspace_size(N, p, q, m1, m2, r, dtype);
     if (!workspace || workspace_bytes < need)
         return fail(KRON_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
@@ -181,31 +187,18 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
         return fail(KRON_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
     const int parts = backward_parts(s, dtype);
     cudaError_t e = cudaSuccess;
-    switch (dtype) {
-        case KRON_F32:
-            if (kron::simt_backward_rows(s) <= 0)
-                return fail(KRON_ERR_UNSUPPORTED, "shape does not fit the FP32 kernel's tile");
-            e = kron::simt_backward((const float *)x, (const float *)S, (const float *)A,
-                                    (const float *)B, (const float *)dY, (float *)dX,
-                                    (float *)workspace, parts, s, cs);
-            if (e != cudaSuccess) return cuda_fail(e, "backward launch");
-            e = kron::reduce_partials((const float *)workspace, parts, S, A, false, (float *)dS,
-                                      (float *)dA, (float *)dB, (float *)dbias, s, cs);
-            break;
-        case KRON_TF32:
-        case KRON_BF16: {
-            const bool bf16 = dtype == KRON_BF16;
-            if (!kron::tc_backward_supported(s, bf16))
-                return fail(KRON_ERR_UNSUPPORTED,
-                            "no tensor-core backward for p=%d q=%d m1=%d m2=%d r=%d (%s)", p, q,
-                            m1, m2, r, bf16 ? "bf16" : "tf32");
-            e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, (float *)dS,
-                                  (float *)dA, (float *)dB, (float *)dbias, bf16, cs);
-            if (e != cudaSuccess) return cuda_fail(e, "backward launch");
-            break;
-        }
-        default:
-            return fail(KRON_ERR_UNSUPPORTED, "dtype %d backward not implemented", (int)dtype);
+    const bool bf16 = dtype == KRON_BF16;
+    if (on_tc) {
+        e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, (float *)dS,
+                              (float *)dA, (float *)dB, (float *)dbias, bf16, cs);
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    } else {
+        // exact-FP32 CUDA-core kernels (every KRON_F32 call; TF32/BF16 shapes with no
+        // compiled tensor-core kernel), then the fixed-order reduction of the partials
+        e = kron::simt_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16, cs);
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+        e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
+                                  (float *)dA, (float *)dB, (float *)dbias, s, cs);
     }
     if (e != cudaSuccess) return cuda_fail(e, "reduction launch");
     return KRON_OK;

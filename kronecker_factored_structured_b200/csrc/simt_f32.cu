@@ -1,4 +1,6 @@
 // simt_f32.cu -- exact-FP32 path of the Kronecker layer on the CUDA cores (FFMA).
+// The I/O tensors may be fp32 or bf16 (converted on load and store); all arithmetic is
+// fp32.  Any shape whose tiles fit shared memory runs here.
 //
 // Both contractions of the vec trick (page "kronecker-layer-benchmark", sections
 // "2. The vec trick" and "3. The vec trick without the loop") are fused per tile of
@@ -19,6 +21,7 @@
 #include "internal.h"
 
 #include <algorithm>
+#include <cuda_bf16.h>
 
 namespace kron {
 namespace {
@@ -94,9 +97,30 @@ __device__ __forceinline__ void smem_mm(const MM &g, bool accumulate) {
     }
 }
 
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Four consecutive elements (16 bytes of fp32, 8 of bf16) as floats.
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+    return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t *>(&lo);
+    u.y = *reinterpret_cast<const uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
 // Row r of a [rows][width] global matrix -> shared rows with stride ld; rows at or
-// beyond N read as zero.  `width` floats per row, 16-byte aligned rows.
-__device__ __forceinline__ void load_rows(const float *__restrict__ g, int64_t n0, int64_t N,
+// beyond N read as zero.  `width` elements per row (a multiple of 4), aligned rows.
+template <typename TI>
+__device__ __forceinline__ void load_rows(const TI *__restrict__ g, int64_t n0, int64_t N,
                                           int rows, int width, float *s, int blk, int ld) {
     // width = nblk * blk; shared row (n, b) of length blk starts at ((n*nblk)+b)*ld
     const int nblk = width / blk;
@@ -104,7 +128,7 @@ __device__ __forceinline__ void load_rows(const float *__restrict__ g, int64_t n
     for (int e = threadIdx.x; e < rows * w4; e += blockDim.x) {
         const int n = e / w4, c4 = (e - n * w4) << 2;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n0 + n < N) v = *reinterpret_cast<const float4 *>(g + (n0 + n) * width + c4);
+        if (n0 + n < N) v = load4(g + (n0 + n) * width + c4);
         const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -173,26 +197,28 @@ BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem) {
 }
 
 // Factor i into shared memory: Bs[j*ldb + k] = B_i[j,k], Cs[a*ldc + c] = S[a,c]*A_i[a,c].
-__device__ __forceinline__ void load_factors(const float *__restrict__ S,
-                                             const float *__restrict__ A,
-                                             const float *__restrict__ B, int i, const Shape &s,
+template <typename TI>
+__device__ __forceinline__ void load_factors(const TI *__restrict__ S,
+                                             const TI *__restrict__ A,
+                                             const TI *__restrict__ B, int i, const Shape &s,
                                              float *Bs, int ldb, float *Cs, int ldc) {
-    const float *Bi = B + (size_t)i * s.m1 * s.m2;
+    const TI *Bi = B + (size_t)i * s.m1 * s.m2;
     for (int e = threadIdx.x; e < s.m1 * s.m2; e += blockDim.x) {
         const int j = e / s.m2, k = e - j * s.m2;
-        Bs[j * ldb + k] = Bi[e];
+        Bs[j * ldb + k] = to_f(Bi[e]);
     }
-    const float *Ai = A + (size_t)i * s.p * s.q;
+    const TI *Ai = A + (size_t)i * s.p * s.q;
     for (int e = threadIdx.x; e < s.p * s.q; e += blockDim.x) {
         const int a = e / s.q, c = e - a * s.q;
-        Cs[a * ldc + c] = S[e] * Ai[e];
+        Cs[a * ldc + c] = to_f(S[e]) * to_f(Ai[e]);
     }
 }
 
+template <typename TI>
 __global__ void __launch_bounds__(kThreads)
-kron_fwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
-                     const float *__restrict__ A, const float *__restrict__ B,
-                     const float *__restrict__ bias, float *__restrict__ y, Shape s,
+kron_fwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
+                     const TI *__restrict__ A, const TI *__restrict__ B,
+                     const TI *__restrict__ bias, TI *__restrict__ y, Shape s,
                      FwdLayout L) {
     extern __shared__ __align__(16) float smem[];
     float *Xs = smem + L.offX, *Bs = smem + L.offB, *Cs = smem + L.offC;
@@ -223,17 +249,18 @@ kron_fwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
         if (n0 + n >= s.N) continue;
         float4 v = *reinterpret_cast<const float4 *>(Ys + n * out + c4);
         if (bias) {
-            const float4 bv = *reinterpret_cast<const float4 *>(bias + c4);
+            const float4 bv = load4(bias + c4);
             v.x += bv.x; v.y += bv.y; v.z += bv.z; v.w += bv.w;
         }
-        *reinterpret_cast<float4 *>(y + (n0 + n) * out + c4) = v;
+        store4(y + (n0 + n) * out + c4, v);
     }
 }
 
+template <typename TI>
 __global__ void __launch_bounds__(kThreads)
-kron_bwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
-                     const float *__restrict__ A, const float *__restrict__ B,
-                     const float *__restrict__ G, float *__restrict__ dX,
+kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
+                     const TI *__restrict__ A, const TI *__restrict__ B,
+                     const TI *__restrict__ G, TI *__restrict__ dX,
                      float *__restrict__ ws, int64_t rows_per_part, size_t ws_stride, Shape s,
                      BwdLayout L) {
     extern __shared__ __align__(16) float smem[];
@@ -301,8 +328,7 @@ kron_bwd_simt_kernel(const float *__restrict__ x, const float *__restrict__ S,
                     const int c = c4 + t, a = c / M1, j = c - a * M1;
                     v[t] = dXs[(n * P + a) * L.ldx + j];
                 }
-                *reinterpret_cast<float4 *>(dX + (n0 + n) * w + c4) =
-                    make_float4(v[0], v[1], v[2], v[3]);
+                store4(dX + (n0 + n) * w + c4, make_float4(v[0], v[1], v[2], v[3]));
             }
         }
     }
@@ -339,42 +365,60 @@ int simt_forward_rows(const Shape &s) {
 
 int simt_backward_rows(const Shape &s) { return bwd_choose(s).R; }
 
-cudaError_t simt_forward(const float *x, const float *S, const float *A, const float *B,
-                         const float *bias, float *y, const Shape &s, cudaStream_t st) {
+namespace {
+
+template <typename TI>
+cudaError_t simt_forward_t(const void *x, const void *S, const void *A, const void *B,
+                           const void *bias, void *y, const Shape &s, cudaStream_t st) {
     const int R = simt_forward_rows(s);
     const FwdLayout L = fwd_layout(s, R);
     const size_t smem = L.total * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(kron_fwd_simt_kernel,
+    cudaError_t e = cudaFuncSetAttribute(kron_fwd_simt_kernel<TI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (s.N + R - 1) / R;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)tiles);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        return cudaLaunchKernelEx(&cfg, kron_fwd_simt_kernel, x, S, A, B, bias, y, s, L);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, kron_fwd_simt_kernel<TI>, (const TI *)x, (const TI *)S,
+                              (const TI *)A, (const TI *)B, (const TI *)bias, (TI *)y, s, L);
 }
 
-cudaError_t simt_backward(const float *x, const float *S, const float *A, const float *B,
-                          const float *dY, float *dX, float *ws, int parts, const Shape &s,
-                          cudaStream_t st) {
+template <typename TI>
+cudaError_t simt_backward_t(const void *x, const void *S, const void *A, const void *B,
+                            const void *dY, void *dX, float *ws, int parts, const Shape &s,
+                            cudaStream_t st) {
     const BwdLayout L = bwd_choose(s);
     const size_t smem = L.total * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(kron_bwd_simt_kernel,
+    cudaError_t e = cudaFuncSetAttribute(kron_bwd_simt_kernel<TI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t rows_per_part = (s.N + parts - 1) / parts;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)parts);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        return cudaLaunchKernelEx(&cfg, kron_bwd_simt_kernel, x, S, A, B, dY, dX, ws, rows_per_part, partial_stride(s), s, L);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)parts);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, kron_bwd_simt_kernel<TI>, (const TI *)x, (const TI *)S,
+                              (const TI *)A, (const TI *)B, (const TI *)dY, (TI *)dX, ws,
+                              rows_per_part, partial_stride(s), s, L);
+}
+
+}  // namespace
+
+cudaError_t simt_forward(const void *x, const void *S, const void *A, const void *B,
+                         const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st) {
+    return bf16 ? simt_forward_t<__nv_bfloat16>(x, S, A, B, bias, y, s, st)
+                : simt_forward_t<float>(x, S, A, B, bias, y, s, st);
+}
+
+cudaError_t simt_backward(const void *x, const void *S, const void *A, const void *B,
+                          const void *dY, void *dX, float *ws, int parts, const Shape &s,
+                          bool bf16, cudaStream_t st) {
+    return bf16 ? simt_backward_t<__nv_bfloat16>(x, S, A, B, dY, dX, ws, parts, s, st)
+                : simt_backward_t<float>(x, S, A, B, dY, dX, ws, parts, s, st);
 }
 
 }  // namespace kron
