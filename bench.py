@@ -27,6 +27,32 @@ if ROOT not in sys.path:
 
 METRIC = "Kron-layer rows/s fwd+bwd (1024², m=32, r=4) & achieved % of roofline"
 UNIT = "rows/s"
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the backward
+# call's kernels (dX + parameter gradients) on the tutorial layer, from one ncu capture
+# (profiles/launches_tutorial_<path>.md), valid only for the kernel sources whose
+# SHA-256 prefix is recorded with it: any later change to them makes the figure null.
+_TRAFFIC = {
+    "tf32": (24.32e6 + 82.00e6 + 0.16e6 + 163.99e6, "924fafee9e667897"),
+    "bf16": (0.09e6 + 41.01e6 + 0.05e6 + 81.99e6, "924fafee9e667897"),
+}
+
+
+def _tc_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "kronecker_factored_structured_b200", "csrc")
+    for f in ("tc_fwd.cu", "tc_bwd.cu", "tc_ptx.cuh"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(path: str, workload: str):
+    rec = _TRAFFIC.get(path)
+    if rec is None or workload != "tutorial" or rec[1] != _tc_sources_sha():
+        return None
+    return rec[0]
 WORKLOAD = "tutorial"
 ROTATE = 3  # independent input sets cycled through, so the working set exceeds L2
 
@@ -303,11 +329,14 @@ def main():
             dist.destroy_process_group()
         return 0
 
-    # ---- roofline of the dominant kernel (the fused backward call) ----
+    # ---- roofline of the dominant call (the backward) ----
     peaks = _peaks()
     bwd_bytes = N * elt * (2 * p * m1 + q * m2)
     bwd_flops = N * (acc.flops_per_row(p, q, m1, m2, r) - acc.flops_per_row(p, q, m1, m2, r, False))
-    if path == "f32":
+    # the tensor-core kernels exist for p = q = m1 = m2 = 32, r = 4; other TF32/BF16 shapes
+    # run the CUDA-core kernels, which are bound by FP32 arithmetic
+    on_tc = path != "f32" and (p, q, m1, m2, r) == (32, 32, 32, 32, 4)
+    if not on_tc:
         peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12   # FFMA TFLOP/s at max clock
         achieved = bwd_flops / (t_bwd / 1e3) / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -317,8 +346,9 @@ def main():
     else:
         achieved = bwd_bytes / (t_bwd / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "kernel": "fused backward call", "peak_source": peaks["source"]}
+                "frac": achieved / peaks["hbm_gbs"], "traffic": _traffic(path, args.workload),
+                "kernel": "backward call: dX kernel + parameter-gradient kernel",
+                "peak_source": peaks["source"]}
 
     step_bytes = N * acc.bytes_per_row(p * m1, q * m2, elt)
     step_flops = N * acc.flops_per_row(p, q, m1, m2, r)
