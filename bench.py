@@ -192,6 +192,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=1024)
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-zero-blocks", action="store_true",
+                    help="pass KRON_FLAG_SKIP_ZERO_BLOCKS (drop products with a zero S entry)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -208,6 +210,7 @@ def main():
     from kronecker_factored_structured_b200 import dp
 
     path = args.path or ("tf32" if "tf32" in kfs.native.IMPLEMENTED_PATHS else "f32")
+    flags = 1 if args.skip_zero_blocks else 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -246,10 +249,11 @@ def main():
         x, G = sets[i % ROTATE]
         if timing is not None:
             timing[0].record(stream)
-        kfs.forward(x, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, out=y)
+        kfs.forward(x, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, flags=flags, out=y)
         if timing is not None:
             timing[1].record(stream)
-        kfs.backward(x, fac["S"], fac["A"], fac["B"], G, dtype=path, workspace=wsb, grads=grads)
+        kfs.backward(x, fac["S"], fac["A"], fac["B"], G, dtype=path, flags=flags, workspace=wsb,
+                     grads=grads)
         if timing is not None:
             timing[2].record(stream)
         if world > 1:
@@ -295,8 +299,9 @@ def main():
     def e2e_step(i):
         xd.copy_(xh[i % ROTATE], non_blocking=True)
         gd.copy_(gh[i % ROTATE], non_blocking=True)
-        kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, out=y)
-        kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, workspace=wsb, grads=grads)
+        kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, flags=flags, out=y)
+        kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, flags=flags, workspace=wsb,
+                     grads=grads)
         if world > 1:
             dp.allreduce_grads(flat)
         yh.copy_(y, non_blocking=True)
@@ -358,6 +363,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": path, "data": "synthetic",
         "config": {"workload": _workload_desc(w), "N": N, "p": p, "q": q, "m1": m1, "m2": m2,
                    "r": r, "path": path, "parallelism": f"dp{world}",
+                   "skip_zero_blocks": bool(flags),
                    "l2": f"inputs rotated over {ROTATE} independent (x, dY) sets "
                          f"({ROTATE * N * elt * (p * m1 + q * m2) / 1e6:.0f} MB > 126 MB L2)"},
         "fwd_ms": t_fwd, "bwd_ms": t_bwd,

@@ -139,7 +139,8 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
                 return fail(KRON_ERR_UNSUPPORTED,
                             "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not "
                             "fit shared memory", p, q, m1, m2, r);
-            e = kron::simt_forward(x, S, A, B, bias, y, s, bf16, cs);
+            e = kron::simt_forward(x, S, A, B, bias, y, s, bf16,
+                                   (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
             break;
         }
         default:
@@ -195,7 +196,8 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
     } else {
         // exact-FP32 CUDA-core kernels (every KRON_F32 call; TF32/BF16 shapes with no
         // compiled tensor-core kernel), then the fixed-order reduction of the partials
-        e = kron::simt_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16, cs);
+        e = kron::simt_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16,
+                                (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
         e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
                                   (float *)dA, (float *)dB, (float *)dbias, s, cs);

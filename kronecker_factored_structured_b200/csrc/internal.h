@@ -34,13 +34,15 @@ inline size_t partial_stride(const Shape &s) {
 // Rows per tile for the SIMT kernels; 0 when the shape does not fit shared memory.
 int simt_forward_rows(const Shape &s);
 int simt_backward_rows(const Shape &s);
-// I/O tensors fp32, or bf16 when bf16 is set (arithmetic fp32 either way).
+// I/O tensors fp32, or bf16 when bf16 is set (arithmetic fp32 either way).  skip drops
+// the products with a zero S entry (KRON_FLAG_SKIP_ZERO_BLOCKS; same results).
 cudaError_t simt_forward(const void *x, const void *S, const void *A, const void *B,
-                         const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st);
+                         const void *bias, void *y, const Shape &s, bool bf16, bool skip,
+                         cudaStream_t st);
 // Writes dX (if non-null) and the per-range partials into ws (parts x partial_stride).
 cudaError_t simt_backward(const void *x, const void *S, const void *A, const void *B,
                           const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                          bool bf16, cudaStream_t st);
+                          bool bf16, bool skip, cudaStream_t st);
 
 // ---- tensor-core paths (tc_fwd.cu, tc_bwd.cu): TF32 (fp32 I/O) or BF16 ----
 bool tc_forward_supported(const Shape &s, bool bf16);

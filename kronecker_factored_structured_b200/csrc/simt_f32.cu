@@ -139,15 +139,16 @@ __device__ __forceinline__ void load_rows(const TI *__restrict__ g, int64_t n0, 
 }
 
 struct FwdLayout {
-    int R, ldx, ldb, ldc, ldt;
-    size_t offX, offB, offC, offT, offY, total;  // in floats
+    int R, ldx, ldb, ldc, ldt, skip;
+    size_t offX, offB, offC, offT, offY, offI, total;  // in floats (offI: int lists)
 };
 
 inline size_t up4(size_t v) { return (v + 3) & ~(size_t)3; }  // 16-byte aligned offsets
 
-FwdLayout fwd_layout(const Shape &s, int R) {
+FwdLayout fwd_layout(const Shape &s, int R, bool skip) {
     FwdLayout L;
     L.R = R;
+    L.skip = skip;
     L.ldx = s.m1 + 1;
     L.ldb = s.m2 + 1;
     L.ldc = s.q + 1;
@@ -158,6 +159,8 @@ FwdLayout fwd_layout(const Shape &s, int R) {
     L.offC = o; o = up4(o + (size_t)s.p * L.ldc);
     L.offT = o; o = up4(o + (size_t)R * s.p * L.ldt);
     L.offY = o; o = up4(o + (size_t)R * s.q * s.m2);
+    // zero-block skip: row map [p], column pointers [q+1], column lists [p*q] (ints)
+    L.offI = o; if (skip) o = up4(o + (size_t)s.p + s.q + 1 + (size_t)s.p * s.q);
     L.total = o;
     return L;
 }
@@ -165,13 +168,14 @@ FwdLayout fwd_layout(const Shape &s, int R) {
 // acc_smem: the dC/dB/dbias accumulators live in shared memory; otherwise (large
 // r*p*q) they are accumulated in place in the CTA's own workspace partial.
 struct BwdLayout {
-    int R, ldx, ldg, ldb, ldc, ldt, acc_smem;
-    size_t offX, offG, offDX, offU, offT, offB, offC, offDC, offDB, offDb, total;
+    int R, ldx, ldg, ldb, ldc, ldt, acc_smem, skip;
+    size_t offX, offG, offDX, offU, offT, offB, offC, offDC, offDB, offDb, offI, total;
 };
 
-BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem) {
+BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem, bool skip) {
     BwdLayout L;
     L.R = R;
+    L.skip = skip;
     L.acc_smem = acc_smem;
     L.ldx = s.m1 + 1;
     L.ldg = s.m2 + 1;
@@ -192,8 +196,95 @@ BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem) {
         L.offDB = o; o = up4(o + (size_t)s.r * s.m1 * s.m2);
         L.offDb = o; o = up4(o + (size_t)s.q * s.m2);
     }
+    // zero-block skip: row pointers [p+1] and row lists [p*q] of S's nonzeros (ints)
+    L.offI = o; if (skip) o = up4(o + (size_t)s.p + 1 + (size_t)s.p * s.q);
     L.total = o;
     return L;
+}
+
+// Nonzero pattern of S for the zero-block skip (KRON_FLAG_SKIP_ZERO_BLOCKS).  C_i = S (.) A_i,
+// so C_i[a,c] = 0 for every rank wherever S[a,c] = 0 (page "kronecker-layer-benchmark",
+// introduction: a zero S entry zeroes a whole block of W); those products are dropped and
+// the others are accumulated in the same order as the dense loops, so the results equal
+// the unflagged ones.
+template <typename TI>
+__device__ __forceinline__ bool s_nz(const TI *S, int e) { return to_f(S[e]) != 0.f; }
+
+// Forward lists: rmap[a] = compact index of row a (-1 if S[a,:] is all zero), colptr /
+// colidx = for each column c the rows a (ascending) with S[a,c] != 0.  Returns the number of
+// nonzero rows.
+template <typename TI>
+__device__ int build_col_lists(const TI *__restrict__ S, const Shape &s, int *rmap, int *colptr,
+                               int *colidx, int *nrows_smem) {
+    const int P = s.p, Q = s.q;
+    for (int a = threadIdx.x; a < P; a += blockDim.x) {
+        int nz = 0;
+        for (int c = 0; c < Q; ++c) nz |= s_nz(S, a * Q + c);
+        rmap[a] = nz;
+    }
+    for (int c = threadIdx.x; c < Q; c += blockDim.x) {
+        int n = 0;
+        for (int a = 0; a < P; ++a) n += s_nz(S, a * Q + c);
+        colptr[c + 1] = n;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int a = 0; a < P; ++a) rmap[a] = rmap[a] ? n++ : -1;
+        *nrows_smem = n;
+        colptr[0] = 0;
+        for (int c = 0; c < Q; ++c) colptr[c + 1] += colptr[c];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < Q; c += blockDim.x) {
+        int t = colptr[c];
+        for (int a = 0; a < P; ++a)
+            if (s_nz(S, a * Q + c)) colidx[t++] = a;
+    }
+    __syncthreads();
+    return *nrows_smem;
+}
+
+// Backward lists: rowptr / rowidx = for each row a the columns c (ascending) with S[a,c] != 0.
+template <typename TI>
+__device__ void build_row_lists(const TI *__restrict__ S, const Shape &s, int *rowptr, int *rowidx) {
+    const int P = s.p, Q = s.q;
+    for (int a = threadIdx.x; a < P; a += blockDim.x) {
+        int n = 0;
+        for (int c = 0; c < Q; ++c) n += s_nz(S, a * Q + c);
+        rowptr[a + 1] = n;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        rowptr[0] = 0;
+        for (int a = 0; a < P; ++a) rowptr[a + 1] += rowptr[a];
+    }
+    __syncthreads();
+    for (int a = threadIdx.x; a < P; a += blockDim.x) {
+        int t = rowptr[a];
+        for (int c = 0; c < Q; ++c)
+            if (s_nz(S, a * Q + c)) rowidx[t++] = c;
+    }
+    __syncthreads();
+}
+
+// x rows of the tile, keeping only the blocks a with rmap[a] >= 0: shared row
+// (n * nra + rmap[a]) of M1 values (stride ld).
+template <typename TI>
+__device__ __forceinline__ void load_rows_compact(const TI *__restrict__ g, int64_t n0, int64_t N,
+                                                  int rows, const Shape &s, const int *rmap,
+                                                  int nra, float *sm, int ld) {
+    const int width = s.p * s.m1, w4 = width >> 2;
+    for (int e = threadIdx.x; e < rows * w4; e += blockDim.x) {
+        const int n = e / w4, c4 = (e - n * w4) << 2;
+        const int a = c4 / s.m1, j = c4 - a * s.m1;
+        const int ca = rmap[a];
+        if (ca < 0) continue;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + n < N) v = load4(g + (n0 + n) * width + c4);
+        float *d = sm + (size_t)(n * nra + ca) * ld + j;
+        d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+    }
 }
 
 // Factor i into shared memory: Bs[j*ldb + k] = B_i[j,k], Cs[a*ldc + c] = S[a,c]*A_i[a,c].
@@ -227,19 +318,46 @@ kron_fwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
     const int64_t n0 = (int64_t)blockIdx.x * R;
     const int P = s.p, Q = s.q, M1 = s.m1, M2 = s.m2;
 
-    load_rows(x, n0, s.N, R, P * M1, Xs, M1, L.ldx);
-
-    for (int i = 0; i < s.r; ++i) {
-        __syncthreads();  // previous stage 2 done with Bs/Cs/Ts
-        load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
-        __syncthreads();
-        // stage 1: T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
-        MM g1{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
-        smem_mm(g1, false);
-        __syncthreads();
-        // stage 2, batched over rows n: Y[(n,c),k] += sum_a C_i[a,c] T[(n,a),k]
-        MM g2{Cs, 0, 1, 0, L.ldc, Ts, P * L.ldt, 0, L.ldt, 1, Ys, Q * M2, M2, R, Q, M2, 1, P};
-        smem_mm(g2, i > 0);
+    if (L.skip) {
+        // zero-block skip: stage 1 only on rows a with a nonzero in S, stage 2 over each
+        // column's nonzero rows (same accumulation order as the dense loops)
+        __shared__ int nra_s;
+        int *rmap = reinterpret_cast<int *>(smem + L.offI), *colptr = rmap + P, *colidx = colptr + Q + 1;
+        const int nra = build_col_lists(S, s, rmap, colptr, colidx, &nra_s);
+        load_rows_compact(x, n0, s.N, R, s, rmap, nra, Xs, L.ldx);
+        for (int i = 0; i < s.r; ++i) {
+            __syncthreads();
+            load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
+            __syncthreads();
+            if (nra > 0) {
+                MM g1{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * nra, M2, 1, M1};
+                smem_mm(g1, false);
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < R * Q * M2; e += blockDim.x) {
+                const int n = e / (Q * M2), c = (e / M2) % Q, k = e % M2;
+                float acc = 0.f;
+                for (int t = colptr[c]; t < colptr[c + 1]; ++t) {
+                    const int a = colidx[t];
+                    acc = fmaf(Cs[a * L.ldc + c], Ts[(n * nra + rmap[a]) * L.ldt + k], acc);
+                }
+                Ys[e] = i > 0 ? Ys[e] + acc : acc;
+            }
+        }
+    } else {
+        load_rows(x, n0, s.N, R, P * M1, Xs, M1, L.ldx);
+        for (int i = 0; i < s.r; ++i) {
+            __syncthreads();  // previous stage 2 done with Bs/Cs/Ts
+            load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
+            __syncthreads();
+            // stage 1: T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
+            MM g1{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
+            smem_mm(g1, false);
+            __syncthreads();
+            // stage 2, batched over rows n: Y[(n,c),k] += sum_a C_i[a,c] T[(n,a),k]
+            MM g2{Cs, 0, 1, 0, L.ldc, Ts, P * L.ldt, 0, L.ldt, 1, Ys, Q * M2, M2, R, Q, M2, 1, P};
+            smem_mm(g2, i > 0);
+        }
     }
     __syncthreads();
     // y = Y + bias, coalesced float4 stores
@@ -279,6 +397,8 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
     for (size_t e = threadIdx.x; e < n_dc; e += blockDim.x) dCs[e] = 0.f;
     for (size_t e = threadIdx.x; e < n_db; e += blockDim.x) dBs[e] = 0.f;
     for (int e = threadIdx.x; e < Q * M2; e += blockDim.x) dbs[e] = 0.f;
+    int *rowptr = reinterpret_cast<int *>(smem + L.offI), *rowidx = rowptr + P + 1;
+    if (L.skip) build_row_lists(S, s, rowptr, rowidx);
 
     for (int64_t n0 = lo; n0 < hi; n0 += R) {
         __syncthreads();
@@ -297,9 +417,21 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
             load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
             __syncthreads();
             // U[(n,a),k] = sum_c C_i[a,c] G[(n,c),k]          (batched over n)
-            MM gu{Cs, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
-                  R, P, M2, 1, Q};
-            smem_mm(gu, false);
+            if (L.skip) {   // only the nonzero S[a,c], in the dense loop's order
+                for (int e = threadIdx.x; e < R * P * M2; e += blockDim.x) {
+                    const int n = e / (P * M2), a = (e / M2) % P, k = e % M2;
+                    float acc = 0.f;
+                    for (int t = rowptr[a]; t < rowptr[a + 1]; ++t) {
+                        const int c = rowidx[t];
+                        acc = fmaf(Cs[a * L.ldc + c], Gs[(n * Q + c) * L.ldg + k], acc);
+                    }
+                    Us[(n * P + a) * L.ldt + k] = acc;
+                }
+            } else {
+                MM gu{Cs, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
+                      R, P, M2, 1, Q};
+                smem_mm(gu, false);
+            }
             // T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
             MM gt{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
             smem_mm(gt, false);
@@ -340,17 +472,22 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
         part[n_dc + n_db + e] = dbs[e];
 }
 
-size_t fwd_bytes(const Shape &s, int R) { return fwd_layout(s, R).total * sizeof(float); }
-size_t bwd_bytes(const Shape &s, int R, bool acc_smem) {
-    return bwd_layout(s, R, acc_smem).total * sizeof(float);
+size_t fwd_bytes(const Shape &s, int R, bool skip) { return fwd_layout(s, R, skip).total * sizeof(float); }
+size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip) {
+    return bwd_layout(s, R, acc_smem, skip).total * sizeof(float);
 }
 
-// Backward tile choice: rows per tile R and where the accumulators live.
-BwdLayout bwd_choose(const Shape &s) {
+// Backward tile choice: rows per tile R and where the accumulators live.  The row split
+// (and with it the summation order of the partials) does not depend on `skip`: R is chosen
+// for the larger (skip) layout whenever that fits.
+BwdLayout bwd_choose(const Shape &s, bool skip) {
     for (int acc = 1; acc >= 0; --acc)
         for (int R : {4, 2, 1})
-            if (bwd_bytes(s, R, acc) <= kMaxSmem) return bwd_layout(s, R, acc);
-    BwdLayout none = bwd_layout(s, 1, false);
+            if (bwd_bytes(s, R, acc, true) <= kMaxSmem) return bwd_layout(s, R, acc, skip);
+    for (int acc = 1; acc >= 0; --acc)
+        for (int R : {4, 2, 1})
+            if (bwd_bytes(s, R, acc, false) <= kMaxSmem) return bwd_layout(s, R, acc, false);
+    BwdLayout none = bwd_layout(s, 1, false, false);
     none.R = 0;
     return none;
 }
@@ -359,19 +496,22 @@ BwdLayout bwd_choose(const Shape &s) {
 
 int simt_forward_rows(const Shape &s) {
     for (int R : {8, 4, 2, 1})
-        if (fwd_bytes(s, R) <= kMaxSmem) return R;
+        if (fwd_bytes(s, R, false) <= kMaxSmem) return R;
     return 0;
 }
 
-int simt_backward_rows(const Shape &s) { return bwd_choose(s).R; }
+int simt_backward_rows(const Shape &s) { return bwd_choose(s, false).R; }
 
 namespace {
 
 template <typename TI>
 cudaError_t simt_forward_t(const void *x, const void *S, const void *A, const void *B,
-                           const void *bias, void *y, const Shape &s, cudaStream_t st) {
-    const int R = simt_forward_rows(s);
-    const FwdLayout L = fwd_layout(s, R);
+                           const void *bias, void *y, const Shape &s, bool skip, cudaStream_t st) {
+    int R = simt_forward_rows(s);
+    // the skip lists need room too; rows of a tile are independent, so R may shrink
+    while (skip && R > 1 && fwd_bytes(s, R, true) > kMaxSmem) R >>= 1;
+    if (skip && fwd_bytes(s, R, true) > kMaxSmem) skip = false;
+    const FwdLayout L = fwd_layout(s, R, skip);
     const size_t smem = L.total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kron_fwd_simt_kernel<TI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -389,8 +529,8 @@ cudaError_t simt_forward_t(const void *x, const void *S, const void *A, const vo
 template <typename TI>
 cudaError_t simt_backward_t(const void *x, const void *S, const void *A, const void *B,
                             const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                            cudaStream_t st) {
-    const BwdLayout L = bwd_choose(s);
+                            bool skip, cudaStream_t st) {
+    const BwdLayout L = bwd_choose(s, skip);
     const size_t smem = L.total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kron_bwd_simt_kernel<TI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -409,16 +549,17 @@ cudaError_t simt_backward_t(const void *x, const void *S, const void *A, const v
 }  // namespace
 
 cudaError_t simt_forward(const void *x, const void *S, const void *A, const void *B,
-                         const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st) {
-    return bf16 ? simt_forward_t<__nv_bfloat16>(x, S, A, B, bias, y, s, st)
-                : simt_forward_t<float>(x, S, A, B, bias, y, s, st);
+                         const void *bias, void *y, const Shape &s, bool bf16, bool skip,
+                         cudaStream_t st) {
+    return bf16 ? simt_forward_t<__nv_bfloat16>(x, S, A, B, bias, y, s, skip, st)
+                : simt_forward_t<float>(x, S, A, B, bias, y, s, skip, st);
 }
 
 cudaError_t simt_backward(const void *x, const void *S, const void *A, const void *B,
                           const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                          bool bf16, cudaStream_t st) {
-    return bf16 ? simt_backward_t<__nv_bfloat16>(x, S, A, B, dY, dX, ws, parts, s, st)
-                : simt_backward_t<float>(x, S, A, B, dY, dX, ws, parts, s, st);
+                          bool bf16, bool skip, cudaStream_t st) {
+    return bf16 ? simt_backward_t<__nv_bfloat16>(x, S, A, B, dY, dX, ws, parts, s, skip, st)
+                : simt_backward_t<float>(x, S, A, B, dY, dX, ws, parts, s, skip, st);
 }
 
 }  // namespace kron
