@@ -10,19 +10,20 @@
 //     T [(i,k),(n,a)] = sum_j  B_i[j,k] X_n[a,j]      A = B_all^T (TMEM), B = x tile
 //     U [(i,a),(n,k)] = sum_c  C_i[a,c] G_n[c,k]      A = C_stack (TMEM), B = G tile MN-major
 //     dC[(i,a),c]    += sum_(n,k) T[n,a,i,k] G_n[c,k]  A = T2 [(i,a)][(n,k)], B = G tile
-//     dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]  A = U2 [(i,k)][(n,a)], B = x tile MN-major
+//     dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]  A = U2 [(i,k)][(n,a)], B = X^T [j][(n,a)]
 //     dbias[c*m2+k]  += sum_n G_n[c,k]
 //   dC and dB accumulate in TMEM over the CTA's fixed, contiguous range of rows and are
 //   written to the workspace as that range's partials; after a grid barrier (cooperative
 //   launch) the same kernel adds the partials in a fixed order and forms dA = dC (.) S and
 //   dS = sum_i dC_i (.) A_i (bitwise reproducible, no separate reduction launch).
 //
-// The x and G tiles serve as K-major operands (T, dC) and as MN-major ones (U, dB): TMA
-// brings each in both shared-memory layouts for TF32 (whose MN-major layout is the 128-byte
-// swizzle with 32-byte atoms), once for BF16 (one swizzled tile is valid both ways).  So no
-// thread ever transposes an input; the only permutes are the two epilogues, which move the
-// T and U accumulators (TMEM -> registers) into the K-major layouts dC and dB read, one
-// 128-byte row segment per warp store.
+// The G tile serves as a K-major operand (dC) and as an MN-major one (U): TMA brings it in
+// both shared-memory layouts for TF32 (whose MN-major layout is the 128-byte swizzle with
+// 32-byte atoms), once for BF16 (one swizzled tile is valid both ways).  dB reads a K-major
+// X^T that the dbias warps write from the x tile (an MN-major x operand costs ~40 clocks
+// more per MMA).  The other permutes are the two epilogues, which move the T and U
+// accumulators (TMEM -> registers) into the K-major layouts dC and dB read, one 128-byte
+// row segment per warp store.
 //
 // Warp roles (736 threads, one CTA per SM, tiles of the CTA's row range in order):
 //   warp 0       TMA producer: an SI-deep ring of input sets (x and G tiles)
@@ -31,7 +32,7 @@
 //   warps 3-18   epilogues in two teams taking alternate tiles (team = tile parity, which
 //                is also its TMEM slot and its T2/U2 buffers): per team, one warp per
 //                TMEM lane quadrant for T -> T2 and one for U -> U2
-//   warps 19-22  dbias column sums of the G tiles
+//   warps 19-22  X^T copies of the x tiles (for dB) and dbias column sums of the G tiles
 // Issuers run their loops as whole warps and let one elected lane issue each burst; every
 // consumer takes the tiles in order, so no mbarrier phase can be mistaken for another.
 #include "internal.h"
@@ -63,6 +64,7 @@ template <> struct BE<__nv_bfloat16> {
 
 constexpr int imin(int a, int b) { return a < b ? a : b; }
 constexpr int kPgThreads = 736;
+constexpr int kPgPrefetch = 3;  // tiles in flight to L2 ahead of the input ring
 
 template <typename T>
 __device__ __forceinline__ float bld(const void *p, size_t i) {
@@ -76,16 +78,19 @@ struct PgCfg {
     using T = T_;
     static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_;
     static constexpr int E = BE<T>::bytes;
-    static constexpr bool TWO = BE<T>::tf32;       // TF32: inputs in two layouts
+    static constexpr bool TWO = BE<T>::tf32;       // TF32: dY in two layouts
     static constexpr int NT = 2;                   // rows per tile
     static constexpr int XR = NT * P, GR = NT * Q; // tile rows: (n,a) and (n,c)
     static constexpr int XRB = M1 * E, GRB = M2 * E;  // tile row bytes = their swizzle width
     static constexpr int X_BYTES = XR * XRB, G_BYTES = GR * GRB;
-    // one input set: x (K-major), G (K-major) [, x MN-major, G MN-major]
+    // one input set: x (K-major), G (K-major) [, G MN-major] by TMA, then X^T [j][(n,a)]
+    // (K-major, 128-byte rows per K-chunk) written by the dbias warps for dB
+    static constexpr int XT_BYTES = M1 * NT * P * E;
     static constexpr int OFF_XK = 0, OFF_GK = X_BYTES;
-    static constexpr int OFF_XM = TWO ? X_BYTES + G_BYTES : OFF_XK;
-    static constexpr int OFF_GM = TWO ? 2 * X_BYTES + G_BYTES : OFF_GK;
-    static constexpr int IN_BYTES = (X_BYTES + G_BYTES) * (TWO ? 2 : 1);
+    static constexpr int OFF_GM = TWO ? X_BYTES + G_BYTES : OFF_GK;
+    static constexpr int TMA_BYTES = X_BYTES + G_BYTES * (TWO ? 2 : 1);
+    static constexpr int OFF_XT = TMA_BYTES;
+    static constexpr int IN_BYTES = TMA_BYTES + XT_BYTES;
     // intermediates: T2 [(i,a)][(n,k)] and U2 [(i,k)][(n,a)], 128 rows, K-major, SW128
     static constexpr int T2K = NT * M2, U2K = NT * P;          // K extents (elements)
     static constexpr int T2_BYTES = 128 * T2K * E, U2_BYTES = 128 * U2K * E;
@@ -113,7 +118,7 @@ struct PgCfg {
     static constexpr uint32_t ID_T = idesc_f32acc(128, XR, BE<T>::fmt);
     static constexpr uint32_t ID_U = idesc_f32acc(128, NT * M2, BE<T>::fmt) | kBMajorMN;
     static constexpr uint32_t ID_DC = idesc_f32acc(128, Q, BE<T>::fmt);
-    static constexpr uint32_t ID_DB = idesc_f32acc(128, M1, BE<T>::fmt) | kBMajorMN;
+    static constexpr uint32_t ID_DB = idesc_f32acc(128, M1, BE<T>::fmt);
     // MN-major layouts of the input tiles: TF32 128-byte rows with 32-byte atoms (4-row
     // groups), BF16 the tile's own swizzle (8-row groups); both put 1 KB per 32-byte K step
     static constexpr uint32_t MN_LAYOUT = TWO ? kLayoutSw128Atom32 : layout_type(XRB);
@@ -127,7 +132,10 @@ struct PgCfg {
     static_assert((T2K * E) % 128 == 0 && (U2K * E) % 128 == 0, "T2/U2 rows: whole 128-byte chunks");
     static_assert(P == 32 && M2 == 32, "epilogue: one 32-column TMEM load per (n, block)");
     static_assert(SI >= 2 && SB >= 2, "rings");
-    static_assert(2 * SI + 4 + 2 * SB + 2 + 2 <= BAR_BYTES / 8, "barrier region");
+    static_assert(TMA_BYTES % 1024 == 0 && XT_BYTES % 1024 == 0 && (NT * P * E) % 128 == 0,
+                  "X^T region: whole 128-byte K-chunks, 1024-aligned");
+    static_assert(M1 == 32, "X^T transpose: lanes take the 32 rows j");
+    static_assert(3 * SI + 4 + 2 * SB + 2 + 3 <= BAR_BYTES / 8, "barrier region");
     static_assert(TM_USED <= TM_COLS, "TMEM budget");
     static_assert(SMEM <= SMEM_MAX, "shared memory budget");
 };
@@ -253,7 +261,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     // barrier indices
     constexpr int IN_FULL = 0, IN_FREE = SI, D_FULL = 2 * SI, D_EMPTY = 2 * SI + 2,
                   I_FULL = 2 * SI + 4, I_EMPTY = I_FULL + SB, DONE = I_FULL + 2 * SB,
-                  DRAIN = DONE + 1, NBARS = DRAIN + 1;
+                  DRAIN = DONE + 1, XT_FULL = DRAIN + 1, NBARS = XT_FULL + SI;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
     const Abort ab{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
     auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -264,6 +272,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         for (int s = 0; s < SI; ++s) {
             mbar_init(bar(IN_FULL + s), 1);
             mbar_init(bar(IN_FREE + s), 1 + 1 + 4);  // issuer A, issuer B, dbias warps
+            mbar_init(bar(XT_FULL + s), 4);          // dbias warps: X^T written
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(bar(D_FULL + d), 1);
@@ -279,10 +288,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         mbar_init_fence();
         prefetch_tmap(&tm_xk);
         prefetch_tmap(&tm_gk);
-        if (Cfg::TWO) {
-            prefetch_tmap(&tm_xm);
-            prefetch_tmap(&tm_gm);
-        }
+        if (Cfg::TWO) prefetch_tmap(&tm_gm);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
     tc_fence_before();
@@ -323,19 +329,27 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
+            // every tile is first pulled into L2 kPgPrefetch tiles ahead of its ring load, so
+            // a ring slot waits on L2 rather than HBM (a slot is held until dC/dB of its tile
+            // are done; the load latency is part of that cycle)
+            auto prefetch = [&](int u) {
+                if (u < nt) {
+                    tma_prefetch_l2_2d(&tm_xk, 0, (t0 + u) * XR);
+                    tma_prefetch_l2_2d(&tm_gk, 0, (t0 + u) * GR);
+                }
+            };
+            for (int u = 0; u < kPgPrefetch; ++u) prefetch(u);
             int issued = 0;
             for (int u = 0; u < nt; ++u) {
+                prefetch(u + kPgPrefetch);
                 const int s = u % SI;
                 if (!mbar_wait(bar(IN_FREE + s), ((u / SI) & 1) ^ 1, ab)) break;
                 const uint32_t dst = sIn + s * Cfg::IN_BYTES;
                 const int tile = t0 + u;
-                mbar_arrive_expect_tx(bar(IN_FULL + s), Cfg::IN_BYTES);
+                mbar_arrive_expect_tx(bar(IN_FULL + s), Cfg::TMA_BYTES);
                 tma_load_2d(dst + Cfg::OFF_XK, &tm_xk, 0, tile * XR, bar(IN_FULL + s));
                 tma_load_2d(dst + Cfg::OFF_GK, &tm_gk, 0, tile * GR, bar(IN_FULL + s));
-                if (Cfg::TWO) {
-                    tma_load_2d(dst + Cfg::OFF_XM, &tm_xm, 0, tile * XR, bar(IN_FULL + s));
-                    tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * GR, bar(IN_FULL + s));
-                }
+                if (Cfg::TWO) tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * GR, bar(IN_FULL + s));
                 issued = u + 1;
             }
             for (int u = (issued > SI ? issued - SI : 0); u < issued; ++u)
@@ -376,7 +390,8 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         for (int u = 0; u < nt; ++u) {
             const int s = u % SI, b = u % SB;
             if (!warp_wait(bar(I_FULL + b), (u / SB) & 1, ab) ||
-                !warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab))
+                !warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab) ||
+                !warp_wait(bar(XT_FULL + s), (u / SI) & 1, ab))
                 break;
             tc_fence_after();
             if (elect_one()) {
@@ -391,12 +406,11 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
                                         Cfg::ID_DC, (u > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
-                for (int kk = 0; kk < Cfg::U2K * E / 32; ++kk) {   // dB, K = (n,a), x MN-major
+                for (int kk = 0; kk < Cfg::U2K * E / 32; ++kk) {   // dB, K = (n,a), B = X^T
                     const int kb = kk * 32;
                     mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DB,
                                         sdesc_kmajor(u2 + (kb / 128) * 128 * 128 + kb % 128, 128),
-                                        sdesc_mn(in + Cfg::OFF_XM + kk * 1024, Cfg::MN_LAYOUT,
-                                                 Cfg::X_BYTES, Cfg::MN_SBO),
+                                        sdesc_kmajor(in + Cfg::OFF_XT + (kb / 128) * M1 * 128 + kb % 128, 128),
                                         Cfg::ID_DB, (u > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(I_EMPTY + b));
@@ -481,6 +495,36 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         for (int u = 0; u < nt; ++u) {
             const int s = u % SI;
             if (!mbar_wait(bar(IN_FULL + s), (u / SI) & 1, ab)) break;
+            // X^T [j][(n,a)] for dB (K-major): lane j reads element j of VPC consecutive x-tile
+            // rows (one 128-byte row segment per warp load) and writes them as one 16-byte
+            // chunk of row j (8 consecutive rows j of a warp hit 8 distinct chunk slots)
+            {
+                constexpr int VPC = 16 / E;
+                const uint32_t xk = sIn + s * Cfg::IN_BYTES + Cfg::OFF_XK;
+                const uint32_t xt = sIn + s * Cfg::IN_BYTES + Cfg::OFF_XT;
+#pragma unroll
+                for (int it = tid; it < M1 * XR / VPC; it += 128) {
+                    const int j = it % M1, kap0 = (it / M1) * VPC;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        if constexpr (BE<T>::tf32) {
+                            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w[h])
+                                         : "r"(xk + koff(kap0 + h, j * E, XR, Cfg::XRB)) : "memory");
+                        } else {
+                            unsigned short lo, hi;
+                            asm volatile("ld.shared.b16 %0, [%1];" : "=h"(lo)
+                                         : "r"(xk + koff(kap0 + 2 * h, j * E, XR, Cfg::XRB)) : "memory");
+                            asm volatile("ld.shared.b16 %0, [%1];" : "=h"(hi)
+                                         : "r"(xk + koff(kap0 + 2 * h + 1, j * E, XR, Cfg::XRB)) : "memory");
+                            w[h] = (uint32_t)lo | ((uint32_t)hi << 16);
+                        }
+                    }
+                    st_shared_v4(xt + koff(j, kap0 * E, M1, 128), w[0], w[1], w[2], w[3]);
+                }
+                fence_proxy_async();
+                mbar_arrive_warp(bar(XT_FULL + s));
+            }
             const uint32_t g = sIn + s * Cfg::IN_BYTES + Cfg::OFF_GK;
 #pragma unroll
             for (int e = 0; e < PER; ++e) {
@@ -556,12 +600,9 @@ cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void
     launch_step() = "tensor map of dY";
     e = make_tmap_2d(&tgk, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GR, Cfg::GRB, false);
     if (e != cudaSuccess) return e;
-    txm = txk;
+    txm = txk;   // unused: dB reads the X^T copy the kernel writes
     tgm = tgk;
     if (Cfg::TWO) {
-        launch_step() = "MN-major tensor map of x";
-        e = make_tmap_2d(&txm, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::M1, Cfg::XR, 128, true);
-        if (e != cudaSuccess) return e;
         launch_step() = "MN-major tensor map of dY";
         e = make_tmap_2d(&tgm, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GR, 128, true);
         if (e != cudaSuccess) return e;
