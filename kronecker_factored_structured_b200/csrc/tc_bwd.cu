@@ -267,7 +267,32 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-    // ---------------- set-up: barriers, TMEM, factors into TMEM ----------------
+    const int t0 = blockIdx.x * args.tiles_per_part;
+    const int t1 = imin(t0 + args.tiles_per_part, args.num_tiles);
+    const int nt = t1 > t0 ? t1 - t0 : 0;
+    // Input ring loads of tile u (the producer's step; a slot's first use needs no wait).
+    // Every tile is first pulled into L2 kPgPrefetch tiles ahead of its ring load, so a ring
+    // slot waits on L2 rather than HBM (a slot is held until dC/dB of its tile are done; the
+    // load latency is part of that cycle).
+    auto prefetch = [&](int u) {
+        if (u < nt) {
+            tma_prefetch_l2_2d(&tm_xk, 0, (t0 + u) * XR);
+            tma_prefetch_l2_2d(&tm_gk, 0, (t0 + u) * GR);
+        }
+    };
+    auto issue = [&](int u) {
+        prefetch(u + kPgPrefetch);
+        const int s = u % SI;
+        const uint32_t dst = sIn + s * Cfg::IN_BYTES;
+        const int tile = t0 + u;
+        mbar_arrive_expect_tx(bar(IN_FULL + s), Cfg::TMA_BYTES);
+        tma_load_2d(dst + Cfg::OFF_XK, &tm_xk, 0, tile * XR, bar(IN_FULL + s));
+        tma_load_2d(dst + Cfg::OFF_GK, &tm_gk, 0, tile * GR, bar(IN_FULL + s));
+        if (Cfg::TWO) tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * GR, bar(IN_FULL + s));
+    };
+    const int pre = imin(SI, nt);   // ring sets filled before the set-up below
+
+    // ---------------- set-up: barriers, first loads, TMEM, factors into TMEM ----------------
     if (threadIdx.x == 0) {
         for (int s = 0; s < SI; ++s) {
             mbar_init(bar(IN_FULL + s), 1);
@@ -289,6 +314,9 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         prefetch_tmap(&tm_xk);
         prefetch_tmap(&tm_gk);
         if (Cfg::TWO) prefetch_tmap(&tm_gm);
+        // the first ring sets stream in while the factors are packed (warp 0 is the producer)
+        for (int u = 0; u < kPgPrefetch; ++u) prefetch(u);
+        for (int u = 0; u < pre; ++u) issue(u);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
     tc_fence_before();
@@ -322,34 +350,13 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     __syncthreads();
     tc_fence_after();
 
-    const int t0 = blockIdx.x * args.tiles_per_part;
-    const int t1 = imin(t0 + args.tiles_per_part, args.num_tiles);
-    const int nt = t1 > t0 ? t1 - t0 : 0;
-
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            // every tile is first pulled into L2 kPgPrefetch tiles ahead of its ring load, so
-            // a ring slot waits on L2 rather than HBM (a slot is held until dC/dB of its tile
-            // are done; the load latency is part of that cycle)
-            auto prefetch = [&](int u) {
-                if (u < nt) {
-                    tma_prefetch_l2_2d(&tm_xk, 0, (t0 + u) * XR);
-                    tma_prefetch_l2_2d(&tm_gk, 0, (t0 + u) * GR);
-                }
-            };
-            for (int u = 0; u < kPgPrefetch; ++u) prefetch(u);
-            int issued = 0;
-            for (int u = 0; u < nt; ++u) {
-                prefetch(u + kPgPrefetch);
-                const int s = u % SI;
-                if (!mbar_wait(bar(IN_FREE + s), ((u / SI) & 1) ^ 1, ab)) break;
-                const uint32_t dst = sIn + s * Cfg::IN_BYTES;
-                const int tile = t0 + u;
-                mbar_arrive_expect_tx(bar(IN_FULL + s), Cfg::TMA_BYTES);
-                tma_load_2d(dst + Cfg::OFF_XK, &tm_xk, 0, tile * XR, bar(IN_FULL + s));
-                tma_load_2d(dst + Cfg::OFF_GK, &tm_gk, 0, tile * GR, bar(IN_FULL + s));
-                if (Cfg::TWO) tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * GR, bar(IN_FULL + s));
+            int issued = pre;
+            for (int u = pre; u < nt; ++u) {
+                if (!mbar_wait(bar(IN_FREE + u % SI), ((u / SI) & 1) ^ 1, ab)) break;
+                issue(u);
                 issued = u + 1;
             }
             for (int u = (issued > SI ? issued - SI : 0); u < issued; ++u)

@@ -172,8 +172,20 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     auto bar = [&](int i) { return smem_u32(bars + i); };
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int my_tiles = (args.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    // x ring load of the CTA's t-th tile (the producer's step; a stage's first use needs no wait)
+    auto issue = [&](int t) {
+        const int s = t % S;
+        const int tile = blockIdx.x + t * gridDim.x;
+        mbar_arrive_expect_tx(bar(B_XFULL + s), Cfg::X_BYTES);
+#pragma unroll
+        for (int kc = 0; kc < Cfg::KC1; ++kc)
+            tma_load_2d(sX + s * Cfg::X_BYTES + kc * N1 * Cfg::SW1, &tmap_x, kc * (Cfg::SW1 / E),
+                        tile * N1, bar(B_XFULL + s));
+    };
+    const int pre = my_tiles < S ? my_tiles : S;   // stages filled before the set-up below
 
-    // ---------------- set-up: barriers, TMEM, packed factors ----------------
+    // ---------------- set-up: barriers, first loads, TMEM, packed factors ----------------
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(bar(B_XFULL + s), 1);
@@ -196,13 +208,18 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         *abort_flag.flag = 0;
         mbar_init_fence();
         prefetch_tmap(&tmap_x);
+        // the first x tiles stream in while the factors are packed (warp 0 is the producer)
+        for (int t = 0; t < pre; ++t) issue(t);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
     }
     // stage-2 B operand: C'[c][(i,a)] = S[a][c] * A_i[a][c]
+    // (thread order: consecutive c for the forward, whose S and A rows run along c;
+    // consecutive (i,a) chunks for the transposed factors, whose rows run along a)
     for (int e = threadIdx.x; e < Q * (R * P / VPC); e += blockDim.x) {
-        const int c = e / (R * P / VPC), ia0 = (e % (R * P / VPC)) * VPC;
+        const int c = TR ? e / (R * P / VPC) : e % Q;
+        const int ia0 = (TR ? e % (R * P / VPC) : e / Q) * VPC;
         float v[8];
 #pragma unroll
         for (int t = 0; t < VPC; ++t) {
@@ -246,22 +263,13 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     __syncthreads();
     tc_fence_after();
 
-    const int my_tiles = (args.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            int issued = 0;
-            for (int t = 0; t < my_tiles; ++t) {
-                const int s = t % S;
-                const uint32_t ph = (t / S) & 1;
-                if (!mbar_wait(bar(B_XEMPTY + s), ph ^ 1, abort_flag)) break;
-                const int tile = blockIdx.x + t * gridDim.x;
-                mbar_arrive_expect_tx(bar(B_XFULL + s), Cfg::X_BYTES);
-#pragma unroll
-                for (int kc = 0; kc < Cfg::KC1; ++kc)
-                    tma_load_2d(sX + s * Cfg::X_BYTES + kc * N1 * Cfg::SW1, &tmap_x,
-                                kc * (Cfg::SW1 / E), tile * N1, bar(B_XFULL + s));
+            int issued = pre;
+            for (int t = pre; t < my_tiles; ++t) {
+                if (!mbar_wait(bar(B_XEMPTY + t % S), ((t / S) & 1) ^ 1, abort_flag)) break;
+                issue(t);
                 issued = t + 1;
             }
             // drain: loads still in flight complete before the CTA may exit
