@@ -33,8 +33,8 @@ UNIT = "rows/s"
 # (profiles/launches_tutorial_<path>.md), valid only for the kernel sources whose
 # SHA-256 prefix is recorded with it: any later change to them makes the figure null.
 _TRAFFIC = {
-    "tf32": (24.32e6 + 82.00e6 + 0.16e6 + 163.99e6, "924fafee9e667897"),
-    "bf16": (0.09e6 + 41.01e6 + 0.05e6 + 81.99e6, "924fafee9e667897"),
+    "tf32": (24.76e6 + 82.00e6 + 0.17e6 + 164.01e6, "f6a7622730a0844c"),
+    "bf16": (0.08e6 + 41.01e6 + 0.08e6 + 82.00e6, "f6a7622730a0844c"),
 }
 
 
@@ -181,6 +181,44 @@ def run_reference(args, w):
     return 0
 
 
+def dense_context(fac, sets, path, steps, dev):
+    """Context only (not the product path): the same layer as a dense x @ W + bias with W
+    materialised (sum_i kron(S*A_i, B_i)), forward and backward (dX = dY W^T, dW = x^T dY,
+    dbias) as three cuBLAS GEMMs through torch, timed like the Kronecker step (CUDA events
+    around `steps` back-to-back steps over the same rotated inputs).  TF32 tensor cores are
+    allowed for the tf32 path and disallowed for f32."""
+    import torch
+    t = torch.bfloat16 if path == "bf16" else torch.float32
+    C = (fac["S"].float()[None] * fac["A"].float())
+    W = sum(torch.kron(C[i], fac["B"].float()[i]) for i in range(C.shape[0])).to(t)
+    bias = fac["bias"].to(t)
+    old = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = path == "tf32"
+    try:
+        def step(i):
+            x, G = sets[i % len(sets)]
+            y = torch.addmm(bias, x, W)
+            dx = G @ W.t()
+            dw = x.t() @ G
+            db = G.sum(0)
+            return y, dx, dw, db
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(steps):
+            step(i)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = old
+    return {"what": "dense x @ W + bias forward and backward (dX, dW, dbias) with W "
+                    "materialised, torch/cuBLAS, same inputs and timer; context only",
+            "matmul": "tf32" if path == "tf32" else path, "ms_per_step": ms}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -190,8 +228,12 @@ def main():
     ap.add_argument("--path", default=None, help="tf32 | f32 | bf16 (default: headline path)")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--ref-rows", type=int, default=1024)
-    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--cpu-rows", type=int, default=None,
+                    help="oracle rows for cpu_baseline (default: the whole batch when it is "
+                         "at most 20000 rows of 1024 + 1024 values, else 1024)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the dense-layer context timing (cuBLAS through torch)")
     ap.add_argument("--skip-zero-blocks", action="store_true",
                     help="pass KRON_FLAG_SKIP_ZERO_BLOCKS (drop products with a zero S entry)")
     args = ap.parse_args()
@@ -262,6 +304,13 @@ def main():
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    # extra device memory of one step beyond the caller's tensors (inputs, outputs and the
+    # workspace are all allocated above): the library allocates nothing itself
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_bytes = torch.cuda.memory_allocated(dev)
+    step(0)
+    torch.cuda.synchronize()
+    peak_extra = torch.cuda.max_memory_allocated(dev) - base_bytes
 
     # ---- timed region: K steps, per-call events on the launching stream ----
     marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
@@ -376,10 +425,17 @@ def main():
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "clocks": clk.summary(),
     }
+    line["memory"] = {"workspace_bytes": int(wsb.numel()), "peak_extra_bytes_per_step": int(peak_extra)}
+    if not args.no_context:
+        ctx = dense_context(fac, sets, path, max(10, min(args.steps, 100)), dev)
+        ctx["kron_ms_per_step"] = ms_step
+        ctx["kron_speedup"] = ctx["ms_per_step"] / ms_step
+        line["context_dense"] = ctx
     if world == 1 and not args.no_cpu_baseline:
-        rows_s, dt, cores = cpu_baseline(w, args.cpu_rows)
+        cpu_rows = args.cpu_rows or (N if N * (w.d_in + w.d_out) <= 20000 * 2048 else 1024)
+        rows_s, dt, cores = cpu_baseline(w, cpu_rows)
         line["cpu_baseline"] = {"value": rows_s, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"first {args.cpu_rows} of {N} rows, forward + "
+                                "sample": f"first {cpu_rows} of {N} rows, forward + "
                                           f"backward, {dt:.1f} s"}
     print(json.dumps(line), flush=True)
     if world > 1:
