@@ -372,17 +372,16 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
             tc_fence_after();
             if (elect_one()) {
                 const uint32_t in = sIn + s * Cfg::IN_BYTES;
+                const uint64_t xd = sdesc_kmajor(in + Cfg::OFF_XK, Cfg::XRB);
+                const uint64_t gd = sdesc_mn(in + Cfg::OFF_GM, Cfg::MN_LAYOUT, Q * Cfg::GRB, Cfg::MN_SBO);
 #pragma unroll
                 for (int kk = 0; kk < M1 * E / 32; ++kk)   // T[(i,k)][(n,a)], K = j
                     mma_ts<BE<T>::tf32>(tmem + Cfg::TM_DT + d * XR, tmem + Cfg::TM_BT + kk * 8,
-                                        sdesc_kmajor(in + Cfg::OFF_XK + kk * 32, Cfg::XRB), Cfg::ID_T,
-                                        kk > 0);
+                                        desc_add(xd, kk * 32), Cfg::ID_T, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < Q * E / 32; ++kk)    // U[(i,a)][(n,k)], K = c, G MN-major
                     mma_ts<BE<T>::tf32>(tmem + Cfg::TM_DU + d * NT * M2, tmem + Cfg::TM_C + kk * 8,
-                                        sdesc_mn(in + Cfg::OFF_GM + kk * 1024, Cfg::MN_LAYOUT,
-                                                 Q * Cfg::GRB, Cfg::MN_SBO),
-                                        Cfg::ID_U, kk > 0);
+                                        desc_add(gd, kk * 1024), Cfg::ID_U, kk > 0);
                 mma_commit(bar(D_FULL + d));
                 mma_commit(bar(IN_FREE + s));
             }
@@ -404,21 +403,22 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
             if (elect_one()) {
                 const uint32_t in = sIn + s * Cfg::IN_BYTES;
                 const uint32_t t2 = sI + b * Cfg::IB, u2 = t2 + Cfg::T2_BYTES;
+                const uint64_t t2d = sdesc_kmajor(t2, 128), u2d = sdesc_kmajor(u2, 128);
+                const uint64_t gkd = sdesc_kmajor(in + Cfg::OFF_GK, Cfg::GRB);
+                const uint64_t xtd = sdesc_kmajor(in + Cfg::OFF_XT, 128);
 #pragma unroll
                 for (int kk = 0; kk < Cfg::T2K * E / 32; ++kk) {   // dC, K = (n,k)
                     const int kb = kk * 32, n = kb / Cfg::GRB, ing = kb % Cfg::GRB;
-                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DC,
-                                        sdesc_kmajor(t2 + (kb / 128) * 128 * 128 + kb % 128, 128),
-                                        sdesc_kmajor(in + Cfg::OFF_GK + n * Q * Cfg::GRB + ing, Cfg::GRB),
-                                        Cfg::ID_DC, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DC, desc_add(t2d, (kb / 128) * 128 * 128 + kb % 128),
+                                        desc_add(gkd, n * Q * Cfg::GRB + ing), Cfg::ID_DC,
+                                        (u > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < Cfg::U2K * E / 32; ++kk) {   // dB, K = (n,a), B = X^T
                     const int kb = kk * 32;
-                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DB,
-                                        sdesc_kmajor(u2 + (kb / 128) * 128 * 128 + kb % 128, 128),
-                                        sdesc_kmajor(in + Cfg::OFF_XT + (kb / 128) * M1 * 128 + kb % 128, 128),
-                                        Cfg::ID_DB, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss<BE<T>::tf32>(tmem + Cfg::TM_DB, desc_add(u2d, (kb / 128) * 128 * 128 + kb % 128),
+                                        desc_add(xtd, (kb / 128) * M1 * 128 + kb % 128), Cfg::ID_DB,
+                                        (u > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(I_EMPTY + b));
                 mma_commit(bar(IN_FREE + s));

@@ -286,11 +286,12 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             tc_fence_after();
             if (elect_one()) {
                 const uint32_t d = tmem + Cfg::TM_D1 + d1 * N1;
+                const uint64_t bd0 = sdesc_kmajor(sX + s * Cfg::X_BYTES, Cfg::SW1);
 #pragma unroll
                 for (int kk = 0; kk < M1 * E / 32; ++kk) {
                     const int kb = kk * 32, ch = kb / Cfg::SW1, in = kb % Cfg::SW1;
-                    const uint64_t bd = sdesc_kmajor(sX + s * Cfg::X_BYTES + ch * N1 * Cfg::SW1 + in, Cfg::SW1);
-                    mma_ts<Elt<T>::tf32>(d, tmem + Cfg::TM_A1 + kk * 8, bd, Cfg::IDESC1, kk > 0);
+                    mma_ts<Elt<T>::tf32>(d, tmem + Cfg::TM_A1 + kk * 8,
+                                         desc_add(bd0, ch * N1 * Cfg::SW1 + in), Cfg::IDESC1, kk > 0);
                 }
                 mma_commit(bar(B_XEMPTY + s));
                 mma_commit(bar(B_D1FULL + d1));
@@ -304,6 +305,7 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         __syncwarp();
     } else if (warp == 2) {
         // ---------------- stage-2 issuer: D2[(n,k)][c] = T . C' ----------------
+        const uint64_t bd0 = sdesc_kmajor(sB2, Cfg::SW2);
         for (int t = 0; t < my_tiles; ++t) {
             const int b = t % TB, d2 = t % D2S;
             if (!warp_wait(bar(B_D2EMPTY + d2), ((t / D2S) & 1) ^ 1, abort_flag) ||
@@ -312,13 +314,12 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
             tc_fence_after();
             if (elect_one()) {
                 const uint32_t d = tmem + Cfg::TM_D2 + d2 * Q;
-                const uint32_t tb = sT + b * Cfg::T_BYTES;
+                const uint64_t ad0 = sdesc_kmajor(sT + b * Cfg::T_BYTES, Cfg::SW2);
 #pragma unroll
                 for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
                     const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
-                    const uint64_t ad = sdesc_kmajor(tb + ch * 128 * Cfg::SW2 + in, Cfg::SW2);
-                    const uint64_t bd = sdesc_kmajor(sB2 + ch * Q * Cfg::SW2 + in, Cfg::SW2);
-                    mma_ss<Elt<T>::tf32>(d, ad, bd, Cfg::IDESC2, kk > 0);
+                    mma_ss<Elt<T>::tf32>(d, desc_add(ad0, ch * 128 * Cfg::SW2 + in),
+                                         desc_add(bd0, ch * Q * Cfg::SW2 + in), Cfg::IDESC2, kk > 0);
                 }
                 mma_commit(bar(B_TEMPTY + b));
                 mma_commit(bar(B_D2FULL + d2));

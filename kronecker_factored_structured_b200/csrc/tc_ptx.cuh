@@ -328,6 +328,13 @@ __device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr, int sw) {
     return d;
 }
 
+// A descriptor for the same operand layout starting byte_off bytes further on.  The start
+// address field holds (address >> 4) in 14 bits; every shared-memory address of a CTA is
+// below 2^18 bytes, so the addition never carries out of the field.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t byte_off) {
+    return desc + (uint64_t)(byte_off >> 4);
+}
+
 // MN-major operand tile: the M (or N) dimension runs along rows of 128 B (TF32, layout
 // type 1 = 128-byte swizzle with 32-byte atoms, 4-row K groups) or of `sw` bytes (16-bit
 // types, the ordinary swizzles, 8-row K groups); `lbo` = byte stride between successive
