@@ -26,7 +26,7 @@
 namespace kron {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr size_t kMaxSmem = 227 * 1024;
 
 // Register-tiled product of shared-memory operands:
