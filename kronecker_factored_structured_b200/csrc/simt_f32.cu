@@ -44,56 +44,95 @@ struct MM {
     int batch, M, N, K1, K0;
 };
 
-__device__ __forceinline__ void smem_mm(const MM &g, bool accumulate) {
-    const int MT = (g.M + 3) >> 2, NT = (g.N + 3) >> 2;
+// Work item `t` of a product: batch b, and the TM x TN output grid {tm + u*MT} x {tn + v*NT}
+// of one thread (MT = ceil(M/TM), NT = ceil(N/TN)).
+template <int TM, int TN>
+__device__ __forceinline__ int mm_items(const MM &g) {
+    return g.batch * ((g.M + TM - 1) / TM) * ((g.N + TN - 1) / TN);
+}
+
+template <int TM, int TN>
+__device__ __forceinline__ void mm_item(const MM &g, int t, bool accumulate) {
+    const int MT = (g.M + TM - 1) / TM, NT = (g.N + TN - 1) / TN;
     const int tiles = MT * NT;
-    for (int t = threadIdx.x; t < g.batch * tiles; t += blockDim.x) {
-        const int b = t / tiles;
-        const int tt = t - b * tiles;
-        const int tm = tt / NT, tn = tt - tm * NT;
-        int row[4], col[4];
-        bool rv[4], cv[4];
+    const int b = t / tiles;
+    const int tt = t - b * tiles;
+    const int tm = tt / NT, tn = tt - tm * NT;
+    int row[TM], col[TN];
+    bool rv[TM], cv[TN];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            row[u] = tm + u * MT;
-            rv[u] = row[u] < g.M;
-            if (!rv[u]) row[u] = 0;
-            col[u] = tn + u * NT;
-            cv[u] = col[u] < g.N;
-            if (!cv[u]) col[u] = 0;
-        }
-        const float *Ab = g.A + (size_t)b * g.sab;
-        const float *Bb = g.B + (size_t)b * g.sbb;
-        float acc[4][4];
+    for (int u = 0; u < TM; ++u) {
+        row[u] = tm + u * MT;
+        rv[u] = row[u] < g.M;
+        if (!rv[u]) row[u] = 0;
+    }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+    for (int v = 0; v < TN; ++v) {
+        col[v] = tn + v * NT;
+        cv[v] = col[v] < g.N;
+        if (!cv[v]) col[v] = 0;
+    }
+    const float *Ab = g.A + (size_t)b * g.sab;
+    const float *Bb = g.B + (size_t)b * g.sbb;
+    float acc[TM][TN];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-        for (int k1 = 0; k1 < g.K1; ++k1) {
-            const float *Ak = Ab + k1 * g.sak1;
-            const float *Bk = Bb + k1 * g.sbk1;
+    for (int u = 0; u < TM; ++u)
+#pragma unroll
+        for (int v = 0; v < TN; ++v) acc[u][v] = 0.f;
+    for (int k1 = 0; k1 < g.K1; ++k1) {
+        const float *Ak = Ab + k1 * g.sak1;
+        const float *Bk = Bb + k1 * g.sbk1;
 #pragma unroll 4
-            for (int k0 = 0; k0 < g.K0; ++k0) {
-                float a[4], bb[4];
+        for (int k0 = 0; k0 < g.K0; ++k0) {
+            float a[TM], bb[TN];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) a[u] = Ak[row[u] * g.sam + k0 * g.sak0];
+            for (int u = 0; u < TM; ++u) a[u] = Ak[row[u] * g.sam + k0 * g.sak0];
 #pragma unroll
-                for (int v = 0; v < 4; ++v) bb[v] = Bk[k0 * g.sbk0 + col[v] * g.sbn];
+            for (int v = 0; v < TN; ++v) bb[v] = Bk[k0 * g.sbk0 + col[v] * g.sbn];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < TM; ++u)
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], bb[v], acc[u][v]);
-            }
+                for (int v = 0; v < TN; ++v) acc[u][v] = fmaf(a[u], bb[v], acc[u][v]);
         }
-        float *Cb = g.C + (size_t)b * g.scb;
+    }
+    float *Cb = g.C + (size_t)b * g.scb;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < TM; ++u)
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-                if (rv[u] && cv[v]) {
-                    float *c = Cb + row[u] * g.scm + col[v];
-                    *c = accumulate ? *c + acc[u][v] : acc[u][v];
-                }
+        for (int v = 0; v < TN; ++v)
+            if (rv[u] && cv[v]) {
+                float *c = Cb + row[u] * g.scm + col[v];
+                *c = accumulate ? *c + acc[u][v] : acc[u][v];
+            }
+}
+
+// One product over the whole CTA with 4 x 4 outputs per work item.
+__device__ __forceinline__ void smem_mm(const MM &g, bool accumulate) {
+    const int n = mm_items<4, 4>(g);
+    for (int t = threadIdx.x; t < n; t += blockDim.x) mm_item<4, 4>(g, t, accumulate);
+}
+
+// Two independent products sharing the CTA's threads (items of the first, then of the
+// second), each with its own output grid per item: products with few outputs take smaller
+// grids, so that every thread has work.
+template <int TM1, int TN1, int TM2, int TN2>
+__device__ __forceinline__ void smem_mm2(const MM &g1, bool acc1, const MM &g2, bool acc2) {
+    const int n1 = mm_items<TM1, TN1>(g1), n2 = mm_items<TM2, TN2>(g2);
+    for (int t = threadIdx.x; t < n1 + n2; t += blockDim.x) {
+        if (t < n1) mm_item<TM1, TN1>(g1, t, acc1);
+        else mm_item<TM2, TN2>(g2, t - n1, acc2);
+    }
+}
+
+// The same for three independent products.
+template <int TM1, int TN1, int TM2, int TN2, int TM3, int TN3>
+__device__ __forceinline__ void smem_mm3(const MM &g1, bool acc1, const MM &g2, bool acc2,
+                                         const MM &g3, bool acc3) {
+    const int n1 = mm_items<TM1, TN1>(g1), n2 = mm_items<TM2, TN2>(g2), n3 = mm_items<TM3, TN3>(g3);
+    for (int t = threadIdx.x; t < n1 + n2 + n3; t += blockDim.x) {
+        if (t < n1) mm_item<TM1, TN1>(g1, t, acc1);
+        else if (t < n1 + n2) mm_item<TM2, TN2>(g2, t - n1, acc2);
+        else mm_item<TM3, TN3>(g3, t - n1 - n2, acc3);
     }
 }
 
@@ -427,26 +466,28 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
                     }
                     Us[(n * P + a) * L.ldt + k] = acc;
                 }
+            }
+            // T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]  (with U when U is a dense product)
+            MM gt{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
+            if (L.skip) {
+                smem_mm(gt, false);
             } else {
                 MM gu{Cs, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
                       R, P, M2, 1, Q};
-                smem_mm(gu, false);
+                smem_mm2<4, 4, 4, 4>(gu, false, gt, false);
             }
-            // T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]
-            MM gt{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
-            smem_mm(gt, false);
             __syncthreads();
             // dX[(n,a),j] += sum_k U[(n,a),k] B_i[j,k]
             MM gx{Us, 0, L.ldt, 0, 1, Bs, 0, 0, 1, L.ldb, dXs, 0, L.ldx, 1, R * P, M1, 1, M2};
-            smem_mm(gx, i > 0);
             // dB_i[j,k] += sum_(n,a) X[(n,a),j] U[(n,a),k]
             MM gb{Xs, 0, 1, 0, L.ldx, Us, 0, 0, L.ldt, 1, dBs + (size_t)i * M1 * M2, 0, M2,
                   1, M1, M2, 1, R * P};
-            smem_mm(gb, true);
             // dC_i[a,c] += sum_n sum_k T[(n,a),k] G[(n,c),k]
             MM gc{Ts, 0, L.ldt, P * L.ldt, 1, Gs, 0, Q * L.ldg, 1, L.ldg,
                   dCs + (size_t)i * P * Q, 0, Q, 1, P, Q, R, M2};
-            smem_mm(gc, true);
+            // three independent products (dX reads U, dB reads X and U, dC reads T and G) in
+            // one pass: dX on 2 x 4 grids, dB and dC, whose outputs are few, on 2 x 2 grids
+            smem_mm3<2, 4, 2, 2, 2, 2>(gx, i > 0, gb, true, gc, true);
         }
         __syncthreads();
         if (dX) {
