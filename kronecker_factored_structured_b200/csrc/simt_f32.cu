@@ -207,14 +207,17 @@ FwdLayout fwd_layout(const Shape &s, int R, bool skip) {
 // acc_smem: the dC/dB/dbias accumulators live in shared memory; otherwise (large
 // r*p*q) they are accumulated in place in the CTA's own workspace partial.
 struct BwdLayout {
-    int R, ldx, ldg, ldb, ldc, ldt, acc_smem, skip;
+    int R, ldx, ldg, ldb, ldc, ldt, acc_smem, skip, resident;
     size_t offX, offG, offDX, offU, offT, offB, offC, offDC, offDB, offDb, offI, total;
 };
 
-BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem, bool skip) {
+// resident: the factors of every rank stay in shared memory for the whole kernel (loaded
+// once); otherwise rank i's are reloaded for each tile.
+BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem, bool skip, bool resident = false) {
     BwdLayout L;
     L.R = R;
     L.skip = skip;
+    L.resident = resident;
     L.acc_smem = acc_smem;
     L.ldx = s.m1 + 1;
     L.ldg = s.m2 + 1;
@@ -227,8 +230,9 @@ BwdLayout bwd_layout(const Shape &s, int R, bool acc_smem, bool skip) {
     L.offDX = o; o = up4(o + (size_t)R * s.p * L.ldx);
     L.offU = o; o = up4(o + (size_t)R * s.p * L.ldt);
     L.offT = o; o = up4(o + (size_t)R * s.p * L.ldt);
-    L.offB = o; o = up4(o + (size_t)s.m1 * L.ldb);
-    L.offC = o; o = up4(o + (size_t)s.p * L.ldc);
+    const size_t nf = resident ? (size_t)s.r : 1;   // ranks held
+    L.offB = o; o = up4(o + nf * s.m1 * L.ldb);
+    L.offC = o; o = up4(o + nf * s.p * L.ldc);
     L.offDC = L.offDB = L.offDb = o;
     if (acc_smem) {
         L.offDC = o; o = up4(o + (size_t)s.r * s.p * s.q);
@@ -438,6 +442,9 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
     for (int e = threadIdx.x; e < Q * M2; e += blockDim.x) dbs[e] = 0.f;
     int *rowptr = reinterpret_cast<int *>(smem + L.offI), *rowidx = rowptr + P + 1;
     if (L.skip) build_row_lists(S, s, rowptr, rowidx);
+    if (L.resident)   // every rank's factors, once (made visible by the first tile's barrier)
+        for (int i = 0; i < s.r; ++i)
+            load_factors(S, A, B, i, s, Bs + (size_t)i * M1 * L.ldb, L.ldb, Cs + (size_t)i * P * L.ldc, L.ldc);
 
     for (int64_t n0 = lo; n0 < hi; n0 += R) {
         __syncthreads();
@@ -453,8 +460,14 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
         }
         for (int i = 0; i < s.r; ++i) {
             __syncthreads();
-            load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
-            __syncthreads();
+            float *Bi = Bs, *Ci = Cs;
+            if (L.resident) {
+                Bi = Bs + (size_t)i * M1 * L.ldb;
+                Ci = Cs + (size_t)i * P * L.ldc;
+            } else {
+                load_factors(S, A, B, i, s, Bs, L.ldb, Cs, L.ldc);
+                __syncthreads();
+            }
             // U[(n,a),k] = sum_c C_i[a,c] G[(n,c),k]          (batched over n)
             if (L.skip) {   // only the nonzero S[a,c], in the dense loop's order
                 for (int e = threadIdx.x; e < R * P * M2; e += blockDim.x) {
@@ -462,23 +475,23 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
                     float acc = 0.f;
                     for (int t = rowptr[a]; t < rowptr[a + 1]; ++t) {
                         const int c = rowidx[t];
-                        acc = fmaf(Cs[a * L.ldc + c], Gs[(n * Q + c) * L.ldg + k], acc);
+                        acc = fmaf(Ci[a * L.ldc + c], Gs[(n * Q + c) * L.ldg + k], acc);
                     }
                     Us[(n * P + a) * L.ldt + k] = acc;
                 }
             }
             // T[(n,a),k] = sum_j X[(n,a),j] B_i[j,k]  (with U when U is a dense product)
-            MM gt{Xs, 0, L.ldx, 0, 1, Bs, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
+            MM gt{Xs, 0, L.ldx, 0, 1, Bi, 0, 0, L.ldb, 1, Ts, 0, L.ldt, 1, R * P, M2, 1, M1};
             if (L.skip) {
                 smem_mm(gt, false);
             } else {
-                MM gu{Cs, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
+                MM gu{Ci, 0, L.ldc, 0, 1, Gs, Q * L.ldg, 0, L.ldg, 1, Us, P * L.ldt, L.ldt,
                       R, P, M2, 1, Q};
                 smem_mm2<4, 4, 4, 4>(gu, false, gt, false);
             }
             __syncthreads();
             // dX[(n,a),j] += sum_k U[(n,a),k] B_i[j,k]
-            MM gx{Us, 0, L.ldt, 0, 1, Bs, 0, 0, 1, L.ldb, dXs, 0, L.ldx, 1, R * P, M1, 1, M2};
+            MM gx{Us, 0, L.ldt, 0, 1, Bi, 0, 0, 1, L.ldb, dXs, 0, L.ldx, 1, R * P, M1, 1, M2};
             // dB_i[j,k] += sum_(n,a) X[(n,a),j] U[(n,a),k]
             MM gb{Xs, 0, 1, 0, L.ldx, Us, 0, 0, L.ldt, 1, dBs + (size_t)i * M1 * M2, 0, M2,
                   1, M1, M2, 1, R * P};
@@ -514,8 +527,8 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
 }
 
 size_t fwd_bytes(const Shape &s, int R, bool skip) { return fwd_layout(s, R, skip).total * sizeof(float); }
-size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip) {
-    return bwd_layout(s, R, acc_smem, skip).total * sizeof(float);
+size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip, bool resident = false) {
+    return bwd_layout(s, R, acc_smem, skip, resident).total * sizeof(float);
 }
 
 // Backward tile choice: rows per tile R and where the accumulators live.  The row split
@@ -524,7 +537,8 @@ size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip) {
 BwdLayout bwd_choose(const Shape &s, bool skip) {
     for (int acc = 1; acc >= 0; --acc)
         for (int R : {4, 2, 1})
-            if (bwd_bytes(s, R, acc, true) <= kMaxSmem) return bwd_layout(s, R, acc, skip);
+            for (int res = 1; res >= 0; --res)
+                if (bwd_bytes(s, R, acc, true, res) <= kMaxSmem) return bwd_layout(s, R, acc, skip, res);
     for (int acc = 1; acc >= 0; --acc)
         for (int R : {4, 2, 1})
             if (bwd_bytes(s, R, acc, false) <= kMaxSmem) return bwd_layout(s, R, acc, false);
