@@ -11,6 +11,9 @@ namespace kron {
 // Name of the host-side step that failed in the last launcher call on this thread.
 const char *&launch_step();
 
+// Multiprocessor count of the current device (tc_fwd.cu).
+namespace tc { int num_sms(); }
+
 struct Shape {
     int64_t N;
     int p, q, m1, m2, r;

@@ -526,6 +526,136 @@ kron_bwd_simt_kernel(const TI *__restrict__ x, const TI *__restrict__ S,
         part[n_dc + n_db + e] = dbs[e];
 }
 
+// ---------------------------------------------------------------------------------------
+// Forward for a compiled shape (P, Q, M1, M2, R rows per tile): the same two stages with
+// compile-time strides, 4 x 8 outputs per thread and 128-bit shared-memory loads, so the
+// inner loops are FFMAs plus few loads; every rank's factors stay in shared memory and each
+// thread keeps its 4 x 8 block of Y in registers across the ranks (no Y tile in shared
+// memory).  Persistent CTAs, two per SM.
+//   stage 1, item (rb, kb): T[4rb+u][8kb+v] = sum_j X[4rb+u][j] B_i[j][8kb+v]
+//   stage 2, item (n, cb, kb): Y_n[4cb+u][8kb+v] += sum_a C_i[a][4cb+u] T[n*P+a][8kb+v]
+constexpr int kF32Threads = 256;
+
+template <int P_, int Q_, int M1_, int M2_, int R_, int RT_>
+struct F32Cfg {
+    static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_, RT = RT_;
+    static constexpr int LDX = M1 + 1;    // A operand of stage 1: scalar loads down a column
+    static constexpr int LDT = M2 + 4;    // 16-byte rows: STS.128 / LDS.128
+    static constexpr int LDB = M2 + 4, LDC = Q + 4;
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_T = OFF_X + RT * P * LDX;
+    static constexpr int OFF_B = (OFF_T + RT * P * LDT + 3) & ~3;
+    static constexpr int OFF_C = OFF_B + R * M1 * LDB;
+    static constexpr int TOTAL = OFF_C + R * P * LDC;   // floats
+    static_assert((RT * P / 4) * (M2 / 8) == kF32Threads, "stage 1: one 4 x 8 block per thread");
+    static_assert(RT * (Q / 4) * (M2 / 8) == kF32Threads, "stage 2: one 4 x 8 block per thread");
+    static_assert(P % 4 == 0 && Q % 4 == 0 && M1 % 4 == 0 && M2 % 8 == 0, "vector widths");
+    static_assert(TOTAL * 4 + 1024 <= 116736, "two CTAs per SM");
+};
+
+template <class Cfg, typename TI>
+__global__ void __launch_bounds__(kF32Threads, 2)
+kron_fwd_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI *__restrict__ A,
+                    const TI *__restrict__ B, const TI *__restrict__ bias, TI *__restrict__ y,
+                    int64_t N) {
+    constexpr int P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R, RT = Cfg::RT;
+    constexpr int LDX = Cfg::LDX, LDT = Cfg::LDT, LDB = Cfg::LDB, LDC = Cfg::LDC;
+    constexpr int KB = M2 / 8, CB = Q / 4;
+    extern __shared__ __align__(16) float smem[];
+    float *Xs = smem + Cfg::OFF_X, *Ts = smem + Cfg::OFF_T, *Bs = smem + Cfg::OFF_B, *Cs = smem + Cfg::OFF_C;
+    const int t = threadIdx.x;
+    // every rank's factors, once: Bs[i][j][k] = B_i[j][k], Cs[i][a][c] = S[a][c] A_i[a][c]
+    for (int e = t; e < R * M1 * M2; e += kF32Threads) {
+        const int i = e / (M1 * M2), j = (e / M2) % M1, k = e % M2;
+        Bs[(i * M1 + j) * LDB + k] = to_f(B[e]);
+    }
+    for (int e = t; e < R * P * Q; e += kF32Threads) {
+        const int i = e / (P * Q), a = (e / Q) % P, c = e % Q;
+        Cs[(i * P + a) * LDC + c] = to_f(S[a * Q + c]) * to_f(A[e]);
+    }
+    // this thread's items
+    const int rb = t / KB, kb1 = t % KB;                          // stage 1
+    const int n2 = t / (CB * KB), cb = (t / KB) % CB, kb2 = t % KB; // stage 2
+    const int64_t tiles = (N + RT - 1) / RT;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int64_t n0 = tile * RT;
+        __syncthreads();   // the previous tile is done with Xs (and the factors are in place)
+        constexpr int W4 = P * M1 / 4;
+        for (int e = t; e < RT * W4; e += kF32Threads) {
+            const int n = e / W4, c4 = (e % W4) * 4, a = c4 / M1, j = c4 % M1;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (n0 + n < N) v = load4(x + (n0 + n) * (P * M1) + c4);
+            float *d = Xs + (n * P + a) * LDX + j;
+            d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+        }
+        float yacc[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) yacc[u][v] = 0.f;
+        for (int i = 0; i < R; ++i) {
+            __syncthreads();   // Xs written / the previous rank's stage 2 is done with Ts
+            {
+                const float *Bi = Bs + i * M1 * LDB + kb1 * 8;
+                const float *Xr = Xs + (rb * 4) * LDX;
+                float acc[4][8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
+#pragma unroll 8
+                for (int j = 0; j < M1; ++j) {
+                    const float4 b0 = *reinterpret_cast<const float4 *>(Bi + j * LDB);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(Bi + j * LDB + 4);
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float a = Xr[u * LDX + j];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(a, bb[v], acc[u][v]);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float *d = Ts + (rb * 4 + u) * LDT + kb1 * 8;
+                    *reinterpret_cast<float4 *>(d) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+                    *reinterpret_cast<float4 *>(d + 4) = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+                }
+            }
+            __syncthreads();
+            {
+                const float *Ci = Cs + i * P * LDC + cb * 4;
+                const float *Tn = Ts + (n2 * P) * LDT + kb2 * 8;
+#pragma unroll 8
+                for (int a = 0; a < P; ++a) {
+                    const float4 c4 = *reinterpret_cast<const float4 *>(Ci + a * LDC);
+                    const float4 t0 = *reinterpret_cast<const float4 *>(Tn + a * LDT);
+                    const float4 t1 = *reinterpret_cast<const float4 *>(Tn + a * LDT + 4);
+                    const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+                    const float tt[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) yacc[u][v] = fmaf(cc[u], tt[v], yacc[u][v]);
+                }
+            }
+        }
+        // y[n][(4cb+u)*M2 + 8kb+v] = Y + bias
+        if (n0 + n2 < N) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int o = (cb * 4 + u) * M2 + kb2 * 8;
+                float v8[8];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) v8[v] = yacc[u][v] + (bias ? to_f(bias[o + v]) : 0.f);
+                TI *dst = y + (n0 + n2) * (Q * M2) + o;
+                store4(dst, make_float4(v8[0], v8[1], v8[2], v8[3]));
+                store4(dst + 4, make_float4(v8[4], v8[5], v8[6], v8[7]));
+            }
+        }
+    }
+}
+
 size_t fwd_bytes(const Shape &s, int R, bool skip) { return fwd_layout(s, R, skip).total * sizeof(float); }
 size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip, bool resident = false) {
     return bwd_layout(s, R, acc_smem, skip, resident).total * sizeof(float);
@@ -559,9 +689,30 @@ int simt_backward_rows(const Shape &s) { return bwd_choose(s, false).R; }
 
 namespace {
 
+template <class Cfg, typename TI>
+cudaError_t launch_fwd_f32(const void *x, const void *S, const void *A, const void *B,
+                           const void *bias, void *y, const Shape &s, cudaStream_t st) {
+    const size_t smem = (size_t)Cfg::TOTAL * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(kron_fwd_f32_kernel<Cfg, TI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (s.N + Cfg::RT - 1) / Cfg::RT;
+    const int64_t slots = (int64_t)tc::num_sms() * 2;   // persistent: two CTAs per SM
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles < slots ? tiles : slots));
+    cfg.blockDim = dim3(kF32Threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, kron_fwd_f32_kernel<Cfg, TI>, (const TI *)x, (const TI *)S,
+                              (const TI *)A, (const TI *)B, (const TI *)bias, (TI *)y, s.N);
+}
+
 template <typename TI>
 cudaError_t simt_forward_t(const void *x, const void *S, const void *A, const void *B,
                            const void *bias, void *y, const Shape &s, bool skip, cudaStream_t st) {
+    // compiled shapes: the tutorial layer (p = q = m1 = m2 = 32, r = 4), 8 rows per tile
+    if (!skip && s.p == 32 && s.q == 32 && s.m1 == 32 && s.m2 == 32 && s.r == 4)
+        return launch_fwd_f32<F32Cfg<32, 32, 32, 32, 4, 8>, TI>(x, S, A, B, bias, y, s, st);
     int R = simt_forward_rows(s);
     // the skip lists need room too; rows of a tile are independent, so R may shrink
     while (skip && R > 1 && fwd_bytes(s, R, true) > kMaxSmem) R >>= 1;

@@ -48,6 +48,10 @@ FUZZ = [
     (251, 48, 24, 64, 32, 4),
     (64, 1, 1, 4, 4, 2),
     (33, 5, 7, 4, 4, 5),
+    # the tutorial layer's shape, which has a compiled FP32 forward (8-row tiles): ragged N
+    (1, 32, 32, 32, 32, 4),
+    (37, 32, 32, 32, 32, 4),
+    (300, 32, 32, 32, 32, 4),
 ]
 
 
