@@ -553,7 +553,10 @@ struct F32Cfg {
     static_assert(TOTAL * 4 + 1024 <= 116736, "two CTAs per SM");
 };
 
-template <class Cfg, typename TI>
+// TR = true computes dX = dY W^T with the same two stages (dX_n = sum_i C_i G_n B_i^T): the
+// kernel's (P, Q, M1, M2) are the layer's (q, p, m2, m1), x is dY, y is dX, there is no bias,
+// and the factors are read transposed while they are packed.
+template <class Cfg, typename TI, bool TR = false>
 __global__ void __launch_bounds__(kF32Threads, 2)
 kron_fwd_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI *__restrict__ A,
                     const TI *__restrict__ B, const TI *__restrict__ bias, TI *__restrict__ y,
@@ -565,13 +568,16 @@ kron_fwd_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI
     float *Xs = smem + Cfg::OFF_X, *Ts = smem + Cfg::OFF_T, *Bs = smem + Cfg::OFF_B, *Cs = smem + Cfg::OFF_C;
     const int t = threadIdx.x;
     // every rank's factors, once: Bs[i][j][k] = B_i[j][k], Cs[i][a][c] = S[a][c] A_i[a][c]
+    // (transposed: B_i[k][j] of the layer's m2' x m1' B_i, and C_i[c][a] of its q' x p' C_i)
     for (int e = t; e < R * M1 * M2; e += kF32Threads) {
         const int i = e / (M1 * M2), j = (e / M2) % M1, k = e % M2;
-        Bs[(i * M1 + j) * LDB + k] = to_f(B[e]);
+        Bs[(i * M1 + j) * LDB + k] = to_f(B[TR ? ((size_t)i * M2 + k) * M1 + j : (size_t)e]);
     }
     for (int e = t; e < R * P * Q; e += kF32Threads) {
         const int i = e / (P * Q), a = (e / Q) % P, c = e % Q;
-        Cs[(i * P + a) * LDC + c] = to_f(S[a * Q + c]) * to_f(A[e]);
+        Cs[(i * P + a) * LDC + c] =
+            TR ? to_f(S[c * P + a]) * to_f(A[((size_t)i * Q + c) * P + a])
+               : to_f(S[a * Q + c]) * to_f(A[e]);
     }
     // this thread's items
     const int rb = t / KB, kb1 = t % KB;                          // stage 1
@@ -656,6 +662,245 @@ kron_fwd_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Parameter-gradient partials for a compiled shape (dX comes from kron_fwd_f32_kernel<TR>).
+// Per tile of RT rows, every product reads both operands with 128-bit shared loads along a
+// contiguous index, from arrays laid out for it:
+//   T  [(n,a)][(i,k)] = sum_j  XT[j][(n,a)] Ball[j][(i,k)]    -> stored as TT[(n,k)][(i,a)]
+//   U  [(n,a)][(i,k)] = sum_c  CT_i[c][a]   G[(n,c)][k]       (batch (n, i))
+//   dB [j][(i,k)]    += sum_(n,a) X[(n,a)][j] U[(n,a)][(i,k)]
+//   dC [(i,a)][c]    += sum_(n,k) TT[(n,k)][(i,a)] GT[(n,k)][c]
+//   dbias[c*m2+k]    += sum_n G[(n,c)][k]
+// dB and dC stay in registers for the CTA's whole row range, each thread summing one half of
+// every tile's K range; the two halves are added in a fixed order at the end and written as
+// the range's partials (the layout reduce.cu sums).  One CTA per SM.
+constexpr int kPgF32Threads = 256;
+
+template <int P_, int Q_, int M1_, int M2_, int R_, int RT_>
+struct PgF32Cfg {
+    static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_, RT = RT_;
+    static constexpr int LX = M1 + 4, LXT = RT * P + 4, LG = M2 + 4, LGT = Q + 4;
+    static constexpr int LTT = R * P + 4, LU = R * M2 + 4, LB = R * M2 + 4, LCT = P + 4;
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_XT = OFF_X + RT * P * LX;
+    static constexpr int OFF_G = OFF_XT + M1 * LXT;
+    static constexpr int OFF_GT = OFF_G + RT * Q * LG;
+    static constexpr int OFF_TT = OFF_GT + RT * M2 * LGT;
+    static constexpr int OFF_U = OFF_TT + RT * M2 * LTT;
+    static constexpr int OFF_B = OFF_U + RT * P * LU;
+    static constexpr int OFF_CT = OFF_B + M1 * LB;
+    static constexpr int TOTAL = OFF_CT + R * Q * LCT;   // floats
+    // work items per product, one 4 x 8 block each
+    static constexpr int NT_T = (RT * P / 4) * (R * M2 / 8);
+    static constexpr int NT_U = RT * R * (P / 4) * (M2 / 8);
+    static constexpr int NT_DB = (M1 / 4) * (R * M2 / 8);
+    static constexpr int NT_DC = (R * P / 4) * (Q / 8);
+    static_assert(NT_T == kPgF32Threads && NT_U == kPgF32Threads, "T and U: one block per thread");
+    static_assert(2 * NT_DB == kPgF32Threads && 2 * NT_DC == kPgF32Threads,
+                  "dB and dC: one block per thread and K half");
+    static_assert((Q * M2) % kPgF32Threads == 0, "dbias columns per thread");
+    static_assert(P % 4 == 0 && Q % 8 == 0 && M1 % 4 == 0 && M2 % 8 == 0 && (RT * P) % 8 == 0 &&
+                  (RT * M2) % 2 == 0, "vector widths and K halves");
+    static_assert(TOTAL * 4 <= 232448, "shared memory");
+};
+
+template <class Cfg, typename TI>
+__global__ void __launch_bounds__(kPgF32Threads, 1)
+kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI *__restrict__ A,
+                      const TI *__restrict__ B, const TI *__restrict__ G, float *__restrict__ ws,
+                      int64_t rows_per_part, size_t ws_stride, int64_t N) {
+    constexpr int P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R, RT = Cfg::RT;
+    constexpr int LX = Cfg::LX, LXT = Cfg::LXT, LG = Cfg::LG, LGT = Cfg::LGT;
+    constexpr int LTT = Cfg::LTT, LU = Cfg::LU, LB = Cfg::LB, LCT = Cfg::LCT;
+    constexpr int DBIAS = Q * M2 / kPgF32Threads;
+    extern __shared__ __align__(16) float smem[];
+    float *X = smem + Cfg::OFF_X, *XT = smem + Cfg::OFF_XT, *Gs = smem + Cfg::OFF_G;
+    float *GT = smem + Cfg::OFF_GT, *TT = smem + Cfg::OFF_TT, *U = smem + Cfg::OFF_U;
+    float *Ball = smem + Cfg::OFF_B, *CT = smem + Cfg::OFF_CT;
+    const int t = threadIdx.x;
+    // factors, once: Ball[j][(i,k)] = B_i[j][k]; CT[i][c][a] = S[a][c] A_i[a][c]
+    for (int e = t; e < R * M1 * M2; e += kPgF32Threads) {
+        const int i = e / (M1 * M2), j = (e / M2) % M1, k = e % M2;
+        Ball[j * LB + i * M2 + k] = to_f(B[e]);
+    }
+    for (int e = t; e < R * P * Q; e += kPgF32Threads) {
+        const int i = e / (P * Q), a = (e / Q) % P, c = e % Q;
+        CT[(i * Q + c) * LCT + a] = to_f(S[a * Q + c]) * to_f(A[e]);
+    }
+    // this thread's blocks
+    const int t_rb = t % (RT * P / 4), t_kb = t / (RT * P / 4);          // T: 4 (n,a) x 8 (i,k)
+    const int u_kb = t % (M2 / 8), u_ab = (t / (M2 / 8)) % (P / 4),        // U: 4 a x 8 k of (n,i)
+              u_b = t / ((M2 / 8) * (P / 4)), u_n = u_b / R, u_i = u_b % R;
+    const int half = t / Cfg::NT_DB;                                       // K half of dB and dC
+    const int db_cb = t % (R * M2 / 8), db_jb = (t % Cfg::NT_DB) / (R * M2 / 8);
+    const int dc_cb = t % (Q / 8), dc_mb = (t % Cfg::NT_DC) / (Q / 8);
+    float dB[4][8], dC[4][8], dbias[DBIAS];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) dB[u][v] = dC[u][v] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DBIAS; ++e) dbias[e] = 0.f;
+
+    const int64_t lo = (int64_t)blockIdx.x * rows_per_part;
+    const int64_t hi = lo + rows_per_part < N ? lo + rows_per_part : N;
+    for (int64_t n0 = lo; n0 < hi; n0 += RT) {
+        __syncthreads();   // the previous tile's dB/dC pass is done with X, G, TT, U
+        // x rows -> X[(n,a)][j] and XT[j][(n,a)]; dY rows -> G[(n,c)][k] and GT[(n,k)][c]
+        // (rows at or past the range end read as zero)
+        for (int e = t; e < RT * P * M1 / 4; e += kPgF32Threads) {
+            const int n = e / (P * M1 / 4), c4 = (e % (P * M1 / 4)) * 4, a = c4 / M1, j = c4 % M1;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (n0 + n < hi) v = load4(x + (n0 + n) * (P * M1) + c4);
+            *reinterpret_cast<float4 *>(X + (n * P + a) * LX + j) = v;
+            XT[(j + 0) * LXT + n * P + a] = v.x;
+            XT[(j + 1) * LXT + n * P + a] = v.y;
+            XT[(j + 2) * LXT + n * P + a] = v.z;
+            XT[(j + 3) * LXT + n * P + a] = v.w;
+        }
+        for (int e = t; e < RT * Q * M2 / 4; e += kPgF32Threads) {
+            const int n = e / (Q * M2 / 4), c4 = (e % (Q * M2 / 4)) * 4, c = c4 / M2, k = c4 % M2;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (n0 + n < hi) v = load4(G + (n0 + n) * (Q * M2) + c4);
+            *reinterpret_cast<float4 *>(Gs + (n * Q + c) * LG + k) = v;
+            GT[(n * M2 + k + 0) * LGT + c] = v.x;
+            GT[(n * M2 + k + 1) * LGT + c] = v.y;
+            GT[(n * M2 + k + 2) * LGT + c] = v.z;
+            GT[(n * M2 + k + 3) * LGT + c] = v.w;
+        }
+        __syncthreads();
+        {   // T block: rows (n,a) = 4 t_rb .. +3, columns (i,k) = 8 t_kb .. +7  -> TT
+            float acc[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
+#pragma unroll 4
+            for (int j = 0; j < M1; ++j) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(XT + j * LXT + t_rb * 4);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Ball + j * LB + t_kb * 8);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Ball + j * LB + t_kb * 8 + 4);
+                const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(aa[u], bb[v], acc[u][v]);
+            }
+            const int n = (t_rb * 4) / P, a0 = (t_rb * 4) % P;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int ik = t_kb * 8 + v, i = ik / M2, k = ik % M2;
+                *reinterpret_cast<float4 *>(TT + (n * M2 + k) * LTT + i * P + a0) =
+                    make_float4(acc[0][v], acc[1][v], acc[2][v], acc[3][v]);
+            }
+        }
+        {   // U block of (n, i): a = 4 u_ab .. +3, k = 8 u_kb .. +7
+            float acc[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
+            const float *Ci = CT + u_i * Q * LCT + u_ab * 4;
+            const float *Gn = Gs + u_n * Q * LG + u_kb * 8;
+#pragma unroll 4
+            for (int c = 0; c < Q; ++c) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(Ci + c * LCT);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Gn + c * LG);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Gn + c * LG + 4);
+                const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(aa[u], bb[v], acc[u][v]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float *d = U + (u_n * P + u_ab * 4 + u) * LU + u_i * M2 + u_kb * 8;
+                *reinterpret_cast<float4 *>(d) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+                *reinterpret_cast<float4 *>(d + 4) = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+            }
+        }
+        // dbias: this thread's columns, summed over the tile's rows
+#pragma unroll
+        for (int e = 0; e < DBIAS; ++e) {
+            const int o = t + e * kPgF32Threads, c = o / M2, k = o % M2;
+#pragma unroll
+            for (int n = 0; n < RT; ++n) dbias[e] += Gs[(n * Q + c) * LG + k];
+        }
+        __syncthreads();
+        {   // dB: j = 4 db_jb .. +3, (i,k) = 8 db_cb .. +7, K = (n,a) in this thread's half
+            constexpr int KH = RT * P / 2;
+            const float *Xk = X + (half * KH) * LX + db_jb * 4;
+            const float *Uk = U + (half * KH) * LU + db_cb * 8;
+#pragma unroll 4
+            for (int kk = 0; kk < KH; ++kk) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(Xk + kk * LX);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Uk + kk * LU);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Uk + kk * LU + 4);
+                const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) dB[u][v] = fmaf(aa[u], bb[v], dB[u][v]);
+            }
+        }
+        {   // dC: (i,a) = 4 dc_mb .. +3, c = 8 dc_cb .. +7, K = (n,k) in this thread's half
+            constexpr int KH = RT * M2 / 2;
+            const float *Tk = TT + (half * KH) * LTT + dc_mb * 4;
+            const float *Gk = GT + (half * KH) * LGT + dc_cb * 8;
+#pragma unroll 4
+            for (int kk = 0; kk < KH; ++kk) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(Tk + kk * LTT);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Gk + kk * LGT);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Gk + kk * LGT + 4);
+                const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) dC[u][v] = fmaf(aa[u], bb[v], dC[u][v]);
+            }
+        }
+    }
+    // the two K halves, added in a fixed order (half 0 + half 1), as this range's partials
+    __syncthreads();
+    float *scratch = smem;   // the tile arrays are free now
+    constexpr int NDB = R * M1 * M2, NDC = R * P * Q;
+    auto db_index = [&](int u, int v) {
+        const int j = db_jb * 4 + u, ik = db_cb * 8 + v, i = ik / M2, k = ik % M2;
+        return (i * M1 + j) * M2 + k;
+    };
+    auto dc_index = [&](int u, int v) {
+        const int ia = dc_mb * 4 + u, i = ia / P, a = ia % P, c = dc_cb * 8 + v;
+        return (i * P + a) * Q + c;
+    };
+    if (half == 1) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                scratch[db_index(u, v)] = dB[u][v];
+                scratch[NDB + dc_index(u, v)] = dC[u][v];
+            }
+    }
+    __syncthreads();
+    float *part = ws + (size_t)blockIdx.x * ws_stride;
+    if (half == 0) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                part[db_index(u, v) + NDC] = dB[u][v] + scratch[db_index(u, v)];
+                part[dc_index(u, v)] = dC[u][v] + scratch[NDB + dc_index(u, v)];
+            }
+    }
+#pragma unroll
+    for (int e = 0; e < DBIAS; ++e) part[NDC + NDB + t + e * kPgF32Threads] = dbias[e];
+}
+
 size_t fwd_bytes(const Shape &s, int R, bool skip) { return fwd_layout(s, R, skip).total * sizeof(float); }
 size_t bwd_bytes(const Shape &s, int R, bool acc_smem, bool skip, bool resident = false) {
     return bwd_layout(s, R, acc_smem, skip, resident).total * sizeof(float);
@@ -689,11 +934,11 @@ int simt_backward_rows(const Shape &s) { return bwd_choose(s, false).R; }
 
 namespace {
 
-template <class Cfg, typename TI>
+template <class Cfg, typename TI, bool TR = false>
 cudaError_t launch_fwd_f32(const void *x, const void *S, const void *A, const void *B,
                            const void *bias, void *y, const Shape &s, cudaStream_t st) {
     const size_t smem = (size_t)Cfg::TOTAL * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(kron_fwd_f32_kernel<Cfg, TI>,
+    cudaError_t e = cudaFuncSetAttribute(kron_fwd_f32_kernel<Cfg, TI, TR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (s.N + Cfg::RT - 1) / Cfg::RT;
@@ -703,7 +948,7 @@ cudaError_t launch_fwd_f32(const void *x, const void *S, const void *A, const vo
     cfg.blockDim = dim3(kF32Threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    return cudaLaunchKernelEx(&cfg, kron_fwd_f32_kernel<Cfg, TI>, (const TI *)x, (const TI *)S,
+    return cudaLaunchKernelEx(&cfg, kron_fwd_f32_kernel<Cfg, TI, TR>, (const TI *)x, (const TI *)S,
                               (const TI *)A, (const TI *)B, (const TI *)bias, (TI *)y, s.N);
 }
 
@@ -736,6 +981,30 @@ template <typename TI>
 cudaError_t simt_backward_t(const void *x, const void *S, const void *A, const void *B,
                             const void *dY, void *dX, float *ws, int parts, const Shape &s,
                             bool skip, cudaStream_t st) {
+    // compiled shape (the tutorial layer): dX by the forward kernel with transposed factors,
+    // the parameter-gradient partials by their own kernel
+    if (!skip && s.p == 32 && s.q == 32 && s.m1 == 32 && s.m2 == 32 && s.r == 4) {
+        using PC = PgF32Cfg<32, 32, 32, 32, 4, 2>;
+        cudaError_t e = cudaSuccess;
+        if (dX) {
+            const Shape ts{s.N, s.q, s.p, s.m2, s.m1, s.r};
+            e = launch_fwd_f32<F32Cfg<32, 32, 32, 32, 4, 8>, TI, true>(dY, S, A, B, nullptr, dX, ts, st);
+            if (e != cudaSuccess) return e;
+        }
+        const size_t smem = (size_t)PC::TOTAL * sizeof(float);
+        e = cudaFuncSetAttribute(kron_pgrad_f32_kernel<PC, TI>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t rows_per_part = (s.N + parts - 1) / parts;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)parts);
+        cfg.blockDim = dim3(kPgF32Threads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        return cudaLaunchKernelEx(&cfg, kron_pgrad_f32_kernel<PC, TI>, (const TI *)x, (const TI *)S,
+                                  (const TI *)A, (const TI *)B, (const TI *)dY, ws, rows_per_part,
+                                  partial_stride(s), s.N);
+    }
     const BwdLayout L = bwd_choose(s, skip);
     const size_t smem = L.total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kron_bwd_simt_kernel<TI>,
