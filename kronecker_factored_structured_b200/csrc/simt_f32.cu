@@ -673,8 +673,10 @@ kron_fwd_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const TI
 //   dbias[c*m2+k]    += sum_n G[(n,c)][k]
 // dB and dC stay in registers for the CTA's whole row range, each thread summing one half of
 // every tile's K range; the two halves are added in a fixed order at the end and written as
-// the range's partials (the layout reduce.cu sums).  One CTA per SM.
-constexpr int kPgF32Threads = 256;
+// the range's partials (the layout reduce.cu sums).  One CTA per SM of two 256-thread
+// groups: group 0 takes the T blocks and then the dB blocks, group 1 the U and dC blocks.
+constexpr int kPgF32Threads = 512;
+constexpr int kPgF32Group = 256;
 
 template <int P_, int Q_, int M1_, int M2_, int R_, int RT_>
 struct PgF32Cfg {
@@ -695,8 +697,8 @@ struct PgF32Cfg {
     static constexpr int NT_U = RT * R * (P / 4) * (M2 / 8);
     static constexpr int NT_DB = (M1 / 4) * (R * M2 / 8);
     static constexpr int NT_DC = (R * P / 4) * (Q / 8);
-    static_assert(NT_T == kPgF32Threads && NT_U == kPgF32Threads, "T and U: one block per thread");
-    static_assert(2 * NT_DB == kPgF32Threads && 2 * NT_DC == kPgF32Threads,
+    static_assert(NT_T == kPgF32Group && NT_U == kPgF32Group, "T and U: one block per thread");
+    static_assert(2 * NT_DB == kPgF32Group && 2 * NT_DC == kPgF32Group,
                   "dB and dC: one block per thread and K half");
     static_assert((Q * M2) % kPgF32Threads == 0, "dbias columns per thread");
     static_assert(P % 4 == 0 && Q % 8 == 0 && M1 % 4 == 0 && M2 % 8 == 0 && (RT * P) % 8 == 0 &&
@@ -727,18 +729,19 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
         const int i = e / (P * Q), a = (e / Q) % P, c = e % Q;
         CT[(i * Q + c) * LCT + a] = to_f(S[a * Q + c]) * to_f(A[e]);
     }
-    // this thread's blocks
-    const int t_rb = t % (RT * P / 4), t_kb = t / (RT * P / 4);          // T: 4 (n,a) x 8 (i,k)
-    const int u_kb = t % (M2 / 8), u_ab = (t / (M2 / 8)) % (P / 4),        // U: 4 a x 8 k of (n,i)
-              u_b = t / ((M2 / 8) * (P / 4)), u_n = u_b / R, u_i = u_b % R;
-    const int half = t / Cfg::NT_DB;                                       // K half of dB and dC
-    const int db_cb = t % (R * M2 / 8), db_jb = (t % Cfg::NT_DB) / (R * M2 / 8);
-    const int dc_cb = t % (Q / 8), dc_mb = (t % Cfg::NT_DC) / (Q / 8);
-    float dB[4][8], dC[4][8], dbias[DBIAS];
+    // this thread's blocks (tl: index within the group)
+    const int grp = t / kPgF32Group, tl = t % kPgF32Group;
+    const int t_rb = tl % (RT * P / 4), t_kb = tl / (RT * P / 4);        // T: 4 (n,a) x 8 (i,k)
+    const int u_kb = tl % (M2 / 8), u_ab = (tl / (M2 / 8)) % (P / 4),      // U: 4 a x 8 k of (n,i)
+              u_b = tl / ((M2 / 8) * (P / 4)), u_n = u_b / R, u_i = u_b % R;
+    const int half = tl / Cfg::NT_DB;                                      // K half of dB and dC
+    const int db_cb = tl % (R * M2 / 8), db_jb = (tl % Cfg::NT_DB) / (R * M2 / 8);
+    const int dc_cb = tl % (Q / 8), dc_mb = (tl % Cfg::NT_DC) / (Q / 8);
+    float acc2[4][8], dbias[DBIAS];   // acc2: dB (group 0) or dC (group 1) over the range
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int v = 0; v < 8; ++v) dB[u][v] = dC[u][v] = 0.f;
+        for (int v = 0; v < 8; ++v) acc2[u][v] = 0.f;
 #pragma unroll
     for (int e = 0; e < DBIAS; ++e) dbias[e] = 0.f;
 
@@ -769,7 +772,7 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
             GT[(n * M2 + k + 3) * LGT + c] = v.w;
         }
         __syncthreads();
-        {   // T block: rows (n,a) = 4 t_rb .. +3, columns (i,k) = 8 t_kb .. +7  -> TT
+        if (grp == 0) {   // T block: rows (n,a) = 4 t_rb .. +3, columns (i,k) = 8 t_kb .. +7  -> TT
             float acc[4][8];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -795,7 +798,7 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
                     make_float4(acc[0][v], acc[1][v], acc[2][v], acc[3][v]);
             }
         }
-        {   // U block of (n, i): a = 4 u_ab .. +3, k = 8 u_kb .. +7
+        else {   // U block of (n, i): a = 4 u_ab .. +3, k = 8 u_kb .. +7
             float acc[4][8];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -830,7 +833,7 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
             for (int n = 0; n < RT; ++n) dbias[e] += Gs[(n * Q + c) * LG + k];
         }
         __syncthreads();
-        {   // dB: j = 4 db_jb .. +3, (i,k) = 8 db_cb .. +7, K = (n,a) in this thread's half
+        if (grp == 0) {   // dB: j = 4 db_jb .. +3, (i,k) = 8 db_cb .. +7, K = (n,a) in this thread's half
             constexpr int KH = RT * P / 2;
             const float *Xk = X + (half * KH) * LX + db_jb * 4;
             const float *Uk = U + (half * KH) * LU + db_cb * 8;
@@ -844,10 +847,9 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) dB[u][v] = fmaf(aa[u], bb[v], dB[u][v]);
+                    for (int v = 0; v < 8; ++v) acc2[u][v] = fmaf(aa[u], bb[v], acc2[u][v]);
             }
-        }
-        {   // dC: (i,a) = 4 dc_mb .. +3, c = 8 dc_cb .. +7, K = (n,k) in this thread's half
+        } else {   // dC: (i,a) = 4 dc_mb .. +3, c = 8 dc_cb .. +7, K = (n,k) in this thread's half
             constexpr int KH = RT * M2 / 2;
             const float *Tk = TT + (half * KH) * LTT + dc_mb * 4;
             const float *Gk = GT + (half * KH) * LGT + dc_cb * 8;
@@ -861,7 +863,7 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) dC[u][v] = fmaf(aa[u], bb[v], dC[u][v]);
+                    for (int v = 0; v < 8; ++v) acc2[u][v] = fmaf(aa[u], bb[v], acc2[u][v]);
             }
         }
     }
@@ -877,14 +879,14 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
         const int ia = dc_mb * 4 + u, i = ia / P, a = ia % P, c = dc_cb * 8 + v;
         return (i * P + a) * Q + c;
     };
+    // scratch[dB | dC] holds half 1; the output index: dB after dC in the partial layout
+    auto sidx = [&](int u, int v) { return grp == 0 ? db_index(u, v) : NDB + dc_index(u, v); };
+    auto pidx = [&](int u, int v) { return grp == 0 ? NDC + db_index(u, v) : dc_index(u, v); };
     if (half == 1) {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                scratch[db_index(u, v)] = dB[u][v];
-                scratch[NDB + dc_index(u, v)] = dC[u][v];
-            }
+            for (int v = 0; v < 8; ++v) scratch[sidx(u, v)] = acc2[u][v];
     }
     __syncthreads();
     float *part = ws + (size_t)blockIdx.x * ws_stride;
@@ -892,10 +894,7 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                part[db_index(u, v) + NDC] = dB[u][v] + scratch[db_index(u, v)];
-                part[dc_index(u, v)] = dC[u][v] + scratch[NDB + dc_index(u, v)];
-            }
+            for (int v = 0; v < 8; ++v) part[pidx(u, v)] = acc2[u][v] + scratch[sidx(u, v)];
     }
 #pragma unroll
     for (int e = 0; e < DBIAS; ++e) part[NDC + NDB + t + e * kPgF32Threads] = dbias[e];
