@@ -443,6 +443,17 @@ def main():
         line["cpu_baseline"] = {"value": rows_s, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"first {cpu_rows} of {N} rows, forward + "
                                           f"backward, {dt:.1f} s"}
+        # the same oracle on one host thread, on a smaller sample (about 16x slower per row)
+        import oracle
+        all_threads = oracle.get_threads()
+        rows1 = max(64, min(cpu_rows, 1024))
+        try:
+            rows_s1, dt1, _ = cpu_baseline(w, rows1, threads=1)
+        finally:
+            oracle.set_threads(all_threads)
+        line["cpu_baseline_single_thread"] = {
+            "value": rows_s1, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {rows1} of {N} rows, forward + backward, {dt1:.1f} s"}
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
