@@ -29,9 +29,9 @@
 //   warp 0       TMA producer: an SI-deep ring of input sets (x and G tiles)
 //   warp 1       issuer A: T and U of tile t into TMEM (two accumulator slots); owns TMEM
 //   warp 2       issuer B: dC and dB of tile t from T2/U2 (an SB-deep ring in shared memory)
-//   warps 3-18   epilogues in two teams taking alternate tiles (team = tile parity, which
-//                is also its TMEM slot and its T2/U2 buffers): per team, one warp per
-//                TMEM lane quadrant for T -> T2 and one for U -> U2
+//   warps 3-18   epilogue: every tile by all 16 warps, per TMEM lane quadrant one warp for
+//                each of T -> T2 and U -> U2 and column block n = 0, 1 (the TMEM slots and
+//                T2/U2 buffers rotate tile by tile)
 //   warps 19-22  X^T copies of the x tiles (for dB) and dbias column sums of the G tiles
 // Issuers run their loops as whole warps and let one elected lane issue each burst; every
 // consumer takes the tiles in order, so no mbarrier phase can be mistaken for another.
@@ -100,7 +100,7 @@ struct PgCfg {
     static constexpr int FREE = SMEM_MAX - 1024 - BAR_BYTES;
     // the input ring holds a set from its load until dC/dB of that tile are done (the
     // longest lifetime in the pipeline), so it gets every byte the intermediates leave
-    static constexpr int SB = FREE - 4 * IB >= 8 * IN_BYTES ? 4 : 2;  // even: two teams
+    static constexpr int SB = FREE - 4 * IB >= 8 * IN_BYTES ? 4 : 2;
     static constexpr int SI = imin(12, (FREE - SB * IB) / IN_BYTES);
     static constexpr int OFF_IN = 0;
     static constexpr int OFF_I = SI * IN_BYTES;
@@ -301,10 +301,10 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(bar(D_FULL + d), 1);
-            mbar_init(bar(D_EMPTY + d), 8);          // the slot's epilogue team
+            mbar_init(bar(D_EMPTY + d), 16);         // every epilogue warp
         }
         for (int b = 0; b < SB; ++b) {
-            mbar_init(bar(I_FULL + b), 8);
+            mbar_init(bar(I_FULL + b), 16);
             mbar_init(bar(I_EMPTY + b), 1);
         }
         mbar_init(bar(DONE), 1);
@@ -431,16 +431,18 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
         if (lane == 0) mbar_wait_drain(bar(DONE), 0);
         __syncwarp();
     } else if (warp < 19) {
-        // ---------------- epilogues: T -> T2 and U -> U2, two teams on alternate tiles ----------------
-        const int team = (warp - 3) >> 3;
-        const bool is_u = ((warp - 3) >> 2) & 1;
+        // ---------------- epilogue: T -> T2 and U -> U2, all 16 warps on every tile ----------------
+        // per TMEM lane quadrant one warp for each of T and U and column block n = 0, 1
+        const int role = (warp - 3) >> 2, team = role >> 1;   // team 0: the n = 0 warps
+        const bool is_u = role & 1;
+        const int nb = role >> 1;                              // this warp's column block n
         const int qd = warp & 3, L = qd * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         // T lane (i,k), columns (n,a) -> T2 row (i,a), K (n,k);
         // U lane (i,a), columns (n,k) -> U2 row (i,k), K (n,a)
         const int i = L / 32, o = L % 32;   // o = k (T) or a (U); p = m2 = 32
         bool ok = true;
-        for (int u = team; u < nt; u += 2) {
+        for (int u = 0; u < nt; ++u) {
             const int d = u & 1, b = u % SB;
             if (!mbar_wait(bar(D_FULL + d), (u >> 1) & 1, ab) ||
                 !mbar_wait(bar(I_EMPTY + b), ((u / SB) & 1) ^ 1, ab)) {
@@ -451,7 +453,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
             const uint32_t src = tmem + lane_addr + (is_u ? Cfg::TM_DU + d * NT * M2 : Cfg::TM_DT + d * XR);
             const uint32_t dst = sI + b * Cfg::IB + (is_u ? Cfg::T2_BYTES : 0);
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {   // column block (n, w), w = a (T) or k (U)
+            for (int n = nb; n < nb + 1; ++n) {   // column block (n, w), w = a (T) or k (U)
                 uint32_t r[32];
                 tmem_load32(src + n * 32, r);
 #pragma unroll
