@@ -701,6 +701,7 @@ struct PgF32Cfg {
     static_assert(2 * NT_DB == kPgF32Group && 2 * NT_DC == kPgF32Group,
                   "dB and dC: one block per thread and K half");
     static_assert((Q * M2) % kPgF32Threads == 0, "dbias columns per thread");
+    static_assert(M1 / 4 == 8 && (R * M2 / 8) % 4 == 0, "dB block order: 8 row blocks, column blocks by 4");
     static_assert(P % 4 == 0 && Q % 8 == 0 && M1 % 4 == 0 && M2 % 8 == 0 && (RT * P) % 8 == 0 &&
                   (RT * M2) % 2 == 0, "vector widths and K halves");
     static_assert(TOTAL * 4 <= 232448, "shared memory");
@@ -735,7 +736,10 @@ kron_pgrad_f32_kernel(const TI *__restrict__ x, const TI *__restrict__ S, const 
     const int u_kb = tl % (M2 / 8), u_ab = (tl / (M2 / 8)) % (P / 4),      // U: 4 a x 8 k of (n,i)
               u_b = tl / ((M2 / 8) * (P / 4)), u_n = u_b / R, u_i = u_b % R;
     const int half = tl / Cfg::NT_DB;                                      // K half of dB and dC
-    const int db_cb = tl % (R * M2 / 8), db_jb = (tl % Cfg::NT_DB) / (R * M2 / 8);
+    // dB blocks: a warp takes 4 column blocks x 8 row blocks, so its 128-bit loads of U touch
+    // 128 contiguous bytes per instruction (one wavefront) instead of 16 spread blocks
+    const int db_h = tl % Cfg::NT_DB;
+    const int db_cb = (db_h % 4) + 4 * (db_h / 32), db_jb = (db_h / 4) % 8;
     const int dc_cb = tl % (Q / 8), dc_mb = (tl % Cfg::NT_DC) / (Q / 8);
     float acc2[4][8], dbias[DBIAS];   // acc2: dB (group 0) or dC (group 1) over the range
 #pragma unroll
