@@ -33,8 +33,8 @@ UNIT = "rows/s"
 # (profiles/launches_tutorial_<path>.md), valid only for the kernel sources whose
 # SHA-256 prefix is recorded with it: any later change to them makes the figure null.
 _TRAFFIC = {
-    "tf32": (24.60e6 + 82.00e6 + 0.15e6 + 164.01e6, "abed0ea9650e076a"),
-    "bf16": (0.04e6 + 41.01e6 + 0.70e6 + 82.00e6, "abed0ea9650e076a"),
+    "tf32": (24.06e6 + 81.99e6 + 0.42e6 + 164.00e6, "519e80ad0f62e269"),
+    "bf16": (0.77e6 + 41.02e6 + 0.32e6 + 81.99e6, "519e80ad0f62e269"),
 }
 
 
