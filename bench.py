@@ -396,6 +396,11 @@ def main():
     # the tensor-core kernels exist for p = q = m1 = m2 = 32, r = 4; other TF32/BF16 shapes
     # run the CUDA-core kernels, which are bound by FP32 arithmetic
     on_tc = path != "f32" and (p, q, m1, m2, r) == (32, 32, 32, 32, 4)
+    # kernels of this library per step: tensor cores: forward, dX, parameter gradients (with
+    # their fused reduction); CUDA cores on the tutorial shape: forward, dX, parameter-gradient
+    # partials, reduction; any other shape: forward, backward, reduction
+    compiled_f32 = path == "f32" and (p, q, m1, m2, r) == (32, 32, 32, 32, 4) and not flags
+    launches_per_step = 4 if compiled_f32 else 3
     if not on_tc:
         peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12   # FFMA TFLOP/s at max clock
         achieved = bwd_flops / (t_bwd / 1e3) / 1e12
@@ -426,7 +431,7 @@ def main():
         "gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "step_roofline_frac_hbm": (step_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3),
         "roofline": roof,
-        "gpu_launches": args.steps * 3,
+        "gpu_launches": args.steps * launches_per_step,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "clocks": clk.summary(),
