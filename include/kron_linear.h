@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define KRON_LINEAR_ABI_VERSION 1
+#define KRON_LINEAR_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define KRON_API __attribute__((visibility("default")))
@@ -117,6 +117,31 @@ KRON_API kron_status_t kron_linear_backward(const void *x, const void *S, const 
                                    int64_t N, int p, int q, int m1, int m2, int r,
                                    kron_dtype_t dtype, unsigned flags,
                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Backward with the l1 penalty on S fused into the dS epilogue.
+ *
+ * The layer is trained with the loss plus l1 * sum_{a,c} |S[a][c]| (page
+ * "kronecker-layer-benchmark", introduction: an l1 penalty on S makes S sparse and with it
+ * W block-sparse; section "Setup": the step's loss is the cross-entropy plus the model's
+ * penalty).  The gradient of that term, l1 * sign(S), is added to dS inside the kernel that
+ * writes dS, so the caller launches nothing for it:
+ *   dS [p][q] = sum_i dC_i (.) A_i + l1 * sign(S)
+ * sign(0) = 0: at S[a][c] = 0 the term is 0, the subgradient that autograd takes for |.|.
+ * The sum is formed in double and rounded once to float32.
+ *   l1   the penalty's weight, finite and >= 0 (else KRON_ERR_INVALID_ARG); with l1 == 0
+ *        the results are bit for bit those of kron_linear_backward.
+ * With N == 0 the factor gradients are zero except dS = l1 * sign(S).
+ * Every other argument, output and rule is kron_linear_backward's.  (The penalty's value is
+ * not computed: the caller adds l1 * sum|S| to the loss it reports if it wants it.)
+ */
+KRON_API kron_status_t kron_linear_backward_l1(const void *x, const void *S, const void *A,
+                                               const void *B, const void *dY, void *dX,
+                                               void *dS, void *dA, void *dB, void *dbias,
+                                               int64_t N, int p, int q, int m1, int m2, int r,
+                                               kron_dtype_t dtype, unsigned flags, double l1,
+                                               void *workspace, size_t workspace_bytes,
+                                               void *stream);
 
 /*
  * Backward without a caller-provided workspace.  (An addition of this library: the

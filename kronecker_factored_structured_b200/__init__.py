@@ -26,36 +26,41 @@ class KronLinearFunction(torch.autograd.Function):
 
     Nothing but the inputs is saved; the backward recomputes X_n B_i on chip.
     Factor gradients come back in float32 and are cast to the parameters' dtype.
+    ``l1`` > 0 makes S's gradient include that of the penalty l1 * sum|S| (added in the
+    library's dS epilogue); the penalty's value is not part of the output.
     """
 
     @staticmethod
-    def forward(ctx, x, S, A, B, bias, dtype, flags):
+    def forward(ctx, x, S, A, B, bias, dtype, flags, l1=0.0):
         ctx.save_for_backward(x, S, A, B)
-        ctx.dtype, ctx.flags, ctx.has_bias = dtype, flags, bias is not None
+        ctx.dtype, ctx.flags, ctx.has_bias, ctx.l1 = dtype, flags, bias is not None, l1
         return forward(x, S, A, B, bias, dtype=dtype, flags=flags)
 
     @staticmethod
     def backward(ctx, dY):
         x, S, A, B = ctx.saved_tensors
         g = backward(x, S, A, B, dY.contiguous(), dtype=ctx.dtype, flags=ctx.flags,
-                     need_dx=ctx.needs_input_grad[0], need_dbias=ctx.has_bias)
+                     need_dx=ctx.needs_input_grad[0], need_dbias=ctx.has_bias, l1=ctx.l1)
         cast = lambda t, like: None if t is None else t.to(like.dtype)
         dbias = cast(g["dbias"], S) if ctx.has_bias else None
         return (g["dX"], cast(g["dS"], S), cast(g["dA"], A), cast(g["dB"], B), dbias,
-                None, None)
+                None, None, None)
 
 
-def kron_linear(x, S, A, B, bias=None, dtype="tf32", flags=0):
-    return KronLinearFunction.apply(x, S, A, B, bias, dtype, flags)
+def kron_linear(x, S, A, B, bias=None, dtype="tf32", flags=0, l1=0.0):
+    return KronLinearFunction.apply(x, S, A, B, bias, dtype, flags, l1)
 
 
 class KronLinear(torch.nn.Module):
     """Drop-in linear layer with W = sum_i kron(S (.) A_i, B_i), W of shape
     (p*m1) x (q*m2); initialised as on the page "kronecker-layer-benchmark"
-    (S = ones, A_i ~ randn/sqrt(p), B_i ~ randn/sqrt(m1), bias = zeros)."""
+    (S = ones, A_i ~ randn/sqrt(p), B_i ~ randn/sqrt(m1), bias = zeros).
+
+    ``l1`` > 0 trains S under the page's penalty l1 * sum|S| with its gradient fused into
+    the backward's dS epilogue; the loss the caller computes then leaves the penalty out."""
 
     def __init__(self, in_features, out_features, block_in, block_out=None, rank=1,
-                 bias=True, dtype="tf32", flags=0, device=None):
+                 bias=True, dtype="tf32", flags=0, device=None, l1=0.0):
         super().__init__()
         block_out = block_in if block_out is None else block_out
         if in_features % block_in or out_features % block_out:
@@ -67,10 +72,10 @@ class KronLinear(torch.nn.Module):
         self.A = torch.nn.Parameter(torch.randn(rank, p, q, **kw) / math.sqrt(p))
         self.B = torch.nn.Parameter(torch.randn(rank, block_in, block_out, **kw) / math.sqrt(block_in))
         self.bias = torch.nn.Parameter(torch.zeros(out_features, **kw)) if bias else None
-        self.path, self.flags = dtype, flags
+        self.path, self.flags, self.l1 = dtype, flags, float(l1)
 
     def forward(self, x):
         shp = x.shape
         y = kron_linear(x.reshape(-1, shp[-1]).contiguous(), self.S, self.A, self.B, self.bias,
-                        self.path, self.flags)
+                        self.path, self.flags, self.l1)
         return y.reshape(*shp[:-1], y.shape[-1])

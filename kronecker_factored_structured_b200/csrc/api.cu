@@ -53,13 +53,13 @@ kron_status_t check_shape(int64_t N, int p, int q, int m1, int m2, int r, kron_d
     return KRON_OK;
 }
 
-// Number of contiguous row ranges of the backward: at most kRowParts, none empty.  A
-// function of the shape and path only, so the summation order is fixed.
 // True when the backward of this shape and dtype runs on the tensor-core kernels.
 bool tc_backward_path(const kron::Shape &s, kron_dtype_t dtype) {
     return dtype != KRON_F32 && kron::tc_backward_supported(s, dtype == KRON_BF16);
 }
 
+// Number of contiguous row ranges of the backward: at most kRowParts, none empty.  A
+// function of the shape and path only, so the summation order is fixed.
 int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
     int rows_per_tile = 0;
     if (tc_backward_path(s, dtype)) rows_per_tile = kron::tc_backward_tile_rows(s);
@@ -150,14 +150,18 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
     return KRON_OK;
 }
 
-kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, const void *B,
+// Both backward entry points.  l1 is the weight of the penalty l1 * sum|S| whose gradient
+// the dS epilogue adds (0: none, and then no term is added at all).
+static kron_status_t backward_impl(const void *x, const void *S, const void *A, const void *B,
                                    const void *dY, void *dX, void *dS, void *dA, void *dB,
                                    void *dbias, int64_t N, int p, int q, int m1, int m2, int r,
-                                   kron_dtype_t dtype, unsigned flags, void *workspace,
-                                   size_t workspace_bytes, void *stream) {
+                                   kron_dtype_t dtype, unsigned flags, double l1,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error[0] = 0;
     kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
     if (st != KRON_OK) return st;
+    if (!(l1 >= 0.0 && l1 <= 1e30))
+        return fail(KRON_ERR_INVALID_ARG, "the l1 weight must be finite and >= 0 (got %g)", l1);
     if (!S || !A || !B || !dS || !dA || !dB || (N > 0 && (!x || !dY)))
         return fail(KRON_ERR_INVALID_ARG,
                     "S, A, B, dS, dA, dB (and x, dY when N > 0) must be non-null");
@@ -167,6 +171,12 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
         return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
     const kron::Shape s{N, p, q, m1, m2, r};
     cudaStream_t cs = (cudaStream_t)stream;
+    if (N == 0 && l1 != 0.0) {  // empty batch: only the penalty's gradient l1 * sign(S)
+        const cudaError_t e = kron::reduce_partials(nullptr, 0, S, A, dtype == KRON_BF16,
+                                                    (float *)dS, (float *)dA, (float *)dB,
+                                                    (float *)dbias, s, l1, cs);
+        return e == cudaSuccess ? KRON_OK : cuda_fail(e, "penalty gradient");
+    }
     if (N == 0) {  // empty batch: every gradient is zero
         cudaError_t e = cudaMemsetAsync(dS, 0, (size_t)p * q * sizeof(float), cs);
         if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, (size_t)r * p * q * sizeof(float), cs);
@@ -191,7 +201,7 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
     const bool bf16 = dtype == KRON_BF16;
     if (on_tc) {
         e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, (float *)dS,
-                              (float *)dA, (float *)dB, (float *)dbias, bf16, cs);
+                              (float *)dA, (float *)dB, (float *)dbias, bf16, l1, cs);
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     } else {
         // exact-FP32 CUDA-core kernels (every KRON_F32 call; TF32/BF16 shapes with no
@@ -200,10 +210,28 @@ kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, 
                                 (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
         e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
-                                  (float *)dA, (float *)dB, (float *)dbias, s, cs);
+                                  (float *)dA, (float *)dB, (float *)dbias, s, l1, cs);
     }
     if (e != cudaSuccess) return cuda_fail(e, "reduction launch");
     return KRON_OK;
+}
+
+kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, const void *B,
+                                   const void *dY, void *dX, void *dS, void *dA, void *dB,
+                                   void *dbias, int64_t N, int p, int q, int m1, int m2, int r,
+                                   kron_dtype_t dtype, unsigned flags, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    return backward_impl(x, S, A, B, dY, dX, dS, dA, dB, dbias, N, p, q, m1, m2, r, dtype, flags,
+                         0.0, workspace, workspace_bytes, stream);
+}
+
+kron_status_t kron_linear_backward_l1(const void *x, const void *S, const void *A, const void *B,
+                                      const void *dY, void *dX, void *dS, void *dA, void *dB,
+                                      void *dbias, int64_t N, int p, int q, int m1, int m2, int r,
+                                      kron_dtype_t dtype, unsigned flags, double l1,
+                                      void *workspace, size_t workspace_bytes, void *stream) {
+    return backward_impl(x, S, A, B, dY, dX, dS, dA, dB, dbias, N, p, q, m1, m2, r, dtype, flags,
+                         l1, workspace, workspace_bytes, stream);
 }
 
 kron_status_t kron_linear_device_error(int clear) {

@@ -59,19 +59,23 @@ bool tc_backward_supported(const Shape &s, bool bf16);
 int tc_backward_tile_rows(const Shape &s);
 // Writes dX (if non-null) and the final dS, dA, dB, dbias (dbias may be null).  ws holds
 // parts x partial_stride floats of row-range partials followed by one grid-barrier word
-// (tc_backward_workspace_extra bytes).
+// (tc_backward_workspace_extra bytes).  l1 != 0 adds l1 * sign(S) to dS.
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                        float *dS, float *dA, float *dB, float *dbias, bool bf16,
+                        float *dS, float *dA, float *dB, float *dbias, bool bf16, double l1,
                         cudaStream_t st);
 constexpr size_t tc_backward_workspace_extra = 256;
 // Device error word of the tensor-core kernels (bounded waits); -1 if unreadable.
 int tc_read_device_error(bool clear);
 
 // ---- deterministic reduction of the row-range partials (reduce.cu) ----
-// S and A are float (is_bf16 = false) or bfloat16 (is_bf16 = true).
+// S and A are float (is_bf16 = false) or bfloat16 (is_bf16 = true).  l1 != 0 adds
+// l1 * sign(S) to dS.  parts == 0 reads nothing from ws (every partial sum is zero).
 cudaError_t reduce_partials(const float *ws, int parts, const void *S, const void *A,
                             bool is_bf16, float *dS, float *dA, float *dB, float *dbias,
-                            const Shape &s, cudaStream_t st);
+                            const Shape &s, double l1, cudaStream_t st);
+
+// sign(v) in {-1, 0, +1} (0 for zero and NaN): the subgradient of |v| that autograd takes.
+__host__ __device__ inline double sign_of(float v) { return (double)((v > 0.f) - (v < 0.f)); }
 
 }  // namespace kron

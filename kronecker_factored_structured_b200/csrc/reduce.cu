@@ -1,9 +1,11 @@
 // reduce.cu -- deterministic reduction of the backward's row-range partials and the
 // factor-gradient epilogue:
 //   dC_i = sum over row ranges of the partial dC_i   (fixed order)
-//   dA_i = dC_i (.) S,   dS = sum_i dC_i (.) A_i,   dB_i and dbias likewise summed.
+//   dA_i = dC_i (.) S,   dS = sum_i dC_i (.) A_i (+ l1 * sign(S)),   dB_i and dbias summed.
 // (dA_i and dS follow from C_i = S (.) A_i by the product rule; W = sum_i kron(C_i, B_i)
-// as on the page "kronecker-layer-benchmark", section "1. Build W, then multiply".)
+// as on the page "kronecker-layer-benchmark", section "1. Build W, then multiply".  The
+// optional l1 term is the gradient of the penalty l1 * sum|S| that the same page's
+// introduction puts on S.)
 //
 // Workspace layout per range g: ws[g*stride + ...] = [dC: r*p*q][dB: r*m1*m2][dbias: q*m2].
 // Each block owns 32 consecutive output columns (for dC: 32 (a,c) positions and all r
@@ -75,7 +77,7 @@ __global__ void __launch_bounds__(32 * kWarps)
 kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
                    const TI *__restrict__ S, const TI *__restrict__ A, float *__restrict__ dS,
                    float *__restrict__ dA, float *__restrict__ dB, float *__restrict__ dbias,
-                   Shape s, int blocks_dc, int blocks_db) {
+                   Shape s, int blocks_dc, int blocks_db, double l1) {
     __shared__ double red[kWarps][33];
     const size_t pq = (size_t)s.p * s.q;
     const size_t n_dc = (size_t)s.r * pq, n_db = (size_t)s.r * s.m1 * s.m2;
@@ -101,7 +103,10 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
                 }
             }
         }
-        if (threadIdx.y == 0 && v) dS[col] = (float)ds;
+        if (threadIdx.y == 0 && v) {
+            if (l1 != 0.0) ds += l1 * sign_of(to_f(S[col]));   // d(l1 * sum|S|)/dS
+            dS[col] = (float)ds;
+        }
         return;
     }
     blk -= blocks_dc;
@@ -127,7 +132,7 @@ kron_reduce_kernel(const float *__restrict__ ws, int parts, size_t stride,
 
 cudaError_t reduce_partials(const float *ws, int parts, const void *S, const void *A,
                             bool is_bf16, float *dS, float *dA, float *dB, float *dbias,
-                            const Shape &s, cudaStream_t st) {
+                            const Shape &s, double l1, cudaStream_t st) {
     const size_t pq = (size_t)s.p * s.q;
     const int blocks_dc = (int)((pq + 31) / 32);
     const int blocks_db = (int)(((size_t)s.r * s.m1 * s.m2 + 31) / 32);
@@ -140,9 +145,9 @@ cudaError_t reduce_partials(const float *ws, int parts, const void *S, const voi
     if (is_bf16)
         return cudaLaunchKernelEx(&cfg, kron_reduce_kernel<__nv_bfloat16>, ws, parts, stride,
                                   (const __nv_bfloat16 *)S, (const __nv_bfloat16 *)A, dS, dA, dB,
-                                  dbias, s, blocks_dc, blocks_db);
+                                  dbias, s, blocks_dc, blocks_db, l1);
     return cudaLaunchKernelEx(&cfg, kron_reduce_kernel<float>, ws, parts, stride, (const float *)S,
-                              (const float *)A, dS, dA, dB, dbias, s, blocks_dc, blocks_db);
+                              (const float *)A, dS, dA, dB, dbias, s, blocks_dc, blocks_db, l1);
 }
 
 }  // namespace kron

@@ -15,7 +15,8 @@
 //   dC and dB accumulate in TMEM over the CTA's fixed, contiguous range of rows and are
 //   written to the workspace as that range's partials; after a grid barrier (cooperative
 //   launch) the same kernel adds the partials in a fixed order and forms dA = dC (.) S and
-//   dS = sum_i dC_i (.) A_i (bitwise reproducible, no separate reduction launch).
+//   dS = sum_i dC_i (.) A_i, plus l1 * sign(S) when the page's l1 penalty on S is fused
+//   (bitwise reproducible, no separate reduction launch).
 //
 // The G tile serves as a K-major operand (dC) and as an MN-major one (U): TMA brings it in
 // both shared-memory layouts for TF32 (whose MN-major layout is the 128-byte swizzle with
@@ -149,6 +150,7 @@ struct PgArgs {
     int *device_error;
     unsigned *arrived;     // grid barrier counter (zeroed by the host before the launch)
     float *dS, *dA, *dB, *dbias;
+    double l1;             // weight of the penalty l1 * sum|S| whose gradient joins dS
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
@@ -164,8 +166,8 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
 // GS groups of threads each sum the ranges g' = ps, ps + GS, ... of one column in double
 // with four accumulators, and the GS group sums are added in a fixed order.  Only `parts`
 // decides the order, so the results are bitwise reproducible.  The epilogue forms
-// dA_i = dC_i (.) S and dS = sum_i dC_i (.) A_i (C_i = S (.) A_i, product rule) and writes
-// dB and dbias.
+// dA_i = dC_i (.) S and dS = sum_i dC_i (.) A_i (C_i = S (.) A_i, product rule), adds
+// l1 * sign(S) to dS when the l1 penalty is fused, and writes dB and dbias.
 template <class Cfg>
 __device__ void reduce_ranges(const PgArgs &args, int parts, double *red, double *vals) {
     using T = typename Cfg::T;
@@ -214,6 +216,7 @@ __device__ void reduce_ranges(const PgArgs &args, int parts, double *red, double
                         args.dA[(size_t)i * P * Q + pos] = (float)(dc * sv);
                         ds += dc * (double)bld<T>(args.A, (size_t)i * P * Q + pos);
                     }
+                    if (args.l1 != 0.0) ds += args.l1 * sign_of((float)sv);
                     args.dS[pos] = (float)ds;
                 }
             } else if (v < NDC + NDB) {
@@ -598,7 +601,7 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
 template <class Cfg>
 cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void *B, const void *dY,
                          float *ws, int parts, const Shape &s, float *dS, float *dA, float *dB,
-                         float *dbias, cudaStream_t st) {
+                         float *dbias, double l1, cudaStream_t st) {
     using T = typename Cfg::T;
     const bool bf16 = !BE<T>::tf32;
     CUtensorMap txk, tgk, txm, tgm;
@@ -628,6 +631,7 @@ cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void
     a.device_error = device_error_ptr();
     a.arrived = reinterpret_cast<unsigned *>(ws + (size_t)parts * a.ws_stride);
     a.dS = dS; a.dA = dA; a.dB = dB; a.dbias = dbias;
+    a.l1 = l1;
     launch_step() = "grid barrier reset";
     e = cudaMemsetAsync(a.arrived, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return e;
@@ -647,7 +651,7 @@ cudaError_t launch_pgrad(const void *x, const void *S, const void *A, const void
 
 using PgFn = cudaError_t (*)(const void *, const void *, const void *, const void *, const void *,
                              float *, int, const Shape &, float *, float *, float *, float *,
-                             cudaStream_t);
+                             double, cudaStream_t);
 struct PgEntry {
     int p, q, m1, m2, r;
     bool bf16;
@@ -676,7 +680,7 @@ int tc_backward_tile_rows(const Shape &) { return 2; }
 
 cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
                         const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                        float *dS, float *dA, float *dB, float *dbias, bool bf16,
+                        float *dS, float *dA, float *dB, float *dbias, bool bf16, double l1,
                         cudaStream_t st) {
     tc::PgFn fn = tc::find_pg(s, bf16);
     if (!fn) return cudaErrorNotSupported;
@@ -684,7 +688,7 @@ cudaError_t tc_backward(const void *x, const void *S, const void *A, const void 
         const cudaError_t e = tc_dx(dY, S, A, B, dX, s, bf16, st);
         if (e != cudaSuccess) return e;
     }
-    return fn(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, st);
+    return fn(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, l1, st);
 }
 
 }  // namespace kron

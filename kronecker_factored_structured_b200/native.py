@@ -28,7 +28,8 @@ STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
           6: "KRON_ERR_TIMEOUT"}
 
 # Every symbol include/kron_linear.h declares.
-EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_noalloc",
+EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_l1",
+           "kron_linear_backward_noalloc",
            "kron_linear_workspace_size",
            "kron_status_string", "kron_last_error", "kron_linear_device_error",
            "kron_linear_abi_version")
@@ -59,6 +60,10 @@ def load(path: str = LIB_PATH):
     lib.kron_linear_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                          i64, I, I, I, I, I, I, U, vp, sz, vp]
     lib.kron_linear_backward.restype = I
+    lib.kron_linear_backward_l1.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            i64, I, I, I, I, I, I, U, ctypes.c_double,
+                                            vp, sz, vp]
+    lib.kron_linear_backward_l1.restype = I
     lib.kron_linear_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                  i64, I, I, I, I, I, I, U, vp]
     lib.kron_linear_backward_noalloc.restype = I
@@ -142,11 +147,13 @@ def forward(x, S, A, B, bias=None, dtype="tf32", flags=0, out=None, stream=None)
 
 
 def backward(x, S, A, B, dY, dtype="tf32", flags=0, need_dx=True, need_dbias=True,
-             workspace=None, grads=None, stream=None):
+             workspace=None, grads=None, stream=None, l1=0.0):
     """Gradients of <dY, y>: returns dict(dX, dS, dA, dB, dbias).
 
     dX has the I/O dtype; dS, dA, dB and dbias are float32.  ``grads`` may hold
     preallocated outputs (same keys); ``workspace`` a preallocated uint8 buffer.
+    ``l1`` > 0 adds the gradient l1 * sign(S) of the penalty l1 * sum|S| to dS inside the
+    library's dS epilogue (kron_linear_backward_l1).
     """
     p, q, m1, m2, r = shapes(S, A, B)
     N = x.shape[0]
@@ -173,8 +180,12 @@ def backward(x, S, A, B, dY, dtype="tf32", flags=0, need_dx=True, need_dbias=Tru
     ws_bytes = workspace_size(N, p, q, m1, m2, r, dtype)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    _check(load().kron_linear_backward(
-        _ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(dY), _ptr(g["dX"]), _ptr(g["dS"]),
-        _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dbias"]), N, p, q, m1, m2, r, DTYPES[dtype], flags,
-        _ptr(workspace), workspace.numel(), _stream(stream)))
+    ptrs = (_ptr(x), _ptr(S), _ptr(A), _ptr(B), _ptr(dY), _ptr(g["dX"]), _ptr(g["dS"]),
+            _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dbias"]), N, p, q, m1, m2, r, DTYPES[dtype],
+            flags)
+    tail = (_ptr(workspace), workspace.numel(), _stream(stream))
+    if l1:
+        _check(load().kron_linear_backward_l1(*ptrs, float(l1), *tail))
+    else:
+        _check(load().kron_linear_backward(*ptrs, *tail))
     return g

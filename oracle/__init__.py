@@ -64,6 +64,7 @@ class Oracle:
         lib.oracle_forward.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, dp]
         lib.oracle_backward.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I,
                                         dp, dp, dp, dp, dp]
+        lib.oracle_l1_grad.argtypes = [dp, I, I, ctypes.c_double, dp]
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_get_threads.restype = I
         self._lib = lib
@@ -115,6 +116,15 @@ class Oracle:
                                   _ptr(dX), _ptr(dS), _ptr(dA), _ptr(dB), _ptr(dbias))
         return {"dX": dX, "dS": dS, "dA": dA, "dB": dB, "dbias": dbias}
 
+    def l1_grad(self, S, lam: float) -> np.ndarray:
+        """Gradient lam * sign(S) of the penalty lam * sum|S| (0 where S is 0)."""
+        S = _f64(S)
+        if S.ndim != 2:
+            raise ValueError("S must be p x q")
+        out = np.empty_like(S)
+        self._lib.oracle_l1_grad(_ptr(S), S.shape[0], S.shape[1], float(lam), _ptr(out))
+        return out
+
 
 _default = None
 
@@ -144,3 +154,7 @@ def forward(x, S, A, B, bias=None) -> np.ndarray:
 
 def backward(x, S, A, B, G, need_dx: bool = True, need_params: bool = True) -> dict:
     return default().backward(x, S, A, B, G, need_dx, need_params)
+
+
+def l1_grad(S, lam: float) -> np.ndarray:
+    return default().l1_grad(S, lam)

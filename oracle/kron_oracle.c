@@ -26,6 +26,10 @@
  *     dS        = sum_i dC_i (.) A_i
  *     dbias     = sum_n G[n]
  *
+ * The tutorial trains S under an l1 penalty lam * sum|S| (same page, introduction);
+ * oracle_l1_grad gives that term's gradient, lam * sign(S), which the library can add
+ * to dS.
+ *
  * Everything is double precision, row-major and contiguous:
  *   x [N][p*m1], y and G [N][q*m2], S [p][q], A [r][p][q], B [r][m1][m2],
  *   bias [q*m2], W [p*m1][q*m2].
@@ -191,4 +195,18 @@ void oracle_backward(const double *x, const double *S, const double *A, const do
         }
     }
     free(W);
+}
+
+/*
+ * Gradient of the l1 penalty lam * sum_{a,c} |S[a][c]| that the page
+ * "kronecker-layer-benchmark" (introduction) puts on S, added to the step's loss
+ * (section "Setup"): out[a][c] = lam * sign(S[a][c]).  |.| has no derivative at 0; the
+ * value taken there is 0, the subgradient autograd uses for abs().
+ */
+void oracle_l1_grad(const double *S, int p, int q, double lam, double *out)
+{
+    for (long ac = 0; ac < (long)p * q; ++ac) {
+        const double v = S[ac];
+        out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);
+    }
 }

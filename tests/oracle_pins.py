@@ -16,7 +16,9 @@ Sources of truth used here (none of them is the oracle's own loop):
   * special shapes that reduce to a plain GEMM,
   * central finite differences of L = <G, y> (exact here: L is affine in each
     single parameter coordinate), and Euler's identity for functions that are
-    linear in one argument.
+    linear in one argument,
+  * for the l1 penalty lam * sum|S| on S: central differences away from the kink at
+    0, and torch's autograd of abs() for the value taken at S = 0.
 """
 from __future__ import annotations
 
@@ -242,6 +244,37 @@ def pin_zero_s_gradient(orc):
     assert np.abs(g["dS"][z]).min() > 1e-8
 
 
+def pin_l1_grad_finite_differences(orc):
+    """Gradient of the penalty lam * sum|S| (page "kronecker-layer-benchmark", introduction:
+    an l1 term on S).  Away from 0, |.| is linear on [v - h, v + h] when h < |v|, so the
+    central difference of the penalty is exact; the entries that are 0 get 0, the
+    subgradient torch's autograd returns for abs() there (checked with torch itself)."""
+    import torch
+    rng = np.random.default_rng(115)
+    p, q, lam = 7, 5, 0.37
+    S = rng.standard_normal((p, q))
+    S[rng.random((p, q)) < 0.3] = 0.0
+    S[0, 0], S[0, 1] = 0.0, -2.5
+    g = orc.l1_grad(S, lam)
+    pen = lambda M: lam * float(np.abs(M).sum())
+    for idx in np.ndindex(S.shape):
+        v = S[idx]
+        if v == 0.0:
+            continue
+        h = 0.5 * abs(v)
+        Sp, Sm = S.copy(), S.copy()
+        Sp[idx], Sm[idx] = v + h, v - h
+        fd = (pen(Sp) - pen(Sm)) / (2 * h)
+        assert abs(fd - g[idx]) < 1e-12 * (1 + abs(fd)), (idx, fd, g[idx])
+    St = torch.tensor(S, dtype=torch.float64, requires_grad=True)
+    (lam * St.abs().sum()).backward()
+    z = S == 0.0
+    assert z.sum() >= 1
+    assert np.array_equal(g[z], St.grad.numpy()[z])
+    assert np.all(g[z] == 0.0)
+    assert np.array_equal(orc.l1_grad(S, 0.0), np.zeros_like(S))
+
+
 ALL_PINS = [
     pin_weight_is_sum_of_numpy_krons,
     pin_forward_brute_force,
@@ -257,4 +290,5 @@ ALL_PINS = [
     pin_linearity_identities,
     pin_backward_numpy_chain_rule,
     pin_zero_s_gradient,
+    pin_l1_grad_finite_differences,
 ]

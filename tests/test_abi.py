@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = native.load()
-    assert lib.kron_linear_abi_version() == 1
+    assert lib.kron_linear_abi_version() == 2
     for code, name in native.STATUS.items():
         assert lib.kron_status_string(code).decode().startswith(name)
 
@@ -94,6 +94,30 @@ def test_backward_rejects(kwargs, status):
 def test_backward_rejects_misaligned_workspace():
     need = kfs.workspace_size(8, 2, 2, 4, 4, 1, "f32")
     assert bwd(ws=V(0x10010), ws_bytes=need) == 3
+
+
+@pytest.mark.parametrize("l1", [-1.0, float("nan"), float("inf"), -1e-300])
+def test_backward_l1_rejects_bad_weight(l1):
+    """The penalty weight must be finite and >= 0; checked before any pointer is read."""
+    lib = native.load()
+    need = kfs.workspace_size(8, 2, 2, 4, 4, 1, "f32")
+    st = lib.kron_linear_backward_l1(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                     ALIGNED, ALIGNED, ALIGNED, None, 8, 2, 2, 4, 4, 1, 0, 0, l1,
+                                     ALIGNED, need, None)
+    assert st == 1
+    assert "l1" in lib.kron_last_error().decode()
+
+
+def test_backward_l1_runs_the_same_checks():
+    lib = native.load()
+    st = lib.kron_linear_backward_l1(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                     None, ALIGNED, ALIGNED, None, 8, 2, 2, 4, 4, 1, 0, 0, 0.5,
+                                     ALIGNED, 1 << 20, None)
+    assert st == 1                                  # dS missing
+    st = lib.kron_linear_backward_l1(MISALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                     ALIGNED, ALIGNED, ALIGNED, None, 8, 2, 2, 4, 4, 1, 0, 0, 0.5,
+                                     ALIGNED, 1 << 20, None)
+    assert st == 3
 
 
 def test_python_binding_raises_without_cuda_tensors():

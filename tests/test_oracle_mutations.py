@@ -37,6 +37,12 @@ MUTATIONS = [
     ("dC_uses_only_first_rank_of_B",
      "B[((long)i * m1 + j) * m2 + k];\n                    dC",
      "B[((long)0 * m1 + j) * m2 + k];\n                    dC", 0),
+    ("l1_grad_wrong_sign", "out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);",
+     "out[ac] = v > 0.0 ? -lam : (v < 0.0 ? lam : 0.0);", 0),
+    ("l1_grad_nonzero_at_kink", "out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);",
+     "out[ac] = v >= 0.0 ? lam : -lam;", 0),
+    ("l1_grad_drops_weight", "out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);",
+     "out[ac] = v > 0.0 ? 1.0 : (v < 0.0 ? -1.0 : 0.0);", 0),
 ]
 
 
