@@ -19,6 +19,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -33,8 +34,8 @@ UNIT = "rows/s"
 # (profiles/launches_tutorial_<path>.md), valid only for the kernel sources whose
 # SHA-256 prefix is recorded with it: any later change to them makes the figure null.
 _TRAFFIC = {
-    "tf32": (24.06e6 + 81.99e6 + 0.42e6 + 164.00e6, "519e80ad0f62e269"),
-    "bf16": (0.77e6 + 41.02e6 + 0.32e6 + 81.99e6, "519e80ad0f62e269"),
+    "tf32": (82.00e6 + 24.35e6 + 163.99e6 + 0.85e6, "8113c98ef788a49a"),
+    "bf16": (41.01e6 + 0.14e6 + 81.99e6 + 0.37e6, "8113c98ef788a49a"),
 }
 
 
@@ -75,8 +76,78 @@ def _workload_desc(w):
             f"m1={w.m1} m2={w.m2}, r={w.r}, {w.dtype} I/O{zero}")
 
 
+class _NvmlRegion:
+    """SM clock and clock-event reasons read through NVML every `period` seconds by a
+    background thread while the timed region runs (nvidia-smi's -lms sampling is too coarse
+    for a region of tens of milliseconds).  Reads only; any NVML failure leaves it empty."""
+    NAMES = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+             ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+             ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+             ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device: int, period: float = 0.002):
+        self.samples, self.period, self.error = [], period, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            self._nv = pynvml
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except pynvml.NVMLError:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                    f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML on this host: the nvidia-smi samples remain
+            self._nv, self.error = None, f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        nv, h = self._nv, self._h
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._nv is not None:
+            try:
+                self._nv.nvmlShutdown()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, bits in self.samples:
+            for name, attr in self.NAMES:
+                if bits & getattr(self._nv, attr):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz for mhz, _ in self.samples),
+                "sm_max_mhz": float(self.max_mhz), "reasons": sorted(reasons),
+                "samples": len(self.samples),
+                "sampler": f"NVML every {self.period * 1e3:.0f} ms inside the timed region"}
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms around the timed region,
+    and NVML every 2 ms inside it (begin_region / end_region); the NVML samples are the
+    record when there are any."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -94,6 +165,14 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def begin_region(self):
+        self.nvml = _NvmlRegion(torch_current_device())
+        self.nvml.start()
+
+    def end_region(self):
+        if getattr(self, "nvml", None) is not None:
+            self.nvml.stop()
 
     def wait_started(self, timeout=5.0):
         """Block until nvidia-smi has printed its first sample (it takes ~0.5 s to start)."""
@@ -116,6 +195,10 @@ class ClockSampler:
             self.lines = [ln for ln in (getattr(self, "first", "") + out).splitlines() if ln.strip()]
 
     def summary(self):
+        fine = self.nvml.summary() if getattr(self, "nvml", None) is not None else None
+        if fine is not None:
+            fine["nvidia_smi_samples"] = len(getattr(self, "lines", []) or [])
+            return fine
         if not getattr(self, "lines", None):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         sm, smax, reasons = [], [], set()
@@ -133,6 +216,11 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def torch_current_device() -> int:
+    import torch
+    return torch.cuda.current_device()
 
 
 def cpu_baseline(w, rows: int, threads: int | None = None):
@@ -320,11 +408,13 @@ def main():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        clk.begin_region()
         start.record(stream)
         for i in range(args.steps):
             step(i)
         end.record(stream)
         torch.cuda.synchronize()
+        clk.end_region()
         if world > 1:
             dist.barrier()
     ms = start.elapsed_time(end)

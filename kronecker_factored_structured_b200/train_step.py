@@ -10,6 +10,10 @@ One step is:
 - backward;
 - an Adam update.
 
+The penalty's gradient takes one of two routes: autograd through |S| (the page's form), or,
+for the model `kron_fused_l1`, the library's backward, which adds lambda * sign(S) where it
+writes dS (the penalty then enters the loss as a value only).
+
 Inputs and labels are random, seeded, and resident on the device.
 
 For context, the same step is timed for the page's dense baselines: three `nn.Linear`, with
@@ -37,17 +41,25 @@ import kronecker_factored_structured_b200 as kfs
 
 
 class KronMLP(nn.Module):
-    def __init__(self, d=1024, classes=10, block=32, rank=4, path="tf32", device="cuda"):
+    """``fused_l1=lam``: the layers' backward adds lam * sign(S) to dS, and penalty()
+    returns sum|S| without a gradient; the caller scales it by the same lam for the loss
+    value it reports."""
+
+    def __init__(self, d=1024, classes=10, block=32, rank=4, path="tf32", device="cuda",
+                 fused_l1=None):
         super().__init__()
-        self.l1 = kfs.KronLinear(d, d, block, rank=rank, dtype=path, device=device)
-        self.l2 = kfs.KronLinear(d, d, block, rank=rank, dtype=path, device=device)
+        lam = 0.0 if fused_l1 is None else float(fused_l1)
+        self.fused_l1 = fused_l1
+        self.l1 = kfs.KronLinear(d, d, block, rank=rank, dtype=path, device=device, l1=lam)
+        self.l2 = kfs.KronLinear(d, d, block, rank=rank, dtype=path, device=device, l1=lam)
         self.head = nn.Linear(d, classes, device=device, dtype=kfs.native.io_dtype(path))
 
     def forward(self, x):
         return self.head(torch.relu(self.l2(torch.relu(self.l1(x)))))
 
     def penalty(self):
-        return self.l1.S.float().abs().sum() + self.l2.S.float().abs().sum()
+        pen = self.l1.S.float().abs().sum() + self.l2.S.float().abs().sum()
+        return pen.detach() if self.fused_l1 is not None else pen
 
 
 class DenseMLP(nn.Module):
@@ -81,6 +93,9 @@ def time_model(model, batch, d, classes, lam, warmup, steps, dtype, seed=0, grap
     step (forward, loss, backward, Adam) is captured once in a CUDA graph and replayed, so
     the host issues one launch per step instead of one per kernel.  Adam keeps its step
     count on the device (capturable) when graphed, or when asked to."""
+    fused = getattr(model, "fused_l1", None)
+    if fused is not None and fused != lam:
+        raise ValueError(f"the model fuses the penalty weight {fused}, the step uses {lam}")
     g = torch.Generator(device="cuda").manual_seed(seed)
     x = torch.randn(batch, d, device="cuda", generator=g).to(dtype)
     labels = torch.randint(0, classes, (batch,), device="cuda", generator=g)
@@ -154,7 +169,9 @@ def main(argv=None):
     try:
         for batch in [int(v) for v in args.batches.split(",")]:
             torch.manual_seed(0)
-            models = {"kron": KronMLP(d, classes, args.block, args.rank, args.path)}
+            models = {"kron": KronMLP(d, classes, args.block, args.rank, args.path),
+                      "kron_fused_l1": KronMLP(d, classes, args.block, args.rank, args.path,
+                                               fused_l1=args.lam)}
             if not args.no_dense:
                 models["dense"] = DenseMLP(d, classes, args.block, False, dtype)
                 models["dense_group_lasso"] = DenseMLP(d, classes, args.block, True, dtype)

@@ -25,12 +25,14 @@ pytestmark = pytest.mark.gpu
 TOL = {"f32": 1e-4, "tf32": 1e-2}
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["autograd_l1", "fused_l1"])
 @pytest.mark.parametrize("path", ["f32", "tf32"])
-def test_mlp_gradients_match_oracle_chain_rule(path):
+def test_mlp_gradients_match_oracle_chain_rule(path, fused):
+    """fused: the penalty's gradient comes from the layers' backward (dS epilogue)."""
     from kronecker_factored_structured_b200.train_step import KronMLP
     torch.manual_seed(11)
     lam = 1e-3
-    model = KronMLP(1024, 10, block=32, rank=4, path=path)
+    model = KronMLP(1024, 10, block=32, rank=4, path=path, fused_l1=lam if fused else None)
     with torch.no_grad():   # non-trivial S (zeros included) and biases
         for l in (model.l1, model.l2):
             l.S.copy_(torch.randn_like(l.S))

@@ -40,3 +40,20 @@ def test_kron_mlp_refuses_cpu_tensors():
     assert float(model.penalty().detach()) == pytest.approx(2 * 64)
     with pytest.raises((ValueError, RuntimeError)):
         model(torch.randn(4, 64))
+
+
+def test_kron_mlp_fused_penalty_is_a_value_only():
+    """With the penalty's gradient fused into the layers' backward, penalty() carries no
+    gradient of its own (else S would get lam * sign(S) twice), and the layers hold lam."""
+    model = KronMLP(d=64, classes=10, block=8, rank=2, path="f32", device="cpu", fused_l1=0.25)
+    pen = model.penalty()
+    assert not pen.requires_grad and float(pen) == pytest.approx(2 * 64)
+    assert model.l1.l1 == 0.25 and model.l2.l1 == 0.25
+    assert KronMLP(d=64, classes=10, block=8, rank=2, path="f32", device="cpu").l1.l1 == 0.0
+
+
+def test_time_model_refuses_mismatched_penalty_weight():
+    from kronecker_factored_structured_b200.train_step import time_model
+    model = KronMLP(d=64, classes=10, block=8, rank=2, path="f32", device="cpu", fused_l1=0.25)
+    with pytest.raises(ValueError):
+        time_model(model, 4, 64, 10, 0.5, warmup=0, steps=1, dtype=torch.float32)
