@@ -87,6 +87,19 @@ class DenseMLP(nn.Module):
         return self._blocks_norm(self.l1.weight) + self._blocks_norm(self.l2.weight)
 
 
+_SIDE = None
+
+
+def _side_stream():
+    """The one side stream that every graph warm-up uses.  A new stream per model would
+    give each its own cuBLAS workspace, kept for the life of the process, and every later
+    model's peak memory would include the earlier ones'."""
+    global _SIDE
+    if _SIDE is None:
+        _SIDE = torch.cuda.Stream()
+    return _SIDE
+
+
 def time_model(model, batch, d, classes, lam, warmup, steps, dtype, seed=0, graph=False,
                capturable=None):
     """Times `steps` training steps after `warmup` untimed ones.  With graph=True the whole
@@ -115,7 +128,7 @@ def time_model(model, batch, d, classes, lam, warmup, steps, dtype, seed=0, grap
 
     if graph:
         # warm-up on a side stream (as torch's whole-network capture requires), then capture
-        side = torch.cuda.Stream()
+        side = _side_stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
             for _ in range(max(3, warmup)):
@@ -157,6 +170,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense baselines")
+    ap.add_argument("--models", default=None,
+                    help="comma-separated models to time, in this order (default: kron, "
+                         "kron_fused_l1, dense, dense_group_lasso; a name may repeat)")
     ap.add_argument("--graph", action="store_true",
                     help="capture each model's whole step in a CUDA graph and replay it")
     args = ap.parse_args(argv)
@@ -168,14 +184,24 @@ def main(argv=None):
     torch.backends.cuda.matmul.allow_tf32 = args.path == "tf32"
     try:
         for batch in [int(v) for v in args.batches.split(",")]:
-            torch.manual_seed(0)
-            models = {"kron": KronMLP(d, classes, args.block, args.rank, args.path),
-                      "kron_fused_l1": KronMLP(d, classes, args.block, args.rank, args.path,
-                                               fused_l1=args.lam)}
-            if not args.no_dense:
-                models["dense"] = DenseMLP(d, classes, args.block, False, dtype)
-                models["dense_group_lasso"] = DenseMLP(d, classes, args.block, True, dtype)
-            for name, model in models.items():
+            # each model is built just before it is timed and released after, so neither
+            # its time nor its peak memory includes another model's state
+            make = {
+                "kron": lambda: KronMLP(d, classes, args.block, args.rank, args.path),
+                "kron_fused_l1": lambda: KronMLP(d, classes, args.block, args.rank, args.path,
+                                                 fused_l1=args.lam),
+                "dense": lambda: DenseMLP(d, classes, args.block, False, dtype),
+                "dense_group_lasso": lambda: DenseMLP(d, classes, args.block, True, dtype),
+            }
+            names = (args.models.split(",") if args.models else
+                     ["kron", "kron_fused_l1"] + ([] if args.no_dense else
+                                                  ["dense", "dense_group_lasso"]))
+            unknown = sorted(set(names) - set(make))
+            if unknown:
+                raise SystemExit(f"unknown model(s) {unknown}; choose from {sorted(make)}")
+            for name in names:
+                torch.manual_seed(0)
+                model = make[name]()
                 r = time_model(model, batch, d, classes, args.lam, args.warmup, args.steps, dtype,
                                graph=args.graph)
                 line = {"benchmark": "mlp_train_step", "model": name, "batch": batch,
