@@ -29,9 +29,11 @@
  *   element types at the boundary (FP32 arithmetic: at least as accurate, slower).
  *
  * Ownership and synchronisation: every pointer except `stream` is a DEVICE pointer
- * owned by the caller.  The library allocates no memory, keeps no state between
- * calls and never synchronises; all work is enqueued on `stream` (a cudaStream_t
- * passed as void*, NULL = legacy default stream).
+ * owned by the caller.  The library allocates no memory and never synchronises; all
+ * work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ * stream).  No result depends on an earlier call.  The only device memory of its own
+ * is compiled in: the error word of kron_linear_device_error and the scratch array of
+ * kron_linear_backward_noalloc.
  *
  * Errors: arguments, shapes, alignment and workspace size are checked on the host
  * before anything is launched; a failing check returns its status and launches
@@ -72,7 +74,7 @@ typedef enum {
     KRON_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                       */
     KRON_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than kron_linear_workspace_size */
     KRON_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed            */
-    KRON_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait gave up           */
+    KRON_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (kron_linear_device_error) */
 } kron_status_t;
 
 /* Skip the work of (a, c) blocks where S is zero (the m1 x m2 block of W is zero,
@@ -129,7 +131,7 @@ KRON_API kron_status_t kron_linear_backward(const void *x, const void *S, const 
  *   dS [p][q] = sum_i dC_i (.) A_i + l1 * sign(S)
  * sign(0) = 0: at S[a][c] = 0 the term is 0, the subgradient that autograd takes for |.|.
  * The sum is formed in double and rounded once to float32.
- *   l1   the penalty's weight, finite and >= 0 (else KRON_ERR_INVALID_ARG); with l1 == 0
+ *   l1   the penalty's weight, 0 <= l1 <= 1e30 (else KRON_ERR_INVALID_ARG); with l1 == 0
  *        the results are bit for bit those of kron_linear_backward.
  * With N == 0 the factor gradients are zero except dS = l1 * sign(S).
  * Every other argument, output and rule is kron_linear_backward's.  (The penalty's value is

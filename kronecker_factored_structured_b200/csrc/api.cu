@@ -161,7 +161,7 @@ static kron_status_t backward_impl(const void *x, const void *S, const void *A, 
     kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
     if (st != KRON_OK) return st;
     if (!(l1 >= 0.0 && l1 <= 1e30))
-        return fail(KRON_ERR_INVALID_ARG, "the l1 weight must be finite and >= 0 (got %g)", l1);
+        return fail(KRON_ERR_INVALID_ARG, "the l1 weight must be in [0, 1e30] (got %g)", l1);
     if (!S || !A || !B || !dS || !dA || !dB || (N > 0 && (!x || !dY)))
         return fail(KRON_ERR_INVALID_ARG,
                     "S, A, B, dS, dA, dB (and x, dY when N > 0) must be non-null");
