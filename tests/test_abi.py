@@ -120,6 +120,13 @@ def test_backward_l1_runs_the_same_checks():
     assert st == 3
 
 
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU or eager fallback: without the built library every call raises."""
+    monkeypatch.setattr(native, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        native.load(str(tmp_path / "libkronlinear.so"))
+
+
 def test_python_binding_raises_without_cuda_tensors():
     import torch
     x = torch.zeros(4, 8)
