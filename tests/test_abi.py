@@ -120,6 +120,30 @@ def test_backward_l1_runs_the_same_checks():
     assert st == 3
 
 
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="needs a host without a usable GPU: the CUDA runtime must refuse")
+@pytest.mark.parametrize("dtype", [0, 1, 2])
+def test_cuda_failure_surfaces_as_kron_err_cuda(dtype):
+    """Arguments that pass every host check on a host whose CUDA runtime cannot run anything:
+    the first CUDA call fails, nothing is launched, and the status is KRON_ERR_CUDA with the
+    failing step in kron_last_error() (the pointers are never dereferenced on the host)."""
+    lib = native.load()
+    st = lib.kron_linear_forward(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, ALIGNED, 8, 32, 32,
+                                 32, 32, 4, dtype, 0, None)
+    assert st == 5
+    assert "forward launch" in lib.kron_last_error().decode()
+    need = lib.kron_linear_workspace_size(8, 32, 32, 32, 32, 4, dtype)
+    st = lib.kron_linear_backward(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                  ALIGNED, ALIGNED, None, 8, 32, 32, 32, 32, 4, dtype, 0,
+                                  V(0x100000), need, None)
+    assert st == 5 and lib.kron_last_error().decode() != ""
+    st = lib.kron_linear_backward_noalloc(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                          ALIGNED, ALIGNED, ALIGNED, None, 8, 32, 32, 32, 32, 4,
+                                          dtype, 0, None)
+    assert st == 5
+    assert lib.kron_linear_device_error(0) == 5
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     """No CPU or eager fallback: without the built library every call raises."""
     monkeypatch.setattr(native, "_lib", None)
