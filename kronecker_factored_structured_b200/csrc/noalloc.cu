@@ -49,6 +49,12 @@ extern "C" kron_status_t kron_linear_backward_noalloc(
     void *dS, void *dA, void *dB, void *dbias, int64_t N, int p, int q, int m1, int m2, int r,
     kron_dtype_t dtype, unsigned flags, void *stream) {
     const size_t need = kron_linear_workspace_size(N, p, q, m1, m2, r, dtype);
+    // need == 0: the sizes or dtype are invalid, or no kernel takes this shape; the
+    // workspace entry point reports which before touching the device (and with N == 0
+    // zeroes the gradients, which needs no scratch)
+    if (need == 0)
+        return kron_linear_backward(x, S, A, B, dY, dX, dS, dA, dB, dbias, N, p, q, m1, m2, r,
+                                    dtype, flags, nullptr, 0, stream);
     if (need > KRON_NOALLOC_SCRATCH_BYTES) {
         char msg[200];
         snprintf(msg, sizeof(msg),

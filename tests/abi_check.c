@@ -1,0 +1,102 @@
+/*
+ * abi_check.c -- the C ABI used from plain C99 (no C++, no Python): the header compiles
+ * with -std=c99 -pedantic -Werror, the library links, and every host-side check of every
+ * entry point returns its documented status before anything touches the device.  The
+ * pointers below are never dereferenced: each call fails a host check.
+ *
+ * Built and run by tests/test_c_abi.py; exits 0 when every check passes, else prints the
+ * failing check and exits 1.
+ */
+#include "kron_linear.h"
+
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+static int failures = 0;
+
+#define CHECK(cond)                                                          \
+    do {                                                                     \
+        if (!(cond)) {                                                       \
+            printf("FAILED line %d: %s (last error: %s)\n", __LINE__, #cond, \
+                   kron_last_error());                                       \
+            ++failures;                                                      \
+        }                                                                    \
+    } while (0)
+
+int main(void) {
+    void *const P = (void *)(uintptr_t)0x10000;     /* 16-byte aligned, never read */
+    void *const MIS = (void *)(uintptr_t)0x10004;   /* misaligned */
+    void *const WS = (void *)(uintptr_t)0x100000;   /* 256-byte aligned, never read */
+    size_t need;
+    int st;
+
+    CHECK(kron_linear_abi_version() == KRON_LINEAR_ABI_VERSION);
+    for (st = KRON_OK; st <= KRON_ERR_TIMEOUT; ++st)
+        CHECK(strncmp(kron_status_string((kron_status_t)st), "KRON_", 5) == 0);
+
+    /* workspace size: a function of the arguments only; 0 for invalid ones */
+    need = kron_linear_workspace_size(20000, 32, 32, 32, 32, 4, KRON_TF32);
+    CHECK(need > 0 && need % 256 == 0);
+    CHECK(need == kron_linear_workspace_size(20000, 32, 32, 32, 32, 4, KRON_TF32));
+    CHECK(kron_linear_workspace_size(20000, 0, 32, 32, 32, 4, KRON_TF32) == 0);
+    CHECK(kron_linear_workspace_size(-1, 32, 32, 32, 32, 4, KRON_F32) == 0);
+    CHECK(kron_linear_workspace_size(8, 2, 2, 4, 4, 1, (kron_dtype_t)9) == 0);
+
+    /* forward */
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 2, 2, 4, 4, 1, (kron_dtype_t)9, 0, NULL) ==
+          KRON_ERR_INVALID_ARG);
+    CHECK(strlen(kron_last_error()) > 0);
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 2, 2, 4, 4, 1, KRON_F32, 8u, NULL) ==
+          KRON_ERR_INVALID_ARG);                                            /* unknown flag */
+    CHECK(kron_linear_forward(NULL, P, P, P, NULL, P, 8, 2, 2, 4, 4, 1, KRON_F32, 0, NULL) ==
+          KRON_ERR_INVALID_ARG);                                            /* x missing */
+    CHECK(kron_linear_forward(MIS, P, P, P, NULL, P, 8, 2, 2, 4, 4, 1, KRON_F32, 0, NULL) ==
+          KRON_ERR_ALIGNMENT);
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 2, 2, 6, 4, 1, KRON_F32, 0, NULL) ==
+          KRON_ERR_UNSUPPORTED);                                            /* m1 % 4 */
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 2, 2, 4, 4, 1, KRON_BF16, 0, NULL) ==
+          KRON_ERR_UNSUPPORTED);                                            /* m1 % 8 */
+    /* N == 0 is a no-op that needs no device at all */
+    CHECK(kron_linear_forward(NULL, P, P, P, NULL, NULL, 0, 2, 2, 4, 4, 1, KRON_F32, 0, NULL) ==
+          KRON_OK);
+    CHECK(strlen(kron_last_error()) == 0);
+
+    /* backward */
+    need = kron_linear_workspace_size(8, 2, 2, 4, 4, 1, KRON_F32);
+    CHECK(kron_linear_backward(P, P, P, P, P, P, NULL, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                               WS, need, NULL) == KRON_ERR_INVALID_ARG);   /* dS missing */
+    CHECK(kron_linear_backward(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                               NULL, 0, NULL) == KRON_ERR_WORKSPACE);
+    CHECK(kron_linear_backward(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                               WS, need - 4, NULL) == KRON_ERR_WORKSPACE);
+    CHECK(kron_linear_backward(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                               (char *)WS + 16, need, NULL) == KRON_ERR_ALIGNMENT);
+    CHECK(kron_linear_backward(P, P, P, P, MIS, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                               WS, need, NULL) == KRON_ERR_ALIGNMENT);     /* dY misaligned */
+
+    /* backward with the fused l1 term: the weight is checked like every other argument */
+    CHECK(kron_linear_backward_l1(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                                  -0.5, WS, need, NULL) == KRON_ERR_INVALID_ARG);
+    CHECK(kron_linear_backward_l1(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                                  1e31, WS, need, NULL) == KRON_ERR_INVALID_ARG);
+    CHECK(kron_linear_backward_l1(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1, KRON_F32, 0,
+                                  0.5, NULL, 0, NULL) == KRON_ERR_WORKSPACE);
+
+    /* backward without a workspace: invalid arguments and oversized problems are refused
+       on the host, before the scratch array's address is looked up */
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1,
+                                       (kron_dtype_t)9, 0, NULL) == KRON_ERR_INVALID_ARG);
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 6, 4, 1,
+                                       KRON_F32, 0, NULL) == KRON_ERR_UNSUPPORTED);
+    /* 20000 rows of the 4096^2 layer with 64x64 blocks and rank 8 need ~41 MB of scratch */
+    CHECK(kron_linear_workspace_size(20000, 64, 64, 64, 64, 8, KRON_F32) >
+          KRON_NOALLOC_SCRATCH_BYTES);
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, P, P, P, NULL, 20000, 64, 64, 64, 64, 8,
+                                       KRON_F32, 0, NULL) == KRON_ERR_WORKSPACE);
+    CHECK(strstr(kron_last_error(), "scratch") != NULL);
+
+    if (failures) return 1;
+    printf("abi_check: all checks passed\n");
+    return 0;
+}
