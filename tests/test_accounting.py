@@ -54,3 +54,34 @@ def test_tutorial_layer_work():
     assert acc.flops_per_row(32, 32, 32, 32, 4) == 1572864
     assert acc.bytes_per_row(1024, 1024, 4) == 20480
     assert acc.flops_per_row(32, 32, 32, 32, 4, backward=False) * 3 == 1572864
+
+
+def test_gpt2_ffn_work_takes_the_cheaper_order():
+    # c_fc 768 -> 3072 (C 24 x 48, B 32 x 64): X.B first is cheaper, 49,152 + 73,728 MACs per
+    # rank; c_proj 3072 -> 768 (C 48 x 24, B 64 x 32): C first, 73,728 + 49,152
+    assert acc.macs_per_row_forward(24, 48, 32, 64, 1) == 122880
+    assert acc.macs_per_row_forward(48, 24, 64, 32, 1) == 122880
+    for r in (1, 4):
+        assert acc.flops_per_row(24, 48, 32, 64, r) == 737280 * r
+        assert acc.flops_per_row(48, 24, 64, 32, r, backward=False) == 245760 * r
+    assert acc.bytes_per_row(768, 3072, 2) == 16896
+    assert acc.bytes_per_row(3072, 768, 2) == 21504
+    assert acc.bytes_per_row(768, 3072, 2, backward=False) == 7680
+
+
+def test_stress_work_with_and_without_the_skip_credit():
+    # 4096^2, m = 64, r = 8: 25,165,824 flop per row with S dense; with 6 of 64 patches
+    # non-zero the two contractions with C (y and U) shrink to 6/64, dC does not
+    assert acc.flops_per_row(64, 64, 64, 64, 8) == 25165824
+    assert acc.flops_per_row(64, 64, 64, 64, 8, skip_fraction=1.0) == 25165824
+    assert acc.flops_per_row(64, 64, 64, 64, 8, skip_fraction=6 / 64) == 17563648
+    assert acc.bytes_per_row(4096, 4096, 2) == 40960
+
+
+def test_sweep_work():
+    # square blocks on the 1024^2 layer: 6144 * r * (m + p) flop per row, p = 1024 / m
+    for m in (8, 16, 64, 128):
+        for r in (1, 2, 8):
+            p = 1024 // m
+            assert acc.flops_per_row(p, p, m, m, r) == 6144 * r * (m + p)
+    assert 20000 * acc.flops_per_row(128, 128, 8, 8, 1) == 16711680000
