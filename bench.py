@@ -30,9 +30,9 @@ METRIC = "Kron-layer rows/s fwd+bwd (1024², m=32, r=4) & achieved % of roofline
 UNIT = "rows/s"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the backward
-# call's kernels (dX + parameter gradients) on the tutorial layer, from one ncu capture
-# (profiles/launches_tutorial_<path>.md), valid only for the kernel sources whose
-# SHA-256 prefix is recorded with it: any later change to them makes the figure null.
+# call's kernels (dX + parameter gradients) on the tutorial layer, from one ncu capture of
+# this command, valid only for the kernel sources whose SHA-256 prefix is recorded with it:
+# any later change to them makes the figure null.
 _TRAFFIC = {
     "tf32": (82.00e6 + 24.35e6 + 163.99e6 + 0.85e6, "8113c98ef788a49a"),
     "bf16": (41.01e6 + 0.14e6 + 81.99e6 + 0.37e6, "8113c98ef788a49a"),
@@ -307,6 +307,174 @@ def dense_context(fac, sets, path, steps, dev):
             "matmul": "tf32" if path == "tf32" else path, "ms_per_step": ms}
 
 
+REPEATS = 5  # repeats of each timed region; the median is reported (and the min)
+
+
+def _path_supported(kfs, w, path):
+    """True when the library has kernels for this workload on this path (the backward's
+    workspace size is 0 exactly when no kernel of the path takes the shape)."""
+    return kfs.workspace_size(max(w.N, 1), w.p, w.q, w.m1, w.m2, w.r, path) > 0
+
+
+def _step_roofline(w, path, ms_step, peaks, flags):
+    """Roofline time of one forward + backward step, max(bytes / HBM, flops / unit peak), and
+    the achieved fraction of it.  The unit peak is the measured BF16 tensor rate for BF16, half
+    of it for TF32 (the nominal TF32:BF16 ratio) and the derived FFMA rate for FP32."""
+    from kronecker_factored_structured_b200 import accounting as acc
+    elt = 2 if path == "bf16" else 4
+    nbytes = w.N * acc.bytes_per_row(w.d_in, w.d_out, elt)
+    skip = None
+    if flags and w.s_zero_patches:
+        skip = 1.0 - w.s_zero_patches / float((w.p // w.s_zero_patch) * (w.q // w.s_zero_patch))
+    flops = w.N * acc.flops_per_row(w.p, w.q, w.m1, w.m2, w.r, skip_fraction=skip)
+    if path == "f32":
+        peak, unit, src = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6, "FFMA", "derived"
+    else:
+        bf = peaks["bf16_tflops"] * 1e12
+        peak, unit, src = (bf, "bf16", peaks["source"]) if path == "bf16" else \
+            (bf / 2, "tf32", peaks["source"] + " bf16 x 1/2")
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_fl = flops / peak
+    t_roof = max(t_hbm, t_fl)
+    return {"bound": "hbm" if t_hbm >= t_fl else ("alu" if path == "f32" else "tensor"),
+            "roofline_us": t_roof * 1e6, "hbm_us": t_hbm * 1e6, "flops_us": t_fl * 1e6,
+            "frac": t_roof / (ms_step / 1e3), "flop_peak": unit, "flop_peak_source": src,
+            "bytes": nbytes, "flops": flops}
+
+
+class _Problem:
+    """Device tensors of one workload on one path: ROTATE (or fewer) independent (x, dY)
+    input sets resident in HBM, the factors, outputs and workspace."""
+
+    def __init__(self, kw, kfs, w, path, dev, rank=0, rotate=ROTATE):
+        import torch
+        self.w, self.path = w, path
+        t_io = kfs.native.io_dtype(path)
+        self.fac = {k: v.to(dev).to(t_io) for k, v in kw.factors(w).items()}
+        self.sets = []
+        for s in range(rotate):
+            ws = dataclasses.replace(w, seed=w.seed + 1000 * s + 100000 * rank) if (s or rank) else w
+            self.sets.append((kw.rows(ws, "x").to(dev).to(t_io), kw.rows(ws, "G").to(dev).to(t_io)))
+        self.y = torch.empty(w.N, w.d_out, dtype=t_io, device=dev)
+        self.wsb = torch.empty(max(kfs.workspace_size(w.N, w.p, w.q, w.m1, w.m2, w.r, path), 1),
+                               dtype=torch.uint8, device=dev)
+
+
+def _time_region(step, steps, repeats, world, dist, stream, clk=None):
+    """Device time (ms) of `steps` back-to-back steps, measured `repeats` times between CUDA
+    events on the launching stream, each repeat bracketed by a barrier and a synchronize;
+    the max over ranks of each repeat.  Returns (median, min, all)."""
+    import torch
+    times = []
+    for rep in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        if clk is not None and rep == 0:
+            clk.begin_region()
+        a.record(stream)
+        for i in range(steps):
+            step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        times.append(ms)
+    if clk is not None:
+        clk.end_region()
+    return statistics.median(times), min(times), times
+
+
+def _split_calls(step, steps, stream):
+    """Mean forward and backward call times (ms) from per-call events over `steps` steps
+    (outside any timed region: the extra event records do not enter a reported value)."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    marks = [(ev(), ev(), ev()) for _ in range(steps)]
+    for i in range(steps):
+        step(i, marks[i])
+    torch.cuda.synchronize()
+    return (statistics.mean(a.elapsed_time(b) for a, b, _ in marks),
+            statistics.mean(b.elapsed_time(c) for _, b, c in marks))
+
+
+def _make_step(kfs, pr, flags, stream, grads, world=1, dp=None, flat=None):
+    def step(i, timing=None):
+        x, G = pr.sets[i % len(pr.sets)]
+        if timing is not None:
+            timing[0].record(stream)
+        kfs.forward(x, pr.fac["S"], pr.fac["A"], pr.fac["B"], pr.fac["bias"], dtype=pr.path,
+                    flags=flags, out=pr.y)
+        if timing is not None:
+            timing[1].record(stream)
+        kfs.backward(x, pr.fac["S"], pr.fac["A"], pr.fac["B"], G, dtype=pr.path, flags=flags,
+                     workspace=pr.wsb, grads=grads)
+        if timing is not None:
+            timing[2].record(stream)
+        if world > 1:
+            dp.allreduce_grads(flat)
+    return step
+
+
+# Further legs of the default run (rank 0 alone, N = 1): the tutorial layer on the other two
+# paths, then every other configuration on its own tensor-core path where the library has
+# one (the workload's BF16 I/O, or TF32 for fp32 I/O), else on the exact-FP32 path for the
+# fp32 workloads.  (workload, path or None for the workload's own, skip-zero-blocks flag)
+LEGS = [("tutorial", "f32", 0), ("tutorial", "bf16", 0),
+        ("gpt2_c_fc_r1", None, 0), ("gpt2_c_fc_r4", None, 0),
+        ("gpt2_c_proj_r1", None, 0), ("gpt2_c_proj_r4", None, 0),
+        ("stress", None, 0), ("stress", None, 1)] + \
+       [(f"sweep_m{m}_r{r}", None, 0) for m in (8, 16, 64, 128) for r in (1, 2, 8)]
+
+
+def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
+    """One further leg: the workload's forward + backward step, median of REPEATS timed
+    regions of `steps` steps; a dict for the JSON line's "legs" list."""
+    import torch
+    w = kw.get(name)
+    if path is None:
+        path = "bf16" if w.dtype == "bf16" else "tf32"
+    if not _path_supported(kfs, w, path):
+        if w.dtype == "bf16":
+            return {"workload": name, "path": path, "flags": flags,
+                    "status": "unsupported: no tensor-core kernel for this shape"}
+        alt = "f32"
+        note = f"no {path} kernel for this shape: exact-FP32 path"
+        path = alt
+    else:
+        note = None
+    if path == "bf16" and w.dtype != "bf16":
+        w = dataclasses.replace(w, dtype="bf16")
+    rotate = ROTATE if w.N * (w.d_in + w.d_out) * (2 if path == "bf16" else 4) < 126e6 else 1
+    pr = _Problem(kw, kfs, w, path, dev, rotate=rotate)
+    grads = {"dX": torch.empty(w.N, w.d_in, dtype=pr.y.dtype, device=dev)}
+    step = _make_step(kfs, pr, flags, stream, grads)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    med, mn, _ = _time_region(step, steps, REPEATS, 1, None, stream)
+    t_fwd, t_bwd = _split_calls(step, steps, stream)
+    ms = med / steps
+    leg = {"workload": _workload_desc(w), "name": name, "path": path, "flags": flags,
+           "N": w.N, "steps": steps, "repeats": REPEATS, "ms_per_step": ms,
+           "ms_per_step_min": mn / steps, "rows_per_s": w.N / (ms / 1e3),
+           "fwd_ms": t_fwd, "bwd_ms": t_bwd,
+           "l2": f"{len(pr.sets)} input set(s), "
+                 f"{len(pr.sets) * w.N * (w.d_in + w.d_out) * (2 if path == 'bf16' else 4) / 1e6:.0f} MB",
+           "roofline": _step_roofline(w, path, ms, peaks, flags)}
+    if note:
+        leg["note"] = note
+    del pr, grads
+    torch.cuda.empty_cache()
+    return leg
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -322,6 +490,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true",
                     help="skip the dense-layer context timing (cuBLAS through torch)")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="time only the headline workload (no further legs)")
+    ap.add_argument("--legs", default=None,
+                    help="comma-separated workload names of the further legs (default: all)")
+    ap.add_argument("--leg-steps", type=int, default=20)
     ap.add_argument("--skip-zero-blocks", action="store_true",
                     help="pass KRON_FLAG_SKIP_ZERO_BLOCKS (drop products with a zero S entry)")
     args = ap.parse_args()
@@ -356,39 +529,18 @@ def main():
     kfs.native.load()
 
     # ---- inputs resident in HBM: ROTATE independent (x, G) sets, factors shared ----
-    fac = {k: v.to(dev) for k, v in kw.factors(w).items()}
-    sets = []
-    for s in range(ROTATE):
-        # each rank holds its own rows (weak scaling): a rank- and set-specific seed
-        ws = dataclasses.replace(w, seed=w.seed + 1000 * s + 100000 * rank) if (s or rank) else w
-        sets.append((kw.rows(ws, "x").to(dev), kw.rows(ws, "G").to(dev)))
+    pr = _Problem(kw, kfs, w, path, dev, rank=rank)
     p, q, m1, m2, r, N = w.p, w.q, w.m1, w.m2, w.r, w.N
     t_io = kfs.native.io_dtype(path)
     elt = 2 if path == "bf16" else 4
-    y = torch.empty(N, q * m2, dtype=t_io, device=dev)
     grads = {"dX": torch.empty(N, p * m1, dtype=t_io, device=dev)}
     # parameter gradients as views of one flat buffer: the one exchange of the data-parallel
     # backward is a single all-reduce of it
     flat, views = dp.flat_grad_buffer(p, q, m1, m2, r, device=dev)
     grads.update(views)
-    wsb = torch.empty(max(kfs.workspace_size(N, p, q, m1, m2, r, path), 1), dtype=torch.uint8,
-                      device=dev)
     stream = torch.cuda.current_stream()
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-
-    def step(i, timing=None):
-        x, G = sets[i % ROTATE]
-        if timing is not None:
-            timing[0].record(stream)
-        kfs.forward(x, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, flags=flags, out=y)
-        if timing is not None:
-            timing[1].record(stream)
-        kfs.backward(x, fac["S"], fac["A"], fac["B"], G, dtype=path, flags=flags, workspace=wsb,
-                     grads=grads)
-        if timing is not None:
-            timing[2].record(stream)
-        if world > 1:
-            dp.allreduce_grads(flat)
+    step = _make_step(kfs, pr, flags, stream, grads, world, dp, flat)
+    fac, sets, wsb = pr.fac, pr.sets, pr.wsb
 
     for i in range(args.warmup):
         step(i)
@@ -401,37 +553,14 @@ def main():
     torch.cuda.synchronize()
     peak_extra = torch.cuda.max_memory_allocated(dev) - base_bytes
 
-    # ---- timed region: K steps between two events on the launching stream ----
-    start, end = ev(), ev()
+    # ---- timed region: REPEATS x (K steps between two events on the launching stream) ----
     with ClockSampler(torch.cuda.current_device()) as clk:
         clk.wait_started()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        clk.begin_region()
-        start.record(stream)
-        for i in range(args.steps):
-            step(i)
-        end.record(stream)
-        torch.cuda.synchronize()
-        clk.end_region()
-        if world > 1:
-            dist.barrier()
-    ms = start.elapsed_time(end)
-    # ---- the split into forward and backward call: K more steps with per-call events
-    # (outside the timed region, so the extra event records do not enter `value`) ----
-    marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(i, marks[i])
-    torch.cuda.synchronize()
-    t_fwd = statistics.mean(a.elapsed_time(b) for a, b, _ in marks)
-    t_bwd = statistics.mean(b.elapsed_time(c) for _, b, c in marks)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_step = ms / args.steps
-    value = world * N * args.steps / (ms / 1e3)
+        ms_med, ms_min, ms_all = _time_region(step, args.steps, REPEATS, world, dist, stream, clk)
+    # ---- the split into forward and backward call (outside the timed region) ----
+    t_fwd, t_bwd = _split_calls(step, args.steps, stream)
+    ms_step = ms_med / args.steps
+    value = world * N * args.steps / (ms_med / 1e3)
 
     # ---- end to end through the public API with pinned host buffers ----
     xh = [s[0].cpu().pin_memory() for s in sets]
@@ -442,14 +571,15 @@ def main():
     xd, gd = torch.empty_like(sets[0][0]), torch.empty_like(sets[0][1])
 
     def e2e_step(i):
-        xd.copy_(xh[i % ROTATE], non_blocking=True)
-        gd.copy_(gh[i % ROTATE], non_blocking=True)
-        kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, flags=flags, out=y)
+        xd.copy_(xh[i % len(sets)], non_blocking=True)
+        gd.copy_(gh[i % len(sets)], non_blocking=True)
+        kfs.forward(xd, fac["S"], fac["A"], fac["B"], fac["bias"], dtype=path, flags=flags,
+                    out=pr.y)
         kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, flags=flags, workspace=wsb,
                      grads=grads)
         if world > 1:
             dp.allreduce_grads(flat)
-        yh.copy_(y, non_blocking=True)
+        yh.copy_(pr.y, non_blocking=True)
         dxh.copy_(grads["dX"], non_blocking=True)
         fh.copy_(flat, non_blocking=True)
 
@@ -457,22 +587,11 @@ def main():
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    s0, s1 = ev(), ev()
-    s0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    s1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = s0.elapsed_time(s1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * N * e2e_steps / (e2e_ms / 1e3)
+    e2e_med, _, _ = _time_region(e2e_step, e2e_steps, 3, world, dist, stream)
+    e2e_value = world * N * e2e_steps / (e2e_med / 1e3)
     h2d = xh[0].numel() * xh[0].element_size() + gh[0].numel() * gh[0].element_size()
     d2h = yh.numel() * yh.element_size() + dxh.numel() * dxh.element_size() + fh.numel() * 4
+    del xh, gh, yh, dxh, fh, xd, gd
 
     if rank != 0:
         if world > 1:
@@ -483,20 +602,20 @@ def main():
     peaks = _peaks()
     bwd_bytes = N * elt * (2 * p * m1 + q * m2)
     bwd_flops = N * (acc.flops_per_row(p, q, m1, m2, r) - acc.flops_per_row(p, q, m1, m2, r, False))
-    # the tensor-core kernels exist for p = q = m1 = m2 = 32, r = 4; other TF32/BF16 shapes
-    # run the CUDA-core kernels, which are bound by FP32 arithmetic
-    on_tc = path != "f32" and (p, q, m1, m2, r) == (32, 32, 32, 32, 4)
-    # kernels of this library per step: tensor cores: forward, dX, parameter gradients (with
-    # their fused reduction); CUDA cores on the tutorial shape: forward, dX, parameter-gradient
-    # partials, reduction; any other shape: forward, backward, reduction
-    compiled_f32 = path == "f32" and (p, q, m1, m2, r) == (32, 32, 32, 32, 4) and not flags
-    launches_per_step = 4 if compiled_f32 else 3
+    on_tc = path != "f32"
+    # kernels of this library per step: tuned tensor-core kernels of the tutorial shape:
+    # forward, dX, parameter gradients (with their fused reduction); CUDA cores on the
+    # tutorial shape: forward, dX, parameter-gradient partials, reduction
+    tutorial_shape = (p, q, m1, m2, r) == (32, 32, 32, 32, 4)
+    compiled_f32 = path == "f32" and tutorial_shape and not flags
+    launches_per_step = 4 if compiled_f32 or (on_tc and not tutorial_shape) else 3
     if not on_tc:
         peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12   # FFMA TFLOP/s at max clock
         achieved = bwd_flops / (t_bwd / 1e3) / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": None,
-                "kernel": "kron_bwd_simt_kernel + reduction (one backward call)",
+                "kernel": "backward call on the CUDA cores (dX, parameter-gradient partials, "
+                          "reduction)",
                 "peak_source": "derived: 148 SMs x 128 FFMA/clk x 2 x max SM clock"}
     else:
         achieved = bwd_bytes / (t_bwd / 1e3) / 1e9
@@ -514,14 +633,16 @@ def main():
         "config": {"workload": _workload_desc(w), "N": N, "p": p, "q": q, "m1": m1, "m2": m2,
                    "r": r, "path": path, "parallelism": f"dp{world}",
                    "skip_zero_blocks": bool(flags),
-                   "l2": f"inputs rotated over {ROTATE} independent (x, dY) sets "
-                         f"({ROTATE * N * elt * (p * m1 + q * m2) / 1e6:.0f} MB > 126 MB L2)"},
+                   "l2": f"inputs rotated over {len(sets)} independent (x, dY) sets "
+                         f"({len(sets) * N * elt * (p * m1 + q * m2) / 1e6:.0f} MB > 126 MB L2)"},
+        "repeats": {"n": REPEATS, "ms_per_step": [t / args.steps for t in ms_all],
+                    "median": ms_step, "min": ms_min / args.steps},
         "fwd_ms": t_fwd, "bwd_ms": t_bwd,
         "tflops": step_flops / (ms_step / 1e3) / 1e12,
         "gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "step_roofline_frac_hbm": (step_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3),
         "roofline": roof,
-        "gpu_launches": args.steps * launches_per_step,
+        "gpu_launches": REPEATS * args.steps * launches_per_step,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "clocks": clk.summary(),
@@ -532,6 +653,17 @@ def main():
         ctx["kron_ms_per_step"] = ms_step
         ctx["kron_speedup"] = ctx["ms_per_step"] / ms_step
         line["context_dense"] = ctx
+    del pr, sets, fac, grads, flat, views, step
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_legs:
+        names = args.legs.split(",") if args.legs else None
+        legs = []
+        for name, lpath, lflags in LEGS:
+            if names is not None and name not in names:
+                continue
+            legs.append(run_leg(kw, kfs, name, lpath, lflags, max(3, min(args.steps, args.leg_steps)),
+                                args.warmup, peaks, dev, stream))
+        line["legs"] = legs
     if world == 1 and not args.no_cpu_baseline:
         cpu_rows = args.cpu_rows or (N if N * (w.d_in + w.d_out) <= 20000 * 2048 else 1024)
         rows_s, dt, cores = cpu_baseline(w, cpu_rows)

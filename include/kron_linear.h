@@ -24,9 +24,11 @@
  *              cores with TF32 operands and FP32 accumulation.
  *   KRON_BF16  x, y, dY, dX, S, A, B and bias are bfloat16; dS, dA, dB and dbias are
  *              float32.  tcgen05 tensor cores with BF16 operands, FP32 accumulation.
- *   The tensor-core kernels are compiled for p = q = m1 = m2 = 32, r = 4.  A TF32 or
- *   BF16 call of any other shape runs the exact-FP32 CUDA-core kernels with the same
- *   element types at the boundary (FP32 arithmetic: at least as accurate, slower).
+ *   KRON_TF32 and KRON_BF16 run only where a tensor-core kernel exists for the shape;
+ *   a call of any other shape returns KRON_ERR_UNSUPPORTED and launches nothing (it is
+ *   never run on another path).  KRON_F32 takes any shape whose FP32 tile fits shared
+ *   memory.  kron_linear_workspace_size returns 0 for a shape the requested path does
+ *   not take, so it also answers whether a backward is supported.
  *
  * Ownership and synchronisation: every pointer except `stream` is a DEVICE pointer
  * owned by the caller.  The library allocates no memory and never synchronises; all
@@ -37,8 +39,8 @@
  *
  * Errors: arguments, shapes, alignment and workspace size are checked on the host
  * before anything is launched; a failing check returns its status and launches
- * nothing.  Shapes no kernel covers (an FP32 tile larger than shared memory) return
- * KRON_ERR_UNSUPPORTED; nothing ever falls back to the CPU.  A failed launch returns KRON_ERR_CUDA;
+ * nothing.  Shapes the requested path has no kernel for return KRON_ERR_UNSUPPORTED;
+ * nothing ever falls back to another path or to the CPU.  A failed launch returns KRON_ERR_CUDA;
  * faults during execution surface at the caller's next synchronisation.
  * kron_last_error() gives a one-line description of the last failure on the
  * calling host thread.
@@ -112,6 +114,12 @@ KRON_API kron_status_t kron_linear_forward(const void *x, const void *S, const v
  * bitwise identical across calls with the same inputs on the same GPU model.
  * `workspace` is device scratch of at least kron_linear_workspace_size(...) bytes,
  * 256-byte aligned, owned by the caller; its contents on entry are ignored.
+ * On the tensor-core paths of the tutorial layer's shape (p = q = m1 = m2 = 32, r = 4)
+ * the parameter-gradient kernel sums the row ranges itself after a grid-wide barrier:
+ * it is a cooperative launch of one CTA per row range (at most 148), all of which must
+ * be resident at once.  On a device or partition that cannot hold them (fewer SMs, or
+ * SMs taken by other work under MPS) the launch fails and the call returns
+ * KRON_ERR_CUDA; the other paths add the ranges with a separate reduction kernel.
  */
 KRON_API kron_status_t kron_linear_backward(const void *x, const void *S, const void *A, const void *B,
                                    const void *dY, void *dX, void *dS, void *dA, void *dB,
@@ -161,7 +169,10 @@ KRON_API kron_status_t kron_linear_backward_l1(const void *x, const void *S, con
  *   - All calls share the one array per device: calls that overlap on the GPU (for
  *     example on two streams) race on it and must be serialised by the caller.
  *   - The first call on a device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current); make that first call before any stream capture.  The address belongs to
+ *     the current CUDA context: it is looked up again after the context changes (after
+ *     cudaDeviceReset, or under a context made current through the driver API), so the
+ *     first call under a new context must also come before any capture.
  * Results are the same as kron_linear_backward's.
  */
 #define KRON_NOALLOC_SCRATCH_BYTES (8u << 20)

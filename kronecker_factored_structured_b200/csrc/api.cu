@@ -53,30 +53,86 @@ kron_status_t check_shape(int64_t N, int p, int q, int m1, int m2, int r, kron_d
     return KRON_OK;
 }
 
-// True when the backward of this shape and dtype runs on the tensor-core kernels.
+// True when the backward of this shape and dtype runs on the tensor-core kernels (the TF32
+// and BF16 paths); KRON_F32 always runs the CUDA-core kernels.
 bool tc_backward_path(const kron::Shape &s, kron_dtype_t dtype) {
     return dtype != KRON_F32 && kron::tc_backward_supported(s, dtype == KRON_BF16);
 }
 
-// Number of contiguous row ranges of the backward: at most kRowParts, none empty.  A
-// function of the shape and path only, so the summation order is fixed.
+// True when some kernel of the requested path takes this shape.
+bool backward_path_exists(const kron::Shape &s, kron_dtype_t dtype) {
+    return dtype == KRON_F32 ? kron::simt_backward_rows(s) > 0 : tc_backward_path(s, dtype);
+}
+
+// Number of contiguous row ranges of the backward: at most the path's maximum, none empty.
+// A function of the shape and path only, so the summation order is fixed.
 int backward_parts(const kron::Shape &s, kron_dtype_t dtype) {
-    int rows_per_tile = 0;
-    if (tc_backward_path(s, dtype)) rows_per_tile = kron::tc_backward_tile_rows(s);
-    else rows_per_tile = kron::simt_backward_rows(s);
-    if (rows_per_tile <= 0) return 0;
+    int rows_per_tile = 0, max_parts = kron::kRowParts;
+    if (tc_backward_path(s, dtype)) {
+        rows_per_tile = kron::tc_backward_tile_rows(s, dtype == KRON_BF16);
+        max_parts = kron::tc_backward_max_parts(s, dtype == KRON_BF16);
+    } else if (dtype == KRON_F32) {
+        rows_per_tile = kron::simt_backward_rows(s);
+    }
+    if (rows_per_tile <= 0 || max_parts <= 0) return 0;
     int64_t tiles = (s.N + rows_per_tile - 1) / rows_per_tile;
     if (tiles < 1) tiles = 1;
-    const int64_t parts0 = tiles < kron::kRowParts ? tiles : kron::kRowParts;
+    const int64_t parts0 = tiles < max_parts ? tiles : max_parts;
     const int64_t per = (tiles + parts0 - 1) / parts0;
     return (int)((tiles + per - 1) / per);
 }
 
 }  // namespace
 
+// Host-side checks shared by every backward entry point: sizes, dtype, flags, the l1
+// weight, pointers, alignment, and that the requested path has a kernel for the shape.
+// Touches no CUDA state.
+static kron_status_t check_backward(const void *x, const void *S, const void *A, const void *B,
+                                    const void *dY, const void *dX, const void *dS,
+                                    const void *dA, const void *dB, const void *dbias, int64_t N,
+                                    int p, int q, int m1, int m2, int r, kron_dtype_t dtype,
+                                    unsigned flags, double l1) {
+    kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
+    if (st != KRON_OK) return st;
+    if (!(l1 >= 0.0 && l1 <= 1e30))
+        return fail(KRON_ERR_INVALID_ARG, "the l1 weight must be in [0, 1e30] (got %g)", l1);
+    if (!S || !A || !B || !dS || !dA || !dB || (N > 0 && (!x || !dY)))
+        return fail(KRON_ERR_INVALID_ARG,
+                    "S, A, B, dS, dA, dB (and x, dY when N > 0) must be non-null");
+    if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(dY) ||
+        !aligned16(dS) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
+        (dbias && !aligned16(dbias)))
+        return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
+    const kron::Shape s{N, p, q, m1, m2, r};
+    if (N > 0 && !backward_path_exists(s, dtype)) {
+        if (dtype == KRON_F32)
+            return fail(KRON_ERR_UNSUPPORTED,
+                        "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not fit "
+                        "shared memory", p, q, m1, m2, r);
+        return fail(KRON_ERR_UNSUPPORTED,
+                    "no tensor-core kernel for p=%d q=%d m1=%d m2=%d r=%d on the %s path "
+                    "(KRON_F32 runs any shape)", p, q, m1, m2, r,
+                    dtype == KRON_BF16 ? "BF16" : "TF32");
+    }
+    return KRON_OK;
+}
+
 namespace kron {
 // Records a failure in this thread's last-error string (for entry points in other files).
 kron_status_t report_failure(kron_status_t st, const char *msg) { return fail(st, "%s", msg); }
+}  // namespace kron
+
+namespace kron {
+// The backward's host-side checks, for entry points in other files (clears the thread's
+// last-error string first, as every entry point does).
+kron_status_t validate_backward(const void *x, const void *S, const void *A, const void *B,
+                                const void *dY, const void *dX, const void *dS, const void *dA,
+                                const void *dB, const void *dbias, int64_t N, int p, int q,
+                                int m1, int m2, int r, kron_dtype_t dtype, unsigned flags) {
+    g_last_error[0] = 0;
+    return check_backward(x, S, A, B, dY, dX, dS, dA, dB, dbias, N, p, q, m1, m2, r, dtype,
+                          flags, 0.0);
+}
 }  // namespace kron
 
 extern "C" {
@@ -124,27 +180,23 @@ kron_status_t kron_linear_forward(const void *x, const void *S, const void *A, c
     const kron::Shape s{N, p, q, m1, m2, r};
     cudaStream_t cs = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
-    switch (dtype) {
-        case KRON_F32:
-        case KRON_TF32:
-        case KRON_BF16: {
-            const bool bf16 = dtype == KRON_BF16;
-            if (dtype != KRON_F32 && kron::tc_forward_supported(s, bf16)) {
-                e = kron::tc_forward(x, S, A, B, bias, y, s, bf16, cs);
-                break;
-            }
-            // exact-FP32 CUDA-core kernels: every KRON_F32 call, and TF32/BF16 shapes with no
-            // compiled tensor-core kernel (fp32 arithmetic, I/O in the caller's dtype)
-            if (kron::simt_forward_rows(s) <= 0)
-                return fail(KRON_ERR_UNSUPPORTED,
-                            "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not "
-                            "fit shared memory", p, q, m1, m2, r);
-            e = kron::simt_forward(x, S, A, B, bias, y, s, bf16,
-                                   (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
-            break;
-        }
-        default:
-            return fail(KRON_ERR_UNSUPPORTED, "dtype %d forward not implemented", (int)dtype);
+    if (dtype == KRON_F32) {
+        // exact FP32 on the CUDA cores: any shape whose tile fits shared memory
+        if (kron::simt_forward_rows(s) <= 0)
+            return fail(KRON_ERR_UNSUPPORTED,
+                        "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not "
+                        "fit shared memory", p, q, m1, m2, r);
+        e = kron::simt_forward(x, S, A, B, bias, y, s,
+                               (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
+    } else {
+        // the tensor-core paths run only where a tcgen05 kernel exists for the shape
+        const bool bf16 = dtype == KRON_BF16;
+        if (!kron::tc_forward_supported(s, bf16))
+            return fail(KRON_ERR_UNSUPPORTED,
+                        "no tensor-core kernel for p=%d q=%d m1=%d m2=%d r=%d on the %s path "
+                        "(KRON_F32 runs any shape)", p, q, m1, m2, r, bf16 ? "BF16" : "TF32");
+        e = kron::tc_forward(x, S, A, B, bias, y, s, bf16,
+                             (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return KRON_OK;
@@ -158,17 +210,9 @@ static kron_status_t backward_impl(const void *x, const void *S, const void *A, 
                                    kron_dtype_t dtype, unsigned flags, double l1,
                                    void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error[0] = 0;
-    kron_status_t st = check_shape(N, p, q, m1, m2, r, dtype, flags);
+    kron_status_t st = check_backward(x, S, A, B, dY, dX, dS, dA, dB, dbias, N, p, q, m1, m2, r,
+                                      dtype, flags, l1);
     if (st != KRON_OK) return st;
-    if (!(l1 >= 0.0 && l1 <= 1e30))
-        return fail(KRON_ERR_INVALID_ARG, "the l1 weight must be in [0, 1e30] (got %g)", l1);
-    if (!S || !A || !B || !dS || !dA || !dB || (N > 0 && (!x || !dY)))
-        return fail(KRON_ERR_INVALID_ARG,
-                    "S, A, B, dS, dA, dB (and x, dY when N > 0) must be non-null");
-    if (!aligned16(x) || !aligned16(S) || !aligned16(A) || !aligned16(B) || !aligned16(dY) ||
-        !aligned16(dS) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
-        (dbias && !aligned16(dbias)))
-        return fail(KRON_ERR_ALIGNMENT, "all tensors must be 16-byte aligned");
     const kron::Shape s{N, p, q, m1, m2, r};
     cudaStream_t cs = (cudaStream_t)stream;
     if (N == 0 && l1 != 0.0) {  // empty batch: only the penalty's gradient l1 * sign(S)
@@ -186,10 +230,6 @@ static kron_status_t backward_impl(const void *x, const void *S, const void *A, 
         return e == cudaSuccess ? KRON_OK : cuda_fail(e, "zero gradients");
     }
     const bool on_tc = tc_backward_path(s, dtype);
-    if (!on_tc && kron::simt_backward_rows(s) <= 0)
-        return fail(KRON_ERR_UNSUPPORTED,
-                    "no kernel for p=%d q=%d m1=%d m2=%d r=%d: the FP32 tile does not fit shared "
-                    "memory", p, q, m1, m2, r);
     const size_t need = kron_linear_workspace_size(N, p, q, m1, m2, r, dtype);
     if (!workspace || workspace_bytes < need)
         return fail(KRON_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
@@ -197,19 +237,18 @@ static kron_status_t backward_impl(const void *x, const void *S, const void *A, 
     if ((uintptr_t)workspace & 255u)
         return fail(KRON_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
     const int parts = backward_parts(s, dtype);
+    const bool skip = (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0;
     cudaError_t e = cudaSuccess;
-    const bool bf16 = dtype == KRON_BF16;
     if (on_tc) {
         e = kron::tc_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, (float *)dS,
-                              (float *)dA, (float *)dB, (float *)dbias, bf16, l1, cs);
+                              (float *)dA, (float *)dB, (float *)dbias, dtype == KRON_BF16, skip,
+                              l1, cs);
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     } else {
-        // exact-FP32 CUDA-core kernels (every KRON_F32 call; TF32/BF16 shapes with no
-        // compiled tensor-core kernel), then the fixed-order reduction of the partials
-        e = kron::simt_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, bf16,
-                                (flags & KRON_FLAG_SKIP_ZERO_BLOCKS) != 0, cs);
+        // exact FP32 on the CUDA cores, then the fixed-order reduction of the partials
+        e = kron::simt_backward(x, S, A, B, dY, dX, (float *)workspace, parts, s, skip, cs);
         if (e != cudaSuccess) return cuda_fail(e, "backward launch");
-        e = kron::reduce_partials((const float *)workspace, parts, S, A, bf16, (float *)dS,
+        e = kron::reduce_partials((const float *)workspace, parts, S, A, false, (float *)dS,
                                   (float *)dA, (float *)dB, (float *)dbias, s, l1, cs);
     }
     if (e != cudaSuccess) return cuda_fail(e, "reduction launch");

@@ -1,6 +1,7 @@
 // simt_f32.cu -- exact-FP32 path of the Kronecker layer on the CUDA cores (FFMA).
-// The I/O tensors may be fp32 or bf16 (converted on load and store); all arithmetic is
-// fp32.  Any shape whose tiles fit shared memory runs here.
+// The kernels are written for an I/O element type TI (converted to fp32 on load); the
+// library instantiates them for fp32 I/O.  All arithmetic is fp32.  Any shape whose
+// tiles fit shared memory runs here.
 //
 // Both contractions of the vec trick (page "kronecker-layer-benchmark", sections
 // "2. The vec trick" and "3. The vec trick without the loop") are fused per tile of
@@ -21,7 +22,6 @@
 #include "internal.h"
 
 #include <algorithm>
-#include <cuda_bf16.h>
 
 namespace kron {
 namespace {
@@ -137,24 +137,10 @@ __device__ __forceinline__ void smem_mm3(const MM &g1, bool acc1, const MM &g2, 
 }
 
 __device__ __forceinline__ float to_f(float v) { return v; }
-__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// Four consecutive elements (16 bytes of fp32, 8 of bf16) as floats.
+// Four consecutive fp32 elements (16 bytes).
 __device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(p);
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
-    return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
-}
 __device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
-__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 u;
-    u.x = *reinterpret_cast<const uint32_t *>(&lo);
-    u.y = *reinterpret_cast<const uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(p) = u;
-}
 
 // Row r of a [rows][width] global matrix -> shared rows with stride ld; rows at or
 // beyond N read as zero.  `width` elements per row (a multiple of 4), aligned rows.
@@ -1027,17 +1013,14 @@ cudaError_t simt_backward_t(const void *x, const void *S, const void *A, const v
 }  // namespace
 
 cudaError_t simt_forward(const void *x, const void *S, const void *A, const void *B,
-                         const void *bias, void *y, const Shape &s, bool bf16, bool skip,
-                         cudaStream_t st) {
-    return bf16 ? simt_forward_t<__nv_bfloat16>(x, S, A, B, bias, y, s, skip, st)
-                : simt_forward_t<float>(x, S, A, B, bias, y, s, skip, st);
+                         const void *bias, void *y, const Shape &s, bool skip, cudaStream_t st) {
+    return simt_forward_t<float>(x, S, A, B, bias, y, s, skip, st);
 }
 
 cudaError_t simt_backward(const void *x, const void *S, const void *A, const void *B,
                           const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                          bool bf16, bool skip, cudaStream_t st) {
-    return bf16 ? simt_backward_t<__nv_bfloat16>(x, S, A, B, dY, dX, ws, parts, s, skip, st)
-                : simt_backward_t<float>(x, S, A, B, dY, dX, ws, parts, s, skip, st);
+                          bool skip, cudaStream_t st) {
+    return simt_backward_t<float>(x, S, A, B, dY, dX, ws, parts, s, skip, st);
 }
 
 }  // namespace kron

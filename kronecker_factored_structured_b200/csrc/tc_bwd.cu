@@ -44,11 +44,6 @@
 namespace kron {
 namespace tc {
 
-int *device_error_ptr();
-cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
-                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw,
-                         bool atom32);
-
 namespace {
 
 template <typename T> struct BE;
@@ -670,25 +665,18 @@ PgFn find_pg(const Shape &s, bool bf16) {
 }
 
 }  // namespace
-}  // namespace tc
 
-bool tc_backward_supported(const Shape &s, bool bf16) {
-    return tc::find_pg(s, bf16) != nullptr && tc_dx_supported(s, bf16);
-}
+// ---- entry points of the tuned parameter-gradient kernel ----
+bool tuned_pgrad_supported(const Shape &s, bool bf16) { return find_pg(s, bf16) != nullptr; }
 
-int tc_backward_tile_rows(const Shape &) { return 2; }
-
-cudaError_t tc_backward(const void *x, const void *S, const void *A, const void *B,
-                        const void *dY, void *dX, float *ws, int parts, const Shape &s,
-                        float *dS, float *dA, float *dB, float *dbias, bool bf16, double l1,
+cudaError_t tuned_pgrad(const void *x, const void *S, const void *A, const void *B,
+                        const void *dY, float *ws, int parts, const Shape &s, float *dS,
+                        float *dA, float *dB, float *dbias, bool bf16, double l1,
                         cudaStream_t st) {
-    tc::PgFn fn = tc::find_pg(s, bf16);
+    PgFn fn = find_pg(s, bf16);
     if (!fn) return cudaErrorNotSupported;
-    if (dX) {
-        const cudaError_t e = tc_dx(dY, S, A, B, dX, s, bf16, st);
-        if (e != cudaSuccess) return e;
-    }
     return fn(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, l1, st);
 }
 
+}  // namespace tc
 }  // namespace kron

@@ -30,14 +30,10 @@
 #include "internal.h"
 #include "tc_ptx.cuh"
 
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
-#include <mutex>
 
 namespace kron {
 namespace tc {
-
-__device__ int g_device_error = 0;
 
 template <typename T> struct Elt;
 template <> struct Elt<float> {
@@ -415,70 +411,6 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2-D tensor map of a row-major [rows][cols] matrix, box = box_cols x box_rows, swizzled
-// by sw bytes (128, 64, 32 or 0); atom32 selects the 128-byte swizzle with 32-byte atoms
-// (the shared-memory layout of MN-major TF32 MMA operands).
-cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t rows,
-                         uint64_t cols, uint32_t box_cols, uint32_t box_rows, int sw,
-                         bool atom32) {
-    auto enc = get_encode();
-    if (!enc) return cudaErrorNotSupported;
-    // The encoder is a driver-API call: make the current device's primary context current
-    // on this host thread first (a thread whose first CUDA call this is has none bound).
-    int dev = 0;
-    cudaError_t ce = cudaGetDevice(&dev);
-    if (ce == cudaSuccess) ce = cudaSetDevice(dev);
-    if (ce != cudaSuccess) return ce;
-    const int E = bf16 ? 2 : 4;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * E};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUtensorMapSwizzle swm = atom32      ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
-                           : sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                           : sw == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
-                           : sw == 32  ? CU_TENSOR_MAP_SWIZZLE_32B
-                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
-    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                     2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, swm, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-// Address of the device error word on the current device (looked up once per device).
-int *device_error_ptr() {
-    static int *ptrs[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = (int *)p;
-    }
-    return ptrs[dev];
-}
-
-int num_sms() {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 template <class Cfg, bool TR>
 cudaError_t launch_fwd(const void *x, const void *S, const void *A, const void *B,
                        const void *bias, void *y, const Shape &s, cudaStream_t st) {
@@ -531,42 +463,18 @@ FwdFn find_fwd(const Shape &s, bool bf16, bool tr) {
     return nullptr;
 }
 
-// The kernel shape of dX = dY W^T: the layer's shape with (p, q) and (m1, m2) swapped.
-Shape transposed(const Shape &s) { return Shape{s.N, s.q, s.p, s.m2, s.m1, s.r}; }
+// ---- entry points of the tuned kernels (tc_dispatch.cu chooses between kernel families) ----
+bool tuned_fwd_supported(const Shape &ks, bool bf16, bool tr) {
+    return find_fwd(ks, bf16, tr) != nullptr;
+}
+
+cudaError_t tuned_fwd(const void *x, const void *S, const void *A, const void *B,
+                      const void *bias, void *y, const Shape &ks, bool bf16, bool tr,
+                      cudaStream_t st) {
+    FwdFn fn = find_fwd(ks, bf16, tr);
+    if (!fn) return cudaErrorNotSupported;
+    return fn(x, S, A, B, tr ? nullptr : bias, y, ks, st);
+}
 
 }  // namespace tc
-
-bool tc_forward_supported(const Shape &s, bool bf16) {
-    return tc::find_fwd(s, bf16, false) != nullptr;
-}
-
-cudaError_t tc_forward(const void *x, const void *S, const void *A, const void *B,
-                       const void *bias, void *y, const Shape &s, bool bf16, cudaStream_t st) {
-    tc::FwdFn fn = tc::find_fwd(s, bf16, false);
-    if (!fn) return cudaErrorNotSupported;
-    return fn(x, S, A, B, bias, y, s, st);
-}
-
-bool tc_dx_supported(const Shape &s, bool bf16) {
-    return tc::find_fwd(tc::transposed(s), bf16, true) != nullptr;
-}
-
-cudaError_t tc_dx(const void *dY, const void *S, const void *A, const void *B, void *dX,
-                  const Shape &s, bool bf16, cudaStream_t st) {
-    const Shape t = tc::transposed(s);
-    tc::FwdFn fn = tc::find_fwd(t, bf16, true);
-    if (!fn) return cudaErrorNotSupported;
-    return fn(dY, S, A, B, nullptr, dX, t, st);
-}
-
-int tc_read_device_error(bool clear) {
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, tc::g_device_error, sizeof(int)) != cudaSuccess) return -1;
-    if (clear && v) {
-        const int z = 0;
-        cudaMemcpyToSymbol(tc::g_device_error, &z, sizeof(int));
-    }
-    return v;
-}
-
 }  // namespace kron

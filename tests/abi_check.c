@@ -95,6 +95,28 @@ int main(void) {
     CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, P, P, P, NULL, 20000, 64, 64, 64, 64, 8,
                                        KRON_F32, 0, NULL) == KRON_ERR_WORKSPACE);
     CHECK(strstr(kron_last_error(), "scratch") != NULL);
+    /* an oversized problem with a bad argument: the argument's own status comes first */
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, NULL, P, P, NULL, 20000, 64, 64, 64, 64,
+                                       8, KRON_F32, 0, NULL) == KRON_ERR_INVALID_ARG);
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, MIS, P, P, P, P, NULL, 20000, 64, 64, 64, 64,
+                                       8, KRON_F32, 0, NULL) == KRON_ERR_ALIGNMENT);
+    CHECK(kron_linear_backward_noalloc(NULL, P, P, P, P, P, P, P, P, NULL, 8, 2, 2, 4, 4, 1,
+                                       KRON_F32, 0, NULL) == KRON_ERR_INVALID_ARG);
+
+    /* the tensor-core paths refuse shapes they have no kernel for (no silent FP32 run):
+       1024^2 with 16x16 blocks (p = q = 64) and rank 2 on TF32; a 15x24 layer on BF16 */
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 64, 64, 16, 16, 2, KRON_TF32, 0, NULL) ==
+          KRON_ERR_UNSUPPORTED);
+    CHECK(strstr(kron_last_error(), "tensor-core") != NULL);
+    CHECK(kron_linear_forward(P, P, P, P, NULL, P, 8, 3, 5, 8, 8, 3, KRON_BF16, 0, NULL) ==
+          KRON_ERR_UNSUPPORTED);
+    CHECK(kron_linear_workspace_size(8, 64, 64, 16, 16, 2, KRON_TF32) == 0);
+    CHECK(kron_linear_backward(P, P, P, P, P, P, P, P, P, NULL, 8, 64, 64, 16, 16, 2, KRON_TF32,
+                               0, WS, 1u << 20, NULL) == KRON_ERR_UNSUPPORTED);
+    CHECK(kron_linear_backward_noalloc(P, P, P, P, P, P, P, P, P, NULL, 8, 3, 5, 8, 8, 3,
+                                       KRON_BF16, 0, NULL) == KRON_ERR_UNSUPPORTED);
+    /* the same shapes run on the exact-FP32 path */
+    CHECK(kron_linear_workspace_size(8, 64, 64, 16, 16, 2, KRON_F32) > 0);
 
     if (failures) return 1;
     printf("abi_check: all checks passed\n");

@@ -96,6 +96,47 @@ def test_backward_rejects_misaligned_workspace():
     assert bwd(ws=V(0x10010), ws_bytes=need) == 3
 
 
+# shapes without a tensor-core kernel: the block-size sweep's 16x16 and 8x8 blocks on TF32,
+# and a small odd-sized layer on BF16
+NO_TC = [(64, 64, 16, 16, 2, 1), (128, 128, 8, 8, 8, 1), (3, 5, 8, 8, 3, 2)]
+
+
+@pytest.mark.parametrize("shape", NO_TC, ids=lambda s: "p{}q{}_m{}x{}_r{}_dt{}".format(*s))
+def test_tensor_core_paths_refuse_shapes_without_a_kernel(shape):
+    """A TF32 or BF16 request on a shape that no tcgen05 kernel covers returns
+    KRON_ERR_UNSUPPORTED from every entry point, before anything touches the device; the
+    exact-FP32 path takes the same shape."""
+    p, q, m1, m2, r, dt = shape
+    lib = native.load()
+    assert fwd(p=p, q=q, m1=m1, m2=m2, r=r, dtype=dt) == 2
+    assert "tensor-core" in lib.kron_last_error().decode()
+    assert lib.kron_linear_workspace_size(8, p, q, m1, m2, r, dt) == 0
+    st = lib.kron_linear_backward(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                  ALIGNED, ALIGNED, None, 8, p, q, m1, m2, r, dt, 0,
+                                  V(0x100000), 1 << 24, None)
+    assert st == 2
+    st = lib.kron_linear_backward_noalloc(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                          ALIGNED, ALIGNED, ALIGNED, None, 8, p, q, m1, m2, r,
+                                          dt, 0, None)
+    assert st == 2
+    assert lib.kron_linear_workspace_size(8, p, q, m1, m2, r, 0) > 0
+
+
+def test_noalloc_checks_arguments_before_the_size_limit():
+    """An oversized problem with a missing or misaligned pointer gets the pointer's status,
+    not KRON_ERR_WORKSPACE: the argument checks come first."""
+    lib = native.load()
+    big = (20000, 64, 64, 64, 64, 8)
+    assert lib.kron_linear_workspace_size(*big, 0) > native.KRON_NOALLOC_SCRATCH_BYTES
+
+    def call(x=ALIGNED, dS=ALIGNED):
+        return lib.kron_linear_backward_noalloc(x, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED,
+                                                dS, ALIGNED, ALIGNED, None, *big, 0, 0, None)
+    assert call() == 4
+    assert call(dS=None) == 1
+    assert call(x=MISALIGNED) == 3
+
+
 @pytest.mark.parametrize("l1", [-1.0, float("nan"), float("inf"), -1e-300])
 def test_backward_l1_rejects_bad_weight(l1):
     """The penalty weight must be finite and >= 0; checked before any pointer is read."""
