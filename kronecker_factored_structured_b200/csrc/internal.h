@@ -101,6 +101,20 @@ cudaError_t tuned_pgrad(const void *x, const void *S, const void *A, const void 
                         const void *dY, float *ws, int parts, const Shape &s, float *dS,
                         float *dA, float *dB, float *dbias, bool bf16, double l1,
                         cudaStream_t st);
+// Generic tensor-core kernels (tc_gen_fwd.cu, tc_gen_pgrad.cu) for the other compiled
+// shapes.  skip = KRON_FLAG_SKIP_ZERO_BLOCKS.
+bool generic_fwd_supported(const Shape &ks, bool bf16, bool tr);
+cudaError_t generic_fwd(const void *x, const void *S, const void *A, const void *B,
+                        const void *bias, void *y, const Shape &ks, bool bf16, bool tr,
+                        bool skip, cudaStream_t st);
+// Row-range partials of dC, dB and dbias into ws (parts x partial_stride floats); the
+// grid is parts x (rank groups) CTAs.  The fixed-order sum over ranges is reduce.cu's.
+bool generic_pgrad_supported(const Shape &s, bool bf16);
+int generic_pgrad_tile_rows(const Shape &s, bool bf16);
+int generic_pgrad_max_parts(const Shape &s, bool bf16);
+cudaError_t generic_pgrad(const void *x, const void *S, const void *A, const void *B,
+                          const void *dY, float *ws, int parts, const Shape &s, bool bf16,
+                          cudaStream_t st);
 }  // namespace tc
 
 // ---- deterministic reduction of the row-range partials (reduce.cu) ----

@@ -49,13 +49,18 @@ cudaError_t current_context_id(int *dev, unsigned long long *id) {
         get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
     });
     cudaError_t e = cudaGetDevice(dev);
-    // make the runtime's context current on this thread (a thread whose first CUDA call
-    // this is has none bound); a context the caller made current stays current
-    if (e == cudaSuccess) e = cudaFree(nullptr);
     if (e != cudaSuccess) return e;
     if (!get_current || !get_id) return cudaErrorNotSupported;
     CUcontext ctx = nullptr;
-    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    if (!ctx) {
+        // no context bound to this thread yet (its first CUDA call): bind the device's
+        // primary context, as the runtime does for a launch (legal under stream capture,
+        // unlike calls that synchronise)
+        e = cudaSetDevice(*dev);
+        if (e != cudaSuccess) return e;
+        if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    }
     if (get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
     return cudaSuccess;
 }
@@ -72,7 +77,7 @@ cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t
     // on this host thread first (a thread whose first CUDA call this is has none bound).
     int dev = 0;
     cudaError_t ce = cudaGetDevice(&dev);
-    if (ce == cudaSuccess) ce = cudaFree(nullptr);
+    if (ce == cudaSuccess) ce = cudaSetDevice(dev);
     if (ce != cudaSuccess) return ce;
     const int E = bf16 ? 2 : 4;
     cuuint64_t dims[2] = {cols, rows};
