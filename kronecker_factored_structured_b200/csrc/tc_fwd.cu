@@ -69,13 +69,22 @@ struct FwdCfg {
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_MAX = 232448;
     static constexpr int FIXED = 1024 + BAR_BYTES + B2_BYTES;
-    // T buffers: as many as leave room for at least 6 x stages (at most 4)
-    static constexpr int TB = (SMEM_MAX - FIXED - 4 * T_BYTES) / X_BYTES >= 6 ? 4
+    // TS2 (TF32, r = 128/m2 = 4 rows per tile, p = m2 = 32): stage 2 reads T from TMEM.  The
+    // stage-1 accumulator block of rank i and row n (lanes i*32.., columns n*32..) belongs,
+    // as stage 2's A operand, at lanes n*32.., columns i*32..: the four diagonal blocks are
+    // in place and the twelve others swap in pairs through a shared-memory scratch (two
+    // buffers of 16 warps x 4 KB), so no T buffer is needed.
+    static constexpr bool TS2 = Elt<T>::tf32 && R == NT && P == 32 && M2 == 32;
+    static constexpr int SWP_BYTES = TS2 ? 2 * 16 * 4096 : 0;
+    // T buffers (SS path): as many as leave room for at least 6 x stages (at most 4)
+    static constexpr int TB = TS2 ? 0
+                            : (SMEM_MAX - FIXED - 4 * T_BYTES) / X_BYTES >= 6 ? 4
                             : (SMEM_MAX - FIXED - 3 * T_BYTES) / X_BYTES >= 6 ? 3 : 2;
-    static constexpr int STAGES = cmin(8, (SMEM_MAX - FIXED - TB * T_BYTES) / X_BYTES);
+    static constexpr int STAGES =
+        cmin(8, (SMEM_MAX - FIXED - SWP_BYTES - TB * T_BYTES) / X_BYTES);
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_T = OFF_B2 + B2_BYTES;
-    static constexpr int OFF_X = OFF_T + TB * T_BYTES;
+    static constexpr int OFF_X = OFF_T + TB * T_BYTES + SWP_BYTES;
     static constexpr int OFF_BAR = OFF_X + STAGES * X_BYTES;
     static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // barriers + alignment slack
     // TMEM columns: D1[3] (N1 each), D2[3] (Q each), stage 1's A operand B_all^T
@@ -99,7 +108,8 @@ struct FwdCfg {
     static_assert(P % 32 == 0 && (32 * E) <= SW2 && SW2 == 128,
                   "a 32-column TMEM chunk maps to one 128B-swizzled row of T");
     static_assert(STAGES >= 3, "x ring");
-    static_assert(2 * STAGES + 2 * D1_SLOTS + 2 * TB + 2 * D2_SLOTS + 2 + 2 <= BAR_BYTES / 8,
+    static_assert(2 * STAGES + 2 * D1_SLOTS + 2 * (TS2 ? D1_SLOTS : TB) + 2 * D2_SLOTS + 2 + 2 <=
+                      BAR_BYTES / 8,
                   "barrier region");
     static_assert(TM_COLS_USED <= 512, "TMEM budget");
     static_assert(SMEM <= SMEM_MAX, "shared memory budget");
@@ -160,8 +170,10 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     const uint32_t sB2 = sbase + Cfg::OFF_B2, sX = sbase + Cfg::OFF_X, sT = sbase + Cfg::OFF_T;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     // barrier indices
+    constexpr bool TS2 = Cfg::TS2;
+    constexpr int NTB = TS2 ? D1S : TB;   // TS2: B_TFULL + d1 = "A operand of slot d1 ready"
     constexpr int B_XFULL = 0, B_XEMPTY = S, B_D1FULL = 2 * S, B_D1EMPTY = 2 * S + D1S,
-                  B_TFULL = 2 * S + 2 * D1S, B_TEMPTY = B_TFULL + TB, B_D2FULL = B_TFULL + 2 * TB,
+                  B_TFULL = 2 * S + 2 * D1S, B_TEMPTY = B_TFULL + NTB, B_D2FULL = B_TFULL + 2 * NTB,
                   B_D2EMPTY = B_D2FULL + D2S, B_DRAIN = B_D2FULL + 2 * D2S, NBARS = B_DRAIN + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
     const Abort abort_flag{reinterpret_cast<volatile int *>(tmem_slot + 1), args.device_error};
@@ -189,9 +201,11 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         }
         for (int b = 0; b < D1S; ++b) {
             mbar_init(bar(B_D1FULL + b), 1);
-            mbar_init(bar(B_D1EMPTY + b), 16);  // epilogue-1 warps
+            // SS path: the epilogue-1 warps free a slot once it is in registers; TS2: the
+            // stage-2 MMAs that read it free it
+            mbar_init(bar(B_D1EMPTY + b), TS2 ? 1 : 16);
         }
-        for (int b = 0; b < TB; ++b) {
+        for (int b = 0; b < NTB; ++b) {
             mbar_init(bar(B_TFULL + b), 16);
             mbar_init(bar(B_TEMPTY + b), 1);
         }
@@ -299,6 +313,32 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         __syncwarp();
         if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 0), 0);
         __syncwarp();
+    } else if (warp == 2 && TS2) {
+        // ---------------- stage-2 issuer, TS2: D2[(n,k)][c] = A2 (TMEM) . C' ----------------
+        const uint64_t bd0 = sdesc_kmajor(sB2, Cfg::SW2);
+        for (int t = 0; t < my_tiles; ++t) {
+            const int d1 = t % D1S, d2 = t % D2S;
+            if (!warp_wait(bar(B_D2EMPTY + d2), ((t / D2S) & 1) ^ 1, abort_flag) ||
+                !warp_wait(bar(B_TFULL + d1), (t / D1S) & 1, abort_flag))
+                break;
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t d = tmem + Cfg::TM_D2 + d2 * Q;
+#pragma unroll
+                for (int kk = 0; kk < Cfg::K2B / 32; ++kk) {
+                    const int kb = kk * 32, ch = kb / Cfg::SW2, in = kb % Cfg::SW2;
+                    mma_ts<true>(d, tmem + Cfg::TM_D1 + d1 * N1 + kk * 8,
+                                 desc_add(bd0, ch * Q * Cfg::SW2 + in), Cfg::IDESC2, kk > 0);
+                }
+                mma_commit(bar(B_D1EMPTY + d1));
+                mma_commit(bar(B_D2FULL + d2));
+            }
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(bar(B_DRAIN + 1));
+        __syncwarp();
+        if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 1), 0);
+        __syncwarp();
     } else if (warp == 2) {
         // ---------------- stage-2 issuer: D2[(n,k)][c] = T . C' ----------------
         const uint64_t bd0 = sdesc_kmajor(sB2, Cfg::SW2);
@@ -326,6 +366,54 @@ kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
         __syncwarp();
         if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 1), 0);
         __syncwarp();
+    } else if (warp < 19 && TS2) {
+        // ---------------- epilogue 1, TS2: swap the off-diagonal blocks in TMEM ----------------
+        // warp (quadrant i, part n) holds block (i, n): lanes (i,k), columns (n, a).  It belongs
+        // at lanes (n,k), columns (i, a), where warp (n, i) holds block (n, i), which belongs
+        // here: the two warps exchange their blocks through the scratch and each stores the
+        // other's into its own place.  Diagonal warps (i == n) have nothing to move.
+        const int quad = warp & 3, part = (warp - 3) >> 2;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const bool diag = quad == part;
+        const int lo = quad < part ? quad : part, hi = quad < part ? part : quad;
+        const int pair_bar = 1 + (lo == 0 ? hi - 1 : lo == 1 ? hi + 1 : 5);   // ids 1..6
+        const uint32_t sswp = sT;   // the scratch sits where the T buffers would be
+        const uint32_t mine = (uint32_t)(quad * 4 + part) * 4096 + (uint32_t)lane * 128;
+        const uint32_t theirs = (uint32_t)(part * 4 + quad) * 4096 + (uint32_t)lane * 128;
+        for (int t = 0; t < my_tiles; ++t) {
+            const int d1 = t % D1S;
+            const uint32_t buf = sswp + (uint32_t)(t & 1) * 16 * 4096;
+            const bool ok = mbar_wait(bar(B_D1FULL + d1), (t / D1S) & 1, abort_flag);
+            if (diag) {
+                if (!ok) break;
+                tc_fence_after();
+                tc_fence_before();
+                mbar_arrive_warp(bar(B_TFULL + d1));
+                continue;
+            }
+            const uint32_t col = tmem + lane_addr + Cfg::TM_D1 + d1 * N1 + part * 32;
+            if (ok) {
+                tc_fence_after();
+                uint32_t r[32];
+                tmem_load32(col, r);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    st_shared_v4(buf + mine + (uint32_t)((j ^ (lane & 7)) << 4), r[4 * j],
+                                 r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            }
+            // both warps of the pair have written (or both leave: one verdict for the pair)
+            if (!named_bar_and(pair_bar, 64, ok)) break;
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t q4[4];
+                ld_shared_v4(buf + theirs + (uint32_t)((j ^ (lane & 7)) << 4), q4);
+                v[4 * j] = q4[0]; v[4 * j + 1] = q4[1]; v[4 * j + 2] = q4[2]; v[4 * j + 3] = q4[3];
+            }
+            tmem_store32(col, v);
+            tc_fence_before();
+            mbar_arrive_warp(bar(B_TFULL + d1));
+        }
     } else if (warp < 19) {
         // ---------------- epilogue 1: D1 (lanes (i,k), columns (n,a)) -> T smem ----------------
         const int quad = warp & 3, part = (warp - 3) >> 2;

@@ -15,11 +15,15 @@
 // stage 2 reads (the page's permute of Z, on chip), and stage 2 accumulates the chunks of
 // a tile into one TMEM accumulator.  Within a chunk the K index of stage 2 runs over
 // (a-group, i, a-in-group) with groups of 16 bytes of a values, so that one MMA K step
-// covers few rows a of S: with KRON_FLAG_SKIP_ZERO_BLOCKS a K step is issued only over the
-// 16-column blocks of c where S has a non-zero in the step's rows a and those columns
-// (the m1 x m2 blocks of W at zero entries of S are zero: page "kronecker-layer-benchmark",
-// introduction).  The first K step of every tile is always issued in full, which also
-// clears the accumulator.
+// covers few rows a of S: with KRON_FLAG_SKIP_ZERO_BLOCKS a K step is not issued when S is
+// zero in all of the step's rows a (the m1 x m2 blocks of W at zero entries of S are zero:
+// page "kronecker-layer-benchmark", introduction), and the epilogue does not store the T
+// values such a step would have read.  Every MMA keeps the one shape N = q (measured: MMAs
+// of mixed N, issued over runs of non-zero 16-column blocks only, ran slower than the dense
+// stage).  The first K step of every tile is always issued, which also clears the
+// accumulator (the T values it reads where C' is zero may be stale, and meet zeros).  A
+// per-16-column-block mask (bit cb of a K step's word) is kept for that reason only as the
+// test of a K step's word against zero.
 //
 // TR = true computes dX = dY W^T with the same kernel: dX_n = sum_i C_i G_n B_i^T is the
 // vec trick with C_i^T and B_i^T, so the kernel's (p, q, m1, m2) are the layer's
@@ -206,21 +210,21 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         st_shared_v4(sCP + b * Cfg::CP_BLK + kmaj(c, kp0 * E, QP, 128), w[0], w[1], w[2], w[3]);
     }
     // zero-block mask: bit cb of mask[b*KS2 + ks] is set when S has a non-zero in the rows a
-    // of K step ks of chunk b and the 16 columns c of block cb
+    // of K step ks of chunk b and the 16 columns c of block cb.  Every thread tests one
+    // (chunk, K position, c block) at a time; the words start at zero.
     if (args.skip) {
-        for (int e = threadIdx.x; e < MB1 * KS2; e += blockDim.x) {
-            const int b = e / KS2, ks = e % KS2;
-            uint32_t m = 0;
-            for (int kp = ks * Cfg::KSTEP; kp < (ks + 1) * Cfg::KSTEP && kp < Cfg::K2; ++kp) {
-                const int g = kp / (IPBE * AG), il = (kp % (IPBE * AG)) / AG;
-                const int a = g * AG + kp % AG;
-                if (b * IPB + il >= R) continue;
-                for (int c = 0; c < Q; ++c) {
-                    const float sv = ld_elt<T>(args.S, TR ? (size_t)c * P + a : (size_t)a * Q + c);
-                    if (sv != 0.f) m |= 1u << (c / 16);
-                }
-            }
-            mask[e] = m;
+        for (int e = threadIdx.x; e < MB1 * KS2; e += blockDim.x) mask[e] = 0;
+        __syncthreads();
+        for (int e = threadIdx.x; e < MB1 * Cfg::K2P * Cfg::NCB; e += blockDim.x) {
+            const int b = e / (Cfg::K2P * Cfg::NCB), rem = e % (Cfg::K2P * Cfg::NCB);
+            const int kp = rem / Cfg::NCB, cb = rem % Cfg::NCB;
+            const int g = kp / (IPBE * AG), il = (kp % (IPBE * AG)) / AG;
+            const int a = g * AG + kp % AG;
+            if (kp >= Cfg::K2 || b * IPB + il >= R) continue;
+            bool nz = false;
+            for (int c = cb * 16; c < cb * 16 + 16 && c < Q; ++c)
+                nz |= ld_elt<T>(args.S, TR ? (size_t)c * P + a : (size_t)a * Q + c) != 0.f;
+            if (nz) atomicOr(&mask[b * KS2 + kp / Cfg::KSTEP], 1u << cb);
         }
     }
     fence_proxy_async();
@@ -302,6 +306,9 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         __syncwarp();
     } else if (warp == 2) {
         // ---------------- stage 2: D2 += T_b . C'_b over the chunks of a tile ----------------
+        // the skip mask words in registers: lane l holds words l and l + 32
+        const uint32_t mw0 = args.skip && lane < MB1 * KS2 ? mask[lane] : 0u;
+        const uint32_t mw1 = args.skip && lane + 32 < MB1 * KS2 ? mask[lane + 32] : 0u;
         bool ok = true;
         for (int t = 0; t < my_tiles && ok; ++t) {
             const int d2 = t % D2S;
@@ -313,30 +320,27 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
                     break;
                 }
                 tc_fence_after();
+                uint32_t msk[KS2];   // this chunk's mask words, warp-uniform
+#pragma unroll
+                for (int ks = 0; ks < KS2; ++ks) {
+                    const int wdx = b * KS2 + ks;
+                    msk[ks] = __shfl_sync(0xffffffffu, wdx < 32 ? mw0 : mw1, wdx & 31);
+                }
                 if (elect_one()) {
                     const uint32_t d = tmem + Cfg::TM_D2 + d2 * QS;
                     const uint64_t ad0 = sdesc_kmajor(sT + tb * Cfg::TC_BYTES, 128);
                     const uint64_t bd0 = sdesc_kmajor(sCP + b * Cfg::CP_BLK, 128);
+#pragma unroll
                     for (int ks = 0; ks < KS2; ++ks) {
                         const int kb = ks * 32, ch = kb / 128, in = kb % 128;
                         const uint64_t ad = desc_add(ad0, ch * 128 * 128 + in);
                         const uint64_t bd = desc_add(bd0, ch * QP * 128 + in);
                         const bool first = b == 0 && ks == 0;
-                        if (!args.skip || first) {
+                        // with the skip flag, a K step whose slice of C' is zero over every
+                        // column is not issued (all MMAs keep one shape)
+                        if (!args.skip || first || msk[ks] != 0u)
                             mma_ss<GE<T>::tf32>(d, ad, bd, idesc_f32acc(128, QP, GE<T>::fmt),
                                                 first ? 0u : 1u);
-                        } else {
-                            // one MMA per run of consecutive non-zero 16-column blocks
-                            uint32_t m = mask[b * KS2 + ks];
-                            while (m) {
-                                const int c0 = __ffs(m) - 1;
-                                const uint32_t rest = ~(m >> c0);
-                                const int len = rest ? __ffs(rest) - 1 : 32 - c0;
-                                mma_ss<GE<T>::tf32>(d + c0 * 16, ad, desc_add(bd, c0 * 16 * 128),
-                                                    idesc_f32acc(128, len * 16, GE<T>::fmt), 1u);
-                                m &= (len + c0 >= 32) ? 0u : ~((1u << (c0 + len)) - 1u);
-                            }
-                        }
                     }
                     mma_commit(bar(B_TEMPTY + tb));
                     if (b == MB1 - 1) mma_commit(bar(B_D2FULL + d2));
@@ -353,7 +357,40 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         const int quad = warp & 3, wi = (warp - 3) >> 2;
         const int L = quad * 32 + lane, il = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        constexpr int NG = N1S / 32;     // 32-column groups of a D1 slot
+        constexpr int NG = N1S / 32;                  // 32-column groups of a D1 slot
+        constexpr int GPW = (NG + 3) / 4;             // groups of one warp (at most 2)
+        constexpr int SPG = 32 / VPC;                 // 16-byte stores per group
+        // byte offsets (within a T chunk) of this lane's 16-byte stores, fixed for the kernel:
+        // column c = (n, a) of lane (i_local, k) goes to row (n, k), K position
+        // (a / AG) * (IPBE * AG) + i_local * AG + a % AG; 0xFFFFFFFF marks a column past N1
+        uint32_t soff[GPW][SPG];
+        uint8_t sks[GPW][SPG];                        // K step of each store
+#pragma unroll
+        for (int gi = 0; gi < GPW; ++gi) {
+#pragma unroll
+            for (int g = 0; g < SPG; ++g) {
+                const int c = (wi + 4 * gi) * 32 + g * VPC;
+                const int n = c / P, a = c % P;
+                const int kp = (a / AG) * (IPBE * AG) + il * AG + a % AG;
+                soff[gi][g] = c < N1 ? kmaj(n * M2 + k, kp * E, 128, 128) : 0xFFFFFFFFu;
+                sks[gi][g] = (uint8_t)(kp / Cfg::KSTEP);
+            }
+        }
+        // with the skip flag, bit (b*GPW + gi)*SPG + g says whether store (gi, g) of chunk b
+        // feeds a K step that stage 2 issues
+        static_assert(MB1 * GPW * SPG <= 64, "live bits");
+        uint64_t keep = ~0ull;
+        if (args.skip) {
+            keep = 0;
+#pragma unroll
+            for (int b = 0; b < MB1; ++b)
+#pragma unroll
+                for (int gi = 0; gi < GPW; ++gi)
+#pragma unroll
+                    for (int g = 0; g < SPG; ++g)
+                        if (mask[b * KS2 + sks[gi][g]] != 0u)
+                            keep |= 1ull << ((b * GPW + gi) * SPG + g);
+        }
         bool ok = true;
         for (int t = 0; t < my_tiles && ok; ++t) {
             for (int b = 0; b < MB1; ++b) {
@@ -370,21 +407,24 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
                     tc_fence_before();
                     mbar_arrive_warp(bar(B_D1EMPTY + d1));
                 }
-                for (int cg = wi; cg < NG; cg += 4) {
-                    uint32_t r[32];
-                    tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1S + cg * 32, r);
-                    if (cg + 4 >= NG) {
-                        tc_fence_before();
-                        mbar_arrive_warp(bar(B_D1EMPTY + d1));
-                    }
-                    if (live) {
 #pragma unroll
-                        for (int g = 0; g < 32 / VPC; ++g) {
-                            const int c = cg * 32 + g * VPC;
-                            if (c < N1) {
-                                const int n = c / P, a = c % P;
-                                const int kp = (a / AG) * (IPBE * AG) + il * AG + a % AG;
-                                st_op16<T>(tbase + kmaj(n * M2 + k, kp * E, 128, 128), &r[g * VPC]);
+                for (int gi = 0; gi < GPW; ++gi) {
+                    const int cg = wi + 4 * gi;
+                    if (cg < NG) {
+                        uint32_t r[32];
+                        tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1S + cg * 32, r);
+                        if (cg + 4 >= NG) {
+                            tc_fence_before();
+                            mbar_arrive_warp(bar(B_D1EMPTY + d1));
+                        }
+                        if (live) {
+#pragma unroll
+                            for (int g = 0; g < SPG; ++g) {
+                                // with the skip flag, T values whose K step multiplies an
+                                // all-zero slice of C' are never used: their store is dropped
+                                if (soff[gi][g] != 0xFFFFFFFFu &&
+                                    ((keep >> ((b * GPW + gi) * SPG + g)) & 1ull))
+                                    st_op16<T>(tbase + soff[gi][g], &r[g * VPC]);
                             }
                         }
                     }
@@ -398,11 +438,16 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         const int quad = warp & 3;
         const int L = quad * 32 + lane, n = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        // bias values of this lane (c*m2 + k), read through the non-coherent path in batches
+        // that precede the y stores of the batch (so no load waits on an earlier store)
+        const unsigned short *bias16 = static_cast<const unsigned short *>(args.bias);
+        const float *bias32 = static_cast<const float *>(args.bias);
         for (int t = 0; t < my_tiles; ++t) {
             const int d2 = t % D2S;
             if (!mbar_wait(bar(B_D2FULL + d2), (t / D2S) & 1, abort_flag)) break;
             tc_fence_after();
             const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
+            const size_t obase = (size_t)row * (Q * M2) + k;
 #pragma unroll 1
             for (int c0 = 0; c0 < QS; c0 += 32) {
                 uint32_t r[32];
@@ -413,14 +458,27 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
                 }
                 if (row < args.N) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int c = c0 + u;
-                        if (c < Q) {
-                            const float bv = args.bias ? ld_elt<T>(args.bias, (size_t)c * M2 + k) : 0.f;
-                            const float v = __uint_as_float(r[u]) + bv;
-                            const size_t o = (size_t)row * (Q * M2) + (size_t)c * M2 + k;
-                            if constexpr (GE<T>::tf32) static_cast<float *>(args.y)[o] = v;
-                            else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
+                    for (int u0 = 0; u0 < 32; u0 += 8) {
+                        float bv[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int c = c0 + u0 + u;
+                            bv[u] = 0.f;
+                            if (args.bias && c < Q) {
+                                if constexpr (GE<T>::tf32) bv[u] = __ldg(bias32 + (size_t)c * M2 + k);
+                                else bv[u] = __bfloat162float(__ushort_as_bfloat16(
+                                         __ldg(bias16 + (size_t)c * M2 + k)));
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int c = c0 + u0 + u;
+                            if (c < Q) {
+                                const float v = __uint_as_float(r[u0 + u]) + bv[u];
+                                const size_t o = obase + (size_t)c * M2;
+                                if constexpr (GE<T>::tf32) static_cast<float *>(args.y)[o] = v;
+                                else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
+                            }
                         }
                     }
                 }

@@ -8,7 +8,8 @@
 //   U [(i,a),(n,k)] = sum_c  C_i[a,c] G_n[c,k]        A = C_stack block (TMEM), B = G tile
 //                                                     read MN-major
 //   dC[(i,a),c]    += sum_(n,k) T[n,a,i,k] G_n[c,k]   A = T2 [(i,a)][(n,k)] (shared), B = G
-//   dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]   A = U2 [(i,k)][(n,a)] (shared), B = X^T
+//   dB[(i,k),j]    += sum_(n,a) U[n,a,i,k] X_n[a,j]   A = U2 [(i,k)][(n,a)] (shared), B = x tile
+//                                                     read MN-major
 //   dbias[c*m2+k]  += sum_n G_n[c,k]                  (rank group 0)
 // T and U are recomputed from x and dY (nothing is kept from the forward).  The epilogue
 // warps move them TMEM -> registers -> shared memory into the K-major layouts dC and dB
@@ -21,12 +22,14 @@
 // about the same time and the second and later reads of a tile mostly hit L2.
 //
 // Warp roles (736 threads, one CTA per SM):
-//   warp 0       TMA producer: an SI-deep ring of input sets (x tile, dY tile [, dY MN-major])
+//   warp 0       TMA producer: an SI-deep ring of input sets (x tile, dY tile)
 //   warp 1       issuer A: T and U of tile t (two TMEM slot sets); owns TMEM
 //   warp 2       issuer B: dC and dB of tile t from T2 / U2 (an SB-deep ring in shared memory)
 //   warps 3-18   epilogue: T -> T2 and U -> U2 (per TMEM lane quadrant four warps share the
 //                32-column groups of every block), then the partials
-//   warps 19-22  X^T copy of each x tile (for dB) and the dbias column sums
+//   warps 19-22  the dbias column sums of the dY tiles (rank group 0)
+// BF16 only: a 128-byte-swizzled BF16 tile is a valid operand both K-major and MN-major, so
+// the x and dY tiles serve as they are loaded (T and dB; dC and U) with no copy.
 #include "internal.h"
 #include "tc_gen_common.cuh"
 
@@ -44,7 +47,6 @@ struct GPgCfg {
     static constexpr int P = P_, Q = Q_, M1 = M1_, M2 = M2_, R = R_, RG = RG_, NT = NT_;
     static constexpr int E = GE<T>::bytes;
     static constexpr int KSTEP = 32 / E, VPC = 16 / E;
-    static constexpr bool TWO = GE<T>::tf32;       // TF32: dY in a second, MN-major layout
     static constexpr int NG = cdiv(R, RG);          // rank groups
     static constexpr int IPT = 128 / M2, MBT = cdiv(RG, IPT);   // T blocks: lanes (i,k)
     static constexpr int IPU = 128 / P, MBU = cdiv(RG, IPU);    // U blocks: lanes (i,a)
@@ -62,12 +64,9 @@ struct GPgCfg {
     static constexpr int KCT = cdiv(KT2 * E, 128), KCU = cdiv(KU2 * E, 128);
     static constexpr int X_BYTES = up(KCX * NTN * SWX, 1024);
     static constexpr int G_BYTES = up(GBR * GRB, 1024);
-    static constexpr int GM_BYTES = TWO ? up(GBR * 128, 1024) : 0;
-    static constexpr int XT_BYTES = up(KCU * M1N * 128, 1024);
-    static constexpr int TMA_BYTES = KCX * NTN * SWX + GBR * GRB + (TWO ? GBR * 128 : 0);
-    static constexpr int OFF_XK = 0, OFF_GK = X_BYTES, OFF_GM = OFF_GK + G_BYTES;
-    static constexpr int OFF_XT = OFF_GM + GM_BYTES;
-    static constexpr int IN_BYTES = OFF_XT + XT_BYTES;
+    static constexpr int TMA_BYTES = KCX * NTN * SWX + GBR * GRB;
+    static constexpr int OFF_XK = 0, OFF_GK = X_BYTES;
+    static constexpr int IN_BYTES = OFF_GK + G_BYTES;
     static constexpr int T2_BLK = KCT * 128 * 128, U2_BLK = KCU * 128 * 128;
     static constexpr int IB = MBU * T2_BLK + MBT * U2_BLK;
     static constexpr int BAR_BYTES = 512;
@@ -90,13 +89,16 @@ struct GPgCfg {
     static constexpr uint32_t ID_U = idesc_f32acc(128, NUN, GE<T>::fmt) | kBMajorMN;
     static constexpr uint32_t ID_DC = idesc_f32acc(128, QN, GE<T>::fmt);
     static constexpr uint32_t ID_DB = idesc_f32acc(128, M1N, GE<T>::fmt);
-    static constexpr uint32_t MN_LAYOUT = TWO ? kLayoutSw128Atom32 : layout_type(GRB);
-    static constexpr uint32_t MN_SBO = TWO ? 4 * 128 : 8 * GRB;
+    static constexpr uint32_t MN_LAYOUT = layout_type(GRB);
+    static constexpr uint32_t MN_SBO = 8 * GRB;
+    static constexpr uint32_t XMN_LAYOUT = layout_type(SWX);
+    static constexpr uint32_t ID_DBX = ID_DB | kBMajorMN;
 
     static_assert(128 % M2 == 0 && M2 % 16 == 0, "m2 divides 128, multiple of 16");
     static_assert(P <= 128 && P % VPC == 0, "p at most 128, whole 16-byte groups");
     static_assert(GRB == 64 || GRB == 128, "dY rows of 64 or 128 bytes (TF32: m2 = 32)");
-    static_assert(!TWO || GRB == 128, "TF32 MN-major dY: 128-byte rows");
+    static_assert(!GE<T>::tf32, "generic parameter gradients: BF16 operands");
+    static_assert(XRB <= 128 && NTN >= KU2, "x tile as dB's MN-major operand: one block of j");
     static_assert(Q % 8 == 0, "dY tile rows of each n start on an 8-row atom");
     static_assert(XRB == 32 || XRB == 64 || XRB % 128 == 0, "x row bytes");
     static_assert(M1 % VPC == 0, "X^T copy");
@@ -121,7 +123,7 @@ struct GPgArgs {
 template <class Cfg>
 __global__ void __launch_bounds__(kGPgThreads, 1)
 kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_g,
-                      const __grid_constant__ CUtensorMap tm_gm, GPgArgs args) {
+                      GPgArgs args) {
     using T = typename Cfg::T;
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
     constexpr int NT = Cfg::NT, RG = Cfg::RG, NG = Cfg::NG, SI = Cfg::SI, SB = Cfg::SB;
@@ -134,7 +136,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     const uint32_t sb = smem_u32(smem);
     const uint32_t sIn = sb + Cfg::OFF_IN, sI = sb + Cfg::OFF_I;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-    constexpr int IN_FULL = 0, IN_FREE = SI, XT_FULL = 2 * SI, D_FULL = 3 * SI, D_EMPTY = D_FULL + 2,
+    constexpr int IN_FULL = 0, IN_FREE = SI, D_FULL = 2 * SI, D_EMPTY = D_FULL + 2,
                   I_FULL = D_EMPTY + 2, I_EMPTY = I_FULL + SB, DONE = I_EMPTY + SB,
                   DRAIN = DONE + 1, NBARS = DRAIN + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
@@ -157,7 +159,6 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             tma_load_2d(dst + Cfg::OFF_XK + kc * Cfg::NTN * Cfg::SWX, &tm_x, kc * (Cfg::SWX / E),
                         tile * NT * P, bar(IN_FULL + s));
         tma_load_2d(dst + Cfg::OFF_GK, &tm_g, 0, tile * NT * Q, bar(IN_FULL + s));
-        if (Cfg::TWO) tma_load_2d(dst + Cfg::OFF_GM, &tm_gm, 0, tile * NT * Q, bar(IN_FULL + s));
     };
     const int pre = gmin(SI, nt);
 
@@ -168,8 +169,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < SI; ++s) {
             mbar_init(bar(IN_FULL + s), 1);
-            mbar_init(bar(IN_FREE + s), 1 + 1 + 4);   // issuer A, issuer B, X^T / dbias warps
-            mbar_init(bar(XT_FULL + s), 4);
+            mbar_init(bar(IN_FREE + s), 1 + 1 + 4);   // issuer A, issuer B, dbias warps
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(bar(D_FULL + d), 1);
@@ -185,7 +185,6 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         mbar_init_fence();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_g);
-        if (Cfg::TWO) prefetch_tmap(&tm_gm);
         for (int u = 0; u < pre; ++u) issue(u);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TM_COLS);
@@ -263,8 +262,8 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             if (elect_one()) {
                 const uint32_t in = sIn + s * Cfg::IN_BYTES;
                 const uint64_t xd = sdesc_kmajor(in + Cfg::OFF_XK, Cfg::SWX);
-                const uint64_t gd = sdesc_mn(in + (Cfg::TWO ? Cfg::OFF_GM : Cfg::OFF_GK),
-                                             Cfg::MN_LAYOUT, Q * Cfg::GRB, Cfg::MN_SBO);
+                const uint64_t gd = sdesc_mn(in + Cfg::OFF_GK, Cfg::MN_LAYOUT, Q * Cfg::GRB,
+                                             Cfg::MN_SBO);
                 for (int bt = 0; bt < MBT; ++bt) {
 #pragma unroll
                     for (int kk = 0; kk < M1 * E / 32; ++kk) {   // T, K = j
@@ -280,7 +279,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                     for (int kk = 0; kk < Cfg::QK / KSTEP; ++kk)   // U, K = c, dY MN-major
                         mma_ts<GE<T>::tf32>(tmem + Cfg::TM_DU + (d * MBU + bu) * Cfg::NUS,
                                             tmem + Cfg::TM_CS + bu * Cfg::CSC + kk * 8,
-                                            desc_add(gd, kk * KSTEP * (Cfg::TWO ? 128 : Cfg::GRB)),
+                                            desc_add(gd, kk * KSTEP * Cfg::GRB),
                                             Cfg::ID_U, kk > 0);
                 }
                 mma_commit(bar(D_FULL + d));
@@ -297,15 +296,16 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         for (int u = 0; u < nt; ++u) {
             const int s = u % SI, b = u % SB;
             if (!warp_wait(bar(I_FULL + b), (u / SB) & 1, ab) ||
-                !warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab) ||
-                !warp_wait(bar(XT_FULL + s), (u / SI) & 1, ab))
+                !warp_wait(bar(IN_FULL + s), (u / SI) & 1, ab))
                 break;
             tc_fence_after();
             if (elect_one()) {
                 const uint32_t in = sIn + s * Cfg::IN_BYTES;
                 const uint32_t ib = sI + b * Cfg::IB;
                 const uint64_t gkd = sdesc_kmajor(in + Cfg::OFF_GK, Cfg::GRB);
-                const uint64_t xtd = sdesc_kmajor(in + Cfg::OFF_XT, 128);
+                // the x tile as dB's B operand: N = j along its rows, K = (n,a) down them
+                const uint64_t xmd = sdesc_mn(in + Cfg::OFF_XK, Cfg::XMN_LAYOUT, Cfg::NTN * Cfg::SWX,
+                                              8 * Cfg::SWX);
                 for (int bu = 0; bu < MBU; ++bu) {
                     const uint64_t t2d = sdesc_kmajor(ib + bu * Cfg::T2_BLK, 128);
 #pragma unroll
@@ -321,12 +321,12 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                 for (int bt = 0; bt < MBT; ++bt) {
                     const uint64_t u2d = sdesc_kmajor(ib + MBU * Cfg::T2_BLK + bt * Cfg::U2_BLK, 128);
 #pragma unroll
-                    for (int kk = 0; kk < Cfg::KU2 / KSTEP; ++kk) {   // dB, K = (n,a), B = X^T
+                    for (int kk = 0; kk < Cfg::KU2 / KSTEP; ++kk) {   // dB, K = (n,a), x MN-major
                         const int kb = kk * 32;
                         mma_ss<GE<T>::tf32>(tmem + Cfg::TM_DB + bt * Cfg::M1S,
                                             desc_add(u2d, (kb / 128) * 128 * 128 + kb % 128),
-                                            desc_add(xtd, (kb / 128) * Cfg::M1N * 128 + kb % 128),
-                                            Cfg::ID_DB, (u > 0 || kk > 0) ? 1u : 0u);
+                                            desc_add(xmd, kk * KSTEP * Cfg::SWX), Cfg::ID_DBX,
+                                            (u > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(bar(I_EMPTY + b));
@@ -355,41 +355,40 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             }
             tc_fence_after();
             const uint32_t ib = sI + b * Cfg::IB;
-            for (int task = wi; task < NTASK; task += 4) {
+#pragma unroll
+            for (int task = 0; task < NTASK; ++task) {
+                if ((task & 3) != wi) continue;
                 uint32_t r[32];
-                if (task < MBT * TG) {
-                    // T block bt, lanes (i,k), columns (n,a) -> T2 of U block i/IPU, row (i%IPU, a)
-                    const int bt = task / TG, cg = task % TG;
-                    tmem_load32(tmem + lane_addr + Cfg::TM_DT + (d * MBT + bt) * Cfg::NTS + cg * 32, r);
-                    const int ir = bt * IPT + L / M2, k = L % M2;
-                    if (ir < rgv) {
-                        const uint32_t dst = ib + (ir / IPU) * Cfg::T2_BLK;
-                        const int rbase = (ir % IPU) * P;
+                const bool is_t = task < MBT * TG;
+                const int blk = is_t ? task / TG : (task - MBT * TG) / UG;
+                const int cg = is_t ? task % TG : (task - MBT * TG) % UG;
+                // T lanes (i,k): row (i%IPU, a) of T2 block i/IPU, K (n,k); U lanes (i,a): row
+                // (i%IPT, k) of U2 block i/IPT, K (n,a).  The lane's own index (k or a) fixes
+                // the K byte of each n; the column fixes the row.
+                tmem_load32(tmem + lane_addr + (is_t ? Cfg::TM_DT + (d * MBT + blk) * Cfg::NTS
+                                                     : Cfg::TM_DU + (d * MBU + blk) * Cfg::NUS) + cg * 32, r);
+                const int ir = is_t ? blk * IPT + L / M2 : blk * IPU + L / P;
+                const int own = is_t ? L % M2 : L % P;            // k (T) or a (U)
+                const int CW = is_t ? P : M2;                     // columns per n: a (T), k (U)
+                const int KW = is_t ? M2 : P;                     // K positions per n
+                const bool valid = (is_t || L < IPU * P) && ir < rgv;
+                const uint32_t dst = ib + (is_t ? (ir / IPU) * Cfg::T2_BLK
+                                                : MBU * Cfg::T2_BLK + (ir / IPT) * Cfg::U2_BLK);
+                const int rbase = is_t ? (ir % IPU) * P : (ir % IPT) * M2;   // a multiple of 8
+                // BF16 pairs: lanes 2m, 2m+1 hold adjacent K positions of the same rows; each
+                // lane stores one 4-byte pair per two columns (even lane: row of column w,
+                // odd lane: row of column w+1)
+                const bool odd = lane & 1;
 #pragma unroll
-                        for (int w = 0; w < 32; ++w) {
-                            const int c = cg * 32 + w;
-                            if (c < NT * P) {
-                                const int n = c / P, a = c % P;
-                                st_op<T>(dst + kmaj(rbase + a, (n * M2 + k) * E, 128, 128), r[w]);
-                            }
-                        }
-                    }
-                } else {
-                    // U block bu, lanes (i,a), columns (n,k) -> U2 of T block i/IPT, row (i%IPT, k)
-                    const int tk = task - MBT * TG, bu = tk / UG, cg = tk % UG;
-                    tmem_load32(tmem + lane_addr + Cfg::TM_DU + (d * MBU + bu) * Cfg::NUS + cg * 32, r);
-                    const int ir = bu * IPU + L / P, a = L % P;
-                    if (L < IPU * P && ir < rgv) {
-                        const uint32_t dst = ib + MBU * Cfg::T2_BLK + (ir / IPT) * Cfg::U2_BLK;
-                        const int rbase = (ir % IPT) * M2;
-#pragma unroll
-                        for (int w = 0; w < 32; ++w) {
-                            const int c = cg * 32 + w;
-                            if (c < NT * M2) {
-                                const int n = c / M2, k = c % M2;
-                                st_op<T>(dst + kmaj(rbase + k, (n * P + a) * E, 128, 128), r[w]);
-                            }
-                        }
+                for (int w = 0; w < 32; w += 2) {
+                    const int c = cg * 32 + w + (odd ? 1 : 0);
+                    const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 1], 1);
+                    if (valid && c < NT * CW) {
+                        const int n = c / CW, row = rbase + c % CW;
+                        const int kb = (n * KW + own - (odd ? 1 : 0)) * E;
+                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 1] : got;
+                        st_shared_u32(dst + kmaj(row, kb, 128, 128),
+                                      pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi)));
                     }
                 }
             }
@@ -429,7 +428,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             }
         }
     } else {
-        // ---------------- X^T copies and dbias column sums ----------------
+        // ---------------- dbias column sums of the dY tiles ----------------
         const int tid = threadIdx.x - 608;
         constexpr int PER = Q * M2 / 128;
         float acc[PER];
@@ -439,32 +438,6 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             const int s = u % SI;
             if (!mbar_wait(bar(IN_FULL + s), (u / SI) & 1, ab)) break;
             const uint32_t in = sIn + s * Cfg::IN_BYTES;
-            // X^T [j][(n,a)] for dB (K-major): VPC consecutive rows (n,a) of column j of the
-            // x tile become one 16-byte chunk of row j
-            for (int it = tid; it < M1 * (NT * P / VPC); it += 128) {
-                const int j = it % M1, kap0 = (it / M1) * VPC;
-                uint32_t w[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    if constexpr (GE<T>::tf32) {
-                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w[h])
-                                     : "r"(in + Cfg::OFF_XK + kmaj(kap0 + h, j * E, Cfg::NTN, Cfg::SWX))
-                                     : "memory");
-                    } else {
-                        unsigned short lo, hi;
-                        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(lo)
-                                     : "r"(in + Cfg::OFF_XK + kmaj(kap0 + 2 * h, j * E, Cfg::NTN, Cfg::SWX))
-                                     : "memory");
-                        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(hi)
-                                     : "r"(in + Cfg::OFF_XK + kmaj(kap0 + 2 * h + 1, j * E, Cfg::NTN, Cfg::SWX))
-                                     : "memory");
-                        w[h] = (uint32_t)lo | ((uint32_t)hi << 16);
-                    }
-                }
-                st_shared_v4(in + Cfg::OFF_XT + kmaj(j, kap0 * E, Cfg::M1N, 128), w[0], w[1], w[2], w[3]);
-            }
-            fence_proxy_async();
-            mbar_arrive_warp(bar(XT_FULL + s));
             if (grp == 0) {
 #pragma unroll
                 for (int e = 0; e < PER; ++e) {
@@ -507,7 +480,7 @@ cudaError_t launch_gpgrad(const void *x, const void *S, const void *A, const voi
                           const void *dY, float *ws, int parts, const Shape &s, cudaStream_t st) {
     using T = typename Cfg::T;
     const bool bf16 = !GE<T>::tf32;
-    CUtensorMap tx, tg, tgm;
+    CUtensorMap tx, tg;
     launch_step() = "tensor map of x";
     cudaError_t e = make_tmap_2d(&tx, x, bf16, (uint64_t)s.N * Cfg::P, Cfg::M1, Cfg::SWX / Cfg::E,
                                  Cfg::NTN, Cfg::SWX, false);
@@ -516,13 +489,6 @@ cudaError_t launch_gpgrad(const void *x, const void *S, const void *A, const voi
     e = make_tmap_2d(&tg, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GBR, Cfg::GRB,
                      false);
     if (e != cudaSuccess) return e;
-    tgm = tg;
-    if (Cfg::TWO) {
-        launch_step() = "MN-major tensor map of dY";
-        e = make_tmap_2d(&tgm, dY, bf16, (uint64_t)s.N * Cfg::Q, Cfg::M2, Cfg::M2, Cfg::GBR, 128,
-                         true);
-        if (e != cudaSuccess) return e;
-    }
     launch_step() = "shared-memory attribute";
     e = cudaFuncSetAttribute(kron_pgrad_gen_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM);
@@ -539,7 +505,7 @@ cudaError_t launch_gpgrad(const void *x, const void *S, const void *A, const voi
     cfg.blockDim = dim3(kGPgThreads);
     cfg.dynamicSmemBytes = Cfg::SMEM;
     cfg.stream = st;
-    return cudaLaunchKernelEx(&cfg, kron_pgrad_gen_kernel<Cfg>, tx, tg, tgm, a);
+    return cudaLaunchKernelEx(&cfg, kron_pgrad_gen_kernel<Cfg>, tx, tg, a);
 }
 
 using GPgFn = cudaError_t (*)(const void *, const void *, const void *, const void *,
