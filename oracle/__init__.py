@@ -8,7 +8,9 @@ The arithmetic lives in ``kron_oracle.c`` (plain C, double precision): it builds
 W = sum_i kron(S (.) A_i, B_i) entry by entry and multiplies naively, as the
 page "kronecker-layer-benchmark", section "1. Build W, then multiply" defines
 the layer; the backward is the chain rule through that explicit W.  This module
-only marshals numpy arrays into that library.
+only marshals numpy arrays into that library, except for the Van Loan fit,
+whose SVD step is numpy's (a library routine serving as one step of the
+algorithm as the page gives it).
 """
 from __future__ import annotations
 
@@ -65,6 +67,7 @@ class Oracle:
         lib.oracle_backward.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I,
                                         dp, dp, dp, dp, dp]
         lib.oracle_l1_grad.argtypes = [dp, I, I, ctypes.c_double, dp]
+        lib.oracle_vanloan_rearrange.argtypes = [dp, I, I, I, I, dp]
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_get_threads.restype = I
         self._lib = lib
@@ -126,6 +129,40 @@ class Oracle:
         return out
 
 
+    def vanloan_rearrange(self, W, p, q, m1, m2) -> np.ndarray:
+        """Wt[(a, c)][(j, k)] = W[a*m1 + j][c*m2 + k], shape (p*q, m1*m2)."""
+        W = _f64(W)
+        if W.shape != (p * m1, q * m2):
+            raise ValueError(f"W has shape {W.shape}, expected ({p * m1}, {q * m2})")
+        Wt = np.empty((p * q, m1 * m2), dtype=np.float64)
+        self._lib.oracle_vanloan_rearrange(_ptr(W), p, q, m1, m2, _ptr(Wt))
+        return Wt
+
+    def vanloan_fit(self, W, p, q, m1, m2, r, normalize: bool = True) -> dict:
+        """Rank-r Kronecker fit of a dense W, in the steps of the page "LLM Compression via
+        Kronecker Product Decomposition" (sections "Van Loan Rearrangement (1993)" and
+        "Adaptive Normalization"):
+
+          1. Wt = R(W), the rearrangement above;
+          2. Wt = U diag(s) V^T (numpy's SVD: the library routine is this step);
+          3. C_i = sqrt(s_i) reshape(u_i, p, q),  B_i = sqrt(s_i) reshape(v_i, m1, m2), i < r;
+          4. alpha = ||W||_F / ||sum_i kron(C_i, B_i)||_F, and with normalize each factor is
+             scaled by sqrt(alpha) (so the fit carries the energy of W).
+
+        Returns dict(A = C stacked [r][p][q], B [r][m1][m2], sigma = s (all of them), alpha).
+        With S = ones, (S, A, B) are factors of this layer.  The sum of r terms is unique
+        when s_{r-1} > s_r; each pair (C_i, B_i) is fixed up to a common sign."""
+        Wt = self.vanloan_rearrange(W, p, q, m1, m2)
+        U, s, Vt = np.linalg.svd(Wt, full_matrices=False)
+        C = np.stack([np.sqrt(s[i]) * U[:, i].reshape(p, q) for i in range(r)])
+        B = np.stack([np.sqrt(s[i]) * Vt[i].reshape(m1, m2) for i in range(r)])
+        Wr = self.weight(np.ones((p, q)), C, B)
+        alpha = float(np.sqrt(np.sum(_f64(W) ** 2)) / np.sqrt(np.sum(Wr ** 2)))
+        if normalize:
+            C, B = C * np.sqrt(alpha), B * np.sqrt(alpha)
+        return {"A": C, "B": B, "sigma": s, "alpha": alpha}
+
+
 _default = None
 
 
@@ -158,3 +195,11 @@ def backward(x, S, A, B, G, need_dx: bool = True, need_params: bool = True) -> d
 
 def l1_grad(S, lam: float) -> np.ndarray:
     return default().l1_grad(S, lam)
+
+
+def vanloan_rearrange(W, p, q, m1, m2) -> np.ndarray:
+    return default().vanloan_rearrange(W, p, q, m1, m2)
+
+
+def vanloan_fit(W, p, q, m1, m2, r, normalize: bool = True) -> dict:
+    return default().vanloan_fit(W, p, q, m1, m2, r, normalize)

@@ -210,3 +210,22 @@ void oracle_l1_grad(const double *S, int p, int q, double lam, double *out)
         out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);
     }
 }
+
+/*
+ * Van Loan rearrangement (page "LLM Compression via Kronecker Product Decomposition",
+ * section "Van Loan Rearrangement (1993)"): the (p*m1) x (q*m2) matrix W becomes the
+ * (p*q) x (m1*m2) matrix Wt whose row (a, c) is block (a, c) of W read row by row:
+ *
+ *     Wt[a*q + c][j*m2 + k] = W[a*m1 + j][c*m2 + k]
+ *
+ * so that W = sum_i kron(C_i, B_i) exactly when Wt = sum_i vec(C_i) vec(B_i)^T.
+ */
+void oracle_vanloan_rearrange(const double *W, int p, int q, int m1, int m2, double *Wt)
+{
+    for (int a = 0; a < p; ++a)
+        for (int c = 0; c < q; ++c)
+            for (int j = 0; j < m1; ++j)
+                for (int k = 0; k < m2; ++k)
+                    Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =
+                        W[((size_t)a * m1 + j) * ((size_t)q * m2) + (size_t)c * m2 + k];
+}

@@ -275,6 +275,91 @@ def pin_l1_grad_finite_differences(orc):
     assert np.array_equal(orc.l1_grad(S, 0.0), np.zeros_like(S))
 
 
+# ---------------------------------------------------------------- Van Loan rank-r fit
+# (page "LLM Compression via Kronecker Product Decomposition", sections "Van Loan
+# Rearrangement (1993)" and "Adaptive Normalization")
+
+def pin_vanloan_rearrangement_of_krons(orc):
+    """R(sum_i kron(C_i, B_i)) = sum_i vec(C_i) vec(B_i)^T, with W built by numpy's kron and
+    the outer products by numpy (the identity the fit rests on), for rectangular blocks; and
+    R is the page's block permutation (numpy reshape / transpose route)."""
+    rng = np.random.default_rng(211)
+    for (p, q, m1, m2, r) in [(3, 4, 2, 5, 2), (2, 5, 4, 3, 3), (1, 3, 3, 1, 1)]:
+        C = rng.standard_normal((r, p, q))
+        B = rng.standard_normal((r, m1, m2))
+        W = sum(np.kron(C[i], B[i]) for i in range(r))
+        Wt = orc.vanloan_rearrange(W, p, q, m1, m2)
+        outer = sum(np.outer(C[i].ravel(), B[i].ravel()) for i in range(r))
+        assert np.allclose(Wt, outer, rtol=0, atol=1e-12), (p, q, m1, m2)
+        perm = W.reshape(p, m1, q, m2).transpose(0, 2, 1, 3).reshape(p * q, m1 * m2)
+        assert np.array_equal(Wt, perm)
+
+
+def pin_vanloan_fit_recovers_exact_rank(orc):
+    """W of Kronecker rank r: the rank-r fit reproduces W (to rounding), alpha = 1 and the
+    singular values past r vanish; the fit of a smaller rank does not reproduce it."""
+    rng = np.random.default_rng(223)
+    p, q, m1, m2, r = 4, 3, 5, 2, 3
+    C = rng.standard_normal((r, p, q))
+    B = rng.standard_normal((r, m1, m2))
+    W = sum(np.kron(C[i], B[i]) for i in range(r))
+    f = orc.vanloan_fit(W, p, q, m1, m2, r)
+    Wr = sum(np.kron(f["A"][i], f["B"][i]) for i in range(r))
+    assert np.abs(Wr - W).max() <= 1e-12 * np.abs(W).max()
+    assert abs(f["alpha"] - 1.0) <= 1e-12
+    assert np.all(f["sigma"][r:] <= 1e-12 * f["sigma"][0]) and f["sigma"][r - 1] > 1e-6
+    f1 = orc.vanloan_fit(W, p, q, m1, m2, r - 1, normalize=False)
+    W1 = sum(np.kron(f1["A"][i], f1["B"][i]) for i in range(r - 1))
+    assert np.abs(W1 - W).max() > 1e-3 * np.abs(W).max()
+
+
+def pin_vanloan_rank_one_closed_form(orc):
+    """W = kron(A, B): R(W) = vec(A) vec(B)^T has the single singular value |A|_F |B|_F, and
+    the rank-1 fit gives back kron(A, B) exactly."""
+    rng = np.random.default_rng(227)
+    A = rng.standard_normal((3, 6))
+    B = rng.standard_normal((4, 2))
+    W = np.kron(A, B)
+    f = orc.vanloan_fit(W, 3, 6, 4, 2, 1)
+    assert abs(f["sigma"][0] - np.linalg.norm(A) * np.linalg.norm(B)) <= 1e-12 * f["sigma"][0]
+    assert np.allclose(np.kron(f["A"][0], f["B"][0]), W, rtol=0, atol=1e-12)
+
+
+def pin_vanloan_best_approximation(orc):
+    """Eckart-Young on R(W): the squared Frobenius error of the rank-r fit of a random W is
+    the sum of the discarded squared singular values, and nudging the fitted factors in
+    random directions never lowers the error (the fit is the best Kronecker sum of r
+    terms)."""
+    rng = np.random.default_rng(229)
+    p, q, m1, m2, r = 3, 4, 4, 3, 2
+    W = rng.standard_normal((p * m1, q * m2))
+    f = orc.vanloan_fit(W, p, q, m1, m2, r, normalize=False)
+    Wr = sum(np.kron(f["A"][i], f["B"][i]) for i in range(r))
+    err2 = np.sum((W - Wr) ** 2)
+    assert abs(err2 - np.sum(f["sigma"][r:] ** 2)) <= 1e-10 * np.sum(W ** 2)
+    for t in range(20):
+        dA = 1e-3 * rng.standard_normal(f["A"].shape)
+        dB = 1e-3 * rng.standard_normal(f["B"].shape)
+        Wp = sum(np.kron(f["A"][i] + dA[i], f["B"][i] + dB[i]) for i in range(r))
+        assert np.sum((W - Wp) ** 2) >= err2 - 1e-12
+
+
+def pin_vanloan_alpha_restores_energy(orc):
+    """alpha = |W|_F / |sum_i kron(C_i, B_i)|_F; after scaling both factors by sqrt(alpha) the
+    fit has the Frobenius norm of W."""
+    rng = np.random.default_rng(233)
+    p, q, m1, m2 = 3, 3, 4, 4
+    W = rng.standard_normal((p * m1, q * m2))
+    for r in (1, 2):
+        f0 = orc.vanloan_fit(W, p, q, m1, m2, r, normalize=False)
+        f1 = orc.vanloan_fit(W, p, q, m1, m2, r, normalize=True)
+        W0 = sum(np.kron(f0["A"][i], f0["B"][i]) for i in range(r))
+        W1 = sum(np.kron(f1["A"][i], f1["B"][i]) for i in range(r))
+        assert abs(f1["alpha"] - np.linalg.norm(W) / np.linalg.norm(W0)) <= 1e-12 * f1["alpha"]
+        assert abs(np.linalg.norm(W1) - np.linalg.norm(W)) <= 1e-12 * np.linalg.norm(W)
+        assert f1["alpha"] > 1.0
+
+
 ALL_PINS = [
     pin_weight_is_sum_of_numpy_krons,
     pin_forward_brute_force,
@@ -285,6 +370,11 @@ ALL_PINS = [
     pin_block_structure,
     pin_rank_one,
     pin_van_loan_rank,
+    pin_vanloan_rearrangement_of_krons,
+    pin_vanloan_fit_recovers_exact_rank,
+    pin_vanloan_rank_one_closed_form,
+    pin_vanloan_best_approximation,
+    pin_vanloan_alpha_restores_energy,
     pin_special_shapes,
     pin_finite_differences,
     pin_linearity_identities,

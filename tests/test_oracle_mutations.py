@@ -43,6 +43,15 @@ MUTATIONS = [
      "out[ac] = v >= 0.0 ? lam : -lam;", 0),
     ("l1_grad_drops_weight", "out[ac] = v > 0.0 ? lam : (v < 0.0 ? -lam : 0.0);",
      "out[ac] = v > 0.0 ? 1.0 : (v < 0.0 ? -1.0 : 0.0);", 0),
+    ("vanloan_rows_transposed",
+     "Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =",
+     "Wt[((size_t)c * p + a) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =", 0),
+    ("vanloan_block_read_transposed",
+     "W[((size_t)a * m1 + j) * ((size_t)q * m2) + (size_t)c * m2 + k];",
+     "W[((size_t)a * m1 + j) * ((size_t)q * m2) + (size_t)k * q + c];", 0),
+    ("vanloan_inner_index_swapped",
+     "Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =",
+     "Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)k * m1 + j] =", 0),
 ]
 
 
