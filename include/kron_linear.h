@@ -183,6 +183,41 @@ KRON_API kron_status_t kron_linear_backward_noalloc(const void *x, const void *S
                                                     kron_dtype_t dtype, unsigned flags,
                                                     void *stream);
 
+/*
+ * Rank-r Kronecker fit of a dense matrix, to initialise the layer's factors from a dense
+ * layer (page "LLM Compression via Kronecker Product Decomposition", sections "Van Loan
+ * Rearrangement (1993)", "Rank-K" and "Adaptive Normalization"):
+ *
+ *   Wt[a*q + c][j*m2 + k] = W[a*m1 + j][c*m2 + k]            ((p*q) x (m1*m2))
+ *   Wt ~ sum_{i<r} sigma_i u_i v_i^T                           (r leading singular pairs)
+ *   A_i = sqrt(sigma_i) reshape(u_i, p, q),  B_i = sqrt(sigma_i) reshape(v_i, m1, m2)
+ *   alpha = |W|_F / |sum_i kron(A_i, B_i)|_F; with normalize != 0, A_i and B_i are both
+ *   scaled by sqrt(alpha) (the fit then has the Frobenius norm of W).
+ *
+ * With S = ones, (S, A, B) are factors of this layer: sum_i kron(S (.) A_i, B_i) is the
+ * best Kronecker sum of r terms to W in the Frobenius norm (times alpha when normalized).
+ * The singular pairs come from randomized subspace iteration (Halko, Martinsson and Tropp,
+ * 2011): Q = orth(Wt Omega), then power_iters times Q = orth(Wt orth(Wt^T Q)), and the
+ * eigenpairs of (Q^T Wt)(Q^T Wt)^T.  The fit is exact (to rounding) when W has Kronecker
+ * rank <= k; otherwise more power iterations and a larger k bring it closer to the exact
+ * truncated SVD.  Sums run in double in a fixed order: results are bitwise reproducible.
+ *   W       [p*m1][q*m2] float32, device
+ *   omega   [k][m1*m2]  float32, device: the random test matrix (e.g. standard normal),
+ *           drawn by the caller; 1 <= r <= k <= 64, k <= p*q, k <= m1*m2
+ *   power_iters  0..16
+ *   A [r][p][q], B [r][m1][m2], sigma [k] (estimated singular values of Wt, largest
+ *   first), alpha [1]: float32 outputs, device, overwritten
+ *   workspace of kron_vanloan_workspace_size(p, q, m1, m2, k) bytes, 256-byte aligned
+ * Every pointer is 16-byte aligned (KRON_ERR_ALIGNMENT).  Bad sizes or pointers return
+ * KRON_ERR_INVALID_ARG before anything is launched; all work is enqueued on `stream`.
+ */
+KRON_API size_t kron_vanloan_workspace_size(int p, int q, int m1, int m2, int k);
+KRON_API kron_status_t kron_vanloan_fit(const void *W, int p, int q, int m1, int m2, int r,
+                                        const void *omega, int k, int power_iters,
+                                        int normalize, void *A, void *B, void *sigma,
+                                        void *alpha, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
 /* Bytes of device workspace kron_linear_backward needs for this problem (0 if the
  * arguments are invalid).  Depends only on the arguments, not on the device. */
 KRON_API size_t kron_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int r,

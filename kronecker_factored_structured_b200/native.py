@@ -30,7 +30,7 @@ STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
 # Every symbol include/kron_linear.h declares.
 EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_l1",
            "kron_linear_backward_noalloc",
-           "kron_linear_workspace_size",
+           "kron_linear_workspace_size", "kron_vanloan_fit", "kron_vanloan_workspace_size",
            "kron_status_string", "kron_last_error", "kron_linear_device_error",
            "kron_linear_abi_version")
 
@@ -67,6 +67,10 @@ def load(path: str = LIB_PATH):
     lib.kron_linear_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                  i64, I, I, I, I, I, I, U, vp]
     lib.kron_linear_backward_noalloc.restype = I
+    lib.kron_vanloan_workspace_size.argtypes = [I, I, I, I, I]
+    lib.kron_vanloan_workspace_size.restype = sz
+    lib.kron_vanloan_fit.argtypes = [vp, I, I, I, I, I, vp, I, I, I, vp, vp, vp, vp, vp, sz, vp]
+    lib.kron_vanloan_fit.restype = I
     lib.kron_linear_workspace_size.argtypes = [i64, I, I, I, I, I, I]
     lib.kron_linear_workspace_size.restype = sz
     lib.kron_status_string.argtypes = [I]
@@ -189,3 +193,32 @@ def backward(x, S, A, B, dY, dtype="tf32", flags=0, need_dx=True, need_dbias=Tru
     else:
         _check(load().kron_linear_backward(*ptrs, *tail))
     return g
+
+
+def vanloan_fit(W, p, q, m1, m2, r, k=None, power_iters=2, normalize=True, omega=None,
+                seed=0, stream=None):
+    """Rank-r Kronecker fit of a dense float32 CUDA matrix W ((p*m1) x (q*m2)) by the
+    library's kron_vanloan_fit; returns dict(S = ones, A [r][p][q], B [r][m1][m2],
+    sigma [k], alpha).  ``omega`` ([k][m1*m2] float32) is the random test matrix; by default
+    it is drawn here with torch (seeded), k = r + 8 capped by the sizes."""
+    if k is None:
+        k = min(r + 8, 64, p * q, m1 * m2)
+    _expect(W, "W", torch.float32, (p * m1, q * m2))
+    dev = W.device
+    if omega is None:
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        omega = torch.randn(k, m1 * m2, device=dev, generator=g)
+    _expect(omega, "omega", torch.float32, (k, m1 * m2))
+    A = torch.empty(r, p, q, device=dev)
+    B = torch.empty(r, m1, m2, device=dev)
+    sigma = torch.empty(k, device=dev)
+    alpha = torch.empty(4, device=dev)
+    lib = load()
+    wsb = int(lib.kron_vanloan_workspace_size(p, q, m1, m2, k))
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    _check(lib.kron_vanloan_fit(_ptr(W), p, q, m1, m2, r, _ptr(omega), k, power_iters,
+                                1 if normalize else 0, _ptr(A), _ptr(B), _ptr(sigma), _ptr(alpha),
+                                _ptr(ws), ws.numel(), _stream(stream)))
+    return {"S": torch.ones(p, q, device=dev), "A": A, "B": B, "sigma": sigma,
+            "alpha": alpha[:1]}

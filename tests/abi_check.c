@@ -118,6 +118,16 @@ int main(void) {
     /* the same shapes run on the exact-FP32 path */
     CHECK(kron_linear_workspace_size(8, 64, 64, 16, 16, 2, KRON_F32) > 0);
 
+    /* Van Loan fit: sizes, rank and pointers are checked on the host */
+    CHECK(kron_vanloan_workspace_size(32, 32, 32, 32, 12) > 0);
+    CHECK(kron_vanloan_workspace_size(32, 32, 32, 32, 65) == 0);
+    CHECK(kron_vanloan_fit(P, 4, 4, 4, 4, 9, P, 8, 2, 1, P, P, P, P, WS, 1u << 24, NULL) ==
+          KRON_ERR_INVALID_ARG);                                        /* r > k */
+    CHECK(kron_vanloan_fit(MIS, 4, 4, 4, 4, 2, P, 8, 2, 1, P, P, P, P, WS, 1u << 24, NULL) ==
+          KRON_ERR_ALIGNMENT);
+    CHECK(kron_vanloan_fit(P, 4, 4, 4, 4, 2, P, 8, 2, 1, P, P, P, P, NULL, 0, NULL) ==
+          KRON_ERR_WORKSPACE);
+
     if (failures) return 1;
     printf("abi_check: all checks passed\n");
     return 0;

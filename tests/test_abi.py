@@ -122,6 +122,33 @@ def test_tensor_core_paths_refuse_shapes_without_a_kernel(shape):
     assert lib.kron_linear_workspace_size(8, p, q, m1, m2, r, 0) > 0
 
 
+@pytest.mark.parametrize("args,status", [
+    (dict(k=0), 1), (dict(k=65), 1), (dict(r=0), 1), (dict(r=9, k=8), 1),
+    (dict(power_iters=17), 1), (dict(W=None), 1), (dict(omega=None), 1),
+    (dict(p=2, q=2, k=8), 1),              # k > p*q
+    (dict(W=MISALIGNED), 3), (dict(ws=None), 4), (dict(ws_bytes=64), 4),
+    (dict(ws=V(0x100010)), 3),
+])
+def test_vanloan_fit_rejects(args, status):
+    """kron_vanloan_fit's host checks, before anything is launched."""
+    lib = native.load()
+    a = dict(W=ALIGNED, p=4, q=4, m1=4, m2=4, r=2, omega=ALIGNED, k=8, power_iters=2,
+             normalize=1, ws=V(0x100000), ws_bytes=1 << 24)
+    a.update(args)
+    st = lib.kron_vanloan_fit(a["W"], a["p"], a["q"], a["m1"], a["m2"], a["r"], a["omega"],
+                              a["k"], a["power_iters"], a["normalize"], ALIGNED, ALIGNED, ALIGNED,
+                              ALIGNED, a["ws"], a["ws_bytes"], None)
+    assert st == status, lib.kron_last_error().decode()
+    assert lib.kron_last_error().decode() != ""
+
+
+def test_vanloan_workspace_size():
+    lib = native.load()
+    assert lib.kron_vanloan_workspace_size(32, 32, 32, 32, 12) >= 4 * 1024 * 1024
+    assert lib.kron_vanloan_workspace_size(32, 32, 32, 32, 0) == 0
+    assert lib.kron_vanloan_workspace_size(2, 2, 32, 32, 8) == 0     # k > p*q
+
+
 def test_noalloc_checks_arguments_before_the_size_limit():
     """An oversized problem with a missing or misaligned pointer gets the pointer's status,
     not KRON_ERR_WORKSPACE: the argument checks come first."""
