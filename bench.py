@@ -404,7 +404,7 @@ def _split_calls(step, steps, stream):
             statistics.mean(b.elapsed_time(c) for _, b, c in marks))
 
 
-def _make_step(kfs, pr, flags, stream, grads, world=1, dp=None, flat=None):
+def _make_step(kfs, pr, flags, stream, grads, world=1, dp=None, flat=None, det=False):
     def step(i, timing=None):
         x, G = pr.sets[i % len(pr.sets)]
         if timing is not None:
@@ -418,7 +418,7 @@ def _make_step(kfs, pr, flags, stream, grads, world=1, dp=None, flat=None):
         if timing is not None:
             timing[2].record(stream)
         if world > 1:
-            dp.allreduce_grads(flat)
+            dp.allreduce_grads(flat, deterministic=det)
     return step
 
 
@@ -497,6 +497,9 @@ def main():
     ap.add_argument("--leg-steps", type=int, default=20)
     ap.add_argument("--skip-zero-blocks", action="store_true",
                     help="pass KRON_FLAG_SKIP_ZERO_BLOCKS (drop products with a zero S entry)")
+    ap.add_argument("--deterministic-exchange", action="store_true",
+                    help="N > 1: sum the ranks' gradients in rank order after an all-gather "
+                         "(bitwise reproducible) instead of one all-reduce")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -539,7 +542,7 @@ def main():
     flat, views = dp.flat_grad_buffer(p, q, m1, m2, r, device=dev)
     grads.update(views)
     stream = torch.cuda.current_stream()
-    step = _make_step(kfs, pr, flags, stream, grads, world, dp, flat)
+    step = _make_step(kfs, pr, flags, stream, grads, world, dp, flat, args.deterministic_exchange)
     fac, sets, wsb = pr.fac, pr.sets, pr.wsb
 
     for i in range(args.warmup):
@@ -578,7 +581,7 @@ def main():
         kfs.backward(xd, fac["S"], fac["A"], fac["B"], gd, dtype=path, flags=flags, workspace=wsb,
                      grads=grads)
         if world > 1:
-            dp.allreduce_grads(flat)
+            dp.allreduce_grads(flat, deterministic=args.deterministic_exchange)
         yh.copy_(pr.y, non_blocking=True)
         dxh.copy_(grads["dX"], non_blocking=True)
         fh.copy_(flat, non_blocking=True)
@@ -632,6 +635,8 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": path, "data": "synthetic",
         "config": {"workload": _workload_desc(w), "N": N, "p": p, "q": q, "m1": m1, "m2": m2,
                    "r": r, "path": path, "parallelism": f"dp{world}",
+                   "exchange": ("all-gather, rank-ordered sum" if args.deterministic_exchange
+                                else "all-reduce") if world > 1 else None,
                    "skip_zero_blocks": bool(flags),
                    "l2": f"inputs rotated over {len(sets)} independent (x, dY) sets "
                          f"({len(sets) * N * elt * (p * m1 + q * m2) / 1e6:.0f} MB > 126 MB L2)"},

@@ -45,9 +45,34 @@ def flat_grad_buffer(p: int, q: int, m1: int, m2: int, r: int,
     return flat, views
 
 
-def allreduce_grads(flat: torch.Tensor, group=None) -> torch.Tensor:
-    """Sum the flat parameter-gradient buffer over the ranks of `group` (in place)."""
+def allreduce_grads(flat: torch.Tensor, group=None, deterministic: bool = False,
+                    gathered: torch.Tensor = None) -> torch.Tensor:
+    """Sum the flat parameter-gradient buffer over the ranks of `group` (in place).
+
+    Default: one NCCL (or gloo) all-reduce.  Its summation order is the library's choice
+    (ring or tree, and on NVSwitch possibly in the switch), so the sum over ranks is not
+    bitwise reproducible across world sizes or runs.
+
+    deterministic=True: every rank all-gathers the ranks' buffers and adds them in rank
+    order, rank 0 first, so every rank gets bitwise the same sum in every run with the same
+    world size (the per-rank gradients are themselves bitwise reproducible).  It moves
+    world-1 buffers to each rank instead of about two: for the tutorial layer's 40 KB of
+    gradients that is latency, not bandwidth.  `gathered` may hold a preallocated buffer of
+    world * numel elements."""
     import torch.distributed as dist
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+    if not (dist.is_available() and dist.is_initialized()):
+        return flat
+    world = dist.get_world_size(group)
+    if world <= 1:
+        return flat
+    if not deterministic:
         dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+        return flat
+    n = flat.numel()
+    if gathered is None:
+        gathered = torch.empty(world * n, dtype=flat.dtype, device=flat.device)
+    dist.all_gather_into_tensor(gathered, flat.contiguous(), group=group)
+    flat.copy_(gathered[:n])
+    for r in range(1, world):
+        flat.add_(gathered[r * n:(r + 1) * n])
     return flat

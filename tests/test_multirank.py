@@ -26,7 +26,7 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, result_q):
+def _rank_main(rank, world, port, result_q, deterministic=False):
     sys.path.insert(0, ROOT)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -47,7 +47,7 @@ def _rank_main(rank, world, port, result_q):
         flat, views = dp.flat_grad_buffer(w.p, w.q, w.m1, w.m2, w.r)
         for k in ("dS", "dA", "dB", "dbias"):
             views[k].copy_(torch.from_numpy(g[k]).float())
-        dp.allreduce_grads(flat)
+        dp.allreduce_grads(flat, deterministic=deterministic)
         result_q.put((rank, start, count, {k: v.double().numpy().copy() for k, v in views.items()},
                       g["dX"]))
     finally:
@@ -77,6 +77,47 @@ def test_flat_buffer_views_cover_it_once():
         v.fill_(i + 1)
     assert torch.all(flat > 0)  # every element belongs to one view
     assert sorted(set(flat.tolist())) == [1.0, 2.0, 3.0, 4.0]
+
+
+def _run_ranks(world, deterministic):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, deterministic))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    out.sort(key=lambda t: t[0])
+    return out
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_deterministic_exchange_is_the_rank_ordered_sum(world):
+    """deterministic=True: every rank holds bitwise the same sum, equal to adding the ranks'
+    fp32 buffers in rank order on the host, and close to the full-batch gradients."""
+    import kron_workloads as kw
+    import oracle
+    from kronecker_factored_structured_b200 import dp
+    out = _run_ranks(world, True)
+    w = kw.get("tiny")
+    d = {k: v.double().numpy() for k, v in kw.inputs(w).items()}
+    parts = []
+    for rank in range(world):
+        start, count = dp.shard_rows(w.N, world, rank)
+        sl = slice(start, start + count)
+        parts.append(oracle.backward(d["x"][sl], d["S"], d["A"], d["B"], d["G"][sl]))
+    full = oracle.backward(d["x"], d["S"], d["A"], d["B"], d["G"])
+    for k in ("dS", "dA", "dB", "dbias"):
+        want = parts[0][k].astype(np.float32)
+        for r in range(1, world):
+            want = want + parts[r][k].astype(np.float32)
+        for rank, _, _, grads, _ in out:
+            assert np.array_equal(grads[k].astype(np.float32), want), (rank, k)
+        assert np.abs(out[0][3][k] - full[k]).max() <= 1e-6 * np.abs(full[k]).max(), k
 
 
 def test_two_gloo_ranks_sum_to_full_batch_gradients():
