@@ -68,6 +68,10 @@ class Oracle:
                                         dp, dp, dp, dp, dp]
         lib.oracle_l1_grad.argtypes = [dp, I, I, ctypes.c_double, dp]
         lib.oracle_vanloan_rearrange.argtypes = [dp, I, I, I, I, dp]
+        lib.oracle_build_weight3.argtypes = [dp, dp, dp, I, I, I, I, I, I, I, dp]
+        lib.oracle_forward3.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, I, I, dp]
+        lib.oracle_backward3.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, I, I,
+                                         dp, dp, dp, dp, dp]
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_get_threads.restype = I
         self._lib = lib
@@ -163,6 +167,48 @@ class Oracle:
         return {"A": C, "B": B, "sigma": s, "alpha": alpha}
 
 
+    # ---- triple Kronecker layer: W = sum_i kron(A_i, kron(B_i, C_i)) ----
+    @staticmethod
+    def _shapes3(A, B, C):
+        r, p, q = A.shape
+        r2, m1, m2 = B.shape
+        r3, s1, s2 = C.shape
+        if r2 != r or r3 != r:
+            raise ValueError("A, B, C must hold the same number of terms")
+        return p, q, m1, m2, s1, s2, r
+
+    def weight3(self, A, B, C) -> np.ndarray:
+        """Dense W = sum_i kron(A_i, kron(B_i, C_i)), shape (p*m1*s1, q*m2*s2)."""
+        A, B, C = _f64(A), _f64(B), _f64(C)
+        p, q, m1, m2, s1, s2, r = self._shapes3(A, B, C)
+        W = np.empty((p * m1 * s1, q * m2 * s2))
+        self._lib.oracle_build_weight3(_ptr(A), _ptr(B), _ptr(C), p, q, m1, m2, s1, s2, r, _ptr(W))
+        return W
+
+    def forward3(self, x, A, B, C, bias=None) -> np.ndarray:
+        x, A, B, C = _f64(x), _f64(A), _f64(B), _f64(C)
+        p, q, m1, m2, s1, s2, r = self._shapes3(A, B, C)
+        N = x.shape[0]
+        if x.shape != (N, p * m1 * s1):
+            raise ValueError(f"x has shape {x.shape}, expected (N, {p * m1 * s1})")
+        bias = None if bias is None else _f64(bias)
+        y = np.empty((N, q * m2 * s2))
+        self._lib.oracle_forward3(_ptr(x), _ptr(A), _ptr(B), _ptr(C), _ptr(bias), N, p, q, m1, m2,
+                                  s1, s2, r, _ptr(y))
+        return y
+
+    def backward3(self, x, A, B, C, G) -> dict:
+        """Gradients of <G, y> for the triple layer: dict(dX, dA, dB, dC, dbias)."""
+        x, A, B, C, G = _f64(x), _f64(A), _f64(B), _f64(C), _f64(G)
+        p, q, m1, m2, s1, s2, r = self._shapes3(A, B, C)
+        N = x.shape[0]
+        dX, dA, dB, dC = np.empty_like(x), np.empty_like(A), np.empty_like(B), np.empty_like(C)
+        dbias = np.empty(q * m2 * s2)
+        self._lib.oracle_backward3(_ptr(x), _ptr(A), _ptr(B), _ptr(C), _ptr(G), N, p, q, m1, m2,
+                                   s1, s2, r, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dbias))
+        return {"dX": dX, "dA": dA, "dB": dB, "dC": dC, "dbias": dbias}
+
+
 _default = None
 
 
@@ -203,3 +249,15 @@ def vanloan_rearrange(W, p, q, m1, m2) -> np.ndarray:
 
 def vanloan_fit(W, p, q, m1, m2, r, normalize: bool = True) -> dict:
     return default().vanloan_fit(W, p, q, m1, m2, r, normalize)
+
+
+def weight3(A, B, C) -> np.ndarray:
+    return default().weight3(A, B, C)
+
+
+def forward3(x, A, B, C, bias=None) -> np.ndarray:
+    return default().forward3(x, A, B, C, bias)
+
+
+def backward3(x, A, B, C, G) -> dict:
+    return default().backward3(x, A, B, C, G)

@@ -229,3 +229,113 @@ void oracle_vanloan_rearrange(const double *W, int p, int q, int m1, int m2, dou
                     Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =
                         W[((size_t)a * m1 + j) * ((size_t)q * m2) + (size_t)c * m2 + k];
 }
+
+/*
+ * Triple Kronecker layer (page "LLM Compression via Kronecker Product Decomposition",
+ * section "Triple Kronecker -- AxBxC (Extreme Compression)"), with r terms:
+ *
+ *     W = sum_i kron(A_i, kron(B_i, C_i)),   A_i p x q,  B_i m1 x m2,  C_i s1 x s2,
+ *     W[(a*m1 + j)*s1 + u][(c*m2 + k)*s2 + v] = sum_i A_i[a][c] B_i[j][k] C_i[u][v],
+ *     y = x W + bias,
+ *
+ * built entry by entry; the backward is the chain rule through that W (dX = G W^T,
+ * dW = x^T G, dA_i[a][c] = sum dW[..] B_i[j][k] C_i[u][v], and likewise for B_i and C_i).
+ * A [r][p][q], B [r][m1][m2], C [r][s1][s2]; x [N][p*m1*s1]; y, G [N][q*m2*s2].
+ */
+void oracle_build_weight3(const double *A, const double *B, const double *C, int p, int q,
+                          int m1, int m2, int s1, int s2, int r, double *W)
+{
+    const long in = (long)p * m1 * s1, out = (long)q * m2 * s2;
+    memset(W, 0, sizeof(double) * (size_t)in * out);
+    for (int i = 0; i < r; ++i)
+        for (int a = 0; a < p; ++a)
+            for (int c = 0; c < q; ++c) {
+                const double av = A[((long)i * p + a) * q + c];
+                for (int j = 0; j < m1; ++j)
+                    for (int k = 0; k < m2; ++k) {
+                        const double bv = B[((long)i * m1 + j) * m2 + k];
+                        for (int u = 0; u < s1; ++u)
+                            for (int v = 0; v < s2; ++v)
+                                W[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] +=
+                                    av * bv * C[((long)i * s1 + u) * s2 + v];
+                    }
+            }
+}
+
+void oracle_forward3(const double *x, const double *A, const double *B, const double *C,
+                     const double *bias, long N, int p, int q, int m1, int m2, int s1, int s2,
+                     int r, double *y)
+{
+    const long in = (long)p * m1 * s1, out = (long)q * m2 * s2;
+    double *W = (double *)malloc(sizeof(double) * (size_t)in * out);
+    oracle_build_weight3(A, B, C, p, q, m1, m2, s1, s2, r, W);
+    oracle_matmul_bias(x, W, bias, N, in, out, y);
+    free(W);
+}
+
+void oracle_backward3(const double *x, const double *A, const double *B, const double *C,
+                      const double *G, long N, int p, int q, int m1, int m2, int s1, int s2,
+                      int r, double *dX, double *dA, double *dB, double *dC, double *dbias)
+{
+    const long in = (long)p * m1 * s1, out = (long)q * m2 * s2;
+    double *W = (double *)malloc(sizeof(double) * (size_t)in * out);
+    double *dW = (double *)calloc((size_t)in * out, sizeof(double));
+    oracle_build_weight3(A, B, C, p, q, m1, m2, s1, s2, r, W);
+    /* dX = G W^T */
+#pragma omp parallel for
+    for (long n = 0; n < N; ++n)
+        for (long u = 0; u < in; ++u) {
+            double s = 0.0;
+            for (long o = 0; o < out; ++o) s += G[n * out + o] * W[u * out + o];
+            dX[n * in + u] = s;
+        }
+    /* dW = x^T G */
+#pragma omp parallel for
+    for (long u = 0; u < in; ++u)
+        for (long n = 0; n < N; ++n) {
+            const double xv = x[n * in + u];
+            for (long o = 0; o < out; ++o) dW[u * out + o] += xv * G[n * out + o];
+        }
+    for (int i = 0; i < r; ++i) {
+        for (int a = 0; a < p; ++a)
+            for (int c = 0; c < q; ++c) {
+                double s = 0.0;
+                for (int j = 0; j < m1; ++j)
+                    for (int k = 0; k < m2; ++k)
+                        for (int u = 0; u < s1; ++u)
+                            for (int v = 0; v < s2; ++v)
+                                s += dW[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] *
+                                     B[((long)i * m1 + j) * m2 + k] * C[((long)i * s1 + u) * s2 + v];
+                dA[((long)i * p + a) * q + c] = s;
+            }
+        for (int j = 0; j < m1; ++j)
+            for (int k = 0; k < m2; ++k) {
+                double s = 0.0;
+                for (int a = 0; a < p; ++a)
+                    for (int c = 0; c < q; ++c)
+                        for (int u = 0; u < s1; ++u)
+                            for (int v = 0; v < s2; ++v)
+                                s += dW[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] *
+                                     A[((long)i * p + a) * q + c] * C[((long)i * s1 + u) * s2 + v];
+                dB[((long)i * m1 + j) * m2 + k] = s;
+            }
+        for (int u = 0; u < s1; ++u)
+            for (int v = 0; v < s2; ++v) {
+                double s = 0.0;
+                for (int a = 0; a < p; ++a)
+                    for (int c = 0; c < q; ++c)
+                        for (int j = 0; j < m1; ++j)
+                            for (int k = 0; k < m2; ++k)
+                                s += dW[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] *
+                                     A[((long)i * p + a) * q + c] * B[((long)i * m1 + j) * m2 + k];
+                dC[((long)i * s1 + u) * s2 + v] = s;
+            }
+    }
+    for (long o = 0; o < out; ++o) {
+        double s = 0.0;
+        for (long n = 0; n < N; ++n) s += G[n * out + o];
+        dbias[o] = s;
+    }
+    free(W);
+    free(dW);
+}

@@ -360,6 +360,70 @@ def pin_vanloan_alpha_restores_energy(orc):
         assert f1["alpha"] > 1.0
 
 
+# ---------------------------------------------------------------- triple Kronecker layer
+# (page "LLM Compression via Kronecker Product Decomposition", section "Triple Kronecker --
+# AxBxC (Extreme Compression)")
+
+def _rand_triple(rng, p, q, m1, m2, s1, s2, r, N=3):
+    A = rng.standard_normal((r, p, q))
+    B = rng.standard_normal((r, m1, m2))
+    C = rng.standard_normal((r, s1, s2))
+    x = rng.standard_normal((N, p * m1 * s1))
+    G = rng.standard_normal((N, q * m2 * s2))
+    bias = rng.standard_normal(q * m2 * s2)
+    return A, B, C, x, G, bias
+
+
+def pin_kron3_weight_is_numpy_triple_kron(orc):
+    """W = sum_i kron(A_i, kron(B_i, C_i)) by numpy's kron, rectangular factors; numpy's kron
+    is associative, so this is also sum_i kron(kron(A_i, B_i), C_i)."""
+    rng = np.random.default_rng(311)
+    A, B, C, *_ = _rand_triple(rng, 2, 3, 3, 2, 2, 4, 2)
+    W = orc.weight3(A, B, C)
+    ref = sum(np.kron(A[i], np.kron(B[i], C[i])) for i in range(2))
+    assert np.allclose(W, ref, rtol=0, atol=1e-12)
+    ref2 = sum(np.kron(np.kron(A[i], B[i]), C[i]) for i in range(2))
+    assert np.allclose(W, ref2, rtol=0, atol=1e-12)
+
+
+def pin_kron3_forward_brute_force(orc):
+    """y[n][(c,k,v)] = sum_{a,j,u} x[n][(a,j,u)] A[a,c] B[j,k] C[u,v] + bias, scalar loops."""
+    rng = np.random.default_rng(313)
+    p, q, m1, m2, s1, s2, r = 2, 2, 2, 3, 3, 2, 2
+    A, B, C, x, G, bias = _rand_triple(rng, p, q, m1, m2, s1, s2, r, N=2)
+    y = orc.forward3(x, A, B, C, bias)
+    for n in range(2):
+        for c, k, v in itertools.product(range(q), range(m2), range(s2)):
+            s = bias[(c * m2 + k) * s2 + v]
+            for a, j, u, i in itertools.product(range(p), range(m1), range(s1), range(r)):
+                s += x[n][(a * m1 + j) * s1 + u] * A[i, a, c] * B[i, j, k] * C[i, u, v]
+            assert abs(y[n][(c * m2 + k) * s2 + v] - s) <= 1e-12 * max(1.0, abs(s))
+
+
+def pin_kron3_finite_differences(orc):
+    """Central differences of L = <G, y> in every input (exact up to rounding: L is affine in
+    each single coordinate)."""
+    rng = np.random.default_rng(317)
+    p, q, m1, m2, s1, s2, r = 2, 3, 2, 2, 2, 3, 2
+    A, B, C, x, G, bias = _rand_triple(rng, p, q, m1, m2, s1, s2, r)
+    g = orc.backward3(x, A, B, C, G)
+    L = lambda x_, A_, B_, C_, b_: float(np.sum(G * orc.forward3(x_, A_, B_, C_, b_)))
+    h = 1e-3
+    args = {"x": x, "A": A, "B": B, "C": C, "bias": bias}
+    names = {"x": "dX", "A": "dA", "B": "dB", "C": "dC", "bias": "dbias"}
+    for key, grad in names.items():
+        base = args[key]
+        for idx in list(np.ndindex(base.shape))[:: max(1, base.size // 9)]:
+            up_, dn_ = base.copy(), base.copy()
+            up_[idx] += h
+            dn_[idx] -= h
+            a_up = dict(args, **{key: up_})
+            a_dn = dict(args, **{key: dn_})
+            num = (L(a_up["x"], a_up["A"], a_up["B"], a_up["C"], a_up["bias"]) -
+                   L(a_dn["x"], a_dn["A"], a_dn["B"], a_dn["C"], a_dn["bias"])) / (2 * h)
+            assert abs(num - g[grad][idx]) <= 1e-7 * max(1.0, abs(num)), (key, idx)
+
+
 ALL_PINS = [
     pin_weight_is_sum_of_numpy_krons,
     pin_forward_brute_force,
@@ -375,6 +439,9 @@ ALL_PINS = [
     pin_vanloan_rank_one_closed_form,
     pin_vanloan_best_approximation,
     pin_vanloan_alpha_restores_energy,
+    pin_kron3_weight_is_numpy_triple_kron,
+    pin_kron3_forward_brute_force,
+    pin_kron3_finite_differences,
     pin_special_shapes,
     pin_finite_differences,
     pin_linearity_identities,

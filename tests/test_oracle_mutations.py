@@ -52,6 +52,15 @@ MUTATIONS = [
     ("vanloan_inner_index_swapped",
      "Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)j * m2 + k] =",
      "Wt[((size_t)a * q + c) * ((size_t)m1 * m2) + (size_t)k * m1 + j] =", 0),
+    ("kron3_weight_swaps_inner_factors",
+     "W[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] +=\n                                    av * bv",
+     "W[(((long)a * m1 + j) * s1 + u) * out + ((long)c * m2 + k) * s2 + v] +=\n                                    av * av", 0),
+    ("kron3_dA_drops_C",
+     "B[((long)i * m1 + j) * m2 + k] * C[((long)i * s1 + u) * s2 + v];\n                dA",
+     "B[((long)i * m1 + j) * m2 + k];\n                dA", 0),
+    ("kron3_dC_uses_B_twice",
+     "A[((long)i * p + a) * q + c] * B[((long)i * m1 + j) * m2 + k];\n                dC",
+     "B[((long)i * m1 + j) * m2 + k] * B[((long)i * m1 + j) * m2 + k];\n                dC", 0),
 ]
 
 
