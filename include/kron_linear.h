@@ -184,6 +184,38 @@ KRON_API kron_status_t kron_linear_backward_noalloc(const void *x, const void *S
                                                     void *stream);
 
 /*
+ * Triple Kronecker layer (page "LLM Compression via Kronecker Product Decomposition",
+ * section "Triple Kronecker -- AxBxC (Extreme Compression)"), with r terms:
+ *
+ *     y = x W + bias,   W = sum_i kron(A_i, kron(B_i, C_i)),
+ *     A [r][p][q], B [r][m1][m2], C [r][s1][s2], x [N][p*m1*s1], y [N][q*m2*s2],
+ *     W[(a*m1 + j)*s1 + u][(c*m2 + k)*s2 + v] = sum_i A_i[a][c] B_i[j][k] C_i[u][v].
+ *
+ * It runs as the two-factor layer above with S = ones and the block factor
+ * kron(B_i, C_i) ((m1*s1) x (m2*s2)), formed in the workspace by each call, so the shapes,
+ * paths, dtypes (KRON_BF16: x, y, dY, dX, A, B, C, bias bf16; gradients fp32) and errors
+ * are those of kron_linear_forward / kron_linear_backward for (p, q, m1*s1, m2*s2, r); in
+ * BF16 the block factor is rounded once to bf16.  The backward returns dA = dC' and chains
+ * the block factor's gradient to dB and dC (fixed-order double sums); dX and dbias may be
+ * NULL.  `workspace` is kron3_linear_workspace_size(..., backward) bytes (forward: 0, backward:
+ * 1), 256-byte aligned, owned by the caller; 0 means the arguments are invalid or the
+ * backward has no kernel for the block shape on this path.
+ */
+KRON_API size_t kron3_linear_workspace_size(int64_t N, int p, int q, int m1, int m2, int s1,
+                                            int s2, int r, kron_dtype_t dtype, int backward);
+KRON_API kron_status_t kron3_linear_forward(const void *x, const void *A, const void *B,
+                                            const void *C, const void *bias, void *y, int64_t N,
+                                            int p, int q, int m1, int m2, int s1, int s2, int r,
+                                            kron_dtype_t dtype, unsigned flags, void *workspace,
+                                            size_t workspace_bytes, void *stream);
+KRON_API kron_status_t kron3_linear_backward(const void *x, const void *A, const void *B,
+                                             const void *C, const void *dY, void *dX, void *dA,
+                                             void *dB, void *dC, void *dbias, int64_t N, int p,
+                                             int q, int m1, int m2, int s1, int s2, int r,
+                                             kron_dtype_t dtype, unsigned flags, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
+/*
  * Rank-r Kronecker fit of a dense matrix, to initialise the layer's factors from a dense
  * layer (page "LLM Compression via Kronecker Product Decomposition", sections "Van Loan
  * Rearrangement (1993)", "Rank-K" and "Adaptive Normalization"):

@@ -159,7 +159,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 kron_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, FwdArgs args) {
     using T = typename Cfg::T;
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
-    constexpr int NT = Cfg::NT, N1 = Cfg::N1, S = Cfg::STAGES, TB = Cfg::TB;
+    // (TS2 has no T buffers: TB stands at 1 in the SS-path code, which TS2 never runs)
+    constexpr int NT = Cfg::NT, N1 = Cfg::N1, S = Cfg::STAGES, TB = Cfg::TB > 0 ? Cfg::TB : 1;
     constexpr int D1S = Cfg::D1_SLOTS, D2S = Cfg::D2_SLOTS;
     constexpr int VPC = 16 / E;  // values per 16-byte chunk
 

@@ -128,7 +128,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     constexpr int E = Cfg::E, P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
     constexpr int NT = Cfg::NT, RG = Cfg::RG, NG = Cfg::NG, SI = Cfg::SI, SB = Cfg::SB;
     constexpr int MBT = Cfg::MBT, MBU = Cfg::MBU, IPT = Cfg::IPT, IPU = Cfg::IPU;
-    constexpr int KSTEP = Cfg::KSTEP, VPC = Cfg::VPC;
+    constexpr int KSTEP = Cfg::KSTEP;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

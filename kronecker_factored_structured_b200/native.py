@@ -31,6 +31,7 @@ STATUS = {0: "KRON_OK", 1: "KRON_ERR_INVALID_ARG", 2: "KRON_ERR_UNSUPPORTED",
 EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_l1",
            "kron_linear_backward_noalloc",
            "kron_linear_workspace_size", "kron_vanloan_fit", "kron_vanloan_workspace_size",
+           "kron3_linear_forward", "kron3_linear_backward", "kron3_linear_workspace_size",
            "kron_status_string", "kron_last_error", "kron_linear_device_error",
            "kron_linear_abi_version")
 
@@ -71,6 +72,14 @@ def load(path: str = LIB_PATH):
     lib.kron_vanloan_workspace_size.restype = sz
     lib.kron_vanloan_fit.argtypes = [vp, I, I, I, I, I, vp, I, I, I, vp, vp, vp, vp, vp, sz, vp]
     lib.kron_vanloan_fit.restype = I
+    lib.kron3_linear_workspace_size.argtypes = [i64, I, I, I, I, I, I, I, I, I]
+    lib.kron3_linear_workspace_size.restype = sz
+    lib.kron3_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, I, I, I, I, I, I, I, I, U,
+                                         vp, sz, vp]
+    lib.kron3_linear_forward.restype = I
+    lib.kron3_linear_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, I, I, I,
+                                          I, I, I, I, I, U, vp, sz, vp]
+    lib.kron3_linear_backward.restype = I
     lib.kron_linear_workspace_size.argtypes = [i64, I, I, I, I, I, I]
     lib.kron_linear_workspace_size.restype = sz
     lib.kron_status_string.argtypes = [I]
@@ -222,3 +231,51 @@ def vanloan_fit(W, p, q, m1, m2, r, k=None, power_iters=2, normalize=True, omega
                                 _ptr(ws), ws.numel(), _stream(stream)))
     return {"S": torch.ones(p, q, device=dev), "A": A, "B": B, "sigma": sigma,
             "alpha": alpha[:1]}
+
+
+def _shapes3(A, B, C):
+    r, p, q = A.shape
+    r2, m1, m2 = B.shape
+    r3, s1, s2 = C.shape
+    if r2 != r or r3 != r:
+        raise ValueError("A, B and C must hold the same number of terms")
+    return p, q, m1, m2, s1, s2, r
+
+
+def forward3(x, A, B, C, bias=None, dtype="tf32", flags=0, stream=None):
+    """Triple Kronecker layer y = x W + bias, W = sum_i kron(A_i, kron(B_i, C_i))."""
+    p, q, m1, m2, s1, s2, r = _shapes3(A, B, C)
+    N = x.shape[0]
+    t = io_dtype(dtype)
+    _expect(x, "x", t, (N, p * m1 * s1))
+    for name, v, shp in (("A", A, (r, p, q)), ("B", B, (r, m1, m2)), ("C", C, (r, s1, s2))):
+        _expect(v, name, t, shp)
+    y = torch.empty(N, q * m2 * s2, dtype=t, device=x.device)
+    lib = load()
+    n = int(lib.kron3_linear_workspace_size(N, p, q, m1, m2, s1, s2, r, DTYPES[dtype], 0))
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.kron3_linear_forward(_ptr(x), _ptr(A), _ptr(B), _ptr(C), _ptr(bias), _ptr(y), N, p,
+                                    q, m1, m2, s1, s2, r, DTYPES[dtype], flags, _ptr(ws),
+                                    ws.numel(), _stream(stream)))
+    return y
+
+
+def backward3(x, A, B, C, dY, dtype="tf32", flags=0, stream=None):
+    """Gradients of <dY, y> for the triple layer: dict(dX, dA, dB, dC, dbias)."""
+    p, q, m1, m2, s1, s2, r = _shapes3(A, B, C)
+    N = x.shape[0]
+    t = io_dtype(dtype)
+    _expect(x, "x", t, (N, p * m1 * s1))
+    _expect(dY, "dY", t, (N, q * m2 * s2))
+    dev = x.device
+    g = {"dX": torch.empty(N, p * m1 * s1, dtype=t, device=dev),
+         "dA": torch.empty(r, p, q, device=dev), "dB": torch.empty(r, m1, m2, device=dev),
+         "dC": torch.empty(r, s1, s2, device=dev), "dbias": torch.empty(q * m2 * s2, device=dev)}
+    lib = load()
+    n = int(lib.kron3_linear_workspace_size(N, p, q, m1, m2, s1, s2, r, DTYPES[dtype], 1))
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+    _check(lib.kron3_linear_backward(_ptr(x), _ptr(A), _ptr(B), _ptr(C), _ptr(dY), _ptr(g["dX"]),
+                                     _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dbias"]),
+                                     N, p, q, m1, m2, s1, s2, r, DTYPES[dtype], flags, _ptr(ws),
+                                     ws.numel(), _stream(stream)))
+    return g

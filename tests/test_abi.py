@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "kron_linear.h")
 
 def header_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"KRON_API\s+[\w\s\*]*?\b(kron_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"KRON_API\s+[\w\s\*]*?\b(kron3?_\w+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -140,6 +140,25 @@ def test_vanloan_fit_rejects(args, status):
                               ALIGNED, a["ws"], a["ws_bytes"], None)
     assert st == status, lib.kron_last_error().decode()
     assert lib.kron_last_error().decode() != ""
+
+
+def test_kron3_host_checks():
+    """The triple Kronecker entry points check sizes, pointers and workspace on the host."""
+    lib = native.load()
+    assert lib.kron3_linear_workspace_size(64, 32, 32, 4, 4, 8, 8, 4, 1, 1) > 0
+    assert lib.kron3_linear_workspace_size(64, 32, 32, 4, 4, 8, 8, 0, 1, 1) == 0     # r = 0
+    assert lib.kron3_linear_workspace_size(64, 3, 5, 2, 2, 4, 4, 1, 2, 1) == 0       # no BF16 kernel
+    assert lib.kron3_linear_workspace_size(64, 3, 5, 2, 2, 4, 4, 1, 0, 1) > 0        # F32 takes it
+    st = lib.kron3_linear_forward(ALIGNED, None, ALIGNED, ALIGNED, None, ALIGNED, 8, 2, 2, 4, 4,
+                                  2, 2, 1, 0, 0, V(0x100000), 1 << 20, None)
+    assert st == 1                                                                  # A missing
+    st = lib.kron3_linear_forward(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, ALIGNED, 8, 2, 2, 4,
+                                  4, 2, 2, 1, 0, 0, None, 0, None)
+    assert st == 4                                                                  # no workspace
+    st = lib.kron3_linear_backward(ALIGNED, ALIGNED, ALIGNED, MISALIGNED, ALIGNED, ALIGNED,
+                                   ALIGNED, ALIGNED, ALIGNED, None, 8, 2, 2, 4, 4, 2, 2, 1, 0, 0,
+                                   V(0x100000), 1 << 20, None)
+    assert st == 3                                                                  # C misaligned
 
 
 def test_vanloan_workspace_size():
