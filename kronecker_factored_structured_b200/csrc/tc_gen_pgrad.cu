@@ -376,17 +376,19 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                                                 : MBU * Cfg::T2_BLK + (ir / IPT) * Cfg::U2_BLK);
                 const int rbase = is_t ? (ir % IPU) * P : (ir % IPT) * M2;   // a multiple of 8
                 // BF16 pairs: lanes 2m, 2m+1 hold adjacent K positions of the same rows; each
-                // lane stores one 4-byte pair per two columns (even lane: row of column w,
-                // odd lane: row of column w+1)
+                // lane stores one 4-byte pair per two columns: the even lane the row of column
+                // w, the odd lane the row of column w+4 (rows four apart: under the 128-byte
+                // swizzle their halves of a warp store land on disjoint banks)
                 const bool odd = lane & 1;
 #pragma unroll
-                for (int w = 0; w < 32; w += 2) {
-                    const int c = cg * 32 + w + (odd ? 1 : 0);
-                    const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 1], 1);
+                for (int w = 0; w < 32; ++w) {
+                    if (w & 4) continue;
+                    const int c = cg * 32 + w + (odd ? 4 : 0);
+                    const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 4], 1);
                     if (valid && c < NT * CW) {
                         const int n = c / CW, row = rbase + c % CW;
                         const int kb = (n * KW + own - (odd ? 1 : 0)) * E;
-                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 1] : got;
+                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 4] : got;
                         st_shared_u32(dst + kmaj(row, kb, 128, 128),
                                       pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi)));
                     }
@@ -430,10 +432,11 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     } else {
         // ---------------- dbias column sums of the dY tiles ----------------
         const int tid = threadIdx.x - 608;
-        constexpr int PER = Q * M2 / 128;
-        float acc[PER];
+        constexpr int PER = Q * M2 / 256;   // pairs (c, k..k+1) per thread
+        static_assert((Q * M2) % 256 == 0 && M2 % 2 == 0, "dbias pairs");
+        float acc[2 * PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+        for (int e = 0; e < 2 * PER; ++e) acc[e] = 0.f;
         for (int u = 0; u < nt; ++u) {
             const int s = u % SI;
             if (!mbar_wait(bar(IN_FULL + s), (u / SI) & 1, ab)) break;
@@ -441,19 +444,15 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             if (grp == 0) {
 #pragma unroll
                 for (int e = 0; e < PER; ++e) {
-                    const int idx = tid + 128 * e, c = idx / M2, k = idx % M2;
+                    const int idx = 2 * (tid + 128 * e), c = idx / M2, k = idx % M2;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        const uint32_t a = in + Cfg::OFF_GK + kmaj(n * Q + c, k * E, Cfg::GBR, Cfg::GRB);
-                        if constexpr (GE<T>::tf32) {
-                            float v;
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-                            acc[e] += v;
-                        } else {
-                            unsigned short hv;
-                            asm volatile("ld.shared.b16 %0, [%1];" : "=h"(hv) : "r"(a) : "memory");
-                            acc[e] += __bfloat162float(__ushort_as_bfloat16(hv));
-                        }
+                        uint32_t v;
+                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v)
+                                     : "r"(in + Cfg::OFF_GK + kmaj(n * Q + c, k * E, Cfg::GBR, Cfg::GRB))
+                                     : "memory");
+                        acc[2 * e] += __bfloat162float(__ushort_as_bfloat16((unsigned short)(v & 0xFFFFu)));
+                        acc[2 * e + 1] += __bfloat162float(__ushort_as_bfloat16((unsigned short)(v >> 16)));
                     }
                 }
             }
@@ -462,7 +461,10 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         if (grp == 0) {
             float *pw = args.ws + (size_t)part * args.ws_stride + (size_t)R * (P * Q + M1 * M2);
 #pragma unroll
-            for (int e = 0; e < PER; ++e) pw[tid + 128 * e] = acc[e];
+            for (int e = 0; e < PER; ++e) {
+                pw[2 * (tid + 128 * e)] = acc[2 * e];
+                pw[2 * (tid + 128 * e) + 1] = acc[2 * e + 1];
+            }
         }
     }
 
