@@ -454,9 +454,18 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
             for (int n = nb; n < nb + 1; ++n) {   // column block (n, w), w = a (T) or k (U)
                 uint32_t r[32];
                 tmem_load32(src + n * 32, r);
+                // rows i*32 + w of the 128B-swizzled K-major region, K byte kb: the 16-byte
+                // chunk index (kb >> 4) & 7 is XORed with the row's low three bits, which are
+                // w & 7 (i*32 is a multiple of 8), so only that XOR varies with w at run time
+                const int kb = (n * 32 + o) * E;
+                const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
+                                      (uint32_t)(kb & 15);
+                const uint32_t c16 = (uint32_t)(kb >> 4) & 7u;
 #pragma unroll
                 for (int w = 0; w < 32; ++w)
-                    st_elem<T>(dst + koff(i * 32 + w, (n * 32 + o) * E, 128, 128), r[w]);
+                    st_elem<T>(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
+                                   ((c16 ^ (uint32_t)(w & 7)) << 4),
+                               r[w]);
             }
             tc_fence_before();
             mbar_arrive_warp(bar(D_EMPTY + d));
