@@ -1,11 +1,11 @@
 """Run one seeded workload's forward + backward through the library a few times, then
 print one timed step (CUDA events).  A small driver for profilers (one kernel per capture):
 
-    python -m kronecker_factored_structured_b200.run_workload WORKLOAD N PATH FLAGS ITERS
+    python -m kronecker_factored_structured_b200.run_workload WORKLOAD N PATH FLAGS ITERS [fwd]
 
 WORKLOAD is a name from kron_workloads (tutorial, gpt2_c_fc_r4, stress, sweep_m64_r2, ...),
 N the number of rows, PATH f32 | tf32 | bf16, FLAGS the flag bits (1 = skip zero blocks),
-ITERS the untimed steps before the timed one."""
+ITERS the untimed steps before the timed one; `fwd` runs the forward only."""
 from __future__ import annotations
 
 import dataclasses
@@ -23,20 +23,24 @@ def main(argv=None):
     import kron_workloads as kw
     import kronecker_factored_structured_b200 as kfs
     name, N, path, flags, iters = argv[0], int(argv[1]), argv[2], int(argv[3]), int(argv[4])
+    fwd_only = len(argv) > 5 and argv[5] == "fwd"
     w = kw.get(name).with_rows(N)
     if path == "bf16":
         w = dataclasses.replace(w, dtype="bf16")
     t = kfs.native.io_dtype(path)
     d = {k: v.to(t).cuda() for k, v in kw.inputs(w).items()}
+    def backward():
+        if not fwd_only:
+            kfs.backward(d["x"], d["S"], d["A"], d["B"], d["G"], dtype=path, flags=flags)
     for _ in range(iters):
         kfs.forward(d["x"], d["S"], d["A"], d["B"], d["bias"], dtype=path, flags=flags)
-        kfs.backward(d["x"], d["S"], d["A"], d["B"], d["G"], dtype=path, flags=flags)
+        backward()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     ev[0].record()
     kfs.forward(d["x"], d["S"], d["A"], d["B"], d["bias"], dtype=path, flags=flags)
     ev[1].record()
-    kfs.backward(d["x"], d["S"], d["A"], d["B"], d["G"], dtype=path, flags=flags)
+    backward()
     ev[2].record()
     torch.cuda.synchronize()
     print(f"{name} N={N} {path} flags={flags}: forward {ev[0].elapsed_time(ev[1]) * 1e3:.1f} us, "
