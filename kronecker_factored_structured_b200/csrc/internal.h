@@ -107,13 +107,15 @@ bool generic_fwd_supported(const Shape &ks, bool bf16, bool tr);
 cudaError_t generic_fwd(const void *x, const void *S, const void *A, const void *B,
                         const void *bias, void *y, const Shape &ks, bool bf16, bool tr,
                         bool skip, cudaStream_t st);
-// Row-range partials of dC, dB and dbias into ws (parts x partial_stride floats); the
-// grid is parts x (rank groups) CTAs.  The fixed-order sum over ranges is reduce.cu's.
+// Parameter gradients: row-range partials of dC, dB and dbias into ws (parts x
+// partial_stride floats, then the grid-barrier word), summed in a fixed order by the same
+// cooperative launch of parts x (rank groups) CTAs, which writes dS, dA, dB and dbias.
 bool generic_pgrad_supported(const Shape &s, bool bf16);
 int generic_pgrad_tile_rows(const Shape &s, bool bf16);
 int generic_pgrad_max_parts(const Shape &s, bool bf16);
 cudaError_t generic_pgrad(const void *x, const void *S, const void *A, const void *B,
-                          const void *dY, float *ws, int parts, const Shape &s, bool bf16,
+                          const void *dY, float *ws, int parts, const Shape &s, float *dS,
+                          float *dA, float *dB, float *dbias, bool bf16, double l1,
                           cudaStream_t st);
 }  // namespace tc
 

@@ -2,8 +2,7 @@
 //
 // The tutorial layer's shape (p = q = m1 = m2 = 32, r = 4) runs the tuned kernels of
 // tc_fwd.cu and tc_bwd.cu; the other compiled shapes run the generic kernels of
-// tc_gen_fwd.cu and tc_gen_pgrad.cu (whose parameter-gradient partials are added by the
-// fixed-order reduction of reduce.cu).  Every other shape is refused with
+// tc_gen_fwd.cu and tc_gen_pgrad.cu.  Every other shape is refused with
 // KRON_ERR_UNSUPPORTED by the caller (api.cu); nothing falls back to another path.
 #include "internal.h"
 
@@ -69,10 +68,7 @@ cudaError_t tc_backward(const void *x, const void *S, const void *A, const void 
         e = tc::generic_fwd(dY, S, A, B, nullptr, dX, tc::transposed(s), bf16, true, skip, st);
         if (e != cudaSuccess) return e;
     }
-    e = tc::generic_pgrad(x, S, A, B, dY, ws, parts, s, bf16, st);
-    if (e != cudaSuccess) return e;
-    launch_step() = "reduction launch";
-    return reduce_partials(ws, parts, S, A, bf16, dS, dA, dB, dbias, s, l1, st);
+    return tc::generic_pgrad(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, bf16, l1, st);
 }
 
 }  // namespace kron

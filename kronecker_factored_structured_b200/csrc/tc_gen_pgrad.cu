@@ -15,8 +15,9 @@
 // warps move them TMEM -> registers -> shared memory into the K-major layouts dC and dB
 // read (T lanes (i,k) become T2 rows (i,a), U lanes (i,a) become U2 rows (i,k)).  dC and
 // dB accumulate in TMEM over the CTA's rows and are written to the workspace as that row
-// range's partials; reduce.cu adds the ranges in a fixed order and forms dA = dC (.) S and
-// dS = sum_i dC_i (.) A_i.  Splitting the ranks over groups keeps the accumulators and
+// range's partials; after a grid barrier (cooperative launch: every CTA resident) the whole
+// grid adds the ranges in a fixed order and forms dA = dC (.) S and dS = sum_i dC_i (.) A_i
+// (plus l1 * sign(S) when the l1 penalty on S is fused) -- no separate reduction launch.  Splitting the ranks over groups keeps the accumulators and
 // the working slots of one CTA inside the 512 TMEM columns for the larger layers; the CTAs
 // of the groups of one row range are adjacent in the grid, so they stream the same rows at
 // about the same time and the second and later reads of a tile mostly hit L2.
@@ -118,7 +119,82 @@ struct GPgArgs {
     int num_tiles;
     int tiles_per_part;
     int *device_error;
+    unsigned *arrived;     // grid-barrier counter, zeroed by the host before the launch
+    float *dS, *dA, *dB, *dbias;
+    double l1;             // weight of the penalty l1 * sum|S| whose gradient joins dS
 };
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Fixed-order sum of every row range's partials, by the whole grid once all are written.
+// Virtual columns: dC ordered (position (a,c), rank i) so that the r ranks of a position
+// are adjacent, then dB, then dbias.  CTA b owns a run of virtual columns (a multiple of r
+// long); in passes of CW columns, GS groups of threads each add ranges g = ps, ps + GS, ...
+// of one column in double (four accumulators) and the group sums are added in a fixed
+// order.  Only `parts` fixes the order: bitwise reproducible.  The epilogue forms
+// dA_i = dC_i (.) S and dS = sum_i dC_i (.) A_i (+ l1 * sign(S)), and writes dB and dbias.
+template <class Cfg>
+__device__ void reduce_parts(const GPgArgs &args, int parts, double *red, double *vals) {
+    using T = typename Cfg::T;
+    constexpr int P = Cfg::P, Q = Cfg::Q, M1 = Cfg::M1, M2 = Cfg::M2, R = Cfg::R;
+    constexpr int NDC = R * P * Q, NDB = R * M1 * M2, NB = Q * M2, NCOL = NDC + NDB + NB;
+    constexpr int CW = R <= 64 ? (64 / R) * R : R;
+    constexpr int GS = kGPgThreads / CW;
+    const int per = ((NCOL + (int)gridDim.x * R - 1) / ((int)gridDim.x * R)) * R;
+    const int v0 = (int)blockIdx.x * per, v1 = gmin(v0 + per, NCOL);
+    const int cs = threadIdx.x % CW, ps = threadIdx.x / CW;
+    for (int c0 = v0; c0 < v1; c0 += CW) {
+        const int v = c0 + cs;
+        if (ps < GS) {
+            double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+            if (v < v1) {
+                const size_t col = v < NDC ? (size_t)(v % R) * P * Q + (size_t)(v / R) : (size_t)v;
+                const float *src = args.ws + col;
+                int g = ps;
+                for (; g + 3 * GS < parts; g += 4 * GS) {
+                    a0 += (double)__ldcg(src + (size_t)g * args.ws_stride);
+                    a1 += (double)__ldcg(src + (size_t)(g + GS) * args.ws_stride);
+                    a2 += (double)__ldcg(src + (size_t)(g + 2 * GS) * args.ws_stride);
+                    a3 += (double)__ldcg(src + (size_t)(g + 3 * GS) * args.ws_stride);
+                }
+                for (; g < parts; g += GS) a0 += (double)__ldcg(src + (size_t)g * args.ws_stride);
+            }
+            red[ps * CW + cs] = (a0 + a1) + (a2 + a3);
+        }
+        __syncthreads();
+        if (threadIdx.x < CW) {
+            double tot = 0.0;
+            for (int k = 0; k < GS; ++k) tot += red[k * CW + threadIdx.x];
+            vals[threadIdx.x] = tot;
+        }
+        __syncthreads();
+        if (threadIdx.x < CW && v < v1) {
+            if (v < NDC) {
+                if (v % R == 0) {   // the rank group of position (a,c) = v / R
+                    const int pos = v / R;
+                    const double sv = (double)ld_elt<T>(args.S, pos);
+                    double ds = 0.0;
+                    for (int i = 0; i < R; ++i) {
+                        const double dc = vals[threadIdx.x + i];
+                        args.dA[(size_t)i * P * Q + pos] = (float)(dc * sv);
+                        ds += dc * (double)ld_elt<T>(args.A, (size_t)i * P * Q + pos);
+                    }
+                    if (args.l1 != 0.0) ds += args.l1 * sign_of((float)sv);
+                    args.dS[pos] = (float)ds;
+                }
+            } else if (v < NDC + NDB) {
+                args.dB[v - NDC] = (float)vals[threadIdx.x];
+            } else if (args.dbias) {
+                args.dbias[v - NDC - NDB] = (float)vals[threadIdx.x];
+            }
+        }
+        __syncthreads();
+    }
+}
 
 template <class Cfg>
 __global__ void __launch_bounds__(kGPgThreads, 1)
@@ -468,18 +544,46 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         }
     }
 
-    // ---------------- teardown ----------------
+    // ---------------- teardown of the tensor-core state ----------------
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::TM_COLS);
     }
+
+    // ---------------- grid barrier, then the fixed-order reduction ----------------
+    // Every CTA arrives (also after an abort, so none waits forever); the launch is
+    // cooperative, so all CTAs are resident.  The wait is bounded like every other.
+    volatile int *grid_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(args.arrived, 1u);
+        const uint64_t w0 = globaltimer();
+        int okb = 1;
+        while (ld_acquire_gpu(args.arrived) < gridDim.x) {
+            if (globaltimer() - w0 > kWaitTimeoutNs) {
+                okb = 0;
+                if (args.device_error) atomicOr(args.device_error, 2);
+                break;
+            }
+            __nanosleep(128);
+        }
+        *grid_ok = okb && !*ab.flag;
+    }
+    __syncthreads();
+    if (*grid_ok) {
+        double *red = reinterpret_cast<double *>(smem);            // input ring: idle now
+        double *vals = red + kGPgThreads + 64;
+        reduce_parts<Cfg>(args, (int)(gridDim.x / NG), red, vals);
+    }
 }
 
 template <class Cfg>
 cudaError_t launch_gpgrad(const void *x, const void *S, const void *A, const void *B,
-                          const void *dY, float *ws, int parts, const Shape &s, cudaStream_t st) {
+                          const void *dY, float *ws, int parts, const Shape &s, float *dS,
+                          float *dA, float *dB, float *dbias, double l1, cudaStream_t st) {
     using T = typename Cfg::T;
     const bool bf16 = !GE<T>::tf32;
     CUtensorMap tx, tg;
@@ -501,17 +605,29 @@ cudaError_t launch_gpgrad(const void *x, const void *S, const void *A, const voi
     a.num_tiles = (int)((s.N + Cfg::NT - 1) / Cfg::NT);
     a.tiles_per_part = (a.num_tiles + parts - 1) / parts;
     a.device_error = device_error_ptr();
-    launch_step() = "kernel launch";
+    a.arrived = reinterpret_cast<unsigned *>(ws + (size_t)parts * a.ws_stride);
+    a.dS = dS; a.dA = dA; a.dB = dB; a.dbias = dbias;
+    a.l1 = l1;
+    launch_step() = "grid barrier reset";
+    e = cudaMemsetAsync(a.arrived, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return e;
+    launch_step() = "kernel launch (cooperative)";
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(parts * Cfg::NG));
     cfg.blockDim = dim3(kGPgThreads);
     cfg.dynamicSmemBytes = Cfg::SMEM;
     cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kron_pgrad_gen_kernel<Cfg>, tx, tg, a);
 }
 
 using GPgFn = cudaError_t (*)(const void *, const void *, const void *, const void *,
-                              const void *, float *, int, const Shape &, cudaStream_t);
+                              const void *, float *, int, const Shape &, float *, float *,
+                              float *, float *, double, cudaStream_t);
 struct GPgEntry {
     int p, q, m1, m2, r;
     bool bf16;
@@ -556,11 +672,12 @@ int generic_pgrad_max_parts(const Shape &s, bool bf16) {
 }
 
 cudaError_t generic_pgrad(const void *x, const void *S, const void *A, const void *B,
-                          const void *dY, float *ws, int parts, const Shape &s, bool bf16,
+                          const void *dY, float *ws, int parts, const Shape &s, float *dS,
+                          float *dA, float *dB, float *dbias, bool bf16, double l1,
                           cudaStream_t st) {
     const gen::GPgEntry *f = gen::find_gpg(s, bf16);
     if (!f) return cudaErrorNotSupported;
-    return f->fn(x, S, A, B, dY, ws, parts, s, st);
+    return f->fn(x, S, A, B, dY, ws, parts, s, dS, dA, dB, dbias, l1, st);
 }
 
 }  // namespace tc
