@@ -457,15 +457,36 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
                 // rows i*32 + w of the 128B-swizzled K-major region, K byte kb: the 16-byte
                 // chunk index (kb >> 4) & 7 is XORed with the row's low three bits, which are
                 // w & 7 (i*32 is a multiple of 8), so only that XOR varies with w at run time
-                const int kb = (n * 32 + o) * E;
-                const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
-                                      (uint32_t)(kb & 15);
-                const uint32_t c16 = (uint32_t)(kb >> 4) & 7u;
+                if constexpr (BE<T>::tf32) {
+                    const int kb = (n * 32 + o) * E;
+                    const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
+                                          (uint32_t)(kb & 15);
+                    const uint32_t c16 = (uint32_t)(kb >> 4) & 7u;
 #pragma unroll
-                for (int w = 0; w < 32; ++w)
-                    st_elem<T>(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
-                                   ((c16 ^ (uint32_t)(w & 7)) << 4),
-                               r[w]);
+                    for (int w = 0; w < 32; ++w)
+                        st_elem<T>(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
+                                       ((c16 ^ (uint32_t)(w & 7)) << 4),
+                                   r[w]);
+                } else {
+                    // BF16 pairs: lanes 2m, 2m+1 hold K positions 2m, 2m+1 of every row w; one
+                    // shuffle gives each a 4-byte pair, the even lane for row w and the odd lane
+                    // for row w + 4 (same 8-row group; under the 128-byte swizzle the two
+                    // halves of the warp store land on disjoint banks)
+                    const bool odd = o & 1;
+                    const int kb = (n * 32 + (o & ~1)) * E;
+                    const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
+                                          (uint32_t)(kb & 15) + (odd ? 4u * 128u : 0u);
+                    const uint32_t c16 = ((uint32_t)(kb >> 4) & 7u) ^ (odd ? 4u : 0u);
+#pragma unroll
+                    for (int w = 0; w < 32; ++w) {
+                        if (w & 4) continue;
+                        const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 4], 1);
+                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 4] : got;
+                        st_shared_u32(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
+                                          ((c16 ^ (uint32_t)(w & 7)) << 4),
+                                      pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi)));
+                    }
+                }
             }
             tc_fence_before();
             mbar_arrive_warp(bar(D_EMPTY + d));
