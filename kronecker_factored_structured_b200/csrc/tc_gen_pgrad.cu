@@ -124,6 +124,16 @@ struct GPgArgs {
     double l1;             // weight of the penalty l1 * sum|S| whose gradient joins dS
 };
 
+// The T and U accumulators hold their M index (i,k) or (i,a) in a permuted lane order: in
+// each aligned group of 16 TMEM lanes, lanes 0-7 hold the even and lanes 8-15 the odd
+// indices of the group.  A 16x256b TMEM load then gives every thread the values of two
+// adjacent M indices (a K pair of T2 or U2) side by side, so the epilogue stores 4-byte
+// BF16 pairs without exchanging values between lanes.  Returns the M index of lane L.
+__device__ __forceinline__ int pair_lane_index(int L) {
+    const int l = L & 15;
+    return (L & ~15) + (l < 8 ? 2 * l : 2 * (l - 8) + 1);
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -272,7 +282,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     //   B_all^T block bt: lane (i,k) = (i0 + bt*IPT + L/m2, L%m2), column j -> B_i[j][k]
     //   C_stack block bu: lane (i,a) = (i0 + bu*IPU + L/p, L%p), column c -> S[a][c] A_i[a][c]
     if (warp >= 3 && warp < 11) {
-        const int qd = warp & 3, L = qd * 32 + lane;
+        const int qd = warp & 3, L = pair_lane_index(qd * 32 + lane);
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         const bool is_c = warp >= 7;
         const int nblk = is_c ? MBU : MBT;
@@ -434,39 +444,39 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
 #pragma unroll
             for (int task = 0; task < NTASK; ++task) {
                 if ((task & 3) != wi) continue;
-                uint32_t r[32];
                 const bool is_t = task < MBT * TG;
                 const int blk = is_t ? task / TG : (task - MBT * TG) / UG;
                 const int cg = is_t ? task % TG : (task - MBT * TG) % UG;
-                // T lanes (i,k): row (i%IPU, a) of T2 block i/IPU, K (n,k); U lanes (i,a): row
-                // (i%IPT, k) of U2 block i/IPT, K (n,a).  The lane's own index (k or a) fixes
-                // the K byte of each n; the column fixes the row.
-                tmem_load32(tmem + lane_addr + (is_t ? Cfg::TM_DT + (d * MBT + blk) * Cfg::NTS
-                                                     : Cfg::TM_DU + (d * MBU + blk) * Cfg::NUS) + cg * 32, r);
-                const int ir = is_t ? blk * IPT + L / M2 : blk * IPU + L / P;
-                const int own = is_t ? L % M2 : L % P;            // k (T) or a (U)
+                const uint32_t src = tmem + (is_t ? Cfg::TM_DT + (d * MBT + blk) * Cfg::NTS
+                                                  : Cfg::TM_DU + (d * MBU + blk) * Cfg::NUS) + cg * 32;
                 const int CW = is_t ? P : M2;                     // columns per n: a (T), k (U)
                 const int KW = is_t ? M2 : P;                     // K positions per n
-                const bool valid = (is_t || L < IPU * P) && ir < rgv;
-                const uint32_t dst = ib + (is_t ? (ir / IPU) * Cfg::T2_BLK
-                                                : MBU * Cfg::T2_BLK + (ir / IPT) * Cfg::U2_BLK);
-                const int rbase = is_t ? (ir % IPU) * P : (ir % IPT) * M2;   // a multiple of 8
-                // BF16 pairs: lanes 2m, 2m+1 hold adjacent K positions of the same rows; each
-                // lane stores one 4-byte pair per two columns: the even lane the row of column
-                // w, the odd lane the row of column w+4 (rows four apart: under the 128-byte
-                // swizzle their halves of a warp store land on disjoint banks)
-                const bool odd = lane & 1;
+                const uint32_t dstb = ib + (is_t ? 0u : (uint32_t)(MBU * Cfg::T2_BLK));
 #pragma unroll
-                for (int w = 0; w < 32; ++w) {
-                    if (w & 4) continue;
-                    const int c = cg * 32 + w + (odd ? 4 : 0);
-                    const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 4], 1);
-                    if (valid && c < NT * CW) {
-                        const int n = c / CW, row = rbase + c % CW;
-                        const int kb = (n * KW + own - (odd ? 1 : 0)) * E;
-                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 4] : got;
-                        st_shared_u32(dst + kmaj(row, kb, 128, 128),
-                                      pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi)));
+                for (int h = 0; h < 2; ++h) {
+                    // this thread's K pair: M indices nat, nat + 1 of lanes g and g + 8 of
+                    // the half; T: (i,k) -> T2 row (i%IPU, a), K (n,k); U: (i,a) -> U2 row
+                    // (i%IPT, k), K (n,a)
+                    uint32_t r[16];
+                    tmem_load16x256_x4(src + ((uint32_t)(qd * 32 + 16 * h) << 16), r);
+                    const int nat = qd * 32 + 16 * h + 2 * (lane >> 2);
+                    const int ir = is_t ? blk * IPT + nat / M2 : blk * IPU + nat / P;
+                    const int own = is_t ? nat % M2 : nat % P;
+                    const bool valid = (is_t || nat < IPU * P) && ir < rgv;
+                    const uint32_t dst = dstb + (is_t ? (ir / IPU) * Cfg::T2_BLK : (ir / IPT) * Cfg::U2_BLK);
+                    const int rbase = is_t ? (ir % IPU) * P : (ir % IPT) * M2;   // a multiple of 8
+#pragma unroll
+                    for (int rp = 0; rp < 4; ++rp) {
+#pragma unroll
+                        for (int dl = 0; dl < 2; ++dl) {
+                            const int c = cg * 32 + rp * 8 + (lane & 3) * 2 + dl;
+                            if (valid && c < NT * CW) {
+                                const int n = c / CW, row = rbase + c % CW;
+                                st_shared_u32(dst + kmaj(row, (n * KW + own) * E, 128, 128),
+                                              pack_bf16x2(__uint_as_float(r[4 * rp + dl]),
+                                                          __uint_as_float(r[4 * rp + 2 + dl])));
+                            }
+                        }
                     }
                 }
             }

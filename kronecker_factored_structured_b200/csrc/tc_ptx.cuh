@@ -280,6 +280,23 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 16 lanes x 32 consecutive 32-bit columns in the 16x256b pattern (four repetitions of
+// 8 columns): with g = t / 4 and c = 2 * (t % 4), registers 4*rep .. 4*rep + 3 of thread
+// t hold (lane g, column 8*rep + c), (lane g, 8*rep + c + 1), (lane g + 8, 8*rep + c) and
+// (lane g + 8, 8*rep + c + 1), lanes counted from the 16-lane base in taddr (which lies in
+// the warp's own quadrant).  Load and wait are one asm statement, as in tmem_load32.
+__device__ __forceinline__ void tmem_load16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 // tmem_load32 split in two: the load is issued here and its registers are only valid
 // after tmem_wait_load32 on the same array, which names them as its outputs so that no
 // use can be scheduled before the wait.
