@@ -323,8 +323,9 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
     const uint32_t tmem = *tmem_slot;
     // A operands in TMEM, one lane per row (two BF16 values per column):
     //   B_all^T: lane (i,k), column j -> B_i[j][k];   C_stack: lane (i,a), column c -> C_i[a][c]
+    // BF16: the rows in the paired lane order of pair_lane_index (the epilogue stores K pairs)
     if (warp >= 3 && warp < 11) {   // team 0 loads the A operands
-        const int qd = warp & 3, L = qd * 32 + lane;
+        const int qd = warp & 3, L = BE<T>::tf32 ? qd * 32 + lane : pair_lane_index(qd * 32 + lane);
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         const bool is_c = warp >= 7;
         const int i = is_c ? L / P : L / M2, o = is_c ? L % P : L % M2;  // o = a or k
@@ -452,12 +453,12 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
             const uint32_t dst = sI + b * Cfg::IB + (is_u ? Cfg::T2_BYTES : 0);
 #pragma unroll
             for (int n = nb; n < nb + 1; ++n) {   // column block (n, w), w = a (T) or k (U)
-                uint32_t r[32];
-                tmem_load32(src + n * 32, r);
                 // rows i*32 + w of the 128B-swizzled K-major region, K byte kb: the 16-byte
                 // chunk index (kb >> 4) & 7 is XORed with the row's low three bits, which are
                 // w & 7 (i*32 is a multiple of 8), so only that XOR varies with w at run time
                 if constexpr (BE<T>::tf32) {
+                    uint32_t r[32];
+                    tmem_load32(src + n * 32, r);
                     const int kb = (n * 32 + o) * E;
                     const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
                                           (uint32_t)(kb & 15);
@@ -468,23 +469,28 @@ kron_pgrad_tc_kernel(const __grid_constant__ CUtensorMap tm_xk, const __grid_con
                                        ((c16 ^ (uint32_t)(w & 7)) << 4),
                                    r[w]);
                 } else {
-                    // BF16 pairs: lanes 2m, 2m+1 hold K positions 2m, 2m+1 of every row w; one
-                    // shuffle gives each a 4-byte pair, the even lane for row w and the odd lane
-                    // for row w + 4 (same 8-row group; under the 128-byte swizzle the two
-                    // halves of the warp store land on disjoint banks)
-                    const bool odd = o & 1;
-                    const int kb = (n * 32 + (o & ~1)) * E;
-                    const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
-                                          (uint32_t)(kb & 15) + (odd ? 4u * 128u : 0u);
-                    const uint32_t c16 = ((uint32_t)(kb >> 4) & 7u) ^ (odd ? 4u : 0u);
+                    // BF16: two 16x256b loads (lane halves h) give thread t the K pair
+                    // o = 16h + 2(t/4), o + 1 of rows w = 8rp + 2(t%4) + {0, 1}; one 4-byte
+                    // store per pair and row (the four rows of a store fall on distinct
+                    // swizzled chunks: no bank conflict)
 #pragma unroll
-                    for (int w = 0; w < 32; ++w) {
-                        if (w & 4) continue;
-                        const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? r[w] : r[w + 4], 1);
-                        const uint32_t lo = odd ? got : r[w], hi = odd ? r[w + 4] : got;
-                        st_shared_u32(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
-                                          ((c16 ^ (uint32_t)(w & 7)) << 4),
-                                      pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi)));
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t q[16];
+                        tmem_load16x256_x4(src - lane_addr + ((uint32_t)(qd * 32 + 16 * h) << 16) + n * 32, q);
+                        const int kb = (n * 32 + 16 * h + 2 * (lane >> 2)) * E;
+                        const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 + (uint32_t)i * 4096 +
+                                              (uint32_t)(kb & 15);
+                        const uint32_t c16 = (uint32_t)(kb >> 4) & 7u;
+#pragma unroll
+                        for (int rp = 0; rp < 4; ++rp)
+#pragma unroll
+                            for (int dl = 0; dl < 2; ++dl) {
+                                const int w = rp * 8 + (lane & 3) * 2 + dl;
+                                st_shared_u32(base + (uint32_t)(w >> 3) * 1024 + (uint32_t)(w & 7) * 128 +
+                                                  ((c16 ^ (uint32_t)(w & 7)) << 4),
+                                              pack_bf16x2(__uint_as_float(q[4 * rp + dl]),
+                                                          __uint_as_float(q[4 * rp + 2 + dl])));
+                            }
                     }
                 }
             }

@@ -124,16 +124,6 @@ struct GPgArgs {
     double l1;             // weight of the penalty l1 * sum|S| whose gradient joins dS
 };
 
-// The T and U accumulators hold their M index (i,k) or (i,a) in a permuted lane order: in
-// each aligned group of 16 TMEM lanes, lanes 0-7 hold the even and lanes 8-15 the odd
-// indices of the group.  A 16x256b TMEM load then gives every thread the values of two
-// adjacent M indices (a K pair of T2 or U2) side by side, so the epilogue stores 4-byte
-// BF16 pairs without exchanging values between lanes.  Returns the M index of lane L.
-__device__ __forceinline__ int pair_lane_index(int L) {
-    const int l = L & 15;
-    return (L & ~15) + (l < 8 ? 2 * l : 2 * (l - 8) + 1);
-}
-
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -281,6 +271,7 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     // A operands in TMEM (zero for lanes past the group's ranks and for K past q):
     //   B_all^T block bt: lane (i,k) = (i0 + bt*IPT + L/m2, L%m2), column j -> B_i[j][k]
     //   C_stack block bu: lane (i,a) = (i0 + bu*IPU + L/p, L%p), column c -> S[a][c] A_i[a][c]
+    // (lanes in the paired order of pair_lane_index: the epilogue stores K pairs)
     if (warp >= 3 && warp < 11) {
         const int qd = warp & 3, L = pair_lane_index(qd * 32 + lane);
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;

@@ -280,6 +280,15 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// Paired lane order of an accumulator whose epilogue stores BF16 pairs of adjacent M
+// indices: in each aligned group of 16 TMEM lanes, lanes 0-7 hold the even and lanes 8-15
+// the odd M indices of the group, so that a 16x256b load (below) gives every thread the
+// values of M indices 2g and 2g + 1 side by side.  Returns the M index held by lane L.
+__device__ __forceinline__ int pair_lane_index(int L) {
+    const int l = L & 15;
+    return (L & ~15) + (l < 8 ? 2 * l : 2 * (l - 8) + 1);
+}
+
 // 16 lanes x 32 consecutive 32-bit columns in the 16x256b pattern (four repetitions of
 // 8 columns): with g = t / 4 and c = 2 * (t % 4), registers 4*rep .. 4*rep + 3 of thread
 // t hold (lane g, column 8*rep + c), (lane g, 8*rep + c + 1), (lane g + 8, 8*rep + c) and
