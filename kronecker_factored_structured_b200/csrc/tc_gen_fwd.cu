@@ -33,12 +33,19 @@
 //   warp 0       TMA producer: x tiles into an S-stage ring
 //   warp 1       stage-1 MMA issuer (owns the TMEM allocation)
 //   warp 2       stage-2 MMA issuer
-//   warps 3-18   epilogue 1: stage-1 accumulator -> T chunk in shared memory
-//   warps 19-22  epilogue 2: stage-2 accumulator + bias -> y
+//   warps 3..     epilogue 1: stage-1 accumulator -> T chunk in shared memory (E1W warps)
+//   ..22          epilogue 2: stage-2 accumulator + bias -> y (E2W = 20 - E1W warps)
+// The twenty epilogue warps are split by the shape.  Epilogue 2 stores y with one scalar
+// store per value and sets the pace of most shapes (a per-role trace: it is busy ~90% of
+// each tile's time), so it gets two warps per TMEM lane quadrant, each over half of the q
+// columns, unless epilogue 1 needs all four of its warps per quadrant (a D1 slot of four
+// or eight 32-column groups); epilogue 1 takes the other 12 or 16 warps.
 #include "internal.h"
 #include "tc_gen_common.cuh"
 
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 namespace kron {
 namespace tc {
@@ -91,6 +98,17 @@ struct GFwdCfg {
     static constexpr int TM_D1 = A1T, TM_D2 = TM_D1 + D1S * N1S;
     static constexpr int TM_COLS = tmem_cols_pow2(TM_D2 + D2S * QS);
     static constexpr uint32_t IDESC1 = idesc_f32acc(128, N1P, GE<T>::fmt);
+    // epilogue warps: H warps per quadrant for epilogue 2
+    static constexpr int NG1 = N1S / 32;                   // 32-column groups of a D1 slot
+#ifdef KRON_GFWD_H
+    static constexpr int H = KRON_GFWD_H;
+#else
+    static constexpr int H = NG1 % 4 == 0 ? 1 : 2;   // measured: 4 warps per quadrant were slower
+#endif
+    static constexpr int E2W = 4 * H, E1W = 20 - E2W, NW1 = E1W / 4;
+    static constexpr int GPW = cdiv(NG1, NW1);            // D1 column groups of one warp
+    static constexpr int CW2 = QS / H;                     // D2 columns of one warp
+    static constexpr int LW2 = gmin(CW2, 32);              // columns per TMEM load
 
     static_assert(128 % M2 == 0 && M2 % 16 == 0, "m2 divides 128 (stage-2 M = 128)");
     static_assert(N1P <= 256, "stage-1 N = (128/m2)*p at most 256");
@@ -100,6 +118,9 @@ struct GFwdCfg {
     static_assert(QP <= 256, "stage-2 N = q at most 256");
     static_assert(NCB <= 32, "c blocks of the skip mask");
     static_assert(STAGES >= 3, "x ring");
+    static_assert(H == 1 || H == 2 || H == 4, "epilogue-2 warps per quadrant");
+    static_assert(CW2 % 8 == 0 && CW2 % LW2 == 0, "epilogue-2 column shares");
+    static_assert(GPW <= 2, "epilogue-1 groups per warp");
     static_assert(2 * STAGES + 2 * D1S + 2 * TBC + 2 * D2S + 2 + 2 <= BAR_BYTES / 8, "barriers");
     static_assert(fits(D1S, D2S), "TMEM budget");
     static_assert(SMEM <= SMEM_MAX, "shared memory budget");
@@ -159,15 +180,15 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         }
         for (int d = 0; d < D1S; ++d) {
             mbar_init(bar(B_D1FULL + d), 1);
-            mbar_init(bar(B_D1EMPTY + d), 16);
+            mbar_init(bar(B_D1EMPTY + d), Cfg::E1W);
         }
         for (int b = 0; b < TBC; ++b) {
-            mbar_init(bar(B_TFULL + b), 16);
+            mbar_init(bar(B_TFULL + b), Cfg::E1W);
             mbar_init(bar(B_TEMPTY + b), 1);
         }
         for (int d = 0; d < D2S; ++d) {
             mbar_init(bar(B_D2FULL + d), 1);
-            mbar_init(bar(B_D2EMPTY + d), 4);
+            mbar_init(bar(B_D2EMPTY + d), Cfg::E2W);
         }
         mbar_init(bar(B_DRAIN + 0), 1);
         mbar_init(bar(B_DRAIN + 1), 1);
@@ -352,13 +373,14 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         __syncwarp();
         if (lane == 0) mbar_wait_drain(bar(B_DRAIN + 1), 0);
         __syncwarp();
-    } else if (warp < 19) {
+    } else if (warp < 3 + Cfg::E1W) {
         // ---------------- epilogue 1: D1 (lanes (i,k), columns (n,a)) -> T chunk ----------------
+        constexpr int NW1 = Cfg::NW1;                 // warps per quadrant
         const int quad = warp & 3, wi = (warp - 3) >> 2;
         const int L = quad * 32 + lane, il = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        constexpr int NG = N1S / 32;                  // 32-column groups of a D1 slot
-        constexpr int GPW = (NG + 3) / 4;             // groups of one warp (at most 2)
+        constexpr int NG = Cfg::NG1;                  // 32-column groups of a D1 slot
+        constexpr int GPW = Cfg::GPW;                 // groups of one warp (at most 2)
         constexpr int SPG = 32 / VPC;                 // 16-byte stores per group
         // byte offsets (within a T chunk) of this lane's 16-byte stores, fixed for the kernel:
         // column c = (n, a) of lane (i_local, k) goes to row (n, k), K position
@@ -369,7 +391,7 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         for (int gi = 0; gi < GPW; ++gi) {
 #pragma unroll
             for (int g = 0; g < SPG; ++g) {
-                const int c = (wi + 4 * gi) * 32 + g * VPC;
+                const int c = (wi + NW1 * gi) * 32 + g * VPC;
                 const int n = c / P, a = c % P;
                 const int kp = (a / AG) * (IPBE * AG) + il * AG + a % AG;
                 soff[gi][g] = c < N1 ? kmaj(n * M2 + k, kp * E, 128, 128) : 0xFFFFFFFFu;
@@ -409,11 +431,11 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
                 }
 #pragma unroll
                 for (int gi = 0; gi < GPW; ++gi) {
-                    const int cg = wi + 4 * gi;
+                    const int cg = wi + NW1 * gi;
                     if (cg < NG) {
                         uint32_t r[32];
                         tmem_load32(tmem + lane_addr + Cfg::TM_D1 + d1 * N1S + cg * 32, r);
-                        if (cg + 4 >= NG) {
+                        if (cg + NW1 >= NG) {
                             tc_fence_before();
                             mbar_arrive_warp(bar(B_D1EMPTY + d1));
                         }
@@ -435,54 +457,69 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
         }
     } else {
         // ---------------- epilogue 2: D2 (lanes (n,k), columns c) + bias -> y ----------------
-        const int quad = warp & 3;
+        // warp HF of its quadrant takes columns [HF * CW2, (HF + 1) * CW2).  The loop is
+        // compiled per HF: with compile-time column bounds the tail tests and store offsets
+        // fold away (a run-time bound measured about three times slower).
+        constexpr int CW2 = Cfg::CW2, LW2 = Cfg::LW2;
+        const int quad = warp & 3, hf = (warp - 3 - Cfg::E1W) >> 2;
         const int L = quad * 32 + lane, n = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         // bias values of this lane (c*m2 + k), read through the non-coherent path in batches
         // that precede the y stores of the batch (so no load waits on an earlier store)
         const unsigned short *bias16 = static_cast<const unsigned short *>(args.bias);
         const float *bias32 = static_cast<const float *>(args.bias);
-        for (int t = 0; t < my_tiles; ++t) {
-            const int d2 = t % D2S;
-            if (!mbar_wait(bar(B_D2FULL + d2), (t / D2S) & 1, abort_flag)) break;
-            tc_fence_after();
-            const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
-            const size_t obase = (size_t)row * (Q * M2) + k;
+        auto run = [&](auto hf_const) {
+            constexpr int HF = decltype(hf_const)::value;
+            for (int t = 0; t < my_tiles; ++t) {
+                const int d2 = t % D2S;
+                if (!mbar_wait(bar(B_D2FULL + d2), (t / D2S) & 1, abort_flag)) break;
+                tc_fence_after();
+                const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
+                const size_t obase = (size_t)row * (Q * M2) + k;
 #pragma unroll 1
-            for (int c0 = 0; c0 < QS; c0 += 32) {
-                uint32_t r[32];
-                tmem_load32(tmem + lane_addr + Cfg::TM_D2 + d2 * QS + c0, r);
-                if (c0 + 32 >= QS) {
-                    tc_fence_before();
-                    mbar_arrive_warp(bar(B_D2EMPTY + d2));
-                }
-                if (row < args.N) {
+                for (int c0 = HF * CW2; c0 < (HF + 1) * CW2; c0 += LW2) {
+                    uint32_t r[LW2];
+                    tmem_load_n<LW2>(tmem + lane_addr + Cfg::TM_D2 + d2 * QS + c0, r);
+                    if (c0 + LW2 >= (HF + 1) * CW2) {
+                        tc_fence_before();
+                        mbar_arrive_warp(bar(B_D2EMPTY + d2));
+                    }
+                    if (row < args.N) {
 #pragma unroll
-                    for (int u0 = 0; u0 < 32; u0 += 8) {
-                        float bv[8];
+                        for (int u0 = 0; u0 < LW2; u0 += 8) {
+                            float bv[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int c = c0 + u0 + u;
-                            bv[u] = 0.f;
-                            if (args.bias && c < Q) {
-                                if constexpr (GE<T>::tf32) bv[u] = __ldg(bias32 + (size_t)c * M2 + k);
-                                else bv[u] = __bfloat162float(__ushort_as_bfloat16(
-                                         __ldg(bias16 + (size_t)c * M2 + k)));
+                            for (int u = 0; u < 8; ++u) {
+                                const int c = c0 + u0 + u;
+                                bv[u] = 0.f;
+                                if (args.bias && c < Q) {
+                                    if constexpr (GE<T>::tf32) bv[u] = __ldg(bias32 + (size_t)c * M2 + k);
+                                    else bv[u] = __bfloat162float(__ushort_as_bfloat16(
+                                             __ldg(bias16 + (size_t)c * M2 + k)));
+                                }
                             }
-                        }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int c = c0 + u0 + u;
-                            if (c < Q) {
-                                const float v = __uint_as_float(r[u0 + u]) + bv[u];
-                                const size_t o = obase + (size_t)c * M2;
-                                if constexpr (GE<T>::tf32) static_cast<float *>(args.y)[o] = v;
-                                else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
+                            for (int u = 0; u < 8; ++u) {
+                                const int c = c0 + u0 + u;
+                                if (c < Q) {
+                                    const float v = __uint_as_float(r[u0 + u]) + bv[u];
+                                    const size_t o = obase + (size_t)c * M2;
+                                    if constexpr (GE<T>::tf32) static_cast<float *>(args.y)[o] = v;
+                                    else static_cast<__nv_bfloat16 *>(args.y)[o] = __float2bfloat16_rn(v);
+                                }
                             }
                         }
                     }
                 }
             }
+        };
+        if (hf == 0) run(std::integral_constant<int, 0>{});
+        if constexpr (Cfg::H >= 2) {
+            if (hf == 1) run(std::integral_constant<int, 1>{});
+        }
+        if constexpr (Cfg::H == 4) {
+            if (hf == 2) run(std::integral_constant<int, 2>{});
+            if (hf == 3) run(std::integral_constant<int, 3>{});
         }
     }
 
