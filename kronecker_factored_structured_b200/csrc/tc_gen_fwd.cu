@@ -201,34 +201,53 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
     // T chunks start at zero: K positions past the chunk's ranks are never written
     zero_smem(sT, TBC * Cfg::TC_BYTES);
     // stage-2 B operand C'_b[c][kpos] = S[a][c] A_i[a][c] for rank i = b*IPB + i_local, with
-    // kpos = (a / AG) * (IPBE * AG) + i_local * AG + a % AG; zero past q, r and p
-    for (int e = threadIdx.x; e < MB1 * QP * (Cfg::K2P / VPC); e += blockDim.x) {
-        const int b = e / (QP * (Cfg::K2P / VPC));
-        const int rem = e % (QP * (Cfg::K2P / VPC));
-        const int c = rem / (Cfg::K2P / VPC), kp0 = (rem % (Cfg::K2P / VPC)) * VPC;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < VPC; ++t) {
-            const int kp = kp0 + t;
-            const int g = kp / (IPBE * AG), il = (kp % (IPBE * AG)) / AG;
-            const int a = g * AG + kp % AG, i = b * IPB + il;
-            float val = 0.f;
-            if (c < Q && a < P && i < R && kp < Cfg::K2) {
-                const size_t sa = TR ? (size_t)c * P + a : (size_t)a * Q + c;
-                const size_t aa = TR ? ((size_t)i * Q + c) * P + a : ((size_t)i * P + a) * Q + c;
-                val = ld_elt<T>(args.S, sa) * ld_elt<T>(args.A, aa);
+    // kpos = (a / AG) * (IPBE * AG) + i_local * AG + a % AG; zero past q, r and p.  One
+    // thread builds one 16-byte chunk (VPC consecutive kpos of one c); consecutive threads
+    // take the chunks whose factor reads are adjacent in memory: consecutive c (S and A
+    // rows run along c), or for TR consecutive a-groups (the transposed factors run along a)
+    {
+        constexpr int NCH = Cfg::K2P / VPC;               // chunks per (b, c)
+        constexpr int NGR = P / AG;                       // a-groups per rank
+#pragma unroll 2
+        for (int e = threadIdx.x; e < MB1 * QP * NCH; e += blockDim.x) {
+            int b, c, kp0;
+            if constexpr (!TR) {
+                b = e / (NCH * QP);
+                const int rem = e % (NCH * QP);
+                kp0 = (rem / QP) * VPC;
+                c = rem % QP;
+            } else {
+                b = e / (QP * NCH);
+                const int rem = e % (QP * NCH);
+                c = rem / NCH;
+                const int ch = rem % NCH, il = ch / NGR, g = ch % NGR;
+                // the chunks past IPBE * NGR are the zero padding of K (kpos >= K2)
+                kp0 = ch < IPBE * NGR ? (g * IPBE + il) * AG : ch * VPC;
             }
-            v[t] = val;
-        }
-        uint32_t w[4];
-        if constexpr (GE<T>::tf32) {
+            float v[8];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) w[t] = tf32_bits(v[t]);
-        } else {
+            for (int t = 0; t < VPC; ++t) {
+                const int kp = kp0 + t;
+                const int g = kp / (IPBE * AG), il = (kp % (IPBE * AG)) / AG;
+                const int a = g * AG + kp % AG, i = b * IPB + il;
+                float val = 0.f;
+                if (c < Q && a < P && i < R && kp < Cfg::K2) {
+                    const size_t sa = TR ? (size_t)c * P + a : (size_t)a * Q + c;
+                    const size_t aa = TR ? ((size_t)i * Q + c) * P + a : ((size_t)i * P + a) * Q + c;
+                    val = ld_elt<T>(args.S, sa) * ld_elt<T>(args.A, aa);
+                }
+                v[t] = val;
+            }
+            uint32_t w[4];
+            if constexpr (GE<T>::tf32) {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
+                for (int t = 0; t < 4; ++t) w[t] = tf32_bits(v[t]);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
+            }
+            st_shared_v4(sCP + b * Cfg::CP_BLK + kmaj(c, kp0 * E, QP, 128), w[0], w[1], w[2], w[3]);
         }
-        st_shared_v4(sCP + b * Cfg::CP_BLK + kmaj(c, kp0 * E, QP, 128), w[0], w[1], w[2], w[3]);
     }
     // zero-block mask: bit cb of mask[b*KS2 + ks] is set when S has a non-zero in the rows a
     // of K step ks of chunk b and the 16 columns c of block cb.  Every thread tests one
@@ -253,14 +272,18 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // stage-1 A operand in TMEM: block b, lane L = (i_local, k) holds B_i[j][k] along j
-    if (warp >= 4 && warp < 8) {
+    // stage-1 A operand in TMEM: block b, lane L = (i_local, k) holds B_i[j][k] along j.
+    // Warps 3-18 (four per TMEM lane quadrant) share the (block, 8-column group) items.
+    if (warp >= 3 && warp < 19) {
         const int L = (warp & 3) * 32 + lane, il = L / M2, k = L % M2;
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-        for (int b = 0; b < MB1; ++b) {
+        constexpr int NCG = Cfg::A1C / 8;
+#pragma unroll 2
+        for (int it = (warp - 3) >> 2; it < MB1 * NCG; it += 4) {
+            const int b = it / NCG, c0 = (it % NCG) * 8;
             const int i = b * IPB + il;
             const uint32_t ta = tmem + lane_addr + Cfg::TM_A1 + b * Cfg::A1C;
-            for (int c0 = 0; c0 < Cfg::A1C; c0 += 8) {
+            {
                 uint32_t w[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {

@@ -103,6 +103,7 @@ struct GPgCfg {
     static_assert(Q % 8 == 0, "dY tile rows of each n start on an 8-row atom");
     static_assert(XRB == 32 || XRB == 64 || XRB % 128 == 0, "x row bytes");
     static_assert(M1 % VPC == 0, "X^T copy");
+    static_assert((M1 * E / 4) % 8 == 0 && (QK * E / 4) % 8 == 0, "whole 8-column groups in TMEM");
     static_assert(NTN <= 256 && NUN <= 256 && QN <= 256 && M1N <= 256 && GBR <= 256, "MMA N / box");
     static_assert(KT2 % KSTEP == 0, "dC K steps");
     static_assert((Q * M2) % 128 == 0, "dbias: whole values per thread");
@@ -271,13 +272,20 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     // A operands in TMEM (zero for lanes past the group's ranks and for K past q):
     //   B_all^T block bt: lane (i,k) = (i0 + bt*IPT + L/m2, L%m2), column j -> B_i[j][k]
     //   C_stack block bu: lane (i,a) = (i0 + bu*IPU + L/p, L%p), column c -> S[a][c] A_i[a][c]
-    // (lanes in the paired order of pair_lane_index: the epilogue stores K pairs)
-    if (warp >= 3 && warp < 11) {
+    // (lanes in the paired order of pair_lane_index: the epilogue stores K pairs).  Warps
+    // 3-18 (four per TMEM lane quadrant) share the work: per quadrant two warps take the
+    // (block, 8-column group) items of B_all^T and two those of C_stack, so that many
+    // factor loads are in flight at once.
+    if (warp >= 3 && warp < 19) {
         const int qd = warp & 3, L = pair_lane_index(qd * 32 + lane);
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
-        const bool is_c = warp >= 7;
+        const int sub = (warp - 3) >> 2;
+        const bool is_c = sub >= 2;
         const int nblk = is_c ? MBU : MBT;
-        for (int blk = 0; blk < nblk; ++blk) {
+        const int ncg = (is_c ? Cfg::QK : M1) * E / 4 / 8;   // 8-column groups per block
+#pragma unroll 2
+        for (int it = sub & 1; it < nblk * ncg; it += 2) {
+            const int blk = it / ncg, c0 = (it % ncg) * 8;
             int i, o;
             bool valid;
             if (is_c) {
@@ -300,16 +308,13 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             };
             const uint32_t base = tmem + lane_addr + (is_c ? Cfg::TM_CS + blk * Cfg::CSC
                                                            : Cfg::TM_BT + blk * Cfg::BTC);
-            const int K = is_c ? Cfg::QK : M1;
-            for (int c0 = 0; c0 < K * E / 4; c0 += 8) {
-                uint32_t w[8];
+            uint32_t w[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if constexpr (GE<T>::tf32) w[u] = tf32_bits(val(c0 + u));
-                    else w[u] = pack_bf16x2(val(2 * (c0 + u)), val(2 * (c0 + u) + 1));
-                }
-                tmem_store8(base + c0, w);
+            for (int u = 0; u < 8; ++u) {
+                if constexpr (GE<T>::tf32) w[u] = tf32_bits(val(c0 + u));
+                else w[u] = pack_bf16x2(val(2 * (c0 + u)), val(2 * (c0 + u) + 1));
             }
+            tmem_store8(base + c0, w);
         }
     }
     tc_fence_before();
