@@ -270,7 +270,7 @@ def run_reference(args, w):
     return 0
 
 
-def dense_context(fac, sets, path, steps, dev):
+def dense_context(fac, sets, path, steps, dev, graph=False):
     """Context only (not the product path): the same layer as a dense x @ W + bias with W
     materialised (sum_i kron(S*A_i, B_i)), forward and backward (dX = dY W^T, dW = x^T dY,
     dbias) as three cuBLAS GEMMs through torch, timed like the Kronecker step (CUDA events
@@ -294,18 +294,22 @@ def dense_context(fac, sets, path, steps, dev):
         for i in range(3):
             step(i)
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for i in range(steps):
-            step(i)
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / steps
+        if graph:
+            ms = _time_graph(step, steps, REPEATS)[0] / steps
+        else:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for i in range(steps):
+                step(i)
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
     finally:
         torch.backends.cuda.matmul.allow_tf32 = old
     return {"what": "dense x @ W + bias forward and backward (dX, dW, dbias) with W "
                     "materialised, torch/cuBLAS, same inputs and timer; context only",
-            "matmul": "tf32" if path == "tf32" else path, "ms_per_step": ms}
+            "matmul": "tf32" if path == "tf32" else path, "ms_per_step": ms,
+            "timer": "CUDA graph replay" if graph else "eager steps between CUDA events"}
 
 
 REPEATS = 5  # repeats of each timed region; the median is reported (and the min)
@@ -392,6 +396,36 @@ def _time_region(step, steps, repeats, world, dist, stream, clk=None):
     return statistics.median(times), min(times), times
 
 
+def _time_graph(step, steps, repeats):
+    """Device time (ms) of `steps` steps captured once in a CUDA graph and replayed
+    `repeats` times between CUDA events (launch overhead excluded: the per-call host work
+    of the Python binding exceeds the device time of the small layers).  Returns (median,
+    min, all)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        step(0)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(steps):
+                step(i)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    del g
+    return statistics.median(times), min(times), times
+
+
 def _split_calls(step, steps, stream):
     """Mean forward and backward call times (ms) from per-call events over `steps` steps
     (outside any timed region: the extra event records do not enter a reported value)."""
@@ -454,23 +488,36 @@ def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
         w = dataclasses.replace(w, dtype="bf16")
     rotate = ROTATE if w.N * (w.d_in + w.d_out) * (2 if path == "bf16" else 4) < 126e6 else 1
     pr = _Problem(kw, kfs, w, path, dev, rotate=rotate)
-    grads = {"dX": torch.empty(w.N, w.d_in, dtype=pr.y.dtype, device=dev)}
+    f32 = torch.float32
+    grads = {"dX": torch.empty(w.N, w.d_in, dtype=pr.y.dtype, device=dev),
+             "dS": torch.empty(w.p, w.q, dtype=f32, device=dev),
+             "dA": torch.empty(w.r, w.p, w.q, dtype=f32, device=dev),
+             "dB": torch.empty(w.r, w.m1, w.m2, dtype=f32, device=dev),
+             "dbias": torch.empty(w.d_out, dtype=f32, device=dev)}
     step = _make_step(kfs, pr, flags, stream, grads)
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    med, mn, _ = _time_region(step, steps, REPEATS, 1, None, stream)
+    # the leg's figure: the steps replayed from one CUDA graph (device time); the same
+    # steps issued eagerly from Python are reported beside it
+    med, mn, _ = _time_graph(step, steps, REPEATS)
+    med_e, _, _ = _time_region(step, steps, REPEATS, 1, None, stream)
     t_fwd, t_bwd = _split_calls(step, steps, stream)
     ms = med / steps
     leg = {"workload": _workload_desc(w), "name": name, "path": path, "flags": flags,
-           "N": w.N, "steps": steps, "repeats": REPEATS, "ms_per_step": ms,
-           "ms_per_step_min": mn / steps, "rows_per_s": w.N / (ms / 1e3),
-           "fwd_ms": t_fwd, "bwd_ms": t_bwd,
+           "N": w.N, "steps": steps, "repeats": REPEATS, "timer": "CUDA graph replay of the steps",
+           "ms_per_step": ms, "ms_per_step_min": mn / steps, "rows_per_s": w.N / (ms / 1e3),
+           "ms_per_step_eager": med_e / steps,
+           "fwd_ms": t_fwd, "bwd_ms": t_bwd, "call_split_timer": "eager, per-call events",
            "l2": f"{len(pr.sets)} input set(s), "
                  f"{len(pr.sets) * w.N * (w.d_in + w.d_out) * (2 if path == 'bf16' else 4) / 1e6:.0f} MB",
            "roofline": _step_roofline(w, path, ms, peaks, flags)}
     if note:
         leg["note"] = note
+    if name.startswith("gpt2"):
+        ctx = dense_context(pr.fac, pr.sets, path, steps, dev, graph=True)
+        ctx["kron_speedup"] = ctx["ms_per_step"] / ms
+        leg["context_dense"] = ctx
     del pr, grads
     torch.cuda.empty_cache()
     return leg
@@ -563,6 +610,8 @@ def main():
         ms_med, ms_min, ms_all = _time_region(step, args.steps, REPEATS, world, dist, stream, clk)
     # ---- the split into forward and backward call (outside the timed region) ----
     t_fwd, t_bwd = _split_calls(step, args.steps, stream)
+    # ---- for information (one GPU): the same steps replayed from one CUDA graph ----
+    graph_ms = _time_graph(step, args.steps, REPEATS)[0] / args.steps if world == 1 else None
     ms_step = ms_med / args.steps
     value = world * N * args.steps / (ms_med / 1e3)
 
@@ -644,6 +693,10 @@ def main():
         "repeats": {"n": REPEATS, "ms_per_step": [t / args.steps for t in ms_all],
                     "median": ms_step, "min": ms_min / args.steps},
         "fwd_ms": t_fwd, "bwd_ms": t_bwd,
+        "graph": None if graph_ms is None else {
+            "ms_per_step": graph_ms, "rows_per_s": N / (graph_ms / 1e3),
+            "what": "the same steps captured once in a CUDA graph and replayed (information; "
+                    "value is the eager figure, the same at every GPU count)"},
         "tflops": step_flops / (ms_step / 1e3) / 1e12,
         "gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "step_roofline_frac_hbm": (step_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms_step / 1e3),
