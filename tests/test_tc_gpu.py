@@ -46,6 +46,24 @@ def test_tc_tutorial_full_size(path):
 
 
 @pytest.mark.parametrize("path", ["tf32", "bf16"])
+def test_tc_no_bias_full_size(path):
+    """N = 20000 with no bias: the forward without a bias vector, and the backward with
+    neither dbias nor anything bias-related requested; every element of y, dX, dS, dA and
+    dB against the oracle's bias-free layer."""
+    import kronecker_factored_structured_b200 as kfs
+    w = _w(path)
+    d = {k: v.cuda() for k, v in _inputs(w).items()}
+    y = kfs.forward(d["x"], d["S"], d["A"], d["B"], None, dtype=path)
+    g = kfs.backward(d["x"], d["S"], d["A"], d["B"], d["G"], dtype=path, need_dbias=False)
+    torch.cuda.synchronize()
+    assert g["dbias"] is None
+    got = {"y": to_np(y)}
+    got.update({k: to_np(v) for k, v in g.items() if v is not None})
+    ref = oracle_run(_inputs(w), with_bias=False)
+    compare(got, ref, path, keys=("y", "dX", "dS", "dA", "dB"))
+
+
+@pytest.mark.parametrize("path", ["tf32", "bf16"])
 def test_tc_s_all_ones_and_dense_zeroes(path):
     """S with no zeros, and S with 90% zeros (dS still exact where S = 0)."""
     for zeros in (0, 922):
