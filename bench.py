@@ -35,8 +35,8 @@ UNIT = "rows/s"
 # SHA-256 prefix is recorded with it: any later change to them makes the figure null.  The
 # write counters miss the part of dX still in L2 when the kernel ends.
 _TRAFFIC = {
-    "tf32": (81.99e6 + 27.67e6 + 164.00e6 + 0.49e6, "2a3c3f2e3bfd9354"),
-    "bf16": (41.01e6 + 0.27e6 + 82.00e6 + 0.37e6, "2a3c3f2e3bfd9354"),
+    "tf32": (81.99e6 + 27.45e6 + 163.99e6 + 0.41e6, "5e81ef99b607a192"),
+    "bf16": (41.01e6 + 0.16e6 + 82.00e6 + 0.09e6, "5e81ef99b607a192"),
 }
 
 
@@ -468,6 +468,32 @@ LEGS = [("tutorial", "f32", 0), ("tutorial", "bf16", 0),
        [(f"sweep_m{m}_r{r}", None, 0) for m in (8, 16, 64, 128) for r in (1, 2, 8)]
 
 
+def _tc_forward_leg(kfs, pr, w, steps, peaks):
+    """TF32 forward call alone on the fp32 tensors of `pr`, replayed from a CUDA graph;
+    None when the library has no TF32 forward kernel for the shape."""
+    fac = pr.fac
+
+    def fwd(i):
+        x, _ = pr.sets[i % len(pr.sets)]
+        kfs.forward(x, fac["S"], fac["A"], fac["B"], fac["bias"], dtype="tf32", out=pr.y)
+    try:
+        fwd(0)
+    except kfs.KronError:
+        return None
+    med, mn, _ = _time_graph(fwd, steps, REPEATS)
+    ms = med / steps
+    nbytes = w.N * 4 * (w.d_in + w.d_out)
+    flops = w.N * 2 * w.r * (w.p * w.m1 * w.m2 + w.p * w.q * w.m2)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_fl = flops / (peaks["bf16_tflops"] * 1e12 / 2)
+    t_roof = max(t_hbm, t_fl)
+    return {"path": "tf32", "ms_per_call": ms, "ms_per_call_min": mn / steps,
+            "timer": "CUDA graph replay", "roofline": {
+                "bound": "hbm" if t_hbm >= t_fl else "tensor", "roofline_us": t_roof * 1e6,
+                "hbm_us": t_hbm * 1e6, "flops_us": t_fl * 1e6, "frac": t_roof / (ms / 1e3),
+                "flop_peak": "tf32 (measured bf16 x 1/2)", "bytes": nbytes, "flops": flops}}
+
+
 def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
     """One further leg: the workload's forward + backward step, median of REPEATS timed
     regions of `steps` steps; a dict for the JSON line's "legs" list."""
@@ -514,6 +540,12 @@ def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
            "roofline": _step_roofline(w, path, ms, peaks, flags)}
     if note:
         leg["note"] = note
+    if note and path == "f32":
+        # the step runs exact FP32; where the TF32 forward has a tensor-core kernel for the
+        # shape, its forward call is timed alone the same way, against the forward roofline
+        fwd_tc = _tc_forward_leg(kfs, pr, w, steps, peaks)
+        if fwd_tc is not None:
+            leg["forward_tf32"] = fwd_tc
     if name.startswith("gpt2"):
         ctx = dense_context(pr.fac, pr.sets, path, steps, dev, graph=True)
         ctx["kron_speedup"] = ctx["ms_per_step"] / ms
