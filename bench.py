@@ -494,6 +494,66 @@ def _tc_forward_leg(kfs, pr, w, steps, peaks):
                 "flop_peak": "tf32 (measured bf16 x 1/2)", "bytes": nbytes, "flops": flops}}
 
 
+def run_extras(kfs, steps, dev):
+    """The two utilities built around the layer, timed on one GPU (rank 0):
+    - the Van Loan rank-r fit of a dense W of the GPT-2 c_fc shape (768 x 3072, C_i 24 x 48,
+      B_i 32 x 64) that is an exact sum of 4 Kronecker products, r = 4, k = 12, two power steps:
+      time per fit (CUDA events around back-to-back fits) and the fit's relative Frobenius
+      error (exact rank: rounding only);
+    - the triple Kronecker layer with A 32 x 32, B 4 x 4, C 8 x 8, r = 4 (blocks of 32 x 32, the
+      tutorial layer's tensor-core kernels) on 20000 rows, TF32: forward + backward step time
+      from a CUDA-graph replay."""
+    import torch
+    from kronecker_factored_structured_b200 import native
+    out = {}
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    p, q, m1, m2, r = 24, 48, 32, 64, 4
+    C = torch.randn(r, p, q, device=dev, generator=g) / p ** 0.5
+    B = torch.randn(r, m1, m2, device=dev, generator=g) / m1 ** 0.5
+    W = sum(torch.kron(C[i], B[i]) for i in range(r)).float().contiguous()
+    omega = torch.randn(12, m1 * m2, device=dev, generator=g)
+    fit = native.vanloan_fit(W, p, q, m1, m2, r, k=12, omega=omega)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(REPEATS):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(10):
+            fit = native.vanloan_fit(W, p, q, m1, m2, r, k=12, omega=omega)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) / 10)
+    Wf = sum(torch.kron(fit["A"][i], fit["B"][i]) for i in range(r))
+    out["vanloan"] = {"what": "kron_vanloan_fit of a 768 x 3072 W of Kronecker rank 4 "
+                              "(GPT-2 c_fc factor shapes), r = 4, k = 12, 2 power steps",
+                      "ms_per_fit": statistics.median(times),
+                      "rel_frobenius_error": float((Wf - W).norm() / W.norm()),
+                      "alpha": float(fit["alpha"][0])}
+    del W, Wf, fit, omega, C, B
+    N, p, q, m1, m2, s1, s2, r = 20000, 32, 32, 4, 4, 8, 8, 4
+    A3 = torch.randn(r, p, q, device=dev, generator=g) / p ** 0.5
+    B3 = torch.randn(r, m1, m2, device=dev, generator=g) / m1 ** 0.5
+    C3 = torch.randn(r, s1, s2, device=dev, generator=g) / s1 ** 0.5
+    bias = 0.1 * torch.randn(q * m2 * s2, device=dev, generator=g)
+    xs = [torch.randn(N, p * m1 * s1, device=dev, generator=g) for _ in range(ROTATE)]
+    Gs = [torch.randn(N, q * m2 * s2, device=dev, generator=g) for _ in range(ROTATE)]
+
+    def step(i):
+        native.forward3(xs[i % ROTATE], A3, B3, C3, bias, dtype="tf32")
+        native.backward3(xs[i % ROTATE], A3, B3, C3, Gs[i % ROTATE], dtype="tf32")
+    step(0)
+    torch.cuda.synchronize()
+    med, _, _ = _time_graph(step, steps, REPEATS)
+    ms = med / steps
+    out["kron3"] = {"what": "triple Kronecker layer, A 32x32, B 4x4, C 8x8, r = 4, N = 20000, "
+                            "TF32, forward + backward (CUDA-graph replay)",
+                    "ms_per_step": ms, "rows_per_s": N / (ms / 1e3)}
+    del xs, Gs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
     """One further leg: the workload's forward + backward step, median of REPEATS timed
     regions of `steps` steps; a dict for the JSON line's "legs" list."""
@@ -755,6 +815,7 @@ def main():
             legs.append(run_leg(kw, kfs, name, lpath, lflags, max(3, min(args.steps, args.leg_steps)),
                                 args.warmup, peaks, dev, stream))
         line["legs"] = legs
+        line["extras"] = run_extras(kfs, max(3, min(args.steps, args.leg_steps)), dev)
     if world == 1 and not args.no_cpu_baseline:
         cpu_rows = args.cpu_rows or (N if N * (w.d_in + w.d_out) <= 20000 * 2048 else 1024)
         rows_s, dt, cores = cpu_baseline(w, cpu_rows)

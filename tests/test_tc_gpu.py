@@ -60,7 +60,8 @@ def test_tc_no_bias_full_size(path):
     got = {"y": to_np(y)}
     got.update({k: to_np(v) for k, v in g.items() if v is not None})
     ref = oracle_run(_inputs(w), with_bias=False)
-    compare(got, ref, path, keys=("y", "dX", "dS", "dA", "dB"))
+    errs = compare(got, ref, path, keys=("y", "dX", "dS", "dA", "dB"))
+    print(path, "no bias", errs)
 
 
 @pytest.mark.parametrize("path", ["tf32", "bf16"])
