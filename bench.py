@@ -169,11 +169,17 @@ class ClockSampler:
 
     def begin_region(self):
         self.nvml = _NvmlRegion(torch_current_device())
+        # the launching thread holds the interpreter lock between library calls; a short
+        # switch interval lets the sampler thread take its 2 ms samples on time
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0002)
         self.nvml.start()
 
     def end_region(self):
         if getattr(self, "nvml", None) is not None:
             self.nvml.stop()
+        if getattr(self, "_switch", None) is not None:
+            sys.setswitchinterval(self._switch)
 
     def wait_started(self, timeout=5.0):
         """Block until nvidia-smi has printed its first sample (it takes ~0.5 s to start)."""
