@@ -461,16 +461,45 @@ kron_pgrad_gen_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                     const bool valid = (is_t || nat < IPU * P) && ir < rgv;
                     const uint32_t dst = dstb + (is_t ? (ir / IPU) * Cfg::T2_BLK : (ir / IPT) * Cfg::U2_BLK);
                     const int rbase = is_t ? (ir % IPU) * P : (ir % IPT) * M2;   // a multiple of 8
-#pragma unroll
-                    for (int rp = 0; rp < 4; ++rp) {
+                    if constexpr (NT == 1) {
+                        // one row per tile: column c of the task is row rbase + c at the fixed K
+                        // byte kb of this thread.  In the 128-byte swizzle the row's low three
+                        // bits, w = 2(t%4) + dl, pick the 16-byte chunk kb/16 XOR w: two offsets
+                        // per thread, and each 8-row group rp adds 1 KB.  Groups past the task's
+                        // columns (c >= p or m2) are dropped at compile time.
+                        const int kb = own * E;
+                        const uint32_t base = dst + (uint32_t)(kb >> 7) * 128 * 128 +
+                                              (uint32_t)((rbase >> 3) + cg * 4) * 1024 + (uint32_t)(kb & 15);
+                        const uint32_t c16 = (uint32_t)(kb >> 4) & 7u;
+                        uint32_t off[2];
 #pragma unroll
                         for (int dl = 0; dl < 2; ++dl) {
-                            const int c = cg * 32 + rp * 8 + (lane & 3) * 2 + dl;
-                            if (valid && c < NT * CW) {
-                                const int n = c / CW, row = rbase + c % CW;
-                                st_shared_u32(dst + kmaj(row, (n * KW + own) * E, 128, 128),
-                                              pack_bf16x2(__uint_as_float(r[4 * rp + dl]),
-                                                          __uint_as_float(r[4 * rp + 2 + dl])));
+                            const uint32_t w = (uint32_t)((lane & 3) * 2 + dl);
+                            off[dl] = w * 128 + ((c16 ^ w) << 4);
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int rp = 0; rp < 4; ++rp) {
+                                if (cg * 32 + rp * 8 >= CW) continue;
+#pragma unroll
+                                for (int dl = 0; dl < 2; ++dl)
+                                    st_shared_u32(base + off[dl] + rp * 1024,
+                                                  pack_bf16x2(__uint_as_float(r[4 * rp + dl]),
+                                                              __uint_as_float(r[4 * rp + 2 + dl])));
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int rp = 0; rp < 4; ++rp) {
+#pragma unroll
+                            for (int dl = 0; dl < 2; ++dl) {
+                                const int c = cg * 32 + rp * 8 + (lane & 3) * 2 + dl;
+                                if (valid && c < NT * CW) {
+                                    const int n = c / CW, row = rbase + c % CW;
+                                    st_shared_u32(dst + kmaj(row, (n * KW + own) * E, 128, 128),
+                                                  pack_bf16x2(__uint_as_float(r[4 * rp + dl]),
+                                                              __uint_as_float(r[4 * rp + 2 + dl])));
+                                }
                             }
                         }
                     }
