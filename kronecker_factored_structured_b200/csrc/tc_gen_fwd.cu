@@ -109,6 +109,9 @@ struct GFwdCfg {
     static constexpr int GPW = cdiv(NG1, NW1);            // D1 column groups of one warp
     static constexpr int CW2 = QS / H;                     // D2 columns of one warp
     static constexpr int LW2 = gmin(CW2, 32);              // columns per TMEM load
+    // one epilogue-2 warp per quadrant over a whole number of 32-column loads: the column
+    // loop is unrolled (measured: stress forward 157 -> 152 us)
+    static constexpr bool E2_UNROLL = H == 1 && Q % 32 == 0;
 
     static_assert(128 % M2 == 0 && M2 % 16 == 0, "m2 divides 128 (stage-2 M = 128)");
     static_assert(N1P <= 256, "stage-1 N = (128/m2)*p at most 256");
@@ -499,11 +502,14 @@ kron_fwd_gen_kernel(const __grid_constant__ CUtensorMap tmap_x, GFwdArgs args) {
                 tc_fence_after();
                 const int64_t row = (int64_t)(blockIdx.x + t * gridDim.x) * NT + n;
                 const size_t obase = (size_t)row * (Q * M2) + k;
-#pragma unroll 1
-                for (int c0 = HF * CW2; c0 < (HF + 1) * CW2; c0 += LW2) {
+                // the column loop: unrolled over the q real columns with one warp per quadrant
+                // (E2_UNROLL), else a loop over this warp's share, padding columns skipped
+                constexpr int C_END = Cfg::E2_UNROLL ? Q : (HF + 1) * CW2;
+#pragma unroll(Cfg::E2_UNROLL ? 8 : 1)
+                for (int c0 = HF * CW2; c0 < C_END; c0 += LW2) {
                     uint32_t r[LW2];
                     tmem_load_n<LW2>(tmem + lane_addr + Cfg::TM_D2 + d2 * QS + c0, r);
-                    if (c0 + LW2 >= (HF + 1) * CW2) {
+                    if (c0 + LW2 >= C_END) {
                         tc_fence_before();
                         mbar_arrive_warp(bar(B_D2EMPTY + d2));
                     }
