@@ -11,6 +11,14 @@ B_i ~ randn/sqrt(m), bias zeros) and the GPT-2 small FFN shapes of the page
 "LLM Compression via Kronecker Product Decomposition" (section "Factor
 Dimensions for GPT-2", c_fc 768->3072 and c_proj 3072->768).
 
+The Kronecker-sparse factors (page "Fast Inference with Kronecker-Sparse
+Matrices": supports kron(I_a, kron(1_{b x c}, I_d)), the factors of Monarch and
+butterfly matrices; the page reports FP32 runs and end-to-end ViT-S/16 and GPT-2
+medium models) get ``KSWorkload`` entries: the two factors of a 1024 x 1024
+Monarch matrix and one radix-2 butterfly factor on the tutorial's 20000 rows, a
+1024 -> 4096 factor at GPT-2 medium's width on 8 x 1024 tokens, and a factor of
+large 128 x 128 blocks.  Values ~ randn/sqrt(b) (each output sums b inputs).
+
 Large row tensors are drawn in fixed chunks of rows, each chunk from its own
 generator seeded by (seed, tensor tag, chunk index), so any subset of rows can
 be re-drawn on the CPU without materialising the whole tensor.
@@ -96,6 +104,71 @@ def all_workloads() -> dict:
 
 def get(name: str) -> Workload:
     return all_workloads()[name]
+
+
+@dataclasses.dataclass(frozen=True)
+class KSWorkload:
+    """One Kronecker-sparse factor of pattern (a, b, c, d): x [N][a*b*d] -> y [N][a*c*d]."""
+    name: str
+    N: int
+    a: int
+    b: int
+    c: int
+    d: int
+    seed: int
+    dtype: str = "f32"
+    x_std: float = 1.0
+    g_std: float = 1.0
+    bias_std: float = 0.1
+
+    @property
+    def pattern(self):
+        return (self.a, self.b, self.c, self.d)
+
+    @property
+    def d_in(self) -> int:
+        return self.a * self.b * self.d
+
+    @property
+    def d_out(self) -> int:
+        return self.a * self.c * self.d
+
+    def with_rows(self, N: int) -> "KSWorkload":
+        return dataclasses.replace(self, N=N, name=f"{self.name}@N{N}")
+
+
+def ks_workloads() -> dict:
+    w = {}
+    for name, N, pat in (("ks_monarch_bd", 20000, (32, 32, 32, 1)),
+                         ("ks_monarch_tr", 20000, (1, 32, 32, 32)),
+                         ("ks_butterfly", 20000, (16, 2, 2, 32)),
+                         ("ks_gpt2m_up", 8192, (1, 32, 128, 32)),
+                         ("ks_block128", 20000, (8, 128, 128, 1))):
+        w[name] = KSWorkload(name=name, N=N, a=pat[0], b=pat[1], c=pat[2], d=pat[3], seed=6)
+    return w
+
+
+def ks_get(name: str) -> KSWorkload:
+    return ks_workloads()[name]
+
+
+def ks_custom(N, a, b, c, d, seed=0) -> KSWorkload:
+    return KSWorkload(name=f"ks_N{N}_{a}x{b}x{c}x{d}", N=N, a=a, b=b, c=c, d=d, seed=seed)
+
+
+def ks_factors(w: KSWorkload) -> dict:
+    """Values w [a][d][b][c] ~ randn/sqrt(b) and bias ~ N(0, bias_std^2) (CPU float32)."""
+    g = _gen(w.seed, 2, w.a, w.b, w.c, w.d)
+    vals = torch.randn(w.a, w.d, w.b, w.c, generator=g) / math.sqrt(w.b)
+    bias = torch.randn(w.d_out, generator=g) * w.bias_std
+    return {"w": vals, "bias": bias}
+
+
+def ks_inputs(w: KSWorkload) -> dict:
+    d = ks_factors(w)
+    d["x"] = rows(w, "x")
+    d["G"] = rows(w, "G")
+    return d
 
 
 def custom(N, p, q, m1, m2, r, dtype="f32", seed=0, s_zero_entries=0, **kw) -> Workload:

@@ -10,7 +10,9 @@ page "kronecker-layer-benchmark", section "1. Build W, then multiply" defines
 the layer; the backward is the chain rule through that explicit W.  This module
 only marshals numpy arrays into that library, except for the Van Loan fit,
 whose SVD step is numpy's (a library routine serving as one step of the
-algorithm as the page gives it).
+algorithm as the page gives it).  The same library holds the Kronecker-sparse
+factor of the page "Fast Inference with Kronecker-Sparse Matrices" (its dense
+matrix built entry by entry from the pattern, then the same naive multiply).
 """
 from __future__ import annotations
 
@@ -72,6 +74,9 @@ class Oracle:
         lib.oracle_forward3.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, I, I, dp]
         lib.oracle_backward3.argtypes = [dp, dp, dp, dp, dp, L, I, I, I, I, I, I, I,
                                          dp, dp, dp, dp, dp]
+        lib.oracle_ks_build.argtypes = [dp, I, I, I, I, dp]
+        lib.oracle_ks_forward.argtypes = [dp, dp, dp, L, I, I, I, I, dp]
+        lib.oracle_ks_backward.argtypes = [dp, dp, dp, L, I, I, I, I, dp, dp, dp]
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_get_threads.restype = I
         self._lib = lib
@@ -209,6 +214,48 @@ class Oracle:
         return {"dX": dX, "dA": dA, "dB": dB, "dC": dC, "dbias": dbias}
 
 
+    # ---- Kronecker-sparse factor: support kron(I_a, kron(1_{b x c}, I_d)) ----
+    @staticmethod
+    def _ks_pattern(w):
+        if w.ndim != 4:
+            raise ValueError("w must have shape (a, d, b, c)")
+        a, d, b, c = w.shape
+        return a, b, c, d
+
+    def ks_dense(self, w) -> np.ndarray:
+        """Dense KS matrix K ((a*b*d) x (a*c*d)) of the values w [a][d][b][c]:
+        K[(al*b + be)*d + de][(al*c + ga)*d + de] = w[al][de][be][ga], zero elsewhere."""
+        w = _f64(w)
+        a, b, c, d = self._ks_pattern(w)
+        K = np.empty((a * b * d, a * c * d))
+        self._lib.oracle_ks_build(_ptr(w), a, b, c, d, _ptr(K))
+        return K
+
+    def ks_forward(self, x, w, bias=None) -> np.ndarray:
+        """y = x K + bias for x of shape (N, a*b*d); returns (N, a*c*d)."""
+        x, w = _f64(x), _f64(w)
+        a, b, c, d = self._ks_pattern(w)
+        N = x.shape[0]
+        if x.shape != (N, a * b * d):
+            raise ValueError(f"x has shape {x.shape}, expected (N, {a * b * d})")
+        bias = None if bias is None else _f64(bias)
+        y = np.empty((N, a * c * d))
+        self._lib.oracle_ks_forward(_ptr(x), _ptr(w), _ptr(bias), N, a, b, c, d, _ptr(y))
+        return y
+
+    def ks_backward(self, x, w, G) -> dict:
+        """Gradients of <G, y>: dict(dX, dw, dbias)."""
+        x, w, G = _f64(x), _f64(w), _f64(G)
+        a, b, c, d = self._ks_pattern(w)
+        N = x.shape[0]
+        if x.shape != (N, a * b * d) or G.shape != (N, a * c * d):
+            raise ValueError("x / G shapes do not match the pattern")
+        dX, dw, dbias = np.empty_like(x), np.empty_like(w), np.empty(a * c * d)
+        self._lib.oracle_ks_backward(_ptr(x), _ptr(w), _ptr(G), N, a, b, c, d, _ptr(dX),
+                                     _ptr(dw), _ptr(dbias))
+        return {"dX": dX, "dw": dw, "dbias": dbias}
+
+
 _default = None
 
 
@@ -261,3 +308,15 @@ def forward3(x, A, B, C, bias=None) -> np.ndarray:
 
 def backward3(x, A, B, C, G) -> dict:
     return default().backward3(x, A, B, C, G)
+
+
+def ks_dense(w) -> np.ndarray:
+    return default().ks_dense(w)
+
+
+def ks_forward(x, w, bias=None) -> np.ndarray:
+    return default().ks_forward(x, w, bias)
+
+
+def ks_backward(x, w, G) -> dict:
+    return default().ks_backward(x, w, G)

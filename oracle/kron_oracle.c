@@ -339,3 +339,77 @@ void oracle_backward3(const double *x, const double *A, const double *B, const d
     free(W);
     free(dW);
 }
+
+/*
+ * Kronecker-sparse (KS) factor (page "Fast Inference with Kronecker-Sparse Matrices",
+ * abstract): a matrix whose support is a Kronecker product of identity and all-ones blocks.
+ * Pattern (a, b, c, d) names the support kron(I_a, kron(1_{b x c}, I_d)) of an
+ * (a*b*d) x (a*c*d) matrix K, used here as the weight of y = x K + bias.  Its a*b*c*d free
+ * entries are the values w [a][d][b][c]:
+ *
+ *     K[(al*b + be)*d + de][(al*c + ga)*d + de] = w[al][de][be][ga],   zero elsewhere.
+ *
+ * The oracle builds K entry by entry and multiplies naively (oracle_matmul_bias); the
+ * backward is the chain rule through that explicit K:
+ *     dX = G K^T,   dK = x^T G,   dw[al][de][be][ga] = dK at the entry w fills,
+ *     dbias = sum_n G[n].
+ * x [N][a*b*d], y and G [N][a*c*d], bias [a*c*d].
+ */
+void oracle_ks_build(const double *w, int a, int b, int c, int d, double *K)
+{
+    const long in = (long)a * b * d, out = (long)a * c * d;
+    memset(K, 0, sizeof(double) * (size_t)in * out);
+    for (int al = 0; al < a; ++al)
+        for (int de = 0; de < d; ++de)
+            for (int be = 0; be < b; ++be)
+                for (int ga = 0; ga < c; ++ga)
+                    K[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + de] =
+                        w[(((long)al * d + de) * b + be) * c + ga];
+}
+
+void oracle_ks_forward(const double *x, const double *w, const double *bias, long N, int a,
+                       int b, int c, int d, double *y)
+{
+    const long in = (long)a * b * d, out = (long)a * c * d;
+    double *K = (double *)malloc(sizeof(double) * (size_t)in * out);
+    oracle_ks_build(w, a, b, c, d, K);
+    oracle_matmul_bias(x, K, bias, N, in, out, y);
+    free(K);
+}
+
+void oracle_ks_backward(const double *x, const double *w, const double *G, long N, int a, int b,
+                        int c, int d, double *dX, double *dw, double *dbias)
+{
+    const long in = (long)a * b * d, out = (long)a * c * d;
+    double *K = (double *)malloc(sizeof(double) * (size_t)in * out);
+    double *dK = (double *)calloc((size_t)in * out, sizeof(double));
+    oracle_ks_build(w, a, b, c, d, K);
+    /* dX = G K^T */
+#pragma omp parallel for
+    for (long n = 0; n < N; ++n)
+        for (long u = 0; u < in; ++u) {
+            double s = 0.0;
+            for (long o = 0; o < out; ++o) s += G[n * out + o] * K[u * out + o];
+            dX[n * in + u] = s;
+        }
+    /* dK = x^T G */
+#pragma omp parallel for
+    for (long u = 0; u < in; ++u)
+        for (long n = 0; n < N; ++n) {
+            const double xv = x[n * in + u];
+            for (long o = 0; o < out; ++o) dK[u * out + o] += xv * G[n * out + o];
+        }
+    for (int al = 0; al < a; ++al)
+        for (int de = 0; de < d; ++de)
+            for (int be = 0; be < b; ++be)
+                for (int ga = 0; ga < c; ++ga)
+                    dw[(((long)al * d + de) * b + be) * c + ga] =
+                        dK[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + de];
+    for (long o = 0; o < out; ++o) {
+        double s = 0.0;
+        for (long n = 0; n < N; ++n) s += G[n * out + o];
+        dbias[o] = s;
+    }
+    free(K);
+    free(dK);
+}

@@ -18,7 +18,12 @@ Sources of truth used here (none of them is the oracle's own loop):
     single parameter coordinate), and Euler's identity for functions that are
     linear in one argument,
   * for the l1 penalty lam * sum|S| on S: central differences away from the kink at
-    0, and torch's autograd of abs() for the value taken at S = 0.
+    0, and torch's autograd of abs() for the value taken at S = 0,
+  * for the Kronecker-sparse factor (page "Fast Inference with Kronecker-Sparse
+    Matrices", abstract: supports that are Kronecker products of identity and all-ones
+    blocks): its support against numpy's kron of eye and ones, scipy's block_diag and
+    hadamard, numpy's kron for tied values, and the two-factor Kronecker layer as a
+    product of two KS factors.
 """
 from __future__ import annotations
 
@@ -424,6 +429,137 @@ def pin_kron3_finite_differences(orc):
             assert abs(num - g[grad][idx]) <= 1e-7 * max(1.0, abs(num)), (key, idx)
 
 
+# ---- Kronecker-sparse factor (pattern (a, b, c, d), values w [a][d][b][c]) ----
+
+KS_PATTERNS = [(2, 3, 4, 5), (1, 4, 2, 3), (3, 2, 5, 1), (2, 1, 1, 3), (1, 3, 3, 1), (4, 2, 2, 2)]
+
+
+def _ks_values(rng, a, b, c, d):
+    """Values bounded away from zero, so the support shows in K != 0."""
+    return rng.uniform(0.5, 1.5, (a, d, b, c)) * rng.choice([-1.0, 1.0], (a, d, b, c))
+
+
+def pin_ks_support_is_kron_of_identity_and_ones(orc):
+    """supp K = kron(I_a, kron(1_{b x c}, I_d)) (numpy's kron of eye and ones), K is
+    (a*b*d) x (a*c*d) and holds exactly a*b*c*d non-zeros, each value once."""
+    rng = np.random.default_rng(401)
+    for a, b, c, d in KS_PATTERNS:
+        w = _ks_values(rng, a, b, c, d)
+        K = orc.ks_dense(w)
+        mask = np.kron(np.eye(a), np.kron(np.ones((b, c)), np.eye(d)))
+        assert K.shape == mask.shape == (a * b * d, a * c * d)
+        assert np.array_equal(K != 0, mask != 0), (a, b, c, d)
+        assert np.array_equal(np.sort(K[K != 0]), np.sort(w.ravel()))
+
+
+def pin_ks_block_diagonal(orc):
+    """d = 1: K is block-diagonal with the a blocks w[al][0] (scipy's block_diag)."""
+    from scipy.linalg import block_diag
+    rng = np.random.default_rng(403)
+    for a, b, c in ((3, 2, 4), (1, 5, 3), (4, 3, 3)):
+        w = rng.standard_normal((a, 1, b, c))
+        assert np.array_equal(orc.ks_dense(w), block_diag(*[w[i, 0] for i in range(a)]))
+
+
+def pin_ks_diagonal(orc):
+    """b = c = 1: K = diag(w) with the values in (al, de) order (numpy's diag)."""
+    rng = np.random.default_rng(409)
+    w = rng.standard_normal((3, 4, 1, 1))
+    assert np.array_equal(orc.ks_dense(w), np.diag(w.reshape(12)))
+
+
+def pin_ks_tied_values_are_numpy_kron(orc):
+    """All a*d blocks equal to one rectangular M: K = kron(I_a, kron(M, I_d)); in particular
+    a = 1 gives kron(M, I_d) and d = 1 gives kron(I_a, M) (numpy's kron)."""
+    rng = np.random.default_rng(419)
+    for a, b, c, d in ((1, 3, 2, 4), (3, 2, 4, 1), (2, 3, 2, 3)):
+        M = rng.standard_normal((b, c))
+        w = np.broadcast_to(M, (a, d, b, c))
+        ref = np.kron(np.eye(a), np.kron(M, np.eye(d)))
+        assert np.array_equal(orc.ks_dense(w), ref), (a, b, c, d)
+
+
+def pin_ks_chain_is_kronecker_layer(orc):
+    """The vec trick as two KS factors: x -> KS(p, m1, m2, 1) with every block B_i, then
+    KS(1, p, q, m2) with every block C_i, summed over i, equals x kron(C_i, B_i) summed over
+    i (numpy's kron) -- the two-factor layer's W with S = ones."""
+    rng = np.random.default_rng(421)
+    p, q, m1, m2, r, N = 3, 2, 2, 4, 2, 5
+    C = rng.standard_normal((r, p, q))
+    B = rng.standard_normal((r, m1, m2))
+    x = rng.standard_normal((N, p * m1))
+    y = np.zeros((N, q * m2))
+    for i in range(r):
+        t = orc.ks_forward(x, np.broadcast_to(B[i], (p, 1, m1, m2)))
+        y += orc.ks_forward(t, np.broadcast_to(C[i], (1, m2, p, q)))
+    ref = x @ sum(np.kron(C[i], B[i]) for i in range(r))
+    assert np.allclose(y, ref, rtol=0, atol=1e-12)
+
+
+def pin_ks_hadamard_chain(orc):
+    """The Walsh-Hadamard transform as a chain of KS factors: with every 2 x 2 block
+    [[1, 1], [1, -1]], the product over l = 1..L of the patterns (2^(l-1), 2, 2, 2^(L-l))
+    is Sylvester's Hadamard matrix of order 2^L (scipy's hadamard)."""
+    from scipy.linalg import hadamard
+    L = 4
+    n = 1 << L
+    H2 = np.array([[1.0, 1.0], [1.0, -1.0]])
+    y = np.eye(n)
+    for l in range(1, L + 1):
+        a, d = 1 << (l - 1), 1 << (L - l)
+        y = orc.ks_forward(y, np.broadcast_to(H2, (a, d, 2, 2)))
+    assert np.array_equal(y, hadamard(n).astype(np.float64))
+
+
+def pin_ks_forward_is_numpy_matmul(orc):
+    """y = x K + bias with numpy's matmul on the oracle's dense K; bias None means 0."""
+    rng = np.random.default_rng(431)
+    a, b, c, d, N = 2, 3, 4, 3, 7
+    w = rng.standard_normal((a, d, b, c))
+    x = rng.standard_normal((N, a * b * d))
+    bias = rng.standard_normal(a * c * d)
+    K = orc.ks_dense(w)
+    assert np.allclose(orc.ks_forward(x, w, bias), x @ K + bias, rtol=0, atol=1e-12)
+    assert np.allclose(orc.ks_forward(x, w), x @ K, rtol=0, atol=1e-12)
+
+
+def pin_ks_finite_differences(orc):
+    """Central differences of L = <G, y> in x, w and bias (exact up to rounding: L is affine
+    in each single coordinate), on a pattern with a, b, c, d all > 1 and b != c."""
+    rng = np.random.default_rng(433)
+    a, b, c, d, N = 2, 3, 2, 2, 3
+    w = rng.standard_normal((a, d, b, c))
+    x = rng.standard_normal((N, a * b * d))
+    G = rng.standard_normal((N, a * c * d))
+    bias = rng.standard_normal(a * c * d)
+    g = orc.ks_backward(x, w, G)
+    Lf = lambda x, w, bias: float(np.sum(G * orc.ks_forward(x, w, bias)))
+    h = 1e-3
+    args = {"x": x, "w": w, "bias": bias}
+    for key, grad in (("x", "dX"), ("w", "dw"), ("bias", "dbias")):
+        base = args[key]
+        for idx in np.ndindex(base.shape):
+            up_, dn_ = base.copy(), base.copy()
+            up_[idx] += h
+            dn_[idx] -= h
+            num = (Lf(**dict(args, **{key: up_})) - Lf(**dict(args, **{key: dn_}))) / (2 * h)
+            assert abs(num - g[grad][idx]) <= 1e-8 * max(1.0, abs(num)), (key, idx)
+
+
+def pin_ks_linearity_identities(orc):
+    """y - bias is linear in x and in w, so <dX, x> = <dw, w> = <G, y - bias> (Euler)."""
+    rng = np.random.default_rng(439)
+    a, b, c, d, N = 3, 2, 3, 2, 6
+    w = rng.standard_normal((a, d, b, c))
+    x = rng.standard_normal((N, a * b * d))
+    G = rng.standard_normal((N, a * c * d))
+    g = orc.ks_backward(x, w, G)
+    ref = float(np.sum(G * orc.ks_forward(x, w)))
+    assert abs(float(np.sum(g["dX"] * x)) - ref) <= 1e-11 * max(1.0, abs(ref))
+    assert abs(float(np.sum(g["dw"] * w)) - ref) <= 1e-11 * max(1.0, abs(ref))
+    assert np.allclose(g["dbias"], G.sum(axis=0), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_weight_is_sum_of_numpy_krons,
     pin_forward_brute_force,
@@ -448,4 +584,13 @@ ALL_PINS = [
     pin_backward_numpy_chain_rule,
     pin_zero_s_gradient,
     pin_l1_grad_finite_differences,
+    pin_ks_support_is_kron_of_identity_and_ones,
+    pin_ks_block_diagonal,
+    pin_ks_diagonal,
+    pin_ks_tied_values_are_numpy_kron,
+    pin_ks_chain_is_kronecker_layer,
+    pin_ks_hadamard_chain,
+    pin_ks_forward_is_numpy_matmul,
+    pin_ks_finite_differences,
+    pin_ks_linearity_identities,
 ]

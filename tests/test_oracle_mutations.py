@@ -61,6 +61,27 @@ MUTATIONS = [
     ("kron3_dC_uses_B_twice",
      "A[((long)i * p + a) * q + c] * B[((long)i * m1 + j) * m2 + k];\n                dC",
      "B[((long)i * m1 + j) * m2 + k] * B[((long)i * m1 + j) * m2 + k];\n                dC", 0),
+    ("ks_rows_in_wrong_interleave",
+     "K[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + de] =",
+     "K[(((long)al * d + de) * b + be) * out + ((long)al * c + ga) * d + de] =", 0),
+    ("ks_cols_in_wrong_interleave",
+     "K[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + de] =",
+     "K[(((long)al * b + be) * d + de) * out + ((long)al * d + de) * c + ga] =", 0),
+    ("ks_block_read_transposed",
+     "w[(((long)al * d + de) * b + be) * c + ga];",
+     "w[(((long)al * d + de) * c + ga) * b + be];", 0),
+    ("ks_blocks_in_wrong_order",
+     "w[(((long)al * d + de) * b + be) * c + ga];",
+     "w[(((long)de * a + al) * b + be) * c + ga];", 0),
+    ("ks_forward_drops_bias", "oracle_matmul_bias(x, K, bias, N, in, out, y);",
+     "oracle_matmul_bias(x, K, NULL, N, in, out, y);", 0),
+    ("ks_dx_wrong_sign", "s += G[n * out + o] * K[u * out + o];",
+     "s -= G[n * out + o] * K[u * out + o];", 0),
+    ("ks_dw_reads_mirrored_delta",
+     "dK[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + de];",
+     "dK[(((long)al * b + be) * d + de) * out + ((long)al * c + ga) * d + (d - 1 - de)];", 0),
+    ("ks_dbias_skips_first_row", "for (long n = 0; n < N; ++n) s += G[n * out + o];",
+     "for (long n = 1; n < N; ++n) s += G[n * out + o];", 2),
 ]
 
 
