@@ -560,6 +560,106 @@ def run_extras(kfs, steps, dev):
     return out
 
 
+def ks_bmm_context(fac, sets, pattern, steps, dev):
+    """Context only (not the product path): the Kronecker-sparse factor computed the way the
+    page "Fast Inference with Kronecker-Sparse Matrices" describes earlier GPU kernels --
+    permute x into a*d contiguous b-column slices, one batched GEMM, permute back (and the
+    same for dY in the backward: dX and dw as two more batched GEMMs), FP32 cuBLAS through
+    torch with TF32 off.  Forward + backward per step, replayed from a CUDA graph."""
+    import torch
+    a, b, c, d = pattern
+    W3 = fac["w"].reshape(a * d, b, c)
+    bias = fac["bias"]
+    old = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        def step(i):
+            x, G = sets[i % len(sets)]
+            N = x.shape[0]
+            xt = x.view(N, a, b, d).permute(1, 3, 0, 2).reshape(a * d, N, b)
+            y = torch.bmm(xt, W3).view(a, d, N, c).permute(2, 0, 3, 1).reshape(N, a * c * d) + bias
+            Gt = G.view(N, a, c, d).permute(1, 3, 0, 2).reshape(a * d, N, c)
+            dx = torch.bmm(Gt, W3.transpose(1, 2)).view(a, d, N, b).permute(2, 0, 3, 1).reshape(
+                N, a * b * d)
+            dw = torch.bmm(xt.transpose(1, 2), Gt)
+            db = G.sum(0)
+            return y, dx, dw, db
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        ms = _time_graph(step, steps, REPEATS)[0] / steps
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = old
+    return {"what": "permute + batched GEMM + permute back (torch/cuBLAS FP32, TF32 off), "
+                    "forward and backward (dX, dw, dbias), same inputs, CUDA graph replay; "
+                    "context only", "ms_per_step": ms}
+
+
+KS_LEGS = ["ks_monarch_bd", "ks_monarch_tr", "ks_butterfly", "ks_gpt2m_up", "ks_block128"]
+
+
+def run_ks_leg(kw, kfs, name, steps, warmup, peaks, dev, stream):
+    """One Kronecker-sparse factor (include/ks_linear.h): forward + backward through the C
+    ABI, exact FP32, CUDA-graph replay of `steps` steps (median of REPEATS), with the
+    roofline max(bytes / HBM, flops / FFMA) and the permute + batched-GEMM context."""
+    import torch
+    from kronecker_factored_structured_b200 import accounting as acc
+    from kronecker_factored_structured_b200 import native
+    w = kw.ks_get(name)
+    a, b, c, d = w.pattern
+    fac = {k: v.to(dev) for k, v in kw.ks_factors(w).items()}
+    rotate = ROTATE if w.N * (w.d_in + w.d_out) * 4 < 126e6 else 1
+    sets = []
+    for s in range(rotate):
+        ws = dataclasses.replace(w, seed=w.seed + 1000 * s) if s else w
+        sets.append((kw.rows(ws, "x").to(dev), kw.rows(ws, "G").to(dev)))
+    y = torch.empty(w.N, w.d_out, device=dev)
+    grads = {"dX": torch.empty(w.N, w.d_in, device=dev), "dw": torch.empty_like(fac["w"]),
+             "dbias": torch.empty(w.d_out, device=dev)}
+    wsb = torch.empty(native.ks_workspace_size(w.N, a, b, c, d), dtype=torch.uint8, device=dev)
+
+    def step(i, timing=None):
+        x, G = sets[i % len(sets)]
+        if timing is not None:
+            timing[0].record(stream)
+        native.ks_forward(x, fac["w"], fac["bias"], out=y)
+        if timing is not None:
+            timing[1].record(stream)
+        native.ks_backward(x, fac["w"], G, workspace=wsb, grads=grads)
+        if timing is not None:
+            timing[2].record(stream)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    med, mn, _ = _time_graph(step, steps, REPEATS)
+    t_fwd, t_bwd = _split_calls(step, steps, stream)
+    ms = med / steps
+    nbytes = w.N * acc.bytes_per_row(w.d_in, w.d_out, 4)
+    flops = w.N * acc.ks_flops_per_row(a, b, c, d)
+    ffma = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6
+    t_hbm, t_fl = nbytes / (peaks["hbm_gbs"] * 1e9), flops / ffma
+    fwd_bytes = w.N * acc.bytes_per_row(w.d_in, w.d_out, 4, backward=False)
+    leg = {"workload": f"Kronecker-sparse factor, pattern (a, b, c, d) = {w.pattern}, "
+                       f"{w.d_in} -> {w.d_out}, N = {w.N}, fp32",
+           "name": name, "path": "f32", "N": w.N, "steps": steps, "repeats": REPEATS,
+           "timer": "CUDA graph replay of the steps", "ms_per_step": ms,
+           "ms_per_step_min": mn / steps, "rows_per_s": w.N / (ms / 1e3),
+           "fwd_ms": t_fwd, "bwd_ms": t_bwd, "call_split_timer": "eager, per-call events",
+           "l2": f"{len(sets)} input set(s), {len(sets) * w.N * (w.d_in + w.d_out) * 4 / 1e6:.0f} MB",
+           "forward_hbm_frac": (fwd_bytes / (peaks["hbm_gbs"] * 1e9)) / (t_fwd / 1e3),
+           "roofline": {"bound": "hbm" if t_hbm >= t_fl else "alu",
+                        "roofline_us": max(t_hbm, t_fl) * 1e6, "hbm_us": t_hbm * 1e6,
+                        "flops_us": t_fl * 1e6, "frac": max(t_hbm, t_fl) / (ms / 1e3),
+                        "flop_peak": "FFMA", "flop_peak_source": "derived", "bytes": nbytes,
+                        "flops": flops}}
+    ctx = ks_bmm_context(fac, sets, w.pattern, steps, dev)
+    ctx["ks_speedup"] = ctx["ms_per_step"] / ms
+    leg["context_bmm"] = ctx
+    del sets, y, grads, wsb, fac
+    torch.cuda.empty_cache()
+    return leg
+
+
 def run_leg(kw, kfs, name, path, flags, steps, warmup, peaks, dev, stream):
     """One further leg: the workload's forward + backward step, median of REPEATS timed
     regions of `steps` steps; a dict for the JSON line's "legs" list."""
@@ -821,6 +921,9 @@ def main():
             legs.append(run_leg(kw, kfs, name, lpath, lflags, max(3, min(args.steps, args.leg_steps)),
                                 args.warmup, peaks, dev, stream))
         line["legs"] = legs
+        line["ks_legs"] = [run_ks_leg(kw, kfs, name, max(3, min(args.steps, args.leg_steps)),
+                                      args.warmup, peaks, dev, stream)
+                           for name in KS_LEGS if names is None or name in names]
         line["extras"] = run_extras(kfs, max(3, min(args.steps, args.leg_steps)), dev)
     if world == 1 and not args.no_cpu_baseline:
         cpu_rows = args.cpu_rows or (N if N * (w.d_in + w.d_out) <= 20000 * 2048 else 1024)

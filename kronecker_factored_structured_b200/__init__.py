@@ -7,6 +7,11 @@ with the vec trick by the hand-written sm_100a kernels of libkronlinear.so; W is
 never materialised.  ``native`` is the ctypes binding of the C ABI
 (include/kron_linear.h); ``KronLinearFunction`` / ``KronLinear`` wrap it for
 autograd.  PyTorch is used for device memory and streams only.
+
+The same library holds the Kronecker-sparse factor of the page "Fast Inference
+with Kronecker-Sparse Matrices" (support kron(I_a, kron(1_{b x c}, I_d)),
+include/ks_linear.h): ``native.ks_forward`` / ``native.ks_backward``, wrapped by
+``KSLinearFunction`` / ``KSLinear``.
 """
 from __future__ import annotations
 
@@ -18,7 +23,8 @@ from . import accounting, native
 from .native import KronError, backward, forward, workspace_size
 
 __all__ = ["native", "accounting", "forward", "backward", "workspace_size", "KronError",
-           "KronLinearFunction", "KronLinear", "kron_linear"]
+           "KronLinearFunction", "KronLinear", "kron_linear", "KSLinearFunction", "KSLinear",
+           "ks_linear"]
 
 
 class KronLinearFunction(torch.autograd.Function):
@@ -78,4 +84,44 @@ class KronLinear(torch.nn.Module):
         shp = x.shape
         y = kron_linear(x.reshape(-1, shp[-1]).contiguous(), self.S, self.A, self.B, self.bias,
                         self.path, self.flags, self.l1)
+        return y.reshape(*shp[:-1], y.shape[-1])
+
+
+class KSLinearFunction(torch.autograd.Function):
+    """Autograd wrapper of the Kronecker-sparse factor; both passes run in the CUDA library."""
+
+    @staticmethod
+    def forward(ctx, x, w, bias):
+        ctx.save_for_backward(x, w)
+        ctx.has_bias = bias is not None
+        return native.ks_forward(x, w, bias)
+
+    @staticmethod
+    def backward(ctx, dY):
+        x, w = ctx.saved_tensors
+        g = native.ks_backward(x, w, dY.contiguous(), need_dx=ctx.needs_input_grad[0],
+                               need_dbias=ctx.has_bias)
+        return g["dX"], g["dw"], g["dbias"]
+
+
+def ks_linear(x, w, bias=None):
+    return KSLinearFunction.apply(x, w, bias)
+
+
+class KSLinear(torch.nn.Module):
+    """Linear layer y = x K + bias whose weight K is Kronecker-sparse with pattern
+    (a, b, c, d): supp K = kron(I_a, kron(1_{b x c}, I_d)), in = a*b*d, out = a*c*d.
+    The a*d dense b x c blocks are initialised with std 1/sqrt(b) (each output sums b
+    inputs); FP32 only.  Butterfly and Monarch layers are sequences of these."""
+
+    def __init__(self, a, b, c, d, bias=True, device=None):
+        super().__init__()
+        kw = dict(device=device, dtype=torch.float32)
+        self.pattern = (a, b, c, d)
+        self.w = torch.nn.Parameter(torch.randn(a, d, b, c, **kw) / math.sqrt(b))
+        self.bias = torch.nn.Parameter(torch.zeros(a * c * d, **kw)) if bias else None
+
+    def forward(self, x):
+        shp = x.shape
+        y = ks_linear(x.reshape(-1, shp[-1]).contiguous(), self.w, self.bias)
         return y.reshape(*shp[:-1], y.shape[-1])

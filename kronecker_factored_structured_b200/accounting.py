@@ -13,6 +13,11 @@ not what a kernel happens to execute:
   the backward is executed work, not credited.
 * bytes per row, forward plus backward: read x, write y; read x and dY, write dX
   -> elt * (3*d_in + 2*d_out).  The factors (kilobytes) are not counted.
+
+The Kronecker-sparse factor of pattern (a, b, c, d) (page "Fast Inference with
+Kronecker-Sparse Matrices") has a*b*c*d non-zeros, a fraction 1/(a*d) of a dense
+(a*b*d) x (a*c*d) matrix; its forward is one multiply-add per non-zero and row, and
+the backward two more (dX and dw), so 6*a*b*c*d flops per row; bytes as above.
 """
 from __future__ import annotations
 
@@ -65,3 +70,13 @@ def bytes_per_row(d_in, d_out, elt_bytes, backward=True):
     if backward:
         return elt_bytes * (3 * d_in + 2 * d_out)
     return elt_bytes * (d_in + d_out)
+
+
+def ks_param_count(a, b, c, d, bias=True):
+    """Values of a Kronecker-sparse factor of pattern (a, b, c, d) (+ bias)."""
+    return a * b * c * d + (a * c * d if bias else 0)
+
+
+def ks_flops_per_row(a, b, c, d, backward=True):
+    """Algorithmic flops per row: 2 per non-zero for y, and as many again for dX and dw."""
+    return 2 * a * b * c * d * (3 if backward else 1)

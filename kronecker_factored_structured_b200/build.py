@@ -27,7 +27,7 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", 
 
 def _deps(src):
     hdrs = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-    hdrs.append(os.path.join(ROOT, "include", "kron_linear.h"))
+    hdrs += glob.glob(os.path.join(ROOT, "include", "*.h"))
     return [src] + hdrs
 
 

@@ -1,4 +1,4 @@
-"""ctypes binding of libkronlinear.so (include/kron_linear.h).
+"""ctypes binding of libkronlinear.so (include/kron_linear.h, include/ks_linear.h).
 
 Argument marshalling only: every step of the layer runs in the library's CUDA
 kernels.  PyTorch supplies device memory and the current CUDA stream.  If the
@@ -33,7 +33,8 @@ EXPORTS = ("kron_linear_forward", "kron_linear_backward", "kron_linear_backward_
            "kron_linear_workspace_size", "kron_vanloan_fit", "kron_vanloan_workspace_size",
            "kron3_linear_forward", "kron3_linear_backward", "kron3_linear_workspace_size",
            "kron_status_string", "kron_last_error", "kron_linear_device_error",
-           "kron_linear_abi_version")
+           "kron_linear_abi_version",
+           "ks_linear_forward", "ks_linear_backward", "ks_linear_workspace_size")
 
 
 class KronError(RuntimeError):
@@ -90,6 +91,12 @@ def load(path: str = LIB_PATH):
     lib.kron_linear_device_error.restype = I
     lib.kron_linear_abi_version.argtypes = []
     lib.kron_linear_abi_version.restype = I
+    lib.ks_linear_forward.argtypes = [vp, vp, vp, vp, i64, I, I, I, I, I, U, vp]
+    lib.ks_linear_forward.restype = I
+    lib.ks_linear_backward.argtypes = [vp, vp, vp, vp, vp, vp, i64, I, I, I, I, I, U, vp, sz, vp]
+    lib.ks_linear_backward.restype = I
+    lib.ks_linear_workspace_size.argtypes = [i64, I, I, I, I, I]
+    lib.ks_linear_workspace_size.restype = sz
     _lib = lib
     return lib
 
@@ -278,4 +285,65 @@ def backward3(x, A, B, C, dY, dtype="tf32", flags=0, stream=None):
                                      _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dbias"]),
                                      N, p, q, m1, m2, s1, s2, r, DTYPES[dtype], flags, _ptr(ws),
                                      ws.numel(), _stream(stream)))
+    return g
+
+
+# ---- Kronecker-sparse factor (include/ks_linear.h) ----
+
+def ks_pattern(w):
+    """(a, b, c, d) of the values w, laid out [a][d][b][c]."""
+    if w.dim() != 4:
+        raise ValueError(f"w must have shape (a, d, b, c), got {tuple(w.shape)}")
+    a, d, b, c = w.shape
+    return a, b, c, d
+
+
+def ks_workspace_size(N, a, b, c, d) -> int:
+    return int(load().ks_linear_workspace_size(N, a, b, c, d, KRON_F32))
+
+
+def ks_forward(x, w, bias=None, out=None, stream=None):
+    """y = x K + bias for the KS matrix K of pattern (a, b, c, d) with values w."""
+    a, b, c, d = ks_pattern(w)
+    N = x.shape[0]
+    f32 = torch.float32
+    _expect(x, "x", f32, (N, a * b * d))
+    _expect(w, "w", f32, (a, d, b, c))
+    if bias is not None:
+        _expect(bias, "bias", f32, (a * c * d,))
+    if out is None:
+        out = torch.empty(N, a * c * d, dtype=f32, device=x.device)
+    _expect(out, "y", f32, (N, a * c * d))
+    _check(load().ks_linear_forward(_ptr(x), _ptr(w), _ptr(bias), _ptr(out), N, a, b, c, d,
+                                    KRON_F32, 0, _stream(stream)))
+    return out
+
+
+def ks_backward(x, w, dY, need_dx=True, need_dbias=True, workspace=None, grads=None,
+                stream=None):
+    """Gradients of <dY, y> for the KS factor: dict(dX, dw, dbias) (None where not asked)."""
+    a, b, c, d = ks_pattern(w)
+    N = x.shape[0]
+    f32 = torch.float32
+    _expect(x, "x", f32, (N, a * b * d))
+    _expect(w, "w", f32, (a, d, b, c))
+    _expect(dY, "dY", f32, (N, a * c * d))
+    dev = x.device
+    g = dict(grads or {})
+    if need_dx and g.get("dX") is None:
+        g["dX"] = torch.empty(N, a * b * d, dtype=f32, device=dev)
+    if not need_dx:
+        g["dX"] = None
+    if g.get("dw") is None:
+        g["dw"] = torch.empty(a, d, b, c, dtype=f32, device=dev)
+    _expect(g["dw"], "dw", f32, (a, d, b, c))
+    if need_dbias and g.get("dbias") is None:
+        g["dbias"] = torch.empty(a * c * d, dtype=f32, device=dev)
+    if not need_dbias:
+        g["dbias"] = None
+    if workspace is None:
+        workspace = torch.empty(ks_workspace_size(N, a, b, c, d), dtype=torch.uint8, device=dev)
+    _check(load().ks_linear_backward(_ptr(x), _ptr(w), _ptr(dY), _ptr(g["dX"]), _ptr(g["dw"]),
+                                     _ptr(g["dbias"]), N, a, b, c, d, KRON_F32, 0,
+                                     _ptr(workspace), workspace.numel(), _stream(stream)))
     return g

@@ -11,12 +11,17 @@ import kronecker_factored_structured_b200 as kfs
 from kronecker_factored_structured_b200 import native
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "kron_linear.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("kron_linear.h", "ks_linear.h")]
 
 
 def header_symbols():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"KRON_API\s+[\w\s\*]*?\b(kron3?_\w+)\s*\(", text)))
+    text = "".join(open(h).read() for h in HEADERS)
+    return sorted(set(re.findall(r"KRON_API\s+[\w\s\*]*?\b((?:kron3?|ks)_\w+)\s*\(", text)))
+
+
+def test_every_header_is_scanned():
+    assert sorted(os.listdir(os.path.join(ROOT, "include"))) == sorted(
+        os.path.basename(h) for h in HEADERS)
 
 
 def test_library_exports_every_declared_symbol():
@@ -244,3 +249,58 @@ def test_python_binding_raises_without_cuda_tensors():
     S, A, B = torch.ones(2, 2), torch.zeros(1, 2, 2), torch.zeros(1, 4, 4)
     with pytest.raises(ValueError):
         kfs.forward(x, S, A, B, dtype="f32")
+
+
+# ---- Kronecker-sparse factor (include/ks_linear.h) ----
+
+def ks_fwd(x=ALIGNED, w=ALIGNED, bias=None, y=ALIGNED, N=8, a=2, b=3, c=4, d=5, dtype=0, flags=0):
+    return native.load().ks_linear_forward(x, w, bias, y, N, a, b, c, d, dtype, flags, None)
+
+
+def ks_bwd(ws=V(0x100000), ws_bytes=1 << 30, N=8, a=2, b=3, c=4, d=5, dtype=0, x=ALIGNED,
+           dw=ALIGNED, dbias=None):
+    return native.load().ks_linear_backward(x, ALIGNED, ALIGNED, ALIGNED, dw, dbias, N, a, b, c,
+                                            d, dtype, 0, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(dtype=7), 1),
+    (dict(flags=1), 1),
+    (dict(N=-1), 1),
+    (dict(a=0), 1),
+    (dict(d=0), 1),
+    (dict(x=None), 1),
+    (dict(w=None, N=0), 1),
+    (dict(a=1, b=1 << 13, d=1 << 12), 1),     # a*b*d above 2^24
+    (dict(dtype=1), 2),                       # TF32: no KS kernel
+    (dict(dtype=2), 2),                       # BF16: no KS kernel
+    (dict(x=V(0x10002)), 3),
+    (dict(bias=V(0x10001)), 3),
+])
+def test_ks_forward_rejects(kwargs, status):
+    assert ks_fwd(**kwargs) == status
+    assert native.load().kron_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(dtype=1), 2),
+    (dict(dw=None), 1),
+    (dict(x=None), 1),
+    (dict(ws=None), 4),
+    (dict(ws_bytes=16), 4),
+    (dict(ws=V(0x100080)), 3),
+    (dict(dbias=V(0x10006)), 3),
+])
+def test_ks_backward_rejects(kwargs, status):
+    assert ks_bwd(**kwargs) == status
+
+
+def test_ks_workspace_size():
+    n = native.ks_workspace_size(20000, 1, 32, 32, 32)
+    assert n > 0 and n % 256 == 0
+    assert n == native.ks_workspace_size(20000, 1, 32, 32, 32)
+    assert native.ks_workspace_size(0, 1, 32, 32, 32) == 256           # empty batch: valid
+    assert native.ks_workspace_size(-1, 1, 32, 32, 32) == 0
+    assert native.load().ks_linear_workspace_size(100, 1, 2, 2, 1, 1) == 0   # TF32: unsupported
+    # the partials grow with the rows until every part has its chunk, then stay fixed
+    assert native.ks_workspace_size(10, 32, 32, 32, 1) <= native.ks_workspace_size(20000, 32, 32, 32, 1)
