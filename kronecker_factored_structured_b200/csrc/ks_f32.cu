@@ -11,7 +11,7 @@
 // it needs in shared memory (the gather happens on chip: x is read once per column tile and
 // y written once, no permuted copy of x or y ever reaches HBM) and runs the whole
 // contraction for its tile.  The same kernel computes dX = dY K^T with the roles of b and c
-// swapped and w read transposed.  dw is a split-N reduction: each CTA sums x^T dY over one
+// swapped, from a copy of the blocks transposed once per call into the workspace.  dw is a split-N reduction: each CTA sums x^T dY over one
 // contiguous row range for one tile of (al, de, be, ga) and writes a partial; a second
 // kernel adds the partials in a fixed order (bitwise reproducible; the row split depends on
 // the sizes only).  dbias rides along in the dw kernel.
@@ -40,12 +40,14 @@ constexpr int64_t kPartTarget = 4 * 148;  // CTAs the backward's row split aims 
 constexpr int64_t kMaxWidth = 1 << 24;    // a*b*d and a*c*d
 
 struct KsTile {
-    int TD;    // deltas per CTA (d when d <= 8, else 8)
+    int TD;    // deltas per CTA: 1, 2, 4 or 8 (the power of two >= d, at most 8)
     int GC;    // column groups: TC = GC * kC columns per tile
     int GR;    // row groups: TM = GR * kR rows (forward) or be values (dw) per tile
-    int KB;    // reduction chunk staged at once (forward: be or ga values; dw: rows)
+    int KB;    // reduction chunk staged at once (forward: be values; dw: rows)
     int KG;    // dw: thread groups that split each chunk's rows (forward: 1)
     int padw;  // padding of the column array's delta stride
+    int vx;    // 1: the row slices are staged with 16-byte loads (alignment allows it)
+    int vw;    // 1: the values (forward) / dY slices (dw) likewise
 };
 
 // Largest power of two gr with 2 gr^2 <= maxg, and gc = maxg / gr: a tile with about as
@@ -57,12 +59,23 @@ void balanced(int maxg, int *gr, int *gc) {
     *gc = maxg / r;
 }
 
-int tile_deltas(int d) { return d <= 8 ? d : 8; }
-int pad_for(int td) { return (td & (td - 1)) == 0 ? (32 / td) % 32 : 1; }
+int tile_deltas(int d) { return d >= 8 ? 8 : (d > 4 ? 8 : (d > 2 ? 4 : d)); }
+int pad_for(int td) { return (32 / td) % 32; }
 int cdiv(int64_t x, int64_t y) { return (int)((x + y - 1) / y); }
+bool a16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Whether one CTA's slice of a row -- elements (k, delta) for k in a chunk starting at a
+// multiple of `kstep` and delta in a tile of TD -- can move as aligned float4 (all four
+// valid or all four outside the matrix): runs of TD (TD < d) need d % 4 == 0; one
+// contiguous run (TD == d) needs its start and length to be multiples of 4.
+bool slice_vec(int kdim, int kstep, int d, int td) {
+    if (td < d) return d % 4 == 0;
+    if (td != d) return false;
+    return ((int64_t)kdim * d) % 4 == 0 && ((int64_t)kstep * d) % 4 == 0;
+}
 
 // Forward / dX tile: kin = contraction length, kout = output block length.
-KsTile fwd_tile(int kin, int kout, int d) {
+KsTile fwd_tile(int kin, int kout, int d, const void *in, const void *w) {
     KsTile t{};
     t.TD = tile_deltas(d);
     t.padw = pad_for(t.TD);
@@ -74,16 +87,21 @@ KsTile fwd_tile(int kin, int kout, int d) {
     if (gc > need_c) {
         gc = need_c;
         gr = maxg / gc < 64 ? maxg / gc : 64;
+        if (gr >= 4) gr &= ~3;
     }
     t.GR = gr;
     t.GC = gc;
     const int step = t.TD * (gr * kR + 4 + gc * kC + t.padw) * 4;
-    const int kb = kSmemTile / step;
-    t.KB = kb < 1 ? 1 : (kb > kin ? kin : kb);
+    int kb = kSmemTile / step;
+    kb = kb < 1 ? 1 : (kb > 256 ? 256 : kb);
+    if (kb < kin && kb >= 4) kb &= ~3;  // chunk starts stay float4-aligned when d is odd
+    t.KB = kb > kin ? kin : kb;
+    t.vx = a16(in) && slice_vec(kin, t.KB, d, t.TD);
+    t.vw = a16(w) && kout % 4 == 0;
     return t;
 }
 
-KsTile dw_tile(int b, int c, int d) {
+KsTile dw_tile(int b, int c, int d, const void *x, const void *g) {
     KsTile t{};
     t.TD = tile_deltas(d);
     t.padw = pad_for(t.TD);
@@ -100,6 +118,8 @@ KsTile dw_tile(int b, int c, int d) {
     const int step = t.TD * (gr * kR + 4 + gc * kC + t.padw) * 4;
     const int kb = kSmemTile / step;
     t.KB = kb < 1 ? 1 : (kb > 256 ? 256 : kb);
+    t.vx = a16(x) && slice_vec(b, gr * kR, d, t.TD);
+    t.vw = a16(g) && slice_vec(c, gc * kC, d, t.TD);
     return t;
 }
 
@@ -116,9 +136,9 @@ struct DwPlan {
     size_t part_stride;  // floats
 };
 
-DwPlan dw_plan(int64_t N, int a, int b, int c, int d) {
+DwPlan dw_plan(int64_t N, int a, int b, int c, int d, const void *x, const void *g) {
     DwPlan P;
-    P.t = dw_tile(b, c, d);
+    P.t = dw_tile(b, c, d, x, g);
     P.tiles_per_part = (int64_t)a * cdiv(d, P.t.TD) * cdiv(b, (int64_t)P.t.GR * kR) *
                        cdiv(c, (int64_t)P.t.GC * kC);
     int64_t parts = 0;
@@ -135,15 +155,128 @@ DwPlan dw_plan(int64_t N, int a, int b, int c, int d) {
     return P;
 }
 
-// y (or dX) tiles.  TR = false: in = x [N][a*kin*d], w [a][d][kin][kout].  TR = true (dX):
-// in = dY [N][a*kin*d], w [a][d][kout][kin] read transposed.
-template <bool TR>
+// Staging of row slices into shared memory.  Element (row rr, slice position u), with
+// u = k*TD + dd for k < kn and dd < TD, comes from
+//     src[(row0 + rr) * row_w + (kbase + k) * d + de0 + dd]
+// and is zero outside the matrix (row0 + rr >= nmax, kbase + k >= kdim or de0 + dd >= d).
+// With vec the slice moves as aligned float4 (4 consecutive u; the host checks that all
+// four are inside or all outside).  No division depends on the element: each thread's
+// assignment is fixed for the launch.
+//
+// stage_cols writes dst[u * S + rr] (the forward's input: rows contiguous per position).
+// Lane pairs take 8 consecutive positions of one row (a whole 32-byte sector), the 16 pairs
+// of a warp 16 consecutive rows; with S = 4 (mod 32) the stores hit 32 distinct banks.
+template <int TD>
+__device__ __forceinline__ void stage_cols(float *__restrict__ dst, int S,
+                                           const float *__restrict__ src, int64_t row_w,
+                                           int64_t row0, int64_t nmax, int nrows, int kbase,
+                                           int kn, int kdim, int d, int de0, bool vec) {
+    const int tid = threadIdx.x;
+    const int span = kn * TD;
+    if (vec) {
+        const int nq = span >> 2;                  // float4 per row slice
+        const int qsel = tid & 1, rl = tid >> 1;   // 2 lanes per group, 128 groups
+        const int R2 = nrows < 128 ? nrows : 128;  // rows per pass
+        const int P2 = 128 / R2;                   // float4 pairs per pass
+        const int rr0 = rl % R2, pl = rl / R2;
+        if (pl >= P2) return;
+        for (int qp = pl; 2 * qp < nq; qp += P2) {
+            const int q = 2 * qp + qsel;
+            if (q >= nq) continue;
+            const int u = 4 * q;
+            const int k = u / TD, dd = u % TD;
+            const bool inside = kbase + k < kdim && de0 + dd < d;
+            const int64_t col = (int64_t)(kbase + k) * d + de0 + dd;
+            for (int rr = rr0; rr < nrows; rr += R2) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (inside && row0 + rr < nmax)
+                    v = *reinterpret_cast<const float4 *>(src + (row0 + rr) * row_w + col);
+                dst[(u + 0) * S + rr] = v.x;
+                dst[(u + 1) * S + rr] = v.y;
+                dst[(u + 2) * S + rr] = v.z;
+                dst[(u + 3) * S + rr] = v.w;
+            }
+        }
+    } else {
+        const int esel = tid & 7, rl = tid >> 3;   // 8 lanes per group, 32 groups
+        const int R8 = nrows < 32 ? nrows : 32;
+        const int P8 = 32 / R8;
+        const int rr0 = rl % R8, pl = rl / R8;
+        if (pl >= P8) return;
+        for (int ep = pl; 8 * ep < span; ep += P8) {
+            const int u = 8 * ep + esel;
+            if (u >= span) continue;
+            const int k = u / TD, dd = u % TD;
+            const bool inside = kbase + k < kdim && de0 + dd < d;
+            const int64_t col = (int64_t)(kbase + k) * d + de0 + dd;
+            for (int rr = rr0; rr < nrows; rr += R8) {
+                float v = 0.f;
+                if (inside && row0 + rr < nmax) v = src[(row0 + rr) * row_w + col];
+                dst[u * S + rr] = v;
+            }
+        }
+    }
+}
+
+// stage_rows writes dst[(rr * TD + dd) * S + k] (the dw operands: positions k contiguous per
+// row and delta).  Consecutive lanes take consecutive units (float4 or float) of one row, so
+// a warp stores within one row wherever a row slice holds 32 units or more; with TD == 1 a
+// float4 lands as one 16-byte store.
+template <int TD>
+__device__ __forceinline__ void stage_rows(float *__restrict__ dst, int S,
+                                           const float *__restrict__ src, int64_t row_w,
+                                           int64_t row0, int64_t nmax, int nrows, int kbase,
+                                           int kn, int kdim, int d, int de0, bool vec) {
+    const int tid = threadIdx.x;
+    const int span = kn * TD;
+    const int nq = vec ? span >> 2 : span;  // units per row slice
+    int q0, qstep, r0, rstep;
+    if (nq <= kThreads) {
+        q0 = tid % nq;
+        qstep = nq;  // one unit per thread and row
+        r0 = tid / nq;
+        rstep = kThreads / nq;
+        if (r0 >= rstep) return;
+    } else {
+        q0 = tid;
+        qstep = kThreads;
+        r0 = 0;
+        rstep = 1;
+    }
+    for (int q = q0; q < nq; q += qstep) {
+        const int u = vec ? 4 * q : q;
+        const int k = u / TD, dd = u % TD;
+        const bool inside = kbase + k < kdim && de0 + dd < d;
+        const int64_t col = (int64_t)(kbase + k) * d + de0 + dd;
+        for (int rr = r0; rr < nrows; rr += rstep) {
+            const bool ok = inside && row0 + rr < nmax;
+            if (vec) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (ok) v = *reinterpret_cast<const float4 *>(src + (row0 + rr) * row_w + col);
+                if (TD == 1) {
+                    *reinterpret_cast<float4 *>(dst + rr * S + u) = v;
+                } else {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[(rr * TD + (u + e) % TD) * S + (u + e) / TD] = vv[e];
+                }
+            } else {
+                dst[(rr * TD + dd) * S + k] = ok ? src[(row0 + rr) * row_w + col] : 0.f;
+            }
+        }
+    }
+}
+
+// y tiles of y = x K + bias, or dX = dY K^T when w holds the transposed blocks.
+//   in [N][a*kin*d], w [a][d][kin][kout], out [N][a*kout*d], bias [a*kout*d] or null.
+template <int TD>
 __global__ void __launch_bounds__(kThreads)
 ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
               const float *__restrict__ bias, float *__restrict__ out, int64_t N, int a, int kin,
               int kout, int d, KsTile t, int64_t tiles) {
     extern __shared__ __align__(16) float smem[];
-    const int TD = t.TD, GC = t.GC, GR = t.GR, TM = GR * kR, TC = GC * kC;
+    const int GC = t.GC, GR = t.GR, TM = GR * kR, TC = GC * kC;
     const int SX = TM + 4, SW = TC + t.padw;
     float *xs = smem;                             // [KB][TD][SX]: input, rows contiguous
     float *ws = smem + (size_t)t.KB * TD * SX;    // [KB][TD][SW]: values, columns contiguous
@@ -152,6 +285,10 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
     const int dl = tid % TD, cg = (tid / TD) % GC, rg = tid / (TD * GC);
     const int64_t in_w = (int64_t)a * kin * d, out_w = (int64_t)a * kout * d;
     const int nj = (kout + TC - 1) / TC, nd = (d + TD - 1) / TD;
+    // fixed per-thread assignment of the value loads: float4 (or float) column jq of rows
+    // s = s0, s0 + sstep, ... of the [kb*TD][TC] value slice
+    const int wcols = t.vw ? GC : TC;
+    const int jq = tid % wcols, s0 = tid / wcols, sstep = kThreads / wcols;
 
     for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int jt = (int)(tile % nj);
@@ -170,36 +307,21 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
 
         for (int k0 = 0; k0 < kin; k0 += t.KB) {
             const int kb = min(t.KB, kin - k0);
-            const int span = kb * TD;  // (k, delta) pairs of one row, contiguous when TD == d
-            for (int e = tid; e < span * TM; e += kThreads) {
-                const int u = e % span, r = e / span;
-                const int de = de0 + u % TD;
-                const int64_t n = n0 + r;
-                float v = 0.f;
-                if (n < N && de < d)
-                    v = in[n * in_w + ((int64_t)al * kin + k0 + u / TD) * d + de];
-                xs[u * SX + r] = v;
-            }
-            for (int e = tid; e < span * TC; e += kThreads) {
-                int kk, dd, jl;
-                if (TR) {
-                    kk = e % kb;
-                    const int q = e / kb;
-                    jl = q % TC;
-                    dd = q / TC;
+            stage_cols<TD>(xs, SX, in, in_w, n0, N, TM, al * kin + k0, kb, al * kin + kin, d,
+                           de0, t.vx);
+            for (int s = s0; s < kb * TD; s += sstep) {
+                const int kk = s / TD, dd = s % TD;
+                const int de = de0 + dd;
+                const float *wrow = w + (((int64_t)al * d + de) * kin + k0 + kk) * kout + j0;
+                if (t.vw) {
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (de < d && j0 + 4 * jq < kout) v = *reinterpret_cast<const float4 *>(wrow + 4 * jq);
+                    *reinterpret_cast<float4 *>(ws + s * SW + 4 * jq) = v;
                 } else {
-                    jl = e % TC;
-                    const int q = e / TC;
-                    kk = q % kb;
-                    dd = q / kb;
+                    float v = 0.f;
+                    if (de < d && j0 + jq < kout) v = wrow[jq];
+                    ws[s * SW + jq] = v;
                 }
-                const int de = de0 + dd, j = j0 + jl;
-                float v = 0.f;
-                if (de < d && j < kout) {
-                    const int64_t blk = (int64_t)al * d + de;
-                    v = TR ? w[(blk * kout + j) * kin + k0 + kk] : w[(blk * kin + k0 + kk) * kout + j];
-                }
-                ws[(kk * TD + dd) * SW + jl] = v;
             }
             __syncthreads();
             if (active) {
@@ -239,15 +361,29 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
     }
 }
 
+// wt[al][de][ga][be] = w[al][de][be][ga]: the blocks of K^T, for dX = dY K^T.
+__global__ void ks_transpose_kernel(const float *__restrict__ w, float *__restrict__ wt,
+                                    int64_t blocks, int b, int c) {
+    const int64_t total = blocks * b * c;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t blk = e / ((int64_t)b * c);
+        const int rem = (int)(e - blk * b * c);
+        const int ga = rem / b, be = rem - ga * b;
+        wt[e] = w[(blk * b + be) * c + ga];
+    }
+}
+
 // Partial sums of dw (and dbias) over one contiguous row range per CTA.  Grid = parts x
 // (al, delta tile, be tile, ga tile); part p writes part[p][0 .. a*b*c*d) (dw layout) and,
 // from the CTAs of the first be tile, part[p][a*b*c*d + (al*c + ga)*d + de] (dbias).
+template <int TD>
 __global__ void __launch_bounds__(kThreads)
 ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__restrict__ part,
              int64_t N, int a, int b, int c, int d, KsTile t, int64_t rows_per_part,
              size_t part_stride) {
     extern __shared__ __align__(16) float smem[];
-    const int TD = t.TD, GC = t.GC, GR = t.GR, KG = t.KG, TB = GR * kR, TC = GC * kC;
+    const int GC = t.GC, GR = t.GR, KG = t.KG, TB = GR * kR, TC = GC * kC;
     const int SX = TB + 4, SW = TC + t.padw;
     float *xs = smem;                             // [KB rows][TD][SX]: be contiguous
     float *gs = smem + (size_t)t.KB * TD * SX;    // [KB rows][TD][SW]: ga contiguous
@@ -283,23 +419,8 @@ ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__
 
     for (int64_t n0 = r0; n0 < r1; n0 += t.KB) {
         const int kb = (int)(r1 - n0 < t.KB ? r1 - n0 : t.KB);
-        const int spx = TB * TD, spg = TC * TD;
-        for (int e = tid; e < kb * spx; e += kThreads) {
-            const int u = e % spx, kr = e / spx;
-            const int bl = u / TD, dd = u % TD;
-            const int be = be0 + bl, de = de0 + dd;
-            float v = 0.f;
-            if (be < b && de < d) v = x[(n0 + kr) * in_w + ((int64_t)al * b + be) * d + de];
-            xs[(kr * TD + dd) * SX + bl] = v;
-        }
-        for (int e = tid; e < kb * spg; e += kThreads) {
-            const int u = e % spg, kr = e / spg;
-            const int gl = u / TD, dd = u % TD;
-            const int ga = ga0 + gl, de = de0 + dd;
-            float v = 0.f;
-            if (ga < c && de < d) v = g[(n0 + kr) * out_w + ((int64_t)al * c + ga) * d + de];
-            gs[(kr * TD + dd) * SW + gl] = v;
-        }
+        stage_rows<TD>(xs, SX, x, in_w, n0, r1, kb, al * b + be0, TB, al * b + b, d, de0, t.vx);
+        stage_rows<TD>(gs, SW, g, out_w, n0, r1, kb, al * c + ga0, TC, al * c + c, d, de0, t.vw);
         __syncthreads();
         if (active) {
             for (int kr = kg; kr < kb; kr += KG) {
@@ -426,20 +547,47 @@ kron_status_t ks_check(int64_t N, int a, int b, int c, int d, kron_dtype_t dtype
 
 bool a4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
 
-cudaError_t launch_fwd(bool tr, const float *in, const float *w, const float *bias, float *out,
-                       int64_t N, int a, int kin, int kout, int d, cudaStream_t st) {
-    const KsTile t = fwd_tile(kin, kout, d);
+template <int TD>
+void fwd_launch_td(unsigned grid, size_t smem, cudaStream_t st, const float *in, const float *w,
+                   const float *bias, float *out, int64_t N, int a, int kin, int kout, int d,
+                   const KsTile &t, int64_t tiles) {
+    ks_fwd_kernel<TD><<<grid, kThreads, smem, st>>>(in, w, bias, out, N, a, kin, kout, d, t,
+                                                    tiles);
+}
+
+// out = in K' (+ bias) for the KS matrix K' with blocks w [a][d][kin][kout].
+cudaError_t launch_fwd(const float *in, const float *w, const float *bias, float *out, int64_t N,
+                       int a, int kin, int kout, int d, cudaStream_t st) {
+    const KsTile t = fwd_tile(kin, kout, d, in, w);
     const int64_t tiles = (N + (int64_t)t.GR * kR - 1) / ((int64_t)t.GR * kR) * a *
                           cdiv(d, t.TD) * cdiv(kout, (int64_t)t.GC * kC);
     const unsigned grid = (unsigned)(tiles < (1 << 30) ? tiles : (1 << 30));
     const size_t smem = tile_smem(t);
-    if (tr)
-        ks_fwd_kernel<true><<<grid, kThreads, smem, st>>>(in, w, nullptr, out, N, a, kin, kout, d,
-                                                          t, tiles);
-    else
-        ks_fwd_kernel<false><<<grid, kThreads, smem, st>>>(in, w, bias, out, N, a, kin, kout, d,
-                                                           t, tiles);
+    switch (t.TD) {
+    case 1: fwd_launch_td<1>(grid, smem, st, in, w, bias, out, N, a, kin, kout, d, t, tiles); break;
+    case 2: fwd_launch_td<2>(grid, smem, st, in, w, bias, out, N, a, kin, kout, d, t, tiles); break;
+    case 4: fwd_launch_td<4>(grid, smem, st, in, w, bias, out, N, a, kin, kout, d, t, tiles); break;
+    default: fwd_launch_td<8>(grid, smem, st, in, w, bias, out, N, a, kin, kout, d, t, tiles); break;
+    }
     return cudaGetLastError();
+}
+
+cudaError_t launch_dw(const DwPlan &P, const float *x, const float *g, float *part, int64_t N,
+                      int a, int b, int c, int d, cudaStream_t st) {
+    const unsigned grid = (unsigned)(P.parts * P.tiles_per_part);
+    const size_t smem = tile_smem(P.t);
+    switch (P.t.TD) {
+    case 1: ks_dw_kernel<1><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
+    case 2: ks_dw_kernel<2><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
+    case 4: ks_dw_kernel<4><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
+    default: ks_dw_kernel<8><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
+    }
+    return cudaGetLastError();
+}
+
+// Workspace: [K^T's blocks: a*b*c*d floats, padded to 64][parts x part_stride partials].
+size_t wt_floats(int a, int b, int c, int d) {
+    return ((size_t)a * b * c * d + 63) & ~(size_t)63;
 }
 
 }  // namespace
@@ -451,9 +599,8 @@ size_t ks_linear_workspace_size(int64_t N, int a, int b, int c, int d, kron_dtyp
     if ((int64_t)a * b * d > kMaxWidth || (int64_t)a * c * d > kMaxWidth ||
         N > ((int64_t)1 << 40))
         return 0;
-    const DwPlan P = dw_plan(N, a, b, c, d);
-    const size_t bytes = (size_t)P.parts * P.part_stride * 4;
-    return bytes < 256 ? 256 : bytes;
+    const DwPlan P = dw_plan(N, a, b, c, d, nullptr, nullptr);  // sizes do not depend on pointers
+    return (wt_floats(a, b, c, d) + (size_t)P.parts * P.part_stride) * 4;
 }
 
 kron_status_t ks_linear_forward(const void *x, const void *w, const void *bias, void *y,
@@ -466,9 +613,8 @@ kron_status_t ks_linear_forward(const void *x, const void *w, const void *bias, 
     if (!a4(x) || !a4(w) || !a4(bias) || !a4(y))
         return ks_fail(KRON_ERR_ALIGNMENT, "tensors must be 4-byte aligned");
     if (N == 0) return KRON_OK;
-    const cudaError_t e = launch_fwd(false, (const float *)x, (const float *)w,
-                                     (const float *)bias, (float *)y, N, a, b, c, d,
-                                     (cudaStream_t)stream);
+    const cudaError_t e = launch_fwd((const float *)x, (const float *)w, (const float *)bias,
+                                     (float *)y, N, a, b, c, d, (cudaStream_t)stream);
     if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS forward launch: %s", cudaGetErrorString(e));
     return KRON_OK;
 }
@@ -498,20 +644,22 @@ kron_status_t ks_linear_backward(const void *x, const void *w, const void *dY, v
         if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS zero fill: %s", cudaGetErrorString(e));
         return KRON_OK;
     }
+    float *wt = static_cast<float *>(workspace);
+    float *part = wt + wt_floats(a, b, c, d);
     if (dX) {
-        e = launch_fwd(true, (const float *)dY, (const float *)w, nullptr, (float *)dX, N, a, c, b,
-                       d, cs);
+        const size_t tb = (nw + 255) / 256;
+        ks_transpose_kernel<<<(unsigned)(tb < 2048 ? tb : 2048), 256, 0, cs>>>(
+            (const float *)w, wt, (int64_t)a * d, b, c);
+        e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = launch_fwd((const float *)dY, wt, nullptr, (float *)dX, N, a, c, b, d, cs);
         if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS dX launch: %s", cudaGetErrorString(e));
     }
-    const DwPlan P = dw_plan(N, a, b, c, d);
-    const int64_t grid = P.parts * P.tiles_per_part;
-    if (grid > 0x7fffffff)
-        return ks_fail(KRON_ERR_UNSUPPORTED, "too many dw tiles (%lld)", (long long)grid);
-    float *part = static_cast<float *>(workspace);
-    ks_dw_kernel<<<(unsigned)grid, kThreads, tile_smem(P.t), cs>>>(
-        (const float *)x, (const float *)dY, part, N, a, b, c, d, P.t, P.rows_per_part,
-        P.part_stride);
-    e = cudaGetLastError();
+    const DwPlan P = dw_plan(N, a, b, c, d, x, dY);
+    if (P.parts * P.tiles_per_part > 0x7fffffff)
+        return ks_fail(KRON_ERR_UNSUPPORTED, "too many dw tiles (%lld)",
+                       (long long)(P.parts * P.tiles_per_part));
+    e = launch_dw(P, (const float *)x, (const float *)dY, part, N, a, b, c, d, cs);
     if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS dw launch: %s", cudaGetErrorString(e));
     const size_t total = nw + (dbias ? nb : 0);
     const size_t blocks = (total + 255) / 256;

@@ -299,7 +299,8 @@ def test_ks_workspace_size():
     n = native.ks_workspace_size(20000, 1, 32, 32, 32)
     assert n > 0 and n % 256 == 0
     assert n == native.ks_workspace_size(20000, 1, 32, 32, 32)
-    assert native.ks_workspace_size(0, 1, 32, 32, 32) == 256           # empty batch: valid
+    n0 = native.ks_workspace_size(0, 1, 32, 32, 32)                  # empty batch: valid
+    assert n0 > 0 and n0 % 256 == 0
     assert native.ks_workspace_size(-1, 1, 32, 32, 32) == 0
     assert native.load().ks_linear_workspace_size(100, 1, 2, 2, 1, 1) == 0   # TF32: unsupported
     # the partials grow with the rows until every part has its chunk, then stay fixed
