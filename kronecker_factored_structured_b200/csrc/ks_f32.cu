@@ -16,10 +16,10 @@
 // kernel adds the partials in a fixed order (bitwise reproducible; the row split depends on
 // the sizes only).  dbias rides along in the dw kernel.
 //
-// Thread work: a thread owns one delta, kR contiguous rows (dw: be values) and kC columns
-// GC apart (GC = column groups of the tile), so that for each of its columns the lanes of a
-// warp, which differ first in delta and then in column group, store consecutive addresses.
-// The delta stride of each shared array is padded so that those lanes hit distinct banks.
+// Thread work: a thread owns one delta, kR contiguous rows (dw: be values) and kC contiguous
+// columns, read from shared memory as float4 each step.  The lanes of a warp differ first in
+// delta (consecutive addresses in y) and then in column group; the delta stride of each
+// shared array is padded so that those lanes hit distinct banks.
 #include "../../include/ks_linear.h"
 #include "internal.h"
 
@@ -34,7 +34,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kR = 8;                   // rows (dw: be values) per thread, contiguous
-constexpr int kC = 4;                   // columns per thread, GC apart
+constexpr int kC = 4;                   // columns per thread, contiguous
 constexpr int kSmemTile = 32 * 1024;    // bytes of staged operands per CTA
 constexpr int64_t kPartTarget = 4 * 148;  // CTAs the backward's row split aims for
 constexpr int64_t kMaxWidth = 1 << 24;    // a*b*d and a*c*d
@@ -153,6 +153,16 @@ DwPlan dw_plan(int64_t N, int a, int b, int c, int d, const void *x, const void 
     const size_t nw = (size_t)a * b * c * d, nb = (size_t)a * c * d;
     P.part_stride = (nw + nb + 63) & ~(size_t)63;
     return P;
+}
+
+// Small blocks: row ranges so that about kSmallTarget threads run (sizes only).
+constexpr int64_t kSmallTarget = 148 * 1024;
+bool small_blocks(int kin, int kout) { return kin <= 4 && kout <= 4; }
+int64_t small_ranges(int64_t N, int a, int d) {
+    if (N <= 0) return 0;
+    const int64_t threads = (int64_t)cdiv((int64_t)a * d, 128) * 128;
+    int64_t r = (kSmallTarget + threads - 1) / threads;
+    return r < 1 ? 1 : (r > N ? N : r);
 }
 
 // Staging of row slices into shared memory.  Element (row rr, slice position u), with
@@ -325,19 +335,22 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
             }
             __syncthreads();
             if (active) {
+                const float *xr = xs + dl * SX + rg * kR;
+                const float *wr = ws + dl * SW + cg * kC;
+                const int xstep = TD * SX, wstep = TD * SW;
+#pragma unroll 2
                 for (int kk = 0; kk < kb; ++kk) {
-                    const float *xr = xs + (kk * TD + dl) * SX + rg * kR;
                     const float4 x0 = *reinterpret_cast<const float4 *>(xr);
                     const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
+                    const float4 w4 = *reinterpret_cast<const float4 *>(wr);
                     const float xv[kR] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    const float *wr = ws + (kk * TD + dl) * SW + cg;
-                    float wv[kC];
-#pragma unroll
-                    for (int jj = 0; jj < kC; ++jj) wv[jj] = wr[jj * GC];
+                    const float wv[kC] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                     for (int i = 0; i < kR; ++i)
 #pragma unroll
                         for (int jj = 0; jj < kC; ++jj) acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
+                    xr += xstep;
+                    wr += wstep;
                 }
             }
             __syncthreads();
@@ -347,7 +360,7 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
             const int de = de0 + dl;
 #pragma unroll
             for (int jj = 0; jj < kC; ++jj) {
-                const int j = j0 + cg + jj * GC;
+                const int j = j0 + cg * kC + jj;
                 if (j >= kout) continue;
                 const int64_t col = ((int64_t)al * kout + j) * d + de;
                 const float bv = bias ? bias[col] : 0.f;
@@ -372,6 +385,96 @@ __global__ void ks_transpose_kernel(const float *__restrict__ w, float *__restri
         const int ga = rem / b, be = rem - ga * b;
         wt[e] = w[(blk * b + be) * c + ga];
     }
+}
+
+// Small blocks (b, c <= 4, e.g. the 2 x 2 blocks of butterfly factors): a stream with no
+// shared memory.  Thread m = al*d + de keeps the b x c block w[al][de] in registers and runs
+// over a range of rows: per row it loads its b inputs (stride d; consecutive threads take
+// consecutive de, so each load instruction of a warp reads consecutive addresses wherever
+// d >= 32) and stores c outputs.  Grid: x over m in blocks of kSmallThreads, y over row
+// ranges of `rows` rows.
+constexpr int kSmallThreads = 128;
+constexpr int kSmallMax = 4;
+
+template <int B, int C>
+__global__ void __launch_bounds__(kSmallThreads)
+ks_small_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
+                    const float *__restrict__ bias, float *__restrict__ out, int64_t N, int a,
+                    int d, int64_t rows) {
+    const int64_t m = (int64_t)blockIdx.x * kSmallThreads + threadIdx.x;
+    if (m >= (int64_t)a * d) return;
+    const int64_t al = m / d, de = m - al * d;
+    float wv[B][C], bv[C];
+#pragma unroll
+    for (int be = 0; be < B; ++be)
+#pragma unroll
+        for (int ga = 0; ga < C; ++ga) wv[be][ga] = w[(m * B + be) * C + ga];
+#pragma unroll
+    for (int ga = 0; ga < C; ++ga) bv[ga] = bias ? bias[(al * C + ga) * d + de] : 0.f;
+    const int64_t in_w = (int64_t)a * B * d, out_w = (int64_t)a * C * d;
+    const float *src = in + al * B * d + de;
+    float *dst = out + al * C * d + de;
+    const int64_t n0 = (int64_t)blockIdx.y * rows;
+    const int64_t n1 = n0 + rows < N ? n0 + rows : N;
+#pragma unroll 4
+    for (int64_t n = n0; n < n1; ++n) {
+        float xv[B];
+#pragma unroll
+        for (int be = 0; be < B; ++be) xv[be] = src[n * in_w + (int64_t)be * d];
+#pragma unroll
+        for (int ga = 0; ga < C; ++ga) {
+            float acc = 0.f;
+#pragma unroll
+            for (int be = 0; be < B; ++be) acc = fmaf(xv[be], wv[be][ga], acc);
+            dst[n * out_w + (int64_t)ga * d] = acc + bv[ga];
+        }
+    }
+}
+
+// dw / dbias partials of small blocks: thread m sums x^T dY of its block over the row range
+// blockIdx.y (rows [y*rows, (y+1)*rows)) and writes part[y] in the layout of ks_dw_kernel.
+template <int B, int C>
+__global__ void __launch_bounds__(kSmallThreads)
+ks_small_dw_kernel(const float *__restrict__ x, const float *__restrict__ g,
+                   float *__restrict__ part, int64_t N, int a, int d, int64_t rows,
+                   size_t part_stride) {
+    const int64_t m = (int64_t)blockIdx.x * kSmallThreads + threadIdx.x;
+    if (m >= (int64_t)a * d) return;
+    const int64_t al = m / d, de = m - al * d;
+    float acc[B][C], bacc[C];
+#pragma unroll
+    for (int ga = 0; ga < C; ++ga) {
+        bacc[ga] = 0.f;
+#pragma unroll
+        for (int be = 0; be < B; ++be) acc[be][ga] = 0.f;
+    }
+    const int64_t in_w = (int64_t)a * B * d, out_w = (int64_t)a * C * d;
+    const float *xs = x + al * B * d + de;
+    const float *gs = g + al * C * d + de;
+    const int64_t n0 = (int64_t)blockIdx.y * rows;
+    const int64_t n1 = n0 + rows < N ? n0 + rows : N;
+#pragma unroll 4
+    for (int64_t n = n0; n < n1; ++n) {
+        float xv[B], gv[C];
+#pragma unroll
+        for (int be = 0; be < B; ++be) xv[be] = xs[n * in_w + (int64_t)be * d];
+#pragma unroll
+        for (int ga = 0; ga < C; ++ga) gv[ga] = gs[n * out_w + (int64_t)ga * d];
+#pragma unroll
+        for (int ga = 0; ga < C; ++ga) {
+            bacc[ga] += gv[ga];
+#pragma unroll
+            for (int be = 0; be < B; ++be) acc[be][ga] = fmaf(xv[be], gv[ga], acc[be][ga]);
+        }
+    }
+    float *pw = part + (size_t)blockIdx.y * part_stride;
+#pragma unroll
+    for (int be = 0; be < B; ++be)
+#pragma unroll
+        for (int ga = 0; ga < C; ++ga) pw[(m * B + be) * C + ga] = acc[be][ga];
+    const size_t nw = (size_t)a * B * C * d;
+#pragma unroll
+    for (int ga = 0; ga < C; ++ga) pw[nw + (al * C + ga) * d + de] = bacc[ga];
 }
 
 // Partial sums of dw (and dbias) over one contiguous row range per CTA.  Grid = parts x
@@ -423,15 +526,17 @@ ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__
         stage_rows<TD>(gs, SW, g, out_w, n0, r1, kb, al * c + ga0, TC, al * c + c, d, de0, t.vw);
         __syncthreads();
         if (active) {
+            const float *xr = xs + (kg * TD + dl) * SX + bg * kR;
+            const float *gr = gs + (kg * TD + dl) * SW + cg * kC;
+            const int xstep = KG * TD * SX, gstep = KG * TD * SW;
             for (int kr = kg; kr < kb; kr += KG) {
-                const float *xr = xs + (kr * TD + dl) * SX + bg * kR;
                 const float4 x0 = *reinterpret_cast<const float4 *>(xr);
                 const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
+                const float4 g4 = *reinterpret_cast<const float4 *>(gr);
                 const float xv[kR] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                const float *gr = gs + (kr * TD + dl) * SW + cg;
-                float gv[kC];
-#pragma unroll
-                for (int jj = 0; jj < kC; ++jj) gv[jj] = gr[jj * GC];
+                const float gv[kC] = {g4.x, g4.y, g4.z, g4.w};
+                xr += xstep;
+                gr += gstep;
 #pragma unroll
                 for (int i = 0; i < kR; ++i)
 #pragma unroll
@@ -486,7 +591,7 @@ ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__
             if (be >= b) continue;
 #pragma unroll
             for (int jj = 0; jj < kC; ++jj) {
-                const int ga = ga0 + cg + jj * GC;
+                const int ga = ga0 + cg * kC + jj;
                 if (ga < c) pw[(((int64_t)al * d + de) * b + be) * c + ga] = acc[i][jj];
             }
         }
@@ -494,7 +599,7 @@ ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__
             const size_t nw = (size_t)a * b * c * d;
 #pragma unroll
             for (int jj = 0; jj < kC; ++jj) {
-                const int ga = ga0 + cg + jj * GC;
+                const int ga = ga0 + cg * kC + jj;
                 if (ga < c) pw[nw + ((size_t)al * c + ga) * d + de] = bacc[jj];
             }
         }
@@ -555,9 +660,51 @@ void fwd_launch_td(unsigned grid, size_t smem, cudaStream_t st, const float *in,
                                                     tiles);
 }
 
+template <int B, int C>
+void small_launch(bool dw, dim3 grid, cudaStream_t st, const float *in, const float *w,
+                  const float *bias, float *out, int64_t N, int a, int d, int64_t rows,
+                  size_t part_stride) {
+    if (dw)
+        ks_small_dw_kernel<B, C><<<grid, kSmallThreads, 0, st>>>(in, w, out, N, a, d, rows,
+                                                                  part_stride);
+    else
+        ks_small_fwd_kernel<B, C><<<grid, kSmallThreads, 0, st>>>(in, w, bias, out, N, a, d, rows);
+}
+
+template <int B>
+void small_launch_c(int c, bool dw, dim3 grid, cudaStream_t st, const float *in, const float *w,
+                    const float *bias, float *out, int64_t N, int a, int d, int64_t rows,
+                    size_t ps) {
+    switch (c) {
+    case 1: small_launch<B, 1>(dw, grid, st, in, w, bias, out, N, a, d, rows, ps); break;
+    case 2: small_launch<B, 2>(dw, grid, st, in, w, bias, out, N, a, d, rows, ps); break;
+    case 3: small_launch<B, 3>(dw, grid, st, in, w, bias, out, N, a, d, rows, ps); break;
+    default: small_launch<B, 4>(dw, grid, st, in, w, bias, out, N, a, d, rows, ps); break;
+    }
+}
+
+// Small-block stream: forward (dw = false: in, w, bias -> out) or dw partials (dw = true:
+// in = x, w = dY, out = partials).  b, c <= 4.
+cudaError_t launch_small(bool dw, const float *in, const float *w, const float *bias, float *out,
+                         int64_t N, int a, int b, int c, int d, size_t part_stride,
+                         cudaStream_t st) {
+    const int64_t R = small_ranges(N, a, d);
+    const int64_t rows = (N + R - 1) / R;
+    const dim3 grid((unsigned)cdiv((int64_t)a * d, kSmallThreads), (unsigned)R);
+    switch (b) {
+    case 1: small_launch_c<1>(c, dw, grid, st, in, w, bias, out, N, a, d, rows, part_stride); break;
+    case 2: small_launch_c<2>(c, dw, grid, st, in, w, bias, out, N, a, d, rows, part_stride); break;
+    case 3: small_launch_c<3>(c, dw, grid, st, in, w, bias, out, N, a, d, rows, part_stride); break;
+    default: small_launch_c<4>(c, dw, grid, st, in, w, bias, out, N, a, d, rows, part_stride); break;
+    }
+    return cudaGetLastError();
+}
+
 // out = in K' (+ bias) for the KS matrix K' with blocks w [a][d][kin][kout].
 cudaError_t launch_fwd(const float *in, const float *w, const float *bias, float *out, int64_t N,
                        int a, int kin, int kout, int d, cudaStream_t st) {
+    if (small_blocks(kin, kout))
+        return launch_small(false, in, w, bias, out, N, a, kin, kout, d, 0, st);
     const KsTile t = fwd_tile(kin, kout, d, in, w);
     const int64_t tiles = (N + (int64_t)t.GR * kR - 1) / ((int64_t)t.GR * kR) * a *
                           cdiv(d, t.TD) * cdiv(kout, (int64_t)t.GC * kC);
@@ -600,7 +747,8 @@ size_t ks_linear_workspace_size(int64_t N, int a, int b, int c, int d, kron_dtyp
         N > ((int64_t)1 << 40))
         return 0;
     const DwPlan P = dw_plan(N, a, b, c, d, nullptr, nullptr);  // sizes do not depend on pointers
-    return (wt_floats(a, b, c, d) + (size_t)P.parts * P.part_stride) * 4;
+    const int64_t parts = small_blocks(b, c) ? small_ranges(N, a, d) : P.parts;
+    return (wt_floats(a, b, c, d) + (size_t)parts * P.part_stride) * 4;
 }
 
 kron_status_t ks_linear_forward(const void *x, const void *w, const void *bias, void *y,
@@ -656,15 +804,22 @@ kron_status_t ks_linear_backward(const void *x, const void *w, const void *dY, v
         if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS dX launch: %s", cudaGetErrorString(e));
     }
     const DwPlan P = dw_plan(N, a, b, c, d, x, dY);
-    if (P.parts * P.tiles_per_part > 0x7fffffff)
-        return ks_fail(KRON_ERR_UNSUPPORTED, "too many dw tiles (%lld)",
-                       (long long)(P.parts * P.tiles_per_part));
-    e = launch_dw(P, (const float *)x, (const float *)dY, part, N, a, b, c, d, cs);
+    int64_t parts = P.parts;
+    if (small_blocks(b, c)) {
+        parts = small_ranges(N, a, d);
+        e = launch_small(true, (const float *)x, (const float *)dY, nullptr, part, N, a, b, c, d,
+                         P.part_stride, cs);
+    } else {
+        if (P.parts * P.tiles_per_part > 0x7fffffff)
+            return ks_fail(KRON_ERR_UNSUPPORTED, "too many dw tiles (%lld)",
+                           (long long)(P.parts * P.tiles_per_part));
+        e = launch_dw(P, (const float *)x, (const float *)dY, part, N, a, b, c, d, cs);
+    }
     if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS dw launch: %s", cudaGetErrorString(e));
     const size_t total = nw + (dbias ? nb : 0);
     const size_t blocks = (total + 255) / 256;
     ks_reduce_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, cs>>>(
-        part, P.parts, P.part_stride, nw, nb, (float *)dw, (float *)dbias);
+        part, parts, P.part_stride, nw, nb, (float *)dw, (float *)dbias);
     e = cudaGetLastError();
     if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS reduce launch: %s", cudaGetErrorString(e));
     return KRON_OK;
