@@ -1,4 +1,5 @@
-"""Data-parallel plumbing for the Kronecker layer: row sharding and the one gradient exchange.
+"""Data-parallel plumbing for the Kronecker layer (and the Kronecker-sparse factor): row sharding
+and the one gradient exchange.
 
 Rows are independent (page "kronecker-layer-benchmark", section "Setup": a batch is just rows
 fed to the layer), so N rows split into contiguous per-rank ranges and the forward needs no
@@ -30,11 +31,28 @@ def param_grad_sizes(p: int, q: int, m1: int, m2: int, r: int) -> Dict[str, tupl
     return {"dS": (p, q), "dA": (r, p, q), "dB": (r, m1, m2), "dbias": (q * m2,)}
 
 
+def ks_param_grad_sizes(a: int, b: int, c: int, d: int) -> Dict[str, tuple]:
+    """Shapes of a Kronecker-sparse factor's parameter gradients (pattern (a, b, c, d))."""
+    return {"dw": (a, d, b, c), "dbias": (a * c * d,)}
+
+
 def flat_grad_buffer(p: int, q: int, m1: int, m2: int, r: int,
                      device="cpu") -> Tuple[torch.Tensor, Dict[str, torch.Tensor]]:
     """One fp32 buffer holding dS, dA, dB, dbias back to back, and a view of it per gradient
     (the layout the backward call writes into through `grads=`)."""
-    shapes = param_grad_sizes(p, q, m1, m2, r)
+    return flat_buffer(param_grad_sizes(p, q, m1, m2, r), device)
+
+
+def ks_flat_grad_buffer(a: int, b: int, c: int, d: int,
+                        device="cpu") -> Tuple[torch.Tensor, Dict[str, torch.Tensor]]:
+    """The same for a Kronecker-sparse factor: dw and dbias as views of one buffer, so its
+    data-parallel backward also exchanges one all-reduce per step."""
+    return flat_buffer(ks_param_grad_sizes(a, b, c, d), device)
+
+
+def flat_buffer(shapes: Dict[str, tuple],
+                device="cpu") -> Tuple[torch.Tensor, Dict[str, torch.Tensor]]:
+    """One zeroed fp32 buffer and a view of it per named shape, back to back in dict order."""
     total = sum(int(torch.Size(s).numel()) for s in shapes.values())
     flat = torch.zeros(total, dtype=torch.float32, device=device)
     views, o = {}, 0

@@ -5,9 +5,11 @@
  * pointers below are never dereferenced: each call fails a host check.
  *
  * Built and run by tests/test_c_abi.py; exits 0 when every check passes, else prints the
- * failing check and exits 1.
+ * failing check and exits 1.  The Kronecker-sparse factor's header (ks_linear.h) is
+ * compiled and checked the same way.
  */
 #include "kron_linear.h"
+#include "ks_linear.h"
 
 #include <stdint.h>
 #include <stdio.h>
@@ -127,6 +129,44 @@ int main(void) {
           KRON_ERR_ALIGNMENT);
     CHECK(kron_vanloan_fit(P, 4, 4, 4, 4, 2, P, 8, 2, 1, P, P, P, P, NULL, 0, NULL) ==
           KRON_ERR_WORKSPACE);
+
+    /* Kronecker-sparse factor: FP32 only, natural 4-byte alignment, host checks first */
+    {
+        void *const MIS2 = (void *)(uintptr_t)0x10002; /* not 4-byte aligned */
+        size_t ks_need = ks_linear_workspace_size(20000, 1, 32, 32, 32, KRON_F32);
+        CHECK(ks_need > 0 && ks_need % 256 == 0);
+        CHECK(ks_need == ks_linear_workspace_size(20000, 1, 32, 32, 32, KRON_F32));
+        CHECK(ks_linear_workspace_size(20000, 1, 32, 32, 32, KRON_TF32) == 0);
+        CHECK(ks_linear_workspace_size(-1, 1, 32, 32, 32, KRON_F32) == 0);
+        CHECK(ks_linear_workspace_size(8, 0, 32, 32, 32, KRON_F32) == 0);
+        CHECK(ks_linear_forward(P, P, NULL, P, 8, 2, 3, 4, 5, (kron_dtype_t)9, 0, NULL) ==
+              KRON_ERR_INVALID_ARG);
+        CHECK(ks_linear_forward(P, P, NULL, P, 8, 2, 3, 4, 5, KRON_TF32, 0, NULL) ==
+              KRON_ERR_UNSUPPORTED);
+        CHECK(ks_linear_forward(P, P, NULL, P, 8, 2, 3, 4, 5, KRON_BF16, 0, NULL) ==
+              KRON_ERR_UNSUPPORTED);
+        CHECK(ks_linear_forward(P, P, NULL, P, 8, 2, 3, 4, 5, KRON_F32, 1u, NULL) ==
+              KRON_ERR_INVALID_ARG);                                        /* no flags */
+        CHECK(ks_linear_forward(P, P, NULL, P, 8, 0, 3, 4, 5, KRON_F32, 0, NULL) ==
+              KRON_ERR_INVALID_ARG);
+        CHECK(ks_linear_forward(NULL, P, NULL, P, 8, 2, 3, 4, 5, KRON_F32, 0, NULL) ==
+              KRON_ERR_INVALID_ARG);
+        CHECK(ks_linear_forward(MIS2, P, NULL, P, 8, 2, 3, 4, 5, KRON_F32, 0, NULL) ==
+              KRON_ERR_ALIGNMENT);
+        CHECK(ks_linear_forward(NULL, P, NULL, NULL, 0, 2, 3, 4, 5, KRON_F32, 0, NULL) ==
+              KRON_OK);                                                     /* N == 0 */
+        ks_need = ks_linear_workspace_size(8, 2, 3, 4, 5, KRON_F32);
+        CHECK(ks_linear_backward(P, P, P, P, NULL, NULL, 8, 2, 3, 4, 5, KRON_F32, 0, WS,
+                                 ks_need, NULL) == KRON_ERR_INVALID_ARG);   /* dw missing */
+        CHECK(ks_linear_backward(P, P, P, P, P, NULL, 8, 2, 3, 4, 5, KRON_F32, 0, NULL, 0,
+                                 NULL) == KRON_ERR_WORKSPACE);
+        CHECK(ks_linear_backward(P, P, P, P, P, NULL, 8, 2, 3, 4, 5, KRON_F32, 0, WS,
+                                 ks_need - 4, NULL) == KRON_ERR_WORKSPACE);
+        CHECK(ks_linear_backward(P, P, P, P, P, NULL, 8, 2, 3, 4, 5, KRON_F32, 0,
+                                 (char *)WS + 16, ks_need, NULL) == KRON_ERR_ALIGNMENT);
+        CHECK(ks_linear_backward(P, P, MIS2, P, P, NULL, 8, 2, 3, 4, 5, KRON_F32, 0, WS,
+                                 ks_need, NULL) == KRON_ERR_ALIGNMENT);     /* dY */
+    }
 
     if (failures) return 1;
     printf("abi_check: all checks passed\n");

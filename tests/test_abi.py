@@ -305,3 +305,18 @@ def test_ks_workspace_size():
     assert native.load().ks_linear_workspace_size(100, 1, 2, 2, 1, 1) == 0   # TF32: unsupported
     # the partials grow with the rows until every part has its chunk, then stay fixed
     assert native.ks_workspace_size(10, 32, 32, 32, 1) <= native.ks_workspace_size(20000, 32, 32, 32, 1)
+
+
+def test_ks_binding_checks_before_any_call():
+    """The binding's shape and dtype checks run before the library is called (CPU tensors)."""
+    import torch
+    w = torch.zeros(2, 5, 3, 4)                      # a = 2, d = 5, b = 3, c = 4
+    assert native.ks_pattern(w) == (2, 3, 4, 5)
+    with pytest.raises(ValueError):
+        native.ks_pattern(torch.zeros(3, 3))
+    with pytest.raises(ValueError):
+        native.ks_forward(torch.zeros(7, 29), w)     # in = a*b*d = 30
+    with pytest.raises(TypeError):
+        native.ks_forward(torch.zeros(7, 30, dtype=torch.float64), w)
+    with pytest.raises(ValueError):
+        native.ks_backward(torch.zeros(7, 30), w, torch.zeros(7, 41))   # out = a*c*d = 40

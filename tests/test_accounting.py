@@ -85,3 +85,19 @@ def test_sweep_work():
             p = 1024 // m
             assert acc.flops_per_row(p, p, m, m, r) == 6144 * r * (m + p)
     assert 20000 * acc.flops_per_row(128, 128, 8, 8, 1) == 16711680000
+
+
+def test_ks_work_counts_the_support():
+    """A KS factor's values, flops and density against the oracle's dense K (its non-zeros)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(5)
+    for a, b, c, d in ((2, 3, 4, 5), (16, 2, 2, 32), (1, 8, 16, 4)):
+        w = rng.uniform(0.5, 1.5, (a, d, b, c))
+        nnz = int(np.count_nonzero(oracle.ks_dense(w)))
+        assert acc.ks_param_count(a, b, c, d, bias=False) == nnz
+        assert acc.ks_param_count(a, b, c, d) == nnz + a * c * d
+        assert acc.ks_flops_per_row(a, b, c, d, backward=False) == 2 * nnz
+        assert acc.ks_flops_per_row(a, b, c, d) == 6 * nnz
+        # density 1 / (a d) of the dense (a b d) x (a c d) matrix
+        assert nnz * a * d == (a * b * d) * (a * c * d)

@@ -1,5 +1,6 @@
 """The C ABI from plain C: tests/abi_check.c is compiled with gcc -std=c99 -pedantic
--Werror against include/kron_linear.h, linked with libkronlinear.so and run on the host.
+-Werror against include/kron_linear.h and include/ks_linear.h, linked with libkronlinear.so and
+run on the host.
 Every call in it fails a host-side check, so no GPU is needed."""
 import os
 import shutil

@@ -158,3 +158,59 @@ def test_reference_arm_prints_once_under_two_ranks():
     import json
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+
+
+def _ks_rank_main(rank, world, port, result_q, deterministic):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+
+    import kron_workloads as kw
+    import oracle
+    from kronecker_factored_structured_b200 import dp
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = kw.ks_custom(53, 2, 3, 4, 5, seed=8)
+        d = {k: v.double().numpy() for k, v in kw.ks_inputs(w).items()}
+        start, count = dp.shard_rows(w.N, world, rank)
+        sl = slice(start, start + count)
+        g = oracle.ks_backward(d["x"][sl], d["w"], d["G"][sl])
+        flat, views = dp.ks_flat_grad_buffer(*w.pattern)
+        for k in ("dw", "dbias"):
+            views[k].copy_(torch.from_numpy(g[k]).float())
+        dp.allreduce_grads(flat, deterministic=deterministic)
+        result_q.put((rank, {k: v.double().numpy().copy() for k, v in views.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_ks_factor_ranks_sum_to_full_batch_gradients(deterministic):
+    """The Kronecker-sparse factor's data-parallel backward: row shards on two gloo ranks, dw
+    and dbias in one flat buffer, one exchange; equal to the full batch's gradients."""
+    import kron_workloads as kw
+    import oracle
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ks_rank_main, args=(r, 2, port, q, deterministic))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w = kw.ks_custom(53, 2, 3, 4, 5, seed=8)
+    d = {k: v.double().numpy() for k, v in kw.ks_inputs(w).items()}
+    full = oracle.ks_backward(d["x"], d["w"], d["G"])
+    for rank, grads in out:
+        for k in ("dw", "dbias"):
+            assert grads[k].shape == full[k].shape
+            assert np.abs(grads[k] - full[k]).max() <= 1e-6 * np.abs(full[k]).max(), (rank, k)
+    if deterministic:
+        for k in ("dw", "dbias"):
+            assert np.array_equal(out[0][1][k], out[1][1][k])
