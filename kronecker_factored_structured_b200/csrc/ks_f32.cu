@@ -11,10 +11,12 @@
 // it needs in shared memory (the gather happens on chip: x is read once per column tile and
 // y written once, no permuted copy of x or y ever reaches HBM) and runs the whole
 // contraction for its tile.  The same kernel computes dX = dY K^T with the roles of b and c
-// swapped, from a copy of the blocks transposed once per call into the workspace.  dw is a split-N reduction: each CTA sums x^T dY over one
-// contiguous row range for one tile of (al, de, be, ga) and writes a partial; a second
-// kernel adds the partials in a fixed order (bitwise reproducible; the row split depends on
-// the sizes only).  dbias rides along in the dw kernel.
+// swapped, from a copy of the blocks transposed once per call into the workspace.  dw is a
+// split-N reduction: each CTA sums x^T dY over one contiguous row range for one tile of
+// (al, de, be, ga) and writes a partial; a second kernel adds the partials in a fixed order
+// (bitwise reproducible; the row split depends on the sizes only).  dbias rides along in the
+// dw kernel.  Blocks of at most 4 x 4 (butterfly factors) skip the tiles: a register-resident
+// stream with one thread per (al, de) runs the forward, dX and the dw partials.
 //
 // Thread work: a thread owns one delta, kR contiguous rows (dw: be values) and kC contiguous
 // columns, read from shared memory as float4 each step.  The lanes of a warp differ first in
@@ -36,7 +38,9 @@ constexpr int kThreads = 256;
 constexpr int kR = 8;                   // rows (dw: be values) per thread, contiguous
 constexpr int kC = 4;                   // columns per thread, contiguous
 constexpr int kSmemTile = 32 * 1024;    // bytes of staged operands per CTA
-constexpr int64_t kPartTarget = 4 * 148;  // CTAs the backward's row split aims for
+constexpr int64_t kPartTarget = 4 * 148;  // CTAs the backward's row split aims for (a
+                                          // constant, not the device's SM count: the split,
+                                          // and so the summation order, depend on sizes only)
 constexpr int64_t kMaxWidth = 1 << 24;    // a*b*d and a*c*d
 
 struct KsTile {
@@ -157,7 +161,8 @@ DwPlan dw_plan(int64_t N, int a, int b, int c, int d, const void *x, const void 
 
 // Small blocks: row ranges so that about kSmallTarget threads run (sizes only).
 constexpr int64_t kSmallTarget = 148 * 1024;
-bool small_blocks(int kin, int kout) { return kin <= 4 && kout <= 4; }
+constexpr int kSmallMax = 4;  // largest b and c of the small-block stream
+bool small_blocks(int kin, int kout) { return kin <= kSmallMax && kout <= kSmallMax; }
 int64_t small_ranges(int64_t N, int a, int d) {
     if (N <= 0) return 0;
     const int64_t threads = (int64_t)cdiv((int64_t)a * d, 128) * 128;
@@ -325,7 +330,8 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
                 const float *wrow = w + (((int64_t)al * d + de) * kin + k0 + kk) * kout + j0;
                 if (t.vw) {
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (de < d && j0 + 4 * jq < kout) v = *reinterpret_cast<const float4 *>(wrow + 4 * jq);
+                    if (de < d && j0 + 4 * jq < kout)
+                        v = *reinterpret_cast<const float4 *>(wrow + 4 * jq);
                     *reinterpret_cast<float4 *>(ws + s * SW + 4 * jq) = v;
                 } else {
                     float v = 0.f;
@@ -348,7 +354,8 @@ ks_fwd_kernel(const float *__restrict__ in, const float *__restrict__ w,
 #pragma unroll
                     for (int i = 0; i < kR; ++i)
 #pragma unroll
-                        for (int jj = 0; jj < kC; ++jj) acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
+                        for (int jj = 0; jj < kC; ++jj)
+                            acc[i][jj] = fmaf(xv[i], wv[jj], acc[i][jj]);
                     xr += xstep;
                     wr += wstep;
                 }
@@ -394,7 +401,6 @@ __global__ void ks_transpose_kernel(const float *__restrict__ w, float *__restri
 // d >= 32) and stores c outputs.  Grid: x over m in blocks of kSmallThreads, y over row
 // ranges of `rows` rows.
 constexpr int kSmallThreads = 128;
-constexpr int kSmallMax = 4;
 
 template <int B, int C>
 __global__ void __launch_bounds__(kSmallThreads)
@@ -570,7 +576,8 @@ ks_dw_kernel(const float *__restrict__ x, const float *__restrict__ g, float *__
 #pragma unroll
                 for (int jj = 0; jj < kC; ++jj) {
                     float s = 0.f;
-                    for (int q = 0; q < KG; ++q) s += red[((size_t)q * items + it) * RS + i * kC + jj];
+                    for (int q = 0; q < KG; ++q)
+                        s += red[((size_t)q * items + it) * RS + i * kC + jj];
                     acc[i][jj] = s;
                 }
 #pragma unroll
@@ -723,11 +730,21 @@ cudaError_t launch_dw(const DwPlan &P, const float *x, const float *g, float *pa
                       int a, int b, int c, int d, cudaStream_t st) {
     const unsigned grid = (unsigned)(P.parts * P.tiles_per_part);
     const size_t smem = tile_smem(P.t);
+    const int64_t rpp = P.rows_per_part;
+    const size_t ps = P.part_stride;
     switch (P.t.TD) {
-    case 1: ks_dw_kernel<1><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
-    case 2: ks_dw_kernel<2><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
-    case 4: ks_dw_kernel<4><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
-    default: ks_dw_kernel<8><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, P.rows_per_part, P.part_stride); break;
+    case 1:
+        ks_dw_kernel<1><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, rpp, ps);
+        break;
+    case 2:
+        ks_dw_kernel<2><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, rpp, ps);
+        break;
+    case 4:
+        ks_dw_kernel<4><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, rpp, ps);
+        break;
+    default:
+        ks_dw_kernel<8><<<grid, kThreads, smem, st>>>(x, g, part, N, a, b, c, d, P.t, rpp, ps);
+        break;
     }
     return cudaGetLastError();
 }
@@ -763,7 +780,8 @@ kron_status_t ks_linear_forward(const void *x, const void *w, const void *bias, 
     if (N == 0) return KRON_OK;
     const cudaError_t e = launch_fwd((const float *)x, (const float *)w, (const float *)bias,
                                      (float *)y, N, a, b, c, d, (cudaStream_t)stream);
-    if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS forward launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess)
+        return ks_fail(KRON_ERR_CUDA, "KS forward launch: %s", cudaGetErrorString(e));
     return KRON_OK;
 }
 
@@ -789,7 +807,8 @@ kron_status_t ks_linear_backward(const void *x, const void *w, const void *dY, v
     if (N == 0) {
         e = cudaMemsetAsync(dw, 0, nw * 4, cs);
         if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, nb * 4, cs);
-        if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS zero fill: %s", cudaGetErrorString(e));
+        if (e != cudaSuccess)
+            return ks_fail(KRON_ERR_CUDA, "KS zero fill: %s", cudaGetErrorString(e));
         return KRON_OK;
     }
     float *wt = static_cast<float *>(workspace);
@@ -801,7 +820,8 @@ kron_status_t ks_linear_backward(const void *x, const void *w, const void *dY, v
         e = cudaGetLastError();
         if (e == cudaSuccess)
             e = launch_fwd((const float *)dY, wt, nullptr, (float *)dX, N, a, c, b, d, cs);
-        if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS dX launch: %s", cudaGetErrorString(e));
+        if (e != cudaSuccess)
+            return ks_fail(KRON_ERR_CUDA, "KS dX launch: %s", cudaGetErrorString(e));
     }
     const DwPlan P = dw_plan(N, a, b, c, d, x, dY);
     int64_t parts = P.parts;
@@ -821,7 +841,8 @@ kron_status_t ks_linear_backward(const void *x, const void *w, const void *dY, v
     ks_reduce_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, cs>>>(
         part, parts, P.part_stride, nw, nb, (float *)dw, (float *)dbias);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return ks_fail(KRON_ERR_CUDA, "KS reduce launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess)
+        return ks_fail(KRON_ERR_CUDA, "KS reduce launch: %s", cudaGetErrorString(e));
     return KRON_OK;
 }
 
