@@ -76,3 +76,28 @@ def test_bf16_workloads_store_bf16():
     for k in ("x", "G", "S", "A", "B", "bias"):
         assert d[k].dtype == torch.bfloat16, k
     assert d["x"].shape == (3, 3072) and d["G"].shape == (3, 768)
+
+
+def test_ks_workloads_shapes_and_draws():
+    """KS workloads: widths from the pattern, values ~ randn/sqrt(b) in the [a][d][b][c] layout,
+    seeded (the same bytes on every draw), and rows re-drawable chunk by chunk."""
+    import math
+
+    import kron_workloads as kw
+    wl = kw.ks_get("ks_monarch_tr")
+    a, b, c, d = wl.pattern
+    assert (wl.d_in, wl.d_out) == (a * b * d, a * c * d) == (1024, 1024)
+    f1, f2 = kw.ks_factors(wl), kw.ks_factors(wl)
+    assert f1["w"].shape == (a, d, b, c) and f1["bias"].shape == (a * c * d,)
+    assert torch.equal(f1["w"], f2["w"]) and torch.equal(f1["bias"], f2["bias"])
+    assert abs(f1["w"].std().item() - 1 / math.sqrt(b)) < 0.02 / math.sqrt(b) * 10
+    assert abs(f1["bias"].std().item() - wl.bias_std) < 0.02
+    small = wl.with_rows(5000)
+    full = kw.rows(small, "x")
+    assert full.shape == (5000, 1024) and full.dtype == torch.float32
+    idx = torch.tensor([4999, 0, 4096, 17])
+    assert torch.equal(kw.rows_at(small, "x", idx), full[idx])
+    assert torch.equal(kw.rows(small, "G", 4000, 4200), kw.rows(small, "G")[4000:4200])
+    # every bench pattern is a valid factor
+    for name, w in kw.ks_workloads().items():
+        assert min(w.pattern) >= 1 and w.N > 0, name
