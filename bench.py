@@ -560,30 +560,35 @@ def run_extras(kfs, steps, dev):
     return out
 
 
-def ks_bmm_context(fac, sets, pattern, steps, dev):
-    """Context only (not the product path): the Kronecker-sparse factor computed the way the
-    page "Fast Inference with Kronecker-Sparse Matrices" describes earlier GPU kernels --
-    permute x into a*d contiguous b-column slices, one batched GEMM, permute back (and the
-    same for dY in the backward: dX and dw as two more batched GEMMs), FP32 cuBLAS through
-    torch with TF32 off.  Forward + backward per step, replayed from a CUDA graph."""
+def ks_permute_bmm_step(x, G, w, bias, pattern):
+    """The Kronecker-sparse factor's forward and backward the way the page "Fast Inference
+    with Kronecker-Sparse Matrices" describes earlier GPU kernels: permute x (and dY) into
+    a*d contiguous slices, batched GEMMs, permute back.  Returns (y, dX, dw, dbias) with dw in
+    the [a][d][b][c] layout.  Context for the bench only (torch ops; any device)."""
     import torch
     a, b, c, d = pattern
-    W3 = fac["w"].reshape(a * d, b, c)
-    bias = fac["bias"]
+    N = x.shape[0]
+    W3 = w.reshape(a * d, b, c)
+    xt = x.view(N, a, b, d).permute(1, 3, 0, 2).reshape(a * d, N, b)
+    y = torch.bmm(xt, W3).view(a, d, N, c).permute(2, 0, 3, 1).reshape(N, a * c * d) + bias
+    Gt = G.view(N, a, c, d).permute(1, 3, 0, 2).reshape(a * d, N, c)
+    dx = torch.bmm(Gt, W3.transpose(1, 2)).view(a, d, N, b).permute(2, 0, 3, 1).reshape(
+        N, a * b * d)
+    dw = torch.bmm(xt.transpose(1, 2), Gt).view(a, d, b, c)
+    db = G.sum(0)
+    return y, dx, dw, db
+
+
+def ks_bmm_context(fac, sets, pattern, steps, dev):
+    """Context only (not the product path): `ks_permute_bmm_step` (FP32 cuBLAS through torch,
+    TF32 off) on the same inputs, forward + backward per step, replayed from a CUDA graph."""
+    import torch
     old = torch.backends.cuda.matmul.allow_tf32
     torch.backends.cuda.matmul.allow_tf32 = False
     try:
         def step(i):
             x, G = sets[i % len(sets)]
-            N = x.shape[0]
-            xt = x.view(N, a, b, d).permute(1, 3, 0, 2).reshape(a * d, N, b)
-            y = torch.bmm(xt, W3).view(a, d, N, c).permute(2, 0, 3, 1).reshape(N, a * c * d) + bias
-            Gt = G.view(N, a, c, d).permute(1, 3, 0, 2).reshape(a * d, N, c)
-            dx = torch.bmm(Gt, W3.transpose(1, 2)).view(a, d, N, b).permute(2, 0, 3, 1).reshape(
-                N, a * b * d)
-            dw = torch.bmm(xt.transpose(1, 2), Gt)
-            db = G.sum(0)
-            return y, dx, dw, db
+            return ks_permute_bmm_step(x, G, fac["w"], fac["bias"], pattern)
         for i in range(3):
             step(i)
         torch.cuda.synchronize()

@@ -93,3 +93,26 @@ def test_without_nvml_the_summary_falls_back(monkeypatch):
     cs.nvml, cs.lines = reg, ["0, 1965, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, Active"]
     s = cs.summary()
     assert s["sm_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 1
+
+
+def test_ks_permute_bmm_context_computes_the_factor():
+    """The bench's permute + batched-GEMM context computes the same factor and gradients as
+    the oracle (so its timing is of the same work)."""
+    import numpy as np
+    import torch
+
+    import bench
+    import oracle
+    a, b, c, d, N = 3, 4, 5, 6, 7
+    g = torch.Generator().manual_seed(0)
+    w = torch.randn(a, d, b, c, generator=g, dtype=torch.float64)
+    bias = torch.randn(a * c * d, generator=g, dtype=torch.float64)
+    x = torch.randn(N, a * b * d, generator=g, dtype=torch.float64)
+    G = torch.randn(N, a * c * d, generator=g, dtype=torch.float64)
+    y, dx, dw, db = bench.ks_permute_bmm_step(x, G, w, bias, (a, b, c, d))
+    ref = oracle.ks_backward(x.numpy(), w.numpy(), G.numpy())
+    assert np.allclose(y.numpy(), oracle.ks_forward(x.numpy(), w.numpy(), bias.numpy()),
+                       rtol=0, atol=1e-12)
+    assert np.allclose(dx.numpy(), ref["dX"], rtol=0, atol=1e-12)
+    assert np.allclose(dw.numpy(), ref["dw"], rtol=0, atol=1e-12)
+    assert np.allclose(db.numpy(), ref["dbias"], rtol=0, atol=1e-12)
